@@ -1,0 +1,371 @@
+"""Pins for the CPU oracle, checked against things other than the oracle itself:
+closed forms, a hand-worked example, other library routines, Monte-Carlo
+moments, brute force on tiny inputs and exact identities from the pages.
+CPU only (no GPU marker)."""
+
+import itertools
+import json
+import math
+import os
+import statistics
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+
+
+RNG = np.random.default_rng(1234)
+
+
+def _x(shape, rng=RNG, scale=1.0):
+    return rng.standard_normal(shape) * scale
+
+
+# ---------------------------------------------------------------- block stats
+
+def test_block_stats_arithmetic_sequence_closed_form():
+    # rows x_r = a + r*delta: mean a + delta (n-1)/2, population variance delta^2 (n^2-1)/12
+    b, N, d = 8, 21, 3            # blocks of 8, 8, 5 rows (ragged tail)
+    a = np.array([0.5, -2.0, 7.0])
+    delta = np.array([1.0, 0.25, -3.0])
+    X = np.zeros((1, 1, 24, d))
+    for i in range(3):
+        for r in range(8):
+            X[0, 0, i * b + r] = a + r * delta
+    X[0, 0, N:] = 1e30                       # padding must never be read
+    mean, var, counts = O.block_stats(X, N, b)
+    assert counts.tolist() == [8, 8, 5]
+    for i, n in enumerate([8, 8, 5]):
+        np.testing.assert_allclose(mean[0, 0, i], a + delta * (n - 1) / 2, rtol=1e-14)
+        np.testing.assert_allclose(var[0, 0, i], delta ** 2 * (n * n - 1) / 12, rtol=1e-12)
+
+
+def test_block_stats_vs_statistics_module():
+    X = _x((2, 3, 40, 4))
+    mean, var, _ = O.block_stats(X, 37, 16)
+    for bb, h, i, m in itertools.product(range(2), range(3), range(3), range(4)):
+        col = X[bb, h, i * 16: min(37, (i + 1) * 16), m].tolist()
+        assert math.isclose(mean[bb, h, i, m], statistics.fmean(col), rel_tol=1e-12, abs_tol=1e-14)
+        assert math.isclose(var[bb, h, i, m], statistics.pvariance(col), rel_tol=1e-10, abs_tol=1e-14)
+
+
+def test_block_stats_shift_invariance_and_nonnegative():
+    X = _x((1, 2, 64, 8))
+    c = _x((8,)) * 100
+    m1, v1, _ = O.block_stats(X, 64, 16)
+    m2, v2, _ = O.block_stats(X + c, 64, 16)
+    np.testing.assert_allclose(m2, m1 + c, rtol=1e-12, atol=1e-10)
+    np.testing.assert_allclose(v2, v1, rtol=1e-8, atol=1e-9)
+    assert (v1 >= 0).all()
+
+
+# ------------------------------------------------------------ hand-worked case
+
+def _golden():
+    here = os.path.join(os.path.dirname(__file__), "golden", "hand_worked_tiny.json")
+    with open(here) as f:
+        return json.load(f)
+
+
+def test_hand_worked_stats_scores_selection():
+    g = _golden()
+    Q = np.array(g["Q"], dtype=float)[None, None]
+    K = np.array(g["K"], dtype=float)[None, None]
+    qm, qv, qc = O.block_stats(Q, 4, g["block"])
+    km, kv, kc = O.block_stats(K, 4, g["block"])
+    np.testing.assert_array_equal(qm[0, 0], g["q_mean"])
+    np.testing.assert_array_equal(qv[0, 0], g["q_var"])
+    np.testing.assert_array_equal(km[0, 0], g["k_mean"])
+    np.testing.assert_array_equal(kv[0, 0], g["k_var"])
+    S = O.corrected_scores(qm, qv, km, kv, kc, g["sm_scale"])
+    P = O.pooled_scores(qm, km, kc, g["sm_scale"])
+    np.testing.assert_allclose(S[0, 0] - math.log(2), g["scores_minus_ln2"], atol=1e-14)
+    np.testing.assert_allclose(P[0, 0] - math.log(2), g["pooled_minus_ln2"], atol=1e-14)
+    k = O.keep_count(g["keep"], 2)
+    idx, cnt = O.select_topk(S, k)
+    assert idx[0, 0].tolist() == g["kept_corrected"]
+    idx, cnt = O.select_topk(P, k)
+    assert idx[0, 0].tolist() == g["kept_pooled"]
+
+
+def test_hand_worked_merge():
+    m = _golden()["merge"]
+    Om, Lm = O.merge_lse(np.array(m["O1"]), np.array(m["L1"]), np.array(m["O2"]),
+                         np.array(math.log(m["L2_is_ln"])))
+    np.testing.assert_allclose(Om, m["O"], atol=1e-15)
+    assert math.isclose(float(Lm), math.log(m["L_is_ln"]), rel_tol=1e-15)
+
+
+# ------------------------------------------------------------ corrected score
+
+def _rand_stats(nq=5, nk=7, d=6, Hq=4, Hkv=2, rng=RNG):
+    qm = rng.standard_normal((1, Hq, nq, d))
+    qv = rng.uniform(0.1, 2.0, (1, Hq, nq, d))
+    km = rng.standard_normal((1, Hkv, nk, d))
+    kv = rng.uniform(0.1, 2.0, (1, Hkv, nk, d))
+    counts = rng.integers(1, 64, nk)
+    return qm, qv, km, kv, counts
+
+
+def test_zero_variance_reduces_to_pooled():
+    # check (3): with zero within-block variance the correction vanishes
+    qm, _, km, _, counts = _rand_stats()
+    S = O.corrected_scores(qm, np.zeros_like(qm), km, np.zeros_like(km), counts, 0.37)
+    P = O.pooled_scores(qm, km, counts, 0.37)
+    np.testing.assert_array_equal(S, P)
+
+
+def test_jensen_correction_is_nonnegative():
+    qm, qv, km, kv, counts = _rand_stats()
+    S = O.corrected_scores(qm, qv, km, kv, counts, 0.37)
+    P = O.pooled_scores(qm, km, counts, 0.37)
+    assert (S >= P).all()
+    assert (S > P).mean() > 0.99
+
+
+def test_identical_token_blocks_pre_equals_post():
+    # every token in a block equal to its block mean: the pre-downsample map
+    # equals the exact post-downsample map (closed form of both)
+    rng = np.random.default_rng(7)
+    b, nb, d = 4, 6, 8
+    N = b * nb - 2                               # ragged last block of 2
+    qb = rng.standard_normal((1, 2, nb, d))
+    kb = rng.standard_normal((1, 1, nb, d)) * 1.5
+    Q = np.repeat(qb, b, axis=2)
+    K = np.repeat(kb, b, axis=2)
+    s = d ** -0.5
+    qm, qv, qc = O.block_stats(Q, N, b)
+    km, kv, kc = O.block_stats(K, N, b)
+    assert np.abs(qv).max() < 1e-24 and np.abs(kv).max() < 1e-24
+    A_pre = O.pre_downsample_map(O.corrected_scores(qm, qv, km, kv, kc, s))
+    A_post = O.post_downsample_map(Q, K, N, b, s)
+    np.testing.assert_allclose(A_pre, A_post, rtol=1e-12, atol=1e-15)
+
+
+def test_mc_variance_of_block_logit():
+    # Var[s q.k] for independent diagonal Gaussians equals s^2 V_ij; each of the
+    # three terms of V carries about a third of the total here, so dropping one
+    # or mis-scaling s fails by far more than the Monte-Carlo error.
+    rng = np.random.default_rng(11)
+    d, n = 6, 1 << 19
+    s = 0.4
+    qbar = rng.uniform(0.8, 1.2, d) * rng.choice([-1, 1], d)
+    kbar = rng.uniform(0.8, 1.2, d) * rng.choice([-1, 1], d)
+    vq = rng.uniform(0.8, 1.2, d)
+    vk = rng.uniform(0.8, 1.2, d)
+    q = qbar + rng.standard_normal((n, d)) * np.sqrt(vq)
+    k = kbar + rng.standard_normal((n, d)) * np.sqrt(vk)
+    x = s * np.einsum("nd,nd->n", q, k)
+    S = O.corrected_scores(qbar[None, None, None], vq[None, None, None],
+                           kbar[None, None, None], vk[None, None, None], [1], s)[0, 0, 0, 0]
+    mean_term = s * qbar @ kbar
+    var_oracle = 2.0 * (S - mean_term)                 # ln m = 0
+    var_mc = x.var()
+    se = var_mc * math.sqrt(2.0 / n) * 3                # generous for the product's kurtosis
+    assert abs(var_mc - var_oracle) < 5 * se, (var_mc, var_oracle, se)
+    assert abs(x.mean() - mean_term) < 5 * math.sqrt(var_mc / n)
+
+
+def test_mc_mgf_single_query_row():
+    # one query row (zero query variance), m keys from N(kbar, diag vk): the
+    # log-mean-exp of the logits converges to s q.kbar + (s^2/2) sum q^2 vk,
+    # which is S~ - ln m. Pins the factor 1/2 and the s^2.
+    rng = np.random.default_rng(5)
+    d, m = 8, 1 << 18
+    s = d ** -0.5
+    q = rng.uniform(0.5, 1.0, d) * rng.choice([-1, 1], d)
+    kbar = rng.standard_normal(d) * 0.5
+    vk = rng.uniform(0.5, 1.5, d)
+    k = kbar + rng.standard_normal((m, d)) * np.sqrt(vk)
+    x = s * (k @ q)
+    lme = np.log(np.mean(np.exp(x - x.max()))) + x.max()
+    S = O.corrected_scores(q[None, None, None], np.zeros((1, 1, 1, d)), kbar[None, None, None],
+                           vk[None, None, None], [m], s)[0, 0, 0, 0]
+    target = S - math.log(m)
+    var_x = float(s * s * (q * q) @ vk)
+    se = math.sqrt((math.exp(var_x) - 1) / m)          # relative s.e. of a lognormal mean
+    assert 0.2 < var_x < 1.5
+    assert abs(lme - target) < 6 * se, (lme, target, se)
+
+
+# ------------------------------------------------------------------ selection
+
+def test_keep_count_values():
+    assert O.keep_count(0.5, 16) == 8
+    assert O.keep_count(0.5, 128) == 64
+    assert [O.keep_count(k, 256) for k in (1.0, 0.5, 0.25)] == [256, 128, 64]
+    assert O.keep_count(0.5, 1024) == 512
+    assert O.keep_count(1e-6, 16) == 1
+    assert O.keep_count(1.0 / 3.0, 3) == 1
+    with pytest.raises(ValueError):
+        O.keep_count(0.0, 4)
+
+
+def test_topk_bruteforce_max_sum_subset():
+    # with distinct scores, the kept set is the size-k subset of maximum total score
+    rng = np.random.default_rng(3)
+    for _ in range(20):
+        nk = 8
+        k = int(rng.integers(1, nk + 1))
+        row = rng.standard_normal(nk)
+        best = max(itertools.combinations(range(nk), k), key=lambda c: sum(row[j] for j in c))
+        idx, cnt = O.select_topk(row[None], k)
+        assert cnt[0] == k
+        assert idx[0].tolist() == sorted(best)
+
+
+def test_topk_ties_prefer_lower_index_and_ascending():
+    row = np.array([[1.0, 2.0, 2.0, 2.0, 0.0, 2.0]])
+    idx, _ = O.select_topk(row, 2, kmax=4)
+    assert idx[0].tolist() == [1, 2, -1, -1]
+    idx, _ = O.select_topk(row, 5)
+    assert idx[0].tolist() == [0, 1, 2, 3, 5]
+
+
+def test_topk_permutation_equivariance_and_keep_all():
+    rng = np.random.default_rng(4)
+    S = rng.standard_normal((3, 12))
+    perm = rng.permutation(12)
+    idx, _ = O.select_topk(S, 5)
+    idx_p, _ = O.select_topk(S[:, perm], 5)
+    for r in range(3):
+        assert sorted(perm[idx_p[r]].tolist()) == idx[r].tolist()
+    idx, cnt = O.select_topk(S, 12)
+    assert (idx == np.arange(12)).all() and (cnt == 12).all()
+
+
+def test_near_tie_band():
+    row = np.array([[0.0, 1.0, 1.0005, 2.0, 1.0 + 2e-3]])
+    # k=3: ranking 3 (2.0), 4 (1.002), 2 (1.0005) -> threshold 1.0005
+    nt = O.near_tie_mask(row, 3)
+    assert nt[0].tolist() == [False, True, True, False, False]
+
+
+# ------------------------------------------------------------------ attention
+
+def _qkv(B=1, Hq=4, Hkv=2, N=200, Na=208, d=16, rng=RNG):
+    Q = rng.standard_normal((B, Hq, Na, d))
+    K = rng.standard_normal((B, Hkv, Na, d))
+    V = rng.standard_normal((B, Hkv, Na, d))
+    Q[:, :, N:] = K[:, :, N:] = V[:, :, N:] = 1e30        # padding must never be read
+    return Q, K, V
+
+
+def test_dense_matches_torch_sdpa():
+    Q, K, V = _qkv()
+    N, s = 200, 16 ** -0.5
+    Od, Ld = O.dense_attention(Q, K, V, N, s)
+    q = torch.from_numpy(Q[:, :, :N])
+    k = torch.from_numpy(np.repeat(K[:, :, :N], 2, axis=1))
+    v = torch.from_numpy(np.repeat(V[:, :, :N], 2, axis=1))
+    ref = torch.nn.functional.scaled_dot_product_attention(q, k, v, scale=s).numpy()
+    np.testing.assert_allclose(Od, ref, rtol=1e-10, atol=1e-12)
+    lse = torch.logsumexp(s * q @ k.transpose(-1, -2), dim=-1).numpy()
+    np.testing.assert_allclose(Ld, lse, rtol=1e-12, atol=1e-12)
+
+
+def test_dense_closed_forms():
+    # identical keys: uniform weights, output = mean of values, LSE = s q.k + ln N
+    rng = np.random.default_rng(9)
+    N, d, s = 50, 8, 0.3
+    Q = rng.standard_normal((1, 1, N, d))
+    K = np.repeat(rng.standard_normal((1, 1, 1, d)), N, axis=2)
+    V = rng.standard_normal((1, 1, N, d))
+    Od, Ld = O.dense_attention(Q, K, V, N, s)
+    np.testing.assert_allclose(Od[0, 0], np.repeat(V[0, 0].mean(0, keepdims=True), N, 0), atol=1e-13)
+    np.testing.assert_allclose(Ld[0, 0], s * Q[0, 0] @ K[0, 0, 0] + math.log(N), atol=1e-12)
+
+
+def test_masked_keep_all_equals_dense():
+    # check (1): keeping every block is dense attention (ragged last block)
+    Q, K, V = _qkv()
+    N, b, s = 200, 32, 16 ** -0.5
+    nb = O.num_blocks(N, b)
+    idx = np.tile(np.arange(nb, dtype=np.int32), (1, 4, nb, 1))
+    cnt = np.full((1, 4, nb), nb, dtype=np.int32)
+    Om, Lm = O.masked_attention(Q, K, V, idx, cnt, N, b, s)
+    Od, Ld = O.dense_attention(Q, K, V, N, s)
+    np.testing.assert_allclose(Om[:, :, :N], Od, rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(Lm[:, :, :N], Ld, rtol=1e-12, atol=1e-12)
+    assert np.isnan(Om[:, :, N:]).all()                  # padding rows untouched
+
+
+def test_merge_of_disjoint_spans_equals_union():
+    # check (2): merging (O, L) over X and over Y equals attention over X u Y
+    Q, K, V = _qkv()
+    N, b, s = 200, 32, 16 ** -0.5
+    nb = O.num_blocks(N, b)
+    rng = np.random.default_rng(2)
+    S = rng.standard_normal((1, 4, nb, nb))
+    idx, cnt = O.select_topk(S, 4, kmax=nb)
+    for split in (1, 3, nb - 1, nb):
+        lo_i, lo_c, hi_i, hi_c = O.split_lists(idx, cnt, split)
+        assert ((lo_c + hi_c) == cnt).all()
+        O1, L1 = O.masked_attention(Q, K, V, lo_i, lo_c, N, b, s)
+        O2, L2 = O.masked_attention(Q, K, V, hi_i, hi_c, N, b, s)
+        Ou, Lu = O.masked_attention(Q, K, V, idx, cnt, N, b, s)
+        Om, Lm = O.merge_lse(O1[:, :, :N], L1[:, :, :N], O2[:, :, :N], L2[:, :, :N])
+        np.testing.assert_allclose(Om, Ou[:, :, :N], rtol=1e-11, atol=1e-12)
+        np.testing.assert_allclose(Lm, Lu[:, :, :N], rtol=1e-12, atol=1e-12)
+
+
+def test_merge_edge_cases():
+    o1 = np.array([[1.0, 2.0], [3.0, 4.0]])
+    o2 = np.array([[5.0, 6.0], [7.0, 8.0]])
+    ninf = -np.inf
+    Om, Lm = O.merge_lse(o1, np.array([0.3, ninf]), o2, np.array([ninf, ninf]))
+    np.testing.assert_array_equal(Om, [[1.0, 2.0], [0.0, 0.0]])
+    assert Lm[0] == 0.3 and np.isneginf(Lm[1])
+    # very different magnitudes stay finite
+    Om, Lm = O.merge_lse(o1[:1], np.array([1000.0]), o2[:1], np.array([-1000.0]))
+    np.testing.assert_allclose(Om, o1[:1], rtol=1e-15)
+
+
+def test_empty_list_gives_zero_and_neginf():
+    Q, K, V = _qkv(N=64, Na=64)
+    idx = np.full((1, 4, 2, 2), -1, dtype=np.int32)
+    cnt = np.zeros((1, 4, 2), dtype=np.int32)
+    Om, Lm = O.masked_attention(Q, K, V, idx, cnt, 64, 32, 0.25)
+    assert (Om == 0).all() and np.isneginf(Lm).all()
+
+
+# ------------------------------------------------- post-downsample (check 4)
+
+def test_post_downsample_two_routes_agree():
+    # brute force over the full probability matrix vs per-block log-normalisers
+    rng = np.random.default_rng(12)
+    N, b, d = 90, 16, 8                       # 6 blocks, ragged last of 10
+    Q = rng.standard_normal((1, 1, N, d))
+    K = rng.standard_normal((1, 1, N, d))
+    V = rng.standard_normal((1, 1, N, d))
+    s = d ** -0.5
+    nb = O.num_blocks(N, b)
+    A = O.post_downsample_map(Q, K, N, b, s)
+    np.testing.assert_allclose(A.sum(-1), 1.0, rtol=1e-13)
+    _, L_full = O.dense_attention(Q, K, V, N, s)
+    L_single = np.empty((nb, N))
+    for j in range(nb):
+        idx = np.full((1, 1, nb, 1), j, dtype=np.int32)
+        cnt = np.ones((1, 1, nb), dtype=np.int32)
+        _, L = O.masked_attention(Q, K, V, idx, cnt, N, b, s)
+        L_single[j] = L[0, 0, :N]
+    A2 = O.block_mass_via_lse(L_single, L_full[0, 0], O.block_counts(N, b))
+    np.testing.assert_allclose(A2, A[0, 0], rtol=1e-11, atol=1e-14)
+
+
+def test_correction_improves_rank_agreement_on_planted_blocks():
+    # diagnostic, not a parity pin: on a planted case the corrected score tracks
+    # the exact map at least as well as the plain pooled score.
+    from block_sparse_attention_ba_b200.workloads import make_inputs
+    Q, K, V, meta = make_inputs("tiny_fp32", N=512)
+    w = meta["workload"]
+    s = w.d ** -0.5
+    qm, qv, _ = O.block_stats(Q, w.N, w.block)
+    km, kv, kc = O.block_stats(K, w.N, w.block)
+    S = O.corrected_scores(qm, qv, km, kv, kc, s)
+    P = O.pooled_scores(qm, km, kc, s)
+    A = O.post_downsample_map(Q, K, w.N, w.block, s)
+    assert O.spearman_vs_post(S, A) >= O.spearman_vs_post(P, A) - 1e-9
+    assert 0.0 <= O.topk_recall_vs_post(S, A, 4) <= 1.0
