@@ -1,0 +1,469 @@
+#!/usr/bin/env python
+"""Benchmark of the BA-Att forward hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload sweep_32k] [--keep 0.5]
+
+One step is one pass of the whole hot path over one batch of synthetic input
+already resident in HBM: block statistics -> corrected scores + top-k ->
+split of the kept lists at a seeded key-block boundary -> block-sparse
+attention over each span -> log-space merge of the two partials (the
+FlashBlock Eq. 9 composition). The default workload is the 32K-token
+diffusion-LM case (B=1, 32 query / 8 KV heads, d=128, block 128, bf16,
+keep 0.5). Prints one JSON line (rank 0).
+
+With N > 1 (torchrun), every rank runs an independent replica of the
+workload (the attention calls are independent units; nothing is exchanged),
+so scaling is weak and `value` sums over ranks using the slowest rank's time.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "BA-Att fwd ms/call and kept-block TFLOP/s @50% keep, N=32K–128K; % of roofline"
+UNIT = "TFLOP/s (kept-block FLOPs)"
+L2_BYTES = 126 * 2 ** 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# --------------------------------------------------------------------------- helpers
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_env():
+    return int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), \
+        int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def kept_flops(cnt_total: int, block: int, d: int) -> float:
+    """Two GEMMs (Q K^T and P V) per kept (query block, key block) pair."""
+    return 4.0 * block * block * d * cnt_total
+
+
+def selector_bytes(w, k: int) -> int:
+    """Algorithmic selector traffic: read Q and K once, write the index lists."""
+    e = 2 if w.dtype == "bf16" else 4
+    qk = (w.B * w.Hq + w.B * w.Hkv) * w.N * w.d * e
+    lists = w.B * w.Hq * w.nb * (k + 1) * 4
+    return qk + lists
+
+
+def kernel_sources_sha(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "block_sparse_attention_ba_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_from_profile(sha: str):
+    """DRAM bytes per sparse-attention launch from the committed ncu summary,
+    if it was taken on the current kernel source."""
+    p = os.path.join(ROOT, "profiles", "attn_tc_traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None, None
+    if d.get("source_sha") != sha:
+        return None, d
+    return d.get("dram_bytes_per_full_step"), d
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 200 ms."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"ba_att_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=self.fh, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in rows for k in range(4) if r[5 + k].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# --------------------------------------------------------------------------- CPU oracle arms
+
+def oracle_sample(w, Q, K, V, keep, seed, n_blocks, n_sel_heads):
+    """Time the oracle (float32, all host cores) on a bounded sample of one
+    step: the selector for `n_sel_heads` query heads (with their KV heads)
+    and masked attention for `n_blocks` query blocks; extrapolate linearly
+    to the full step. Returns (seconds per full step, description)."""
+    import oracle as O
+    rng = np.random.default_rng(seed)
+    s = w.d ** -0.5
+    k = O.keep_count(keep, w.nb)
+    G = w.Hq // w.Hkv
+    heads = sorted(rng.choice(w.Hq, size=n_sel_heads, replace=False).tolist())
+    t0 = time.perf_counter()
+    kv_heads = sorted({h // G for h in heads})
+    qm, qv, _ = O.block_stats(Q[:, heads], w.N, w.block, dtype=np.float32)
+    km, kv, kc = O.block_stats(K[:, kv_heads], w.N, w.block, dtype=np.float32)
+    # corrected_scores maps query head -> KV head by position; lay the
+    # sampled KV heads out so that each sampled query head finds its own
+    kmap = [kv_heads.index(h // G) for h in heads]
+    S = O.corrected_scores(qm, qv, km[:, kmap], kv[:, kmap], kc, s, dtype=np.float32)
+    idx, cnt = O.select_topk(S, k)
+    t_sel = time.perf_counter() - t0
+    blocks = [(0, heads[int(rng.integers(len(heads)))], int(rng.integers(w.nb))) for _ in range(n_blocks)]
+    idx_full = np.zeros((w.B, w.Hq, w.nb, k), dtype=np.int32)
+    cnt_full = np.full((w.B, w.Hq, w.nb), k, dtype=np.int32)
+    for hi, h in enumerate(heads):
+        idx_full[:, h] = idx[:, hi]
+    t1 = time.perf_counter()
+    O.masked_attention(Q, K, V, idx_full, cnt_full, w.N, w.block, s, query_blocks=blocks, dtype=np.float32)
+    t_att = time.perf_counter() - t1
+    per_step = t_sel * (w.Hq / n_sel_heads) + t_att * (w.B * w.Hq * w.nb / n_blocks)
+    desc = (f"oracle float32 on host cores: selector for {n_sel_heads}/{w.Hq} query heads, masked attention for "
+            f"{n_blocks}/{w.B * w.Hq * w.nb} query blocks; extrapolated linearly to one full step")
+    return per_step, desc, t_sel + t_att
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+# --------------------------------------------------------------------------- our arm
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from block_sparse_attention_ba_b200 import api
+    from block_sparse_attention_ba_b200.workloads import WORKLOADS, make_inputs
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+    api.load_library()
+
+    w0 = WORKLOADS[args.workload]
+    w = w0.with_(split=True)
+    keep = args.keep
+    Q, K, V, meta = make_inputs(w)
+    split_block = meta["split_block"]
+    dev = torch.device("cuda", local)
+    Qd = torch.from_numpy(Q).to(torch.bfloat16).to(dev)
+    Kd = torch.from_numpy(K).to(torch.bfloat16).to(dev)
+    Vd = torch.from_numpy(V).to(torch.bfloat16).to(dev)
+    shape = api.Shape.of(Qd, Kd, w.N, w.block)
+    k = api.keep_count(shape, keep)
+    nb = shape.nb
+    # all buffers allocated once, outside the timed region
+    stats_buf = (torch.empty((w.B, w.Hq, nb, w.d), device=dev), torch.empty((w.B, w.Hq, nb, w.d), device=dev),
+                 torch.empty((w.B, w.Hkv, nb, w.d), device=dev), torch.empty((w.B, w.Hkv, nb, w.d), device=dev))
+    idx = torch.empty((w.B, w.Hq, nb, k), device=dev, dtype=torch.int32)
+    cnt = torch.empty((w.B, w.Hq, nb), device=dev, dtype=torch.int32)
+    lists = (torch.empty_like(idx), torch.empty_like(cnt), torch.empty_like(idx), torch.empty_like(cnt))
+    O1, O2, Om = torch.empty_like(Qd), torch.empty_like(Qd), torch.empty_like(Qd)
+    L1, L2, Lm = (torch.empty((w.B, w.Hq, w.N_alloc), device=dev) for _ in range(3))
+    stream = torch.cuda.current_stream(dev)
+
+    names = ("stats", "select", "split", "sparse_lo", "sparse_hi", "merge")
+
+    def step(events=None):
+        def mark(i):
+            if events is not None:
+                events[i].record(stream)
+        mark(0)
+        api.stats(Qd, Kd, shape, out=stats_buf)
+        mark(1)
+        api.select(stats_buf, shape, keep, out=(idx, cnt, None))
+        mark(2)
+        api.split_lists(idx, cnt, shape, split_block, out=lists)
+        mark(3)
+        api.sparse_fwd(Qd, Kd, Vd, lists[0], lists[1], shape, out=(O1, L1))
+        mark(4)
+        api.sparse_fwd(Qd, Kd, Vd, lists[2], lists[3], shape, out=(O2, L2))
+        mark(5)
+        api.merge_lse(O1, L1, O2, L2, out=(Om, Lm))
+        mark(6)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st, word = api.get_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error word {word:#x} during warm-up")
+    cnt_total = int(cnt.sum().item())
+    flops = kept_flops(cnt_total, w.block, w.d)
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    t_start.record(stream)
+    for s_i in range(args.steps):
+        step(ev[s_i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    stage_ms = {n: float(np.mean([ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(args.steps)]))
+                for i, n in enumerate(names)}
+    st, word = api.get_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error word {word:#x} during timing")
+
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    ms_per_step = elapsed_ms / args.steps
+    value = world * flops / (ms_per_step * 1e-3) / 1e12
+
+    result = None
+    if rank == 0:
+        peaks, peak_src = load_peaks()
+        sparse_ms = stage_ms["sparse_lo"] + stage_ms["sparse_hi"]
+        achieved = flops / (sparse_ms * 1e-3) / 1e12
+        sha = kernel_sources_sha(["attn_tc.cuh", "common.cuh"])
+        traffic, prof = traffic_from_profile(sha)
+        roofline = {"bound": "tensor", "kernel": "attn_tc_kernel (both span launches of a step)",
+                    "achieved": round(achieved, 1), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                    "frac": round(achieved / peaks["bf16_tflops"], 4),
+                    "frac_vs_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4),
+                    "peak_source": f"{peak_src} (dense bf16 burst)", "traffic": traffic,
+                    "units": f"{cnt_total} kept (query block, key block) pairs x 4*b^2*d FLOP"}
+        sel_ms = stage_ms["stats"] + stage_ms["select"]
+        sel_bytes = selector_bytes(w, k)
+        selector = {"bound": "hbm", "achieved": round(sel_bytes / (sel_ms * 1e-3) / 1e9, 1),
+                    "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": round(sel_bytes / (sel_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+                    "bytes": sel_bytes, "ms": round(sel_ms, 4),
+                    "stats_frac": round((sel_bytes - w.B * w.Hq * nb * (k + 1) * 4) / (stage_ms["stats"] * 1e-3)
+                                        / 1e9 / peaks["hbm_gbs"], 4)}
+        result = {
+            "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"{w.name}: B={w.B} Hq={w.Hq} Hkv={w.Hkv} N={w.N} d={w.d} block={w.block} "
+                                   f"bf16 keep={keep}; step = stats+select+split(block {split_block})"
+                                   f"+2x sparse_fwd+merge_lse",
+                       "keep": keep, "kept_blocks_per_query_block": k, "split_block": split_block,
+                       "parallelism": f"{world} independent replica(s)",
+                       "l2": f"inputs {(Qd.numel() + Kd.numel() + Vd.numel()) * 2 / 2**20:.0f} MiB > L2 "
+                             f"126 MiB; no flush"},
+            "roofline": roofline, "selector": selector,
+            "stages_ms": {n: round(v, 4) for n, v in stage_ms.items()},
+            "gpu_launches": 6 * args.steps, "clocks": clk,
+        }
+    return result, dict(Qd=Qd, Kd=Kd, Vd=Vd, shape=shape, keep=keep, w=w, Q=Q, K=K, V=V, split_block=split_block,
+                        step=step, flops=flops, world=world, rank=rank, dev=dev,
+                        bufs=(stats_buf, idx, cnt, lists, O1, O2, Om, L1, L2, Lm))
+
+
+def run_e2e(ctx, steps, warmup):
+    """Same step through the public API from pinned host buffers: H2D of Q, K,
+    V, the step, and D2H of O and LSE, all inside the timed region."""
+    import torch
+    from block_sparse_attention_ba_b200 import api
+
+    dev = ctx["dev"]
+    Qh = torch.from_numpy(ctx["Q"]).to(torch.bfloat16).pin_memory()
+    Kh = torch.from_numpy(ctx["K"]).to(torch.bfloat16).pin_memory()
+    Vh = torch.from_numpy(ctx["V"]).to(torch.bfloat16).pin_memory()
+    Oh = torch.empty(Qh.shape, dtype=torch.bfloat16).pin_memory()
+    Lh = torch.empty(ctx["bufs"][9].shape, dtype=torch.float32).pin_memory()
+    Qd, Kd, Vd = ctx["Qd"], ctx["Kd"], ctx["Vd"]
+    Om, Lm = ctx["bufs"][6], ctx["bufs"][9]
+    stream = torch.cuda.current_stream(dev)
+
+    def e2e_step():
+        Qd.copy_(Qh, non_blocking=True)
+        Kd.copy_(Kh, non_blocking=True)
+        Vd.copy_(Vh, non_blocking=True)
+        ctx["step"]()
+        Oh.copy_(Om, non_blocking=True)
+        Lh.copy_(Lm, non_blocking=True)
+
+    for _ in range(warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    st, word = api.get_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error word {word:#x} in e2e")
+    ms = a.elapsed_time(b) / steps
+    h2d = (Qh.numel() + Kh.numel() + Vh.numel()) * 2
+    d2h = Oh.numel() * 2 + Lh.numel() * 4
+    return {"value": round(ctx["world"] * ctx["flops"] / (ms * 1e-3) / 1e12, 2), "unit": UNIT,
+            "ms_per_step": round(ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def run_dense(ctx, steps=3):
+    """The GPU path's own dense run: keep = 1.0, single pass (stats, select, sparse_fwd)."""
+    import torch
+    from block_sparse_attention_ba_b200 import api
+
+    shape, dev = ctx["shape"], ctx["dev"]
+    w = ctx["w"]
+    st = api.stats(ctx["Qd"], ctx["Kd"], shape)
+    idx, cnt = api.select(st, shape, 1.0)
+    O, L = api.sparse_fwd(ctx["Qd"], ctx["Kd"], ctx["Vd"], idx, cnt, shape)
+    torch.cuda.synchronize()
+    a, b, c = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+    stream = torch.cuda.current_stream(dev)
+    a.record(stream)
+    for _ in range(steps):
+        api.stats(ctx["Qd"], ctx["Kd"], shape, out=st)
+        api.select(st, shape, 1.0, out=(idx, cnt, None))
+    b.record(stream)
+    for _ in range(steps):
+        api.sparse_fwd(ctx["Qd"], ctx["Kd"], ctx["Vd"], idx, cnt, shape, out=(O, L))
+    c.record(stream)
+    torch.cuda.synchronize()
+    sel_ms = a.elapsed_time(b) / steps
+    att_ms = b.elapsed_time(c) / steps
+    fl = kept_flops(int(cnt.sum().item()), w.block, w.d)
+    return {"keep": 1.0, "ms_per_call": round(sel_ms + att_ms, 4), "sparse_fwd_ms": round(att_ms, 4),
+            "tflops": round(fl / ((sel_ms + att_ms) * 1e-3) / 1e12, 1),
+            "sparse_fwd_tflops": round(fl / (att_ms * 1e-3) / 1e12, 1)}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--workload", default="sweep_32k")
+    ap.add_argument("--keep", type=float, default=0.5)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    world, rank, _ = dist_env()
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        run_reference(args)
+        return
+
+    result, ctx = run_ours(args)
+    e2e = run_e2e(ctx, max(3, args.steps // 2), 3)
+    dense = run_dense(ctx)
+    if rank == 0:
+        result["e2e"] = e2e
+        result["dense_keep1"] = dense
+        if not args.no_cpu_baseline:
+            per_step, desc, spent = oracle_sample(ctx["w"], ctx["Q"], ctx["K"], ctx["V"], ctx["keep"], 0,
+                                                  n_blocks=48, n_sel_heads=2)
+            result["cpu_baseline"] = {"value": round(ctx["flops"] / per_step / 1e12, 6), "unit": UNIT,
+                                      "cores": cpu_cores(), "kind": "oracle", "sample": desc,
+                                      "sample_seconds": round(spent, 1)}
+        print(json.dumps(result), flush=True)
+    if ctx["world"] > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_reference(args):
+    """The oracle as it stands, timed on the host cores on bounded samples of
+    the same workload; each step is one sample, extrapolated to a full step."""
+    from block_sparse_attention_ba_b200.workloads import WORKLOADS, make_inputs
+    import oracle as O
+
+    w = WORKLOADS[args.workload].with_(split=True)
+    Q, K, V, meta = make_inputs(w)
+    k = O.keep_count(args.keep, w.nb)
+    flops = kept_flops(w.B * w.Hq * w.nb * k, w.block, w.d)
+    for i in range(args.warmup):
+        oracle_sample(w, Q, K, V, args.keep, 1000 + i, n_blocks=2, n_sel_heads=1)
+    per = []
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        ps, desc, _ = oracle_sample(w, Q, K, V, args.keep, i, n_blocks=8, n_sel_heads=1)
+        per.append(ps)
+    wall = time.perf_counter() - t0
+    ms = float(np.mean(per)) * 1e3
+    value = flops / (ms * 1e-3) / 1e12
+    out = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": 1,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 1), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+           "config": {"workload": f"{w.name}: B={w.B} Hq={w.Hq} Hkv={w.Hkv} N={w.N} d={w.d} block={w.block} "
+                                  f"keep={args.keep}", "keep": args.keep},
+           "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+                            "sample": desc + "; one sample per step", "wall_seconds": round(wall, 1)},
+           "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+           "gpu_launches": 0}
+    print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

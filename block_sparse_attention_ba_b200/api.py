@@ -1,0 +1,241 @@
+"""Thin ctypes binding over libbaatt.so (declared in include/ba_att.h).
+
+Argument marshalling only: every step of the hot path runs in the library's
+CUDA kernels. PyTorch supplies device memory and the current stream; outputs
+not passed in are allocated with ``torch.empty`` on the inputs' device. A
+missing library, a CPU tensor, or a non-OK status raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import threading
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+
+BA_OK = 0
+STATUS_NAMES = {0: "BA_OK", 1: "BA_ERR_INVALID_ARG", 2: "BA_ERR_UNSUPPORTED", 3: "BA_ERR_MISALIGNED",
+                4: "BA_ERR_CUDA", 5: "BA_ERR_DEVICE", 6: "BA_ERR_TIMEOUT"}
+DTYPE_F32, DTYPE_BF16 = 0, 1
+
+# Entry points declared in include/ba_att.h: name -> (restype, argtypes)
+_P = ctypes.c_void_p
+_I32 = ctypes.c_int32
+
+
+class CShape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32), ("N", ctypes.c_int32),
+                ("N_alloc", ctypes.c_int32), ("d", ctypes.c_int32), ("block", ctypes.c_int32),
+                ("dtype", ctypes.c_int32), ("sm_scale", ctypes.c_float)]
+
+
+_SIGS = {
+    "ba_att_version": (ctypes.c_char_p, []),
+    "ba_att_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "ba_att_num_blocks": (_I32, [ctypes.POINTER(CShape)]),
+    "ba_att_keep_count": (_I32, [ctypes.POINTER(CShape), ctypes.c_float]),
+    "ba_att_stats": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _P, _P, _P, _P, _P]),
+    "ba_att_select": (ctypes.c_int, [ctypes.POINTER(CShape), ctypes.c_float, _P, _P, _P, _P, _P, _P, _I32, _P, _P]),
+    "ba_att_split_lists": (ctypes.c_int, [ctypes.POINTER(CShape), _I32, _P, _P, _I32, _P, _P, _P, _P, _P]),
+    "ba_att_sparse_fwd": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _P, _P, _P, _I32, _P, _P, _P]),
+    "ba_att_merge_lse": (ctypes.c_int, [ctypes.c_int64, _I32, _I32, _P, _P, _P, _P, _P, _P, _P]),
+    "ba_att_get_device_error": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_uint32)]),
+    "ba_att_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_uint32, _P]),
+}
+
+_lib = None
+_lock = threading.Lock()
+
+
+class BaAttError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {STATUS_NAMES.get(status, status)}")
+
+
+def library_path() -> str:
+    return os.environ.get("BA_ATT_LIB", os.path.join(_HERE, "libbaatt.so"))
+
+
+def load_library():
+    """Load libbaatt.so (once). Raises if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            path = library_path()
+            if not os.path.exists(path):
+                raise RuntimeError(f"{path} is missing: build it with `python -m block_sparse_attention_ba_b200.build`")
+            lib = ctypes.CDLL(path)
+            for name, (res, args) in _SIGS.items():
+                fn = getattr(lib, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = lib
+    return _lib
+
+
+def _check(fn: str, status: int):
+    if status != BA_OK:
+        raise BaAttError(fn, status)
+
+
+@dataclass(frozen=True)
+class Shape:
+    B: int
+    Hq: int
+    Hkv: int
+    N: int
+    N_alloc: int
+    d: int
+    block: int
+    dtype: int
+    sm_scale: float = 0.0
+
+    @property
+    def nb(self) -> int:
+        return -(-self.N // self.block)
+
+    @property
+    def scale(self) -> float:
+        return self.sm_scale if self.sm_scale > 0 else 1.0 / math.sqrt(self.d)
+
+    def c(self) -> CShape:
+        return CShape(self.B, self.Hq, self.Hkv, self.N, self.N_alloc, self.d, self.block, self.dtype,
+                      float(self.sm_scale))
+
+    @staticmethod
+    def of(Q: torch.Tensor, K: torch.Tensor, N: int | None = None, block: int = 128,
+           sm_scale: float = 0.0) -> "Shape":
+        B, Hq, N_alloc, d = Q.shape
+        dt = {torch.float32: DTYPE_F32, torch.bfloat16: DTYPE_BF16}.get(Q.dtype)
+        if dt is None:
+            raise TypeError(f"unsupported dtype {Q.dtype}")
+        return Shape(B, Hq, K.shape[1], N_alloc if N is None else N, N_alloc, d, block, dt, sm_scale)
+
+
+def _stream(t: torch.Tensor | None = None):
+    dev = t.device if t is not None else torch.device("cuda")
+    return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+
+def _dev(t: torch.Tensor, name: str) -> ctypes.c_void_p:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def num_blocks(shape: Shape) -> int:
+    return int(load_library().ba_att_num_blocks(ctypes.byref(shape.c())))
+
+
+def keep_count(shape: Shape, keep: float) -> int:
+    return int(load_library().ba_att_keep_count(ctypes.byref(shape.c()), ctypes.c_float(keep)))
+
+
+def stats(Q: torch.Tensor, K: torch.Tensor, shape: Shape, out=None):
+    """Per-block mean / population variance of Q and K (fp32)."""
+    lib = load_library()
+    dev = Q.device
+    if out is None:
+        out = (torch.empty((shape.B, shape.Hq, shape.nb, shape.d), device=dev, dtype=torch.float32),
+               torch.empty((shape.B, shape.Hq, shape.nb, shape.d), device=dev, dtype=torch.float32),
+               torch.empty((shape.B, shape.Hkv, shape.nb, shape.d), device=dev, dtype=torch.float32),
+               torch.empty((shape.B, shape.Hkv, shape.nb, shape.d), device=dev, dtype=torch.float32))
+    qm, qv, km, kv = out
+    _check("ba_att_stats", lib.ba_att_stats(ctypes.byref(shape.c()), _dev(Q, "Q"), _dev(K, "K"), _dev(qm, "q_mean"),
+                                            _dev(qv, "q_var"), _dev(km, "k_mean"), _dev(kv, "k_var"), _stream(Q)))
+    return out
+
+
+def select(stats_out, shape: Shape, keep: float, kmax: int | None = None, with_scores: bool = False, out=None):
+    """Corrected block scores + top-k; returns (idx, cnt) or (idx, cnt, scores)."""
+    lib = load_library()
+    qm, qv, km, kv = stats_out
+    k = keep_count(shape, keep)
+    if k < 1:
+        raise BaAttError("ba_att_keep_count", 1)
+    kmax = k if kmax is None else kmax
+    dev = qm.device
+    if out is None:
+        idx = torch.empty((shape.B, shape.Hq, shape.nb, kmax), device=dev, dtype=torch.int32)
+        cnt = torch.empty((shape.B, shape.Hq, shape.nb), device=dev, dtype=torch.int32)
+        sc = torch.empty((shape.B, shape.Hq, shape.nb, shape.nb), device=dev, dtype=torch.float32) \
+            if with_scores else None
+    else:
+        idx, cnt, sc = out
+    _check("ba_att_select", lib.ba_att_select(
+        ctypes.byref(shape.c()), ctypes.c_float(keep), _dev(qm, "q_mean"), _dev(qv, "q_var"), _dev(km, "k_mean"),
+        _dev(kv, "k_var"), _dev(idx, "kv_idx"), _dev(cnt, "kv_cnt"), idx.shape[-1],
+        _dev(sc, "block_scores") if sc is not None else None, _stream(qm)))
+    return (idx, cnt, sc) if sc is not None else (idx, cnt)
+
+
+def split_lists(idx: torch.Tensor, cnt: torch.Tensor, shape: Shape, split_block: int, out=None):
+    """Partition kept lists at a key-block boundary -> (lo_idx, lo_cnt, hi_idx, hi_cnt)."""
+    lib = load_library()
+    if out is None:
+        out = (torch.empty_like(idx), torch.empty_like(cnt), torch.empty_like(idx), torch.empty_like(cnt))
+    lo_i, lo_c, hi_i, hi_c = out
+    _check("ba_att_split_lists", lib.ba_att_split_lists(
+        ctypes.byref(shape.c()), int(split_block), _dev(idx, "kv_idx"), _dev(cnt, "kv_cnt"), idx.shape[-1],
+        _dev(lo_i, "lo_idx"), _dev(lo_c, "lo_cnt"), _dev(hi_i, "hi_idx"), _dev(hi_c, "hi_cnt"), _stream(idx)))
+    return out
+
+
+def sparse_fwd(Q, K, V, idx, cnt, shape: Shape, out=None):
+    """Block-sparse attention over the kept blocks -> (O, LSE)."""
+    lib = load_library()
+    if out is None:
+        out = (torch.empty_like(Q),
+               torch.empty((shape.B, shape.Hq, shape.N_alloc), device=Q.device, dtype=torch.float32))
+    O, LSE = out
+    _check("ba_att_sparse_fwd", lib.ba_att_sparse_fwd(
+        ctypes.byref(shape.c()), _dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), _dev(idx, "kv_idx"), _dev(cnt, "kv_cnt"),
+        idx.shape[-1], _dev(O, "O"), _dev(LSE, "LSE"), _stream(Q)))
+    return out
+
+
+def merge_lse(O1, L1, O2, L2, out=None):
+    """Log-space merge of two partial attentions -> (O, L). out may alias (O1, L1)."""
+    lib = load_library()
+    d = O1.shape[-1]
+    rows = O1.numel() // d
+    dt = {torch.float32: DTYPE_F32, torch.bfloat16: DTYPE_BF16}[O1.dtype]
+    if out is None:
+        out = (torch.empty_like(O1), torch.empty_like(L1))
+    O, L = out
+    _check("ba_att_merge_lse", lib.ba_att_merge_lse(
+        rows, d, dt, _dev(O1, "O1"), _dev(L1, "L1"), _dev(O2, "O2"), _dev(L2, "L2"), _dev(O, "O"), _dev(L, "L"),
+        _stream(O1)))
+    return out
+
+
+def forward(Q, K, V, N: int, block: int, keep: float, sm_scale: float = 0.0):
+    """Full BA-Att forward: stats -> select -> sparse attention. Returns (O, LSE, idx, cnt)."""
+    shape = Shape.of(Q, K, N, block, sm_scale)
+    st = stats(Q, K, shape)
+    idx, cnt = select(st, shape, keep)
+    O, LSE = sparse_fwd(Q, K, V, idx, cnt, shape)
+    return O, LSE, idx, cnt
+
+
+def get_device_error(device=None):
+    """Synchronise the current stream, read and clear the device error word -> (status, word)."""
+    lib = load_library()
+    word = ctypes.c_uint32(0)
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    st = lib.ba_att_get_device_error(ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream),
+                                     ctypes.byref(word))
+    return int(st), int(word.value)
+
+
+def selftest_bounded_wait(timeout_us: int):
+    lib = load_library()
+    _check("ba_att_selftest_bounded_wait", lib.ba_att_selftest_bounded_wait(int(timeout_us), _stream()))

@@ -1,0 +1,314 @@
+// ba_att.cu — host side of the C ABI declared in include/ba_att.h.
+//
+// Every entry point validates its arguments on the host first and launches
+// nothing on a bad argument. Launches are asynchronous on the caller's
+// stream; no call synchronises except ba_att_get_device_error. The library
+// allocates no device memory: its only global state is the device error word
+// (a __device__ variable) and a cache of per-device SM counts.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "common.cuh"
+#include "stats.cuh"
+#include "select.cuh"
+#include "merge.cuh"
+#include "attn_simt.cuh"
+#include "attn_tc.cuh"
+
+using namespace baatt;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+int num_sms_of_current_device() {
+  static int cache[kMaxDevices] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+ba_status check_shape(const ba_att_shape *s) {
+  if (s == nullptr) return BA_ERR_INVALID_ARG;
+  if (s->B < 1 || s->Hq < 1 || s->Hkv < 1 || s->N < 1 || s->N_alloc < s->N) return BA_ERR_INVALID_ARG;
+  if (s->Hq % s->Hkv != 0) return BA_ERR_INVALID_ARG;
+  if (s->B > 65535 || s->Hq > 65535) return BA_ERR_UNSUPPORTED;
+  if (s->dtype != BA_DTYPE_F32 && s->dtype != BA_DTYPE_BF16) return BA_ERR_INVALID_ARG;
+  if (s->d != 64 && s->d != 128) return BA_ERR_UNSUPPORTED;
+  if (s->block < 16 || s->block > 256 || s->block % 16 != 0) return BA_ERR_UNSUPPORTED;
+  if (std::isnan(s->sm_scale) || std::isinf(s->sm_scale)) return BA_ERR_INVALID_ARG;
+  const long long rows = static_cast<long long>(s->B) * (s->Hq > s->Hkv ? s->Hq : s->Hkv) * s->N_alloc;
+  if (rows > (1LL << 36)) return BA_ERR_UNSUPPORTED;
+  return BA_OK;
+}
+
+int nblocks(const ba_att_shape *s) { return (s->N + s->block - 1) / s->block; }
+
+float effective_scale(const ba_att_shape *s) {
+  return s->sm_scale > 0.f ? s->sm_scale : 1.0f / std::sqrt(static_cast<float>(s->d));
+}
+
+ba_status from_cuda(cudaError_t e) { return e == cudaSuccess ? BA_OK : BA_ERR_CUDA; }
+
+// ---- tensor maps (driver entry point fetched through the runtime, so the
+// library links no libcuda stub)
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// [BH, rows, d] bf16 head-major tensor; rows >= N_valid read as zeros.
+bool make_head_map(CUtensorMap *map, const void *ptr, int d, int N_valid, int N_alloc, long long BH) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N_valid), static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2u, static_cast<cuuint64_t>(N_alloc) * d * 2u};
+  cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(tc::kTileRows), 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool use_tensor_core_path(const ba_att_shape *s) {
+  return s->dtype == BA_DTYPE_BF16 && s->d == 128 && s->block == 128;
+}
+
+__global__ void bounded_wait_selftest_kernel(unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait_bounded(smem_u32(&bar), 0, nullptr, limit_ns);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *ba_att_version(void) { return "0.1.0 sm_100a"; }
+
+const char *ba_att_status_string(ba_status st) {
+  switch (st) {
+    case BA_OK: return "BA_OK";
+    case BA_ERR_INVALID_ARG: return "BA_ERR_INVALID_ARG";
+    case BA_ERR_UNSUPPORTED: return "BA_ERR_UNSUPPORTED";
+    case BA_ERR_MISALIGNED: return "BA_ERR_MISALIGNED";
+    case BA_ERR_CUDA: return "BA_ERR_CUDA";
+    case BA_ERR_DEVICE: return "BA_ERR_DEVICE";
+    case BA_ERR_TIMEOUT: return "BA_ERR_TIMEOUT";
+  }
+  return "BA_ERR_UNKNOWN";
+}
+
+int32_t ba_att_num_blocks(const ba_att_shape *shape) {
+  if (check_shape(shape) != BA_OK) return -1;
+  return nblocks(shape);
+}
+
+int32_t ba_att_keep_count(const ba_att_shape *shape, float keep) {
+  if (check_shape(shape) != BA_OK) return -1;
+  if (!(keep > 0.f && keep <= 1.f)) return -1;
+  const int nk = nblocks(shape);
+  const double kk = std::ceil(static_cast<double>(keep) * nk - 1e-9);
+  int k = static_cast<int>(kk);
+  if (k < 1) k = 1;
+  if (k > nk) k = nk;
+  return k;
+}
+
+ba_status ba_att_stats(const ba_att_shape *s, const void *Q, const void *K, float *q_mean, float *q_var,
+                       float *k_mean, float *k_var, ba_stream_t stream) {
+  ba_status st = check_shape(s);
+  if (st != BA_OK) return st;
+  if (!Q || !K || !q_mean || !q_var || !k_mean || !k_var) return BA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(q_mean) || !aligned16(q_var) || !aligned16(k_mean) ||
+      !aligned16(k_var))
+    return BA_ERR_MISALIGNED;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (s->dtype == BA_DTYPE_BF16) {
+    auto q = static_cast<const __nv_bfloat16 *>(Q);
+    auto k = static_cast<const __nv_bfloat16 *>(K);
+    e = s->d == 128 ? launch_stats<__nv_bfloat16, 128>(q, k, q_mean, q_var, k_mean, k_var, s->B, s->Hq, s->Hkv, s->N,
+                                                       s->N_alloc, s->block, cs)
+                    : launch_stats<__nv_bfloat16, 64>(q, k, q_mean, q_var, k_mean, k_var, s->B, s->Hq, s->Hkv, s->N,
+                                                      s->N_alloc, s->block, cs);
+  } else {
+    auto q = static_cast<const float *>(Q);
+    auto k = static_cast<const float *>(K);
+    e = s->d == 128 ? launch_stats<float, 128>(q, k, q_mean, q_var, k_mean, k_var, s->B, s->Hq, s->Hkv, s->N,
+                                               s->N_alloc, s->block, cs)
+                    : launch_stats<float, 64>(q, k, q_mean, q_var, k_mean, k_var, s->B, s->Hq, s->Hkv, s->N,
+                                              s->N_alloc, s->block, cs);
+  }
+  return from_cuda(e);
+}
+
+ba_status ba_att_select(const ba_att_shape *s, float keep, const float *q_mean, const float *q_var,
+                        const float *k_mean, const float *k_var, int32_t *kv_idx, int32_t *kv_cnt, int32_t kmax,
+                        float *block_scores, ba_stream_t stream) {
+  ba_status st = check_shape(s);
+  if (st != BA_OK) return st;
+  if (!q_mean || !q_var || !k_mean || !k_var || !kv_idx || !kv_cnt) return BA_ERR_INVALID_ARG;
+  if (!aligned16(q_mean) || !aligned16(q_var) || !aligned16(k_mean) || !aligned16(k_var) || !aligned16(kv_idx) ||
+      !aligned16(kv_cnt) || (block_scores && !aligned16(block_scores)))
+    return BA_ERR_MISALIGNED;
+  const int k = ba_att_keep_count(s, keep);
+  if (k < 1) return BA_ERR_INVALID_ARG;
+  if (kmax < k) return BA_ERR_INVALID_ARG;
+  const int nb = nblocks(s);
+  if (nb > 4096) return BA_ERR_UNSUPPORTED;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  const float scale = effective_scale(s);
+  cudaError_t e = s->d == 128 ? launch_select<128>(q_mean, q_var, k_mean, k_var, kv_idx, kv_cnt, block_scores, s->B,
+                                                   s->Hq, s->Hkv, s->N, s->block, k, kmax, scale, cs)
+                              : launch_select<64>(q_mean, q_var, k_mean, k_var, kv_idx, kv_cnt, block_scores, s->B,
+                                                  s->Hq, s->Hkv, s->N, s->block, k, kmax, scale, cs);
+  return from_cuda(e);
+}
+
+ba_status ba_att_split_lists(const ba_att_shape *s, int32_t split_block, const int32_t *kv_idx, const int32_t *kv_cnt,
+                             int32_t kmax, int32_t *lo_idx, int32_t *lo_cnt, int32_t *hi_idx, int32_t *hi_cnt,
+                             ba_stream_t stream) {
+  ba_status st = check_shape(s);
+  if (st != BA_OK) return st;
+  if (!kv_idx || !kv_cnt || !lo_idx || !lo_cnt || !hi_idx || !hi_cnt) return BA_ERR_INVALID_ARG;
+  if (!aligned16(kv_idx) || !aligned16(kv_cnt) || !aligned16(lo_idx) || !aligned16(lo_cnt) || !aligned16(hi_idx) ||
+      !aligned16(hi_cnt))
+    return BA_ERR_MISALIGNED;
+  const int nb = nblocks(s);
+  if (kmax < 1 || split_block < 0 || split_block > nb) return BA_ERR_INVALID_ARG;
+  const long long n_lists = static_cast<long long>(s->B) * s->Hq * nb;
+  return from_cuda(launch_split(kv_idx, kv_cnt, lo_idx, lo_cnt, hi_idx, hi_cnt, n_lists, kmax, nb, split_block,
+                                num_sms_of_current_device(), reinterpret_cast<cudaStream_t>(stream)));
+}
+
+ba_status ba_att_sparse_fwd(const ba_att_shape *s, const void *Q, const void *K, const void *V, const int32_t *kv_idx,
+                            const int32_t *kv_cnt, int32_t kmax, void *O, float *LSE, ba_stream_t stream) {
+  ba_status st = check_shape(s);
+  if (st != BA_OK) return st;
+  if (!Q || !K || !V || !kv_idx || !kv_cnt || !O || !LSE) return BA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(kv_idx) || !aligned16(kv_cnt) || !aligned16(O) ||
+      !aligned16(LSE))
+    return BA_ERR_MISALIGNED;
+  if (kmax < 1) return BA_ERR_INVALID_ARG;
+  const int nb = nblocks(s);
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  const float scale = effective_scale(s);
+  if (use_tensor_core_path(s)) {
+    CUtensorMap mq, mk, mv;
+    if (!make_head_map(&mq, Q, s->d, s->N, s->N_alloc, static_cast<long long>(s->B) * s->Hq) ||
+        !make_head_map(&mk, K, s->d, s->N, s->N_alloc, static_cast<long long>(s->B) * s->Hkv) ||
+        !make_head_map(&mv, V, s->d, s->N, s->N_alloc, static_cast<long long>(s->B) * s->Hkv))
+      return BA_ERR_CUDA;
+    cudaError_t e = cudaFuncSetAttribute(tc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(tc::kDynSmem));
+    if (e != cudaSuccess) return BA_ERR_CUDA;
+    const long long tiles = static_cast<long long>(s->B) * s->Hq * nb;
+    if (tiles > 0x7FFFFFFFLL) return BA_ERR_UNSUPPORTED;
+    tc::attn_tc_kernel<<<static_cast<unsigned>(tiles), tc::kThreads, tc::kDynSmem, cs>>>(
+        mq, mk, mv, kv_idx, kv_cnt, kmax, static_cast<__nv_bfloat16 *>(O), LSE, s->Hq, s->Hkv, s->N, s->N_alloc, nb,
+        scale * 1.4426950408889634f);
+    return from_cuda(cudaGetLastError());
+  }
+  cudaError_t e;
+  if (s->dtype == BA_DTYPE_BF16) {
+    auto q = static_cast<const __nv_bfloat16 *>(Q);
+    auto k = static_cast<const __nv_bfloat16 *>(K);
+    auto v = static_cast<const __nv_bfloat16 *>(V);
+    auto o = static_cast<__nv_bfloat16 *>(O);
+    e = s->d == 128 ? launch_attn_simt<__nv_bfloat16, 128>(q, k, v, kv_idx, kv_cnt, kmax, o, LSE, s->B, s->Hq, s->Hkv,
+                                                           s->N, s->N_alloc, s->block, scale, cs)
+                    : launch_attn_simt<__nv_bfloat16, 64>(q, k, v, kv_idx, kv_cnt, kmax, o, LSE, s->B, s->Hq, s->Hkv,
+                                                          s->N, s->N_alloc, s->block, scale, cs);
+  } else {
+    auto q = static_cast<const float *>(Q);
+    auto k = static_cast<const float *>(K);
+    auto v = static_cast<const float *>(V);
+    auto o = static_cast<float *>(O);
+    e = s->d == 128 ? launch_attn_simt<float, 128>(q, k, v, kv_idx, kv_cnt, kmax, o, LSE, s->B, s->Hq, s->Hkv, s->N,
+                                                   s->N_alloc, s->block, scale, cs)
+                    : launch_attn_simt<float, 64>(q, k, v, kv_idx, kv_cnt, kmax, o, LSE, s->B, s->Hq, s->Hkv, s->N,
+                                                  s->N_alloc, s->block, scale, cs);
+  }
+  return from_cuda(e);
+}
+
+ba_status ba_att_merge_lse(int64_t rows, int32_t d, int32_t dtype, const void *O1, const float *L1, const void *O2,
+                           const float *L2, void *O, float *L, ba_stream_t stream) {
+  if (rows < 0) return BA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return BA_ERR_UNSUPPORTED;
+  if (dtype != BA_DTYPE_F32 && dtype != BA_DTYPE_BF16) return BA_ERR_INVALID_ARG;
+  if (!O1 || !L1 || !O2 || !L2 || !O || !L) return BA_ERR_INVALID_ARG;
+  if (!aligned16(O1) || !aligned16(O2) || !aligned16(O) || (reinterpret_cast<uintptr_t>(L1) & 3u) ||
+      (reinterpret_cast<uintptr_t>(L2) & 3u) || (reinterpret_cast<uintptr_t>(L) & 3u))
+    return BA_ERR_MISALIGNED;
+  if (rows == 0) return BA_OK;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  const int sms = num_sms_of_current_device();
+  cudaError_t e;
+  if (dtype == BA_DTYPE_BF16) {
+    auto o1 = static_cast<const __nv_bfloat16 *>(O1);
+    auto o2 = static_cast<const __nv_bfloat16 *>(O2);
+    auto o = static_cast<__nv_bfloat16 *>(O);
+    e = d == 128 ? launch_merge<__nv_bfloat16, 128>(o1, L1, o2, L2, o, L, rows, sms, cs)
+                 : launch_merge<__nv_bfloat16, 64>(o1, L1, o2, L2, o, L, rows, sms, cs);
+  } else {
+    auto o1 = static_cast<const float *>(O1);
+    auto o2 = static_cast<const float *>(O2);
+    auto o = static_cast<float *>(O);
+    e = d == 128 ? launch_merge<float, 128>(o1, L1, o2, L2, o, L, rows, sms, cs)
+                 : launch_merge<float, 64>(o1, L1, o2, L2, o, L, rows, sms, cs);
+  }
+  return from_cuda(e);
+}
+
+ba_status ba_att_get_device_error(ba_stream_t stream, uint32_t *word_out) {
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(cs) != cudaSuccess) return BA_ERR_CUDA;
+  unsigned int word = 0;
+  if (cudaMemcpyFromSymbol(&word, g_error_word, sizeof(word)) != cudaSuccess) return BA_ERR_CUDA;
+  const unsigned int zero = 0;
+  if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return BA_ERR_CUDA;
+  if (word_out) *word_out = word;
+  if (word == 0) return BA_OK;
+  if (word & BA_DEVERR_WAIT_TIMEOUT) return BA_ERR_TIMEOUT;
+  return BA_ERR_DEVICE;
+}
+
+ba_status ba_att_selftest_bounded_wait(uint32_t timeout_us, ba_stream_t stream) {
+  if (timeout_us < 1 || timeout_us > 2000000u) return BA_ERR_INVALID_ARG;
+  bounded_wait_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<unsigned long long>(timeout_us) * 1000ull);
+  return from_cuda(cudaGetLastError());
+}
+
+}  // extern "C"

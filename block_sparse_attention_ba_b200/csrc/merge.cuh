@@ -1,0 +1,144 @@
+// merge.cuh — K9: log-space merge of two partial attentions, and the list
+// split that produces the two partial key sets.
+//
+// "FlashBlock: Attention Caching for Efficient Long-Context Block Diffusion",
+// Eq. 5 (attention over a key set splits exactly into the contributions of
+// two disjoint parts) and Eq. 9 (the parts are recombined from their outputs
+// and log-normalisers after subtracting the larger normaliser).
+#pragma once
+
+#include "common.cuh"
+
+namespace baatt {
+
+constexpr int kMergeThreads = 256;
+
+// One 16-byte vector of a row per thread; rows are independent. HBM-bound:
+// reads O1, O2, L1, L2 once and writes O, L once.
+template <typename T, int D>
+__global__ void __launch_bounds__(kMergeThreads) merge_lse_kernel(const T *O1,
+                                                                  const float *L1, const T *O2,
+                                                                  const float *L2, T *O, float *L,
+                                                                  long long rows) {
+  constexpr int VEC = Elem<T>::kVec;
+  constexpr int VPR = D / VEC;                         // vectors per row
+  const long long total = rows * VPR;
+  const int lane = threadIdx.x & 31;
+  // A row's VPR threads sit in one warp (VPR divides 32), so a __syncwarp()
+  // between the reads and the writes makes the in-place forms (O == O1,
+  // L == L1, ...) safe. The loop bound is warp-uniform for that reason.
+  for (long long base = blockIdx.x * static_cast<long long>(kMergeThreads) + (threadIdx.x & ~31); base < total;
+       base += static_cast<long long>(gridDim.x) * kMergeThreads) {
+    const long long v = base + lane;
+    const bool act = v < total;
+    const long long r = act ? v / VPR : 0;
+    const int c = static_cast<int>(v % VPR);
+    float out[VEC];
+    float lse = 0.f;
+    if (act) {
+      const float l1 = L1[r], l2 = L2[r];
+      const float m = fmaxf(l1, l2);
+      const bool empty = (m == -INFINITY);
+      const float w1 = empty ? 0.f : expf(l1 - m);
+      const float w2 = empty ? 0.f : expf(l2 - m);
+      const float den = w1 + w2;
+      const float inv = empty ? 0.f : 1.f / den;
+      const uint4 a = *(reinterpret_cast<const uint4 *>(O1 + r * D) + c);
+      const uint4 bb = *(reinterpret_cast<const uint4 *>(O2 + r * D) + c);
+      float fa[VEC], fb[VEC];
+      Elem<T>::unpack(a, fa);
+      Elem<T>::unpack(bb, fb);
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) out[e] = (w1 * fa[e] + w2 * fb[e]) * inv;
+      lse = empty ? -INFINITY : m + logf(den);
+    }
+    __syncwarp();
+    if (act) {
+      uint4 res;
+      if constexpr (VEC == 8) {
+        res.x = pack_bf16x2(out[0], out[1]);
+        res.y = pack_bf16x2(out[2], out[3]);
+        res.z = pack_bf16x2(out[4], out[5]);
+        res.w = pack_bf16x2(out[6], out[7]);
+      } else {
+        res.x = __float_as_uint(out[0]);
+        res.y = __float_as_uint(out[1]);
+        res.z = __float_as_uint(out[2]);
+        res.w = __float_as_uint(out[3]);
+      }
+      reinterpret_cast<uint4 *>(O + r * D)[c] = res;
+      if (c == 0) L[r] = lse;
+    }
+  }
+}
+
+template <typename T, int D>
+cudaError_t launch_merge(const T *O1, const float *L1, const T *O2, const float *L2, T *O, float *L, long long rows,
+                         int num_sms, cudaStream_t stream) {
+  constexpr int VPR = D / Elem<T>::kVec;
+  const long long total = rows * VPR;
+  long long blocks = (total + kMergeThreads - 1) / kMergeThreads;
+  const long long cap = static_cast<long long>(num_sms) * 8;     // 8 resident CTAs per SM
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  merge_lse_kernel<T, D><<<static_cast<unsigned>(blocks), kMergeThreads, 0, stream>>>(O1, L1, O2, L2, O, L, rows);
+  return cudaGetLastError();
+}
+
+// One warp per list: entries below split_block go to the "lo" list, the rest
+// to the "hi" list; both stay ascending. Out-of-range entries are dropped and
+// flagged.
+__global__ void split_lists_kernel(const int32_t *__restrict__ idx, const int32_t *__restrict__ cnt, int32_t *lo_idx,
+                                   int32_t *lo_cnt, int32_t *hi_idx, int32_t *hi_cnt, long long n_lists, int kmax,
+                                   int nk, int split) {
+  const unsigned full = 0xFFFFFFFFu;
+  const int lane = threadIdx.x & 31;
+  const unsigned lt_mask = (1u << lane) - 1u;
+  const long long warps_total = static_cast<long long>(gridDim.x) * (blockDim.x / 32);
+  for (long long row = blockIdx.x * static_cast<long long>(blockDim.x / 32) + (threadIdx.x >> 5); row < n_lists;
+       row += warps_total) {
+    int c = __ldg(cnt + row);
+    if (c < 0 || c > kmax) {
+      if (lane == 0) raise_error(BA_DEVERR_BAD_COUNT);
+      c = c < 0 ? 0 : kmax;
+    }
+    const int32_t *in = idx + row * kmax;
+    int32_t *lo = lo_idx + row * kmax;
+    int32_t *hi = hi_idx + row * kmax;
+    int nlo = 0, nhi = 0;
+    for (int t0 = 0; t0 < c; t0 += 32) {
+      const int t = t0 + lane;
+      const int j = t < c ? __ldg(in + t) : -1;
+      const bool ok = t < c && j >= 0 && j < nk;
+      if (t < c && !ok) raise_error(BA_DEVERR_BAD_INDEX);
+      const bool is_lo = ok && j < split;
+      const bool is_hi = ok && j >= split;
+      const unsigned bl = __ballot_sync(full, is_lo);
+      const unsigned bh = __ballot_sync(full, is_hi);
+      if (is_lo) lo[nlo + __popc(bl & lt_mask)] = j;
+      if (is_hi) hi[nhi + __popc(bh & lt_mask)] = j;
+      nlo += __popc(bl);
+      nhi += __popc(bh);
+    }
+    for (int t = nlo + lane; t < kmax; t += 32) lo[t] = -1;
+    for (int t = nhi + lane; t < kmax; t += 32) hi[t] = -1;
+    if (lane == 0) {
+      lo_cnt[row] = nlo;
+      hi_cnt[row] = nhi;
+    }
+  }
+}
+
+inline cudaError_t launch_split(const int32_t *idx, const int32_t *cnt, int32_t *lo_idx, int32_t *lo_cnt,
+                                int32_t *hi_idx, int32_t *hi_cnt, long long n_lists, int kmax, int nk, int split,
+                                int num_sms, cudaStream_t stream) {
+  long long blocks = (n_lists + 7) / 8;
+  const long long cap = static_cast<long long>(num_sms) * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  split_lists_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(idx, cnt, lo_idx, lo_cnt, hi_idx, hi_cnt,
+                                                                          n_lists, kmax, nk, split);
+  return cudaGetLastError();
+}
+
+}  // namespace baatt

@@ -1,0 +1,222 @@
+/*
+ * ba_att.h — C ABI of the BA-Att hot path on NVIDIA B200 (sm_100a).
+ *
+ * Block Approximate Sparse Attention (BA-Att) has two stages:
+ *   1. a block-wise pre-downsample selector: per-block means and diagonal
+ *      variances of Q and K, a covariance-compensated block-score map, and
+ *      norm sorting that keeps the top fraction of key blocks per query block;
+ *   2. block-sparse bidirectional attention over the kept blocks, emitting the
+ *      output O and the per-row log-sum-exp (LSE).
+ * A companion call merges two partial attentions (O, LSE) in log space.
+ *
+ * Sources: "Efficient Long-Context Modeling in Diffusion Language Models via
+ * Block Approximate Sparse Attention" (abstract, "Core claim", "What carries
+ * the argument", Figure 4) and "FlashBlock: Attention Caching for Efficient
+ * Long-Context Block Diffusion" (Eq. 5, Eq. 9). The pages give the method in
+ * prose only; the formulas stated below are the plain reading of that prose.
+ *
+ * Conventions shared by every call
+ *  - Tensors are dense, row-major, head-major: Q is [B, Hq, N_alloc, d];
+ *    K and V are [B, Hkv, N_alloc, d]. Only rows n < N of each head are
+ *    tokens; rows N..N_alloc-1 are padding that is never read as a token and
+ *    never written.
+ *  - Blocks: block size b for queries and keys alike; nq = nk = ceil(N / b);
+ *    block i covers rows [i*b, min(N, (i+1)*b)) (the last may be ragged).
+ *  - Grouped-query attention: query head h uses KV head h / (Hq / Hkv).
+ *  - Memory: the caller allocates and owns every buffer. Device pointers are
+ *    CUDA device (or managed) memory, 16-byte aligned. The library allocates
+ *    no device memory; its only global state is one device-side error word.
+ *  - Streams: every call is asynchronous on `stream` (NULL = legacy default
+ *    stream) and never synchronises, except ba_att_get_device_error.
+ *  - Errors: arguments are checked on the host before anything is launched;
+ *    a bad argument returns a status and launches nothing. A failed launch
+ *    returns BA_ERR_CUDA. Inconsistent data discovered on the device (an
+ *    out-of-range block index, a count above kmax, a list not strictly
+ *    ascending) never traps: the offending entry is skipped, a bit is set in
+ *    the device error word, and ba_att_get_device_error reports it later.
+ */
+#ifndef BA_ATT_H
+#define BA_ATT_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t; declared here so the header needs no CUDA. */
+typedef struct CUstream_st *ba_stream_t;
+
+typedef enum {
+  BA_OK = 0,
+  BA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, keep outside (0,1], ... */
+  BA_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. d = 96)        */
+  BA_ERR_MISALIGNED = 3,    /* a pointer is not 16-byte aligned               */
+  BA_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed           */
+  BA_ERR_DEVICE = 5,        /* device-side data check failed (see error word) */
+  BA_ERR_TIMEOUT = 6        /* a bounded device-side wait ran out             */
+} ba_status;
+
+typedef enum { BA_DTYPE_F32 = 0, BA_DTYPE_BF16 = 1 } ba_dtype;
+
+/* Device error word bits (ba_att_get_device_error). */
+#define BA_DEVERR_BAD_INDEX     0x1u  /* block index outside [0, nk)          */
+#define BA_DEVERR_BAD_COUNT     0x2u  /* count outside [0, kmax]              */
+#define BA_DEVERR_NOT_ASCENDING 0x4u  /* list entries not strictly ascending  */
+#define BA_DEVERR_WAIT_TIMEOUT  0x8u  /* a bounded barrier wait gave up       */
+
+typedef struct {
+  int32_t B;        /* batch                                   >= 1          */
+  int32_t Hq;       /* query heads                             >= 1          */
+  int32_t Hkv;      /* key/value heads, divides Hq             >= 1          */
+  int32_t N;        /* valid tokens per head                   >= 1          */
+  int32_t N_alloc;  /* rows allocated per head                 >= N          */
+  int32_t d;        /* head dimension: 64 or 128                             */
+  int32_t block;    /* block size b: a multiple of 16 in [16, 256]           */
+  int32_t dtype;    /* ba_dtype of Q, K, V and O                             */
+  float sm_scale;   /* softmax scale s; <= 0 selects d^-1/2                  */
+} ba_att_shape;
+
+/* Library version string, e.g. "0.1.0 sm_100a". Never NULL. */
+const char *ba_att_version(void);
+
+/* Human-readable name of a status. Never NULL. */
+const char *ba_att_status_string(ba_status status);
+
+/* nq = nk = ceil(N / block); -1 if the shape is invalid. */
+int32_t ba_att_num_blocks(const ba_att_shape *shape);
+
+/* Kept blocks per query block: max(1, ceil(keep * nk)) (the selector keeps
+ * the top fraction of key blocks; "Core claim"). -1 if keep is outside (0,1]
+ * or the shape is invalid. */
+int32_t ba_att_keep_count(const ba_att_shape *shape, float keep);
+
+/*
+ * ba_att_stats — stage one, block-wise pre-downsample statistics
+ * (BA-Att abstract: "block-wise pre-downsampled operation"; diagonal Q/K
+ * variances from "Core claim").
+ *
+ * For every block i and head h, over the valid rows r of the block:
+ *   mean[i, m] = (1/n_i) sum_r x[r, m]
+ *   var [i, m] = (1/n_i) sum_r (x[r, m] - mean[i, m])^2     (population)
+ * computed in fp32 (two passes over register-resident data).
+ *
+ * Q, K      device, [B,Hq|Hkv,N_alloc,d] of shape->dtype; read once.
+ * q_mean, q_var   device fp32 [B, Hq,  nq, d]  (written)
+ * k_mean, k_var   device fp32 [B, Hkv, nk, d]  (written)
+ */
+ba_status ba_att_stats(const ba_att_shape *shape, const void *Q, const void *K,
+                       float *q_mean, float *q_var, float *k_mean, float *k_var,
+                       ba_stream_t stream);
+
+/*
+ * ba_att_select — covariance-compensated block scores + norm sorting
+ * (BA-Att abstract and "Core claim": score blocks in the downsampled space,
+ * correct the pooled score with diagonal Q/K variances, sort, keep the top
+ * fraction; Figure 2 names the sorted metric).
+ *
+ *   S~[i, j] = s * qbar_i . kbar_j
+ *            + (s^2/2) * sum_m ( vq_i,m kbar_j,m^2 + qbar_i,m^2 vk_j,m + vq_i,m vk_j,m )
+ *            + ln m_j
+ * i.e. ln E[e^x] for the Gaussian model x = s q.k with q, k independent with
+ * the block means and diagonal variances, summed over the m_j keys of block j.
+ * Per (batch, query head, query block) the key blocks are ranked by S~
+ * descending (ties: lower j first) and the first k = ba_att_keep_count(keep)
+ * are kept and written in ascending order.
+ *
+ * q_mean..k_var   device fp32, as written by ba_att_stats.
+ * kv_idx          device int32 [B, Hq, nq, kmax]: kept key-block indices,
+ *                 ascending; entries at positions >= count are set to -1.
+ * kv_cnt          device int32 [B, Hq, nq]: number kept (= k).
+ * kmax            row stride of kv_idx; must be >= k.
+ * block_scores    nullable device fp32 [B, Hq, nq, nk]: if non-NULL, S~ is
+ *                 also written there.
+ * Requires nk <= 4096.
+ */
+ba_status ba_att_select(const ba_att_shape *shape, float keep,
+                        const float *q_mean, const float *q_var,
+                        const float *k_mean, const float *k_var,
+                        int32_t *kv_idx, int32_t *kv_cnt, int32_t kmax,
+                        float *block_scores, ba_stream_t stream);
+
+/*
+ * ba_att_split_lists — partition every kept-block list at a key-block
+ * boundary into a block-external span (blocks < split_block) and a
+ * block-internal span (blocks >= split_block) (FlashBlock Eq. 5: the two
+ * parts are attended separately and merged with ba_att_merge_lse).
+ *
+ * kv_idx, kv_cnt        device int32 input lists, layout as ba_att_select.
+ * lo_idx/lo_cnt, hi_idx/hi_cnt   device int32 outputs, same layouts and kmax;
+ *                       unused entries are -1. Input entries that are out of
+ *                       range are dropped and flagged in the error word.
+ * 0 <= split_block <= nk.
+ */
+ba_status ba_att_split_lists(const ba_att_shape *shape, int32_t split_block,
+                             const int32_t *kv_idx, const int32_t *kv_cnt, int32_t kmax,
+                             int32_t *lo_idx, int32_t *lo_cnt,
+                             int32_t *hi_idx, int32_t *hi_cnt, ba_stream_t stream);
+
+/*
+ * ba_att_sparse_fwd — block-sparse bidirectional attention forward
+ * (BA-Att abstract and Figure 4: attention evaluated only over the kept
+ * blocks, no causal mask).
+ *
+ * For every valid row r of query block i, with C_i the valid keys of blocks
+ * kv_idx[i, 0..kv_cnt[i]):
+ *   LSE[r] = ln sum_{c in C_i} exp(s q_r . k_c)
+ *   O[r]   = sum_{c in C_i} exp(s q_r . k_c - LSE[r]) v_c
+ * computed with an online softmax over the kept blocks, fp32 accumulation,
+ * O rounded to nearest-even into shape->dtype. An empty list gives O[r] = 0
+ * and LSE[r] = -inf. Rows >= N are not written.
+ *
+ * Q, K, V   device, shape->dtype, layouts as above.
+ * kv_idx, kv_cnt, kmax   device int32 lists as written by ba_att_select
+ *           (any strictly ascending lists in [0, nk) are accepted).
+ * O         device [B, Hq, N_alloc, d] of shape->dtype (written).
+ * LSE       device fp32 [B, Hq, N_alloc], natural log (written).
+ * Paths: bf16 with d = 128 and block = 128 runs the tcgen05/TMEM tensor-core
+ * kernel; every other supported shape runs an fp32 CUDA-core kernel.
+ */
+ba_status ba_att_sparse_fwd(const ba_att_shape *shape,
+                            const void *Q, const void *K, const void *V,
+                            const int32_t *kv_idx, const int32_t *kv_cnt, int32_t kmax,
+                            void *O, float *LSE, ba_stream_t stream);
+
+/*
+ * ba_att_merge_lse — log-space merge of two partial attentions over disjoint
+ * key sets (FlashBlock Eq. 9, decomposition of Eq. 5):
+ *   m = max(L1, L2), w_k = exp(L_k - m),
+ *   O = (w1 O1 + w2 O2) / (w1 + w2),  L = m + ln(w1 + w2);
+ * both L = -inf gives O = 0, L = -inf.
+ *
+ * rows      number of rows (e.g. B*Hq*N_alloc); d in {64, 128}.
+ * O1, O2, O device [rows, d] of dtype; L1, L2, L device fp32 [rows].
+ * O may alias O1 or O2 and L may alias L1 or L2 (in-place merge).
+ */
+ba_status ba_att_merge_lse(int64_t rows, int32_t d, int32_t dtype,
+                           const void *O1, const float *L1,
+                           const void *O2, const float *L2,
+                           void *O, float *L, ba_stream_t stream);
+
+/*
+ * ba_att_get_device_error — synchronise `stream`, read the device error word
+ * of the current device, clear it, and return BA_OK (word 0), BA_ERR_TIMEOUT
+ * (timeout bit set) or BA_ERR_DEVICE (any other bit). *word_out (nullable)
+ * receives the raw bits.
+ */
+ba_status ba_att_get_device_error(ba_stream_t stream, uint32_t *word_out);
+
+/*
+ * ba_att_selftest_bounded_wait — launch one CTA that waits on a shared-memory
+ * barrier no thread ever arrives on, giving up after timeout_us microseconds
+ * (1 <= timeout_us <= 2000000). It exercises the bounded-wait path every
+ * pipelined kernel here uses: the wait must end, set BA_DEVERR_WAIT_TIMEOUT
+ * and leave the context usable. No counterpart on the pages.
+ */
+ba_status ba_att_selftest_bounded_wait(uint32_t timeout_us, ba_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BA_ATT_H */

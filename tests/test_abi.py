@@ -1,0 +1,119 @@
+"""The C-ABI library loads without a GPU, exports every symbol the header
+declares, and rejects bad arguments on the host before launching anything.
+CPU only: no call here reaches a kernel launch."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from block_sparse_attention_ba_b200 import api
+from block_sparse_attention_ba_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ba_att.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return api.load_library()
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(ba_att_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = header_functions()
+    for n in ("ba_att_stats", "ba_att_select", "ba_att_sparse_fwd", "ba_att_merge_lse", "ba_att_split_lists",
+              "ba_att_num_blocks", "ba_att_keep_count", "ba_att_get_device_error", "ba_att_status_string",
+              "ba_att_version"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in header_functions():
+        assert hasattr(lib, name), name
+    assert set(header_functions()) == set(api._SIGS)
+
+
+def test_version_and_status_strings(lib):
+    assert lib.ba_att_version().decode().endswith("sm_100a")
+    for code, name in api.STATUS_NAMES.items():
+        assert lib.ba_att_status_string(code).decode() == name
+
+
+def shape(**kw):
+    base = dict(B=1, Hq=4, Hkv=2, N=1000, N_alloc=1024, d=128, block=128, dtype=api.DTYPE_BF16, sm_scale=0.0)
+    base.update(kw)
+    return api.CShape(**base)
+
+
+def test_num_blocks_and_keep_count(lib):
+    s = shape()
+    assert lib.ba_att_num_blocks(ctypes.byref(s)) == 8
+    assert lib.ba_att_keep_count(ctypes.byref(s), ctypes.c_float(0.5)) == 4
+    assert lib.ba_att_keep_count(ctypes.byref(s), ctypes.c_float(1.0)) == 8
+    assert lib.ba_att_keep_count(ctypes.byref(s), ctypes.c_float(1e-4)) == 1
+    assert lib.ba_att_keep_count(ctypes.byref(s), ctypes.c_float(0.0)) == -1
+    assert lib.ba_att_keep_count(ctypes.byref(s), ctypes.c_float(1.5)) == -1
+    for n, keep, k in ((256, 0.5, 128), (256, 0.25, 64), (1024, 0.5, 512), (16, 0.5, 8)):
+        s = shape(N=n * 128, N_alloc=n * 128)
+        assert lib.ba_att_keep_count(ctypes.byref(s), ctypes.c_float(keep)) == k
+
+
+P = ctypes.c_void_p(0x10000)       # aligned, never dereferenced: every call below fails validation
+MIS = ctypes.c_void_p(0x10008)
+
+
+@pytest.mark.parametrize("bad,status", [
+    (dict(d=96), 2), (dict(block=100), 2), (dict(block=512), 2), (dict(Hq=3, Hkv=2), 1), (dict(N=0), 1),
+    (dict(N_alloc=10), 1), (dict(dtype=7), 1), (dict(B=0), 1), (dict(sm_scale=float("nan")), 1),
+])
+def test_bad_shapes_rejected(lib, bad, status):
+    s = shape(**bad)
+    assert lib.ba_att_stats(ctypes.byref(s), P, P, P, P, P, P, None) == status
+    assert lib.ba_att_sparse_fwd(ctypes.byref(s), P, P, P, P, P, 4, P, P, None) == status
+    assert lib.ba_att_select(ctypes.byref(s), ctypes.c_float(0.5), P, P, P, P, P, P, 8, None, None) == status
+    assert lib.ba_att_num_blocks(ctypes.byref(s)) == -1
+
+
+def test_null_and_misaligned_pointers(lib):
+    s = shape()
+    assert lib.ba_att_stats(None, P, P, P, P, P, P, None) == 1
+    assert lib.ba_att_stats(ctypes.byref(s), None, P, P, P, P, P, None) == 1
+    assert lib.ba_att_stats(ctypes.byref(s), MIS, P, P, P, P, P, None) == 3
+    assert lib.ba_att_sparse_fwd(ctypes.byref(s), P, P, P, P, P, 4, None, P, None) == 1
+    assert lib.ba_att_sparse_fwd(ctypes.byref(s), P, P, MIS, P, P, 4, P, P, None) == 3
+    assert lib.ba_att_select(ctypes.byref(s), ctypes.c_float(0.5), P, P, P, P, P, MIS, 8, None, None) == 3
+    assert lib.ba_att_merge_lse(10, 128, 1, P, P, None, P, P, P, None) == 1
+    assert lib.ba_att_merge_lse(10, 128, 1, MIS, P, P, P, P, P, None) == 3
+
+
+def test_selection_arguments(lib):
+    s = shape()
+    # keep outside (0, 1]
+    assert lib.ba_att_select(ctypes.byref(s), ctypes.c_float(0.0), P, P, P, P, P, P, 8, None, None) == 1
+    assert lib.ba_att_select(ctypes.byref(s), ctypes.c_float(1.01), P, P, P, P, P, P, 8, None, None) == 1
+    # kmax below the kept count (keep 0.5 of 8 blocks = 4)
+    assert lib.ba_att_select(ctypes.byref(s), ctypes.c_float(0.5), P, P, P, P, P, P, 3, None, None) == 1
+    # too many blocks for the in-shared-memory selector
+    big = shape(N=4097 * 16, N_alloc=4097 * 16, block=16)
+    assert lib.ba_att_select(ctypes.byref(big), ctypes.c_float(0.5), P, P, P, P, P, P, 4097, None, None) == 2
+    # split point outside [0, nb]
+    assert lib.ba_att_split_lists(ctypes.byref(s), 9, P, P, 8, P, P, P, P, None) == 1
+    assert lib.ba_att_split_lists(ctypes.byref(s), -1, P, P, 8, P, P, P, P, None) == 1
+    assert lib.ba_att_sparse_fwd(ctypes.byref(s), P, P, P, P, P, 0, P, P, None) == 1
+
+
+def test_merge_and_selftest_arguments(lib):
+    assert lib.ba_att_merge_lse(10, 96, 1, P, P, P, P, P, P, None) == 2
+    assert lib.ba_att_merge_lse(10, 128, 5, P, P, P, P, P, P, None) == 1
+    assert lib.ba_att_merge_lse(-1, 128, 1, P, P, P, P, P, P, None) == 1
+    assert lib.ba_att_merge_lse(0, 128, 1, P, P, P, P, P, P, None) == 0     # nothing to do
+    assert lib.ba_att_selftest_bounded_wait(0, None) == 1
+    assert lib.ba_att_selftest_bounded_wait(3_000_000, None) == 1
