@@ -217,7 +217,10 @@ def run_ours(args):
     idx = torch.empty((w.B, w.Hq, nb, k), device=dev, dtype=torch.int32)
     cnt = torch.empty((w.B, w.Hq, nb), device=dev, dtype=torch.int32)
     lists = (torch.empty_like(idx), torch.empty_like(cnt), torch.empty_like(idx), torch.empty_like(cnt))
-    O1, O2, Om = torch.empty_like(Qd), torch.empty_like(Qd), torch.empty_like(Qd)
+    # span partials stay in fp32 so the merged output is rounded to bf16 once
+    O1 = torch.empty(Qd.shape, device=dev, dtype=torch.float32)
+    O2 = torch.empty(Qd.shape, device=dev, dtype=torch.float32)
+    Om = torch.empty_like(Qd)
     L1, L2, Lm = (torch.empty((w.B, w.Hq, w.N_alloc), device=dev) for _ in range(3))
     stream = torch.cuda.current_stream(dev)
 

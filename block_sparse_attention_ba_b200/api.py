@@ -42,8 +42,8 @@ _SIGS = {
     "ba_att_stats": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _P, _P, _P, _P, _P]),
     "ba_att_select": (ctypes.c_int, [ctypes.POINTER(CShape), ctypes.c_float, _P, _P, _P, _P, _P, _P, _I32, _P, _P]),
     "ba_att_split_lists": (ctypes.c_int, [ctypes.POINTER(CShape), _I32, _P, _P, _I32, _P, _P, _P, _P, _P]),
-    "ba_att_sparse_fwd": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _P, _P, _P, _I32, _P, _P, _P]),
-    "ba_att_merge_lse": (ctypes.c_int, [ctypes.c_int64, _I32, _I32, _P, _P, _P, _P, _P, _P, _P]),
+    "ba_att_sparse_fwd": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _P, _P, _P, _I32, _P, _I32, _P, _P]),
+    "ba_att_merge_lse": (ctypes.c_int, [ctypes.c_int64, _I32, _I32, _I32, _P, _P, _P, _P, _P, _P, _P]),
     "ba_att_get_device_error": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_uint32)]),
     "ba_att_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_uint32, _P]),
 }
@@ -189,31 +189,40 @@ def split_lists(idx: torch.Tensor, cnt: torch.Tensor, shape: Shape, split_block:
     return out
 
 
-def sparse_fwd(Q, K, V, idx, cnt, shape: Shape, out=None):
-    """Block-sparse attention over the kept blocks -> (O, LSE)."""
+_TORCH_DT = {torch.float32: DTYPE_F32, torch.bfloat16: DTYPE_BF16}
+
+
+def sparse_fwd(Q, K, V, idx, cnt, shape: Shape, out=None, out_dtype=None):
+    """Block-sparse attention over the kept blocks -> (O, LSE).
+
+    out_dtype=torch.float32 keeps O in fp32 (for partials merged later)."""
     lib = load_library()
     if out is None:
-        out = (torch.empty_like(Q),
+        odt = Q.dtype if out_dtype is None else out_dtype
+        out = (torch.empty(Q.shape, device=Q.device, dtype=odt),
                torch.empty((shape.B, shape.Hq, shape.N_alloc), device=Q.device, dtype=torch.float32))
     O, LSE = out
     _check("ba_att_sparse_fwd", lib.ba_att_sparse_fwd(
         ctypes.byref(shape.c()), _dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), _dev(idx, "kv_idx"), _dev(cnt, "kv_cnt"),
-        idx.shape[-1], _dev(O, "O"), _dev(LSE, "LSE"), _stream(Q)))
+        idx.shape[-1], _dev(O, "O"), _TORCH_DT[O.dtype], _dev(LSE, "LSE"), _stream(Q)))
     return out
 
 
-def merge_lse(O1, L1, O2, L2, out=None):
-    """Log-space merge of two partial attentions -> (O, L). out may alias (O1, L1)."""
+def merge_lse(O1, L1, O2, L2, out=None, out_dtype=None):
+    """Log-space merge of two partial attentions -> (O, L).
+
+    out may alias (O1, L1) when the dtypes agree; out_dtype=torch.bfloat16
+    rounds fp32 partials once into a bf16 output."""
     lib = load_library()
     d = O1.shape[-1]
     rows = O1.numel() // d
-    dt = {torch.float32: DTYPE_F32, torch.bfloat16: DTYPE_BF16}[O1.dtype]
     if out is None:
-        out = (torch.empty_like(O1), torch.empty_like(L1))
+        out = (torch.empty(O1.shape, device=O1.device, dtype=O1.dtype if out_dtype is None else out_dtype),
+               torch.empty_like(L1))
     O, L = out
     _check("ba_att_merge_lse", lib.ba_att_merge_lse(
-        rows, d, dt, _dev(O1, "O1"), _dev(L1, "L1"), _dev(O2, "O2"), _dev(L2, "L2"), _dev(O, "O"), _dev(L, "L"),
-        _stream(O1)))
+        rows, d, _TORCH_DT[O1.dtype], _TORCH_DT[O.dtype], _dev(O1, "O1"), _dev(L1, "L1"), _dev(O2, "O2"),
+        _dev(L2, "L2"), _dev(O, "O"), _dev(L, "L"), _stream(O1)))
     return out
 
 

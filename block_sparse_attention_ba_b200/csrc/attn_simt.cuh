@@ -30,10 +30,10 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-template <typename T, int D>
+template <typename T, typename TO, int D>
 __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(
     const T *__restrict__ Q, const T *__restrict__ K, const T *__restrict__ V, const int32_t *__restrict__ kv_idx,
-    const int32_t *__restrict__ kv_cnt, int kmax, T *__restrict__ O, float *__restrict__ LSE, int Hq, int Hkv, int N,
+    const int32_t *__restrict__ kv_cnt, int kmax, TO *__restrict__ O, float *__restrict__ LSE, int Hq, int Hkv, int N,
     int N_alloc, int block, int nb, int subs, float scale_log2) {
   constexpr int DPL = D / 32;
   constexpr int RPW = kSimtRows / (kSimtThreads / 32);      // rows per warp
@@ -129,22 +129,22 @@ __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(
     if (r >= nrows) break;
     const bool has = lrow[rr] > 0.f;
     const float inv = has ? 1.f / lrow[rr] : 0.f;
-    T *orow = O + (qhead + row0 + r) * D;
+    TO *orow = O + (qhead + row0 + r) * D;
 #pragma unroll
     for (int tt = 0; tt < DPL; ++tt) store_out(orow + lane + 32 * tt, o[rr][tt] * inv);
     if (lane == 0) LSE[qhead + row0 + r] = has ? (mrow[rr] + log2f(lrow[rr])) * kLn2 : -INFINITY;
   }
 }
 
-template <typename T, int D>
-cudaError_t launch_attn_simt(const T *Q, const T *K, const T *V, const int32_t *idx, const int32_t *cnt, int kmax, T *O,
+template <typename T, typename TO, int D>
+cudaError_t launch_attn_simt(const T *Q, const T *K, const T *V, const int32_t *idx, const int32_t *cnt, int kmax, TO *O,
                              float *LSE, int B, int Hq, int Hkv, int N, int N_alloc, int block, float sm_scale,
                              cudaStream_t stream) {
   const int nb = (N + block - 1) / block;
   const int subs = (block + kSimtRows - 1) / kSimtRows;
   dim3 grid(static_cast<unsigned>(nb * subs), Hq, B);
   const float scale_log2 = sm_scale * 1.4426950408889634f;
-  attn_simt_kernel<T, D><<<grid, kSimtThreads, 0, stream>>>(Q, K, V, idx, cnt, kmax, O, LSE, Hq, Hkv, N, N_alloc,
+  attn_simt_kernel<T, TO, D><<<grid, kSimtThreads, 0, stream>>>(Q, K, V, idx, cnt, kmax, O, LSE, Hq, Hkv, N, N_alloc,
                                                              block, nb, subs, scale_log2);
   return cudaGetLastError();
 }

@@ -59,10 +59,13 @@ __device__ __forceinline__ bool entry_ok(const int32_t *list, int t, int nb, int
   return true;
 }
 
+// TO: output element type, bf16 (final output) or float (a partial that is
+// merged later, so the merged result is rounded only once).
+template <typename TO>
 __global__ void __launch_bounds__(kThreads, 2)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const int32_t *__restrict__ kv_idx,
-                   const int32_t *__restrict__ kv_cnt, int kmax, __nv_bfloat16 *__restrict__ O,
+                   const int32_t *__restrict__ kv_cnt, int kmax, TO *__restrict__ O,
                    float *__restrict__ LSE, int Hq, int Hkv, int N, int N_alloc, int nb, float scale_log2) {
   extern __shared__ uint8_t dyn_smem[];
   __shared__ Ctl ctl;
@@ -248,7 +251,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       if (qrow < N) {
         uint4 *dst = reinterpret_cast<uint4 *>(O + orow * kHeadDim);
 #pragma unroll
-        for (int v = 0; v < kHeadDim / 8; ++v) dst[v] = make_uint4(0, 0, 0, 0);
+        for (int v = 0; v < kHeadDim * static_cast<int>(sizeof(TO)) / 16; ++v) dst[v] = make_uint4(0, 0, 0, 0);
         LSE[orow] = -INFINITY;
       }
     } else if (ok) {
@@ -264,14 +267,26 @@ __global__ void __launch_bounds__(kThreads, 2)
           tmem_ld32(tO + q * 32, orr);
           tmem_ld_wait();
           if (qrow < N) {
+            if constexpr (sizeof(TO) == 2) {
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              uint4 pkt;
-              pkt.x = pack_bf16x2(__uint_as_float(orr[8 * v + 0]) * inv, __uint_as_float(orr[8 * v + 1]) * inv);
-              pkt.y = pack_bf16x2(__uint_as_float(orr[8 * v + 2]) * inv, __uint_as_float(orr[8 * v + 3]) * inv);
-              pkt.z = pack_bf16x2(__uint_as_float(orr[8 * v + 4]) * inv, __uint_as_float(orr[8 * v + 5]) * inv);
-              pkt.w = pack_bf16x2(__uint_as_float(orr[8 * v + 6]) * inv, __uint_as_float(orr[8 * v + 7]) * inv);
-              dst[q * 4 + v] = pkt;
+              for (int v = 0; v < 4; ++v) {
+                uint4 pkt;
+                pkt.x = pack_bf16x2(__uint_as_float(orr[8 * v + 0]) * inv, __uint_as_float(orr[8 * v + 1]) * inv);
+                pkt.y = pack_bf16x2(__uint_as_float(orr[8 * v + 2]) * inv, __uint_as_float(orr[8 * v + 3]) * inv);
+                pkt.z = pack_bf16x2(__uint_as_float(orr[8 * v + 4]) * inv, __uint_as_float(orr[8 * v + 5]) * inv);
+                pkt.w = pack_bf16x2(__uint_as_float(orr[8 * v + 6]) * inv, __uint_as_float(orr[8 * v + 7]) * inv);
+                dst[q * 4 + v] = pkt;
+              }
+            } else {
+#pragma unroll
+              for (int v = 0; v < 8; ++v) {
+                uint4 pkt;
+                pkt.x = __float_as_uint(__uint_as_float(orr[4 * v + 0]) * inv);
+                pkt.y = __float_as_uint(__uint_as_float(orr[4 * v + 1]) * inv);
+                pkt.z = __float_as_uint(__uint_as_float(orr[4 * v + 2]) * inv);
+                pkt.w = __float_as_uint(__uint_as_float(orr[4 * v + 3]) * inv);
+                dst[q * 8 + v] = pkt;
+              }
             }
           }
         }

@@ -212,10 +212,12 @@ ba_status ba_att_split_lists(const ba_att_shape *s, int32_t split_block, const i
 }
 
 ba_status ba_att_sparse_fwd(const ba_att_shape *s, const void *Q, const void *K, const void *V, const int32_t *kv_idx,
-                            const int32_t *kv_cnt, int32_t kmax, void *O, float *LSE, ba_stream_t stream) {
+                            const int32_t *kv_cnt, int32_t kmax, void *O, int32_t o_dtype, float *LSE,
+                            ba_stream_t stream) {
   ba_status st = check_shape(s);
   if (st != BA_OK) return st;
   if (!Q || !K || !V || !kv_idx || !kv_cnt || !O || !LSE) return BA_ERR_INVALID_ARG;
+  if (o_dtype != s->dtype && o_dtype != BA_DTYPE_F32) return BA_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(kv_idx) || !aligned16(kv_cnt) || !aligned16(O) ||
       !aligned16(LSE))
     return BA_ERR_MISALIGNED;
@@ -223,50 +225,58 @@ ba_status ba_att_sparse_fwd(const ba_att_shape *s, const void *Q, const void *K,
   const int nb = nblocks(s);
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   const float scale = effective_scale(s);
+  const bool out_f32 = (o_dtype == BA_DTYPE_F32);
   if (use_tensor_core_path(s)) {
     CUtensorMap mq, mk, mv;
     if (!make_head_map(&mq, Q, s->d, s->N, s->N_alloc, static_cast<long long>(s->B) * s->Hq) ||
         !make_head_map(&mk, K, s->d, s->N, s->N_alloc, static_cast<long long>(s->B) * s->Hkv) ||
         !make_head_map(&mv, V, s->d, s->N, s->N_alloc, static_cast<long long>(s->B) * s->Hkv))
       return BA_ERR_CUDA;
-    cudaError_t e = cudaFuncSetAttribute(tc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(tc::kDynSmem));
-    if (e != cudaSuccess) return BA_ERR_CUDA;
     const long long tiles = static_cast<long long>(s->B) * s->Hq * nb;
     if (tiles > 0x7FFFFFFFLL) return BA_ERR_UNSUPPORTED;
-    tc::attn_tc_kernel<<<static_cast<unsigned>(tiles), tc::kThreads, tc::kDynSmem, cs>>>(
-        mq, mk, mv, kv_idx, kv_cnt, kmax, static_cast<__nv_bfloat16 *>(O), LSE, s->Hq, s->Hkv, s->N, s->N_alloc, nb,
-        scale * 1.4426950408889634f);
+    const float sl2 = scale * 1.4426950408889634f;
+    cudaError_t e;
+    if (out_f32) {
+      e = cudaFuncSetAttribute(tc::attn_tc_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(tc::kDynSmem));
+      if (e != cudaSuccess) return BA_ERR_CUDA;
+      tc::attn_tc_kernel<float><<<static_cast<unsigned>(tiles), tc::kThreads, tc::kDynSmem, cs>>>(
+          mq, mk, mv, kv_idx, kv_cnt, kmax, static_cast<float *>(O), LSE, s->Hq, s->Hkv, s->N, s->N_alloc, nb, sl2);
+    } else {
+      e = cudaFuncSetAttribute(tc::attn_tc_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(tc::kDynSmem));
+      if (e != cudaSuccess) return BA_ERR_CUDA;
+      tc::attn_tc_kernel<__nv_bfloat16><<<static_cast<unsigned>(tiles), tc::kThreads, tc::kDynSmem, cs>>>(
+          mq, mk, mv, kv_idx, kv_cnt, kmax, static_cast<__nv_bfloat16 *>(O), LSE, s->Hq, s->Hkv, s->N, s->N_alloc,
+          nb, sl2);
+    }
     return from_cuda(cudaGetLastError());
   }
   cudaError_t e;
+#define BA_SIMT(T, TO, DD)                                                                                      \
+  launch_attn_simt<T, TO, DD>(static_cast<const T *>(Q), static_cast<const T *>(K), static_cast<const T *>(V), \
+                              kv_idx, kv_cnt, kmax, static_cast<TO *>(O), LSE, s->B, s->Hq, s->Hkv, s->N,       \
+                              s->N_alloc, s->block, scale, cs)
   if (s->dtype == BA_DTYPE_BF16) {
-    auto q = static_cast<const __nv_bfloat16 *>(Q);
-    auto k = static_cast<const __nv_bfloat16 *>(K);
-    auto v = static_cast<const __nv_bfloat16 *>(V);
-    auto o = static_cast<__nv_bfloat16 *>(O);
-    e = s->d == 128 ? launch_attn_simt<__nv_bfloat16, 128>(q, k, v, kv_idx, kv_cnt, kmax, o, LSE, s->B, s->Hq, s->Hkv,
-                                                           s->N, s->N_alloc, s->block, scale, cs)
-                    : launch_attn_simt<__nv_bfloat16, 64>(q, k, v, kv_idx, kv_cnt, kmax, o, LSE, s->B, s->Hq, s->Hkv,
-                                                          s->N, s->N_alloc, s->block, scale, cs);
+    if (out_f32)
+      e = s->d == 128 ? BA_SIMT(__nv_bfloat16, float, 128) : BA_SIMT(__nv_bfloat16, float, 64);
+    else
+      e = s->d == 128 ? BA_SIMT(__nv_bfloat16, __nv_bfloat16, 128) : BA_SIMT(__nv_bfloat16, __nv_bfloat16, 64);
   } else {
-    auto q = static_cast<const float *>(Q);
-    auto k = static_cast<const float *>(K);
-    auto v = static_cast<const float *>(V);
-    auto o = static_cast<float *>(O);
-    e = s->d == 128 ? launch_attn_simt<float, 128>(q, k, v, kv_idx, kv_cnt, kmax, o, LSE, s->B, s->Hq, s->Hkv, s->N,
-                                                   s->N_alloc, s->block, scale, cs)
-                    : launch_attn_simt<float, 64>(q, k, v, kv_idx, kv_cnt, kmax, o, LSE, s->B, s->Hq, s->Hkv, s->N,
-                                                  s->N_alloc, s->block, scale, cs);
+    e = s->d == 128 ? BA_SIMT(float, float, 128) : BA_SIMT(float, float, 64);
   }
+#undef BA_SIMT
   return from_cuda(e);
 }
 
-ba_status ba_att_merge_lse(int64_t rows, int32_t d, int32_t dtype, const void *O1, const float *L1, const void *O2,
-                           const float *L2, void *O, float *L, ba_stream_t stream) {
+ba_status ba_att_merge_lse(int64_t rows, int32_t d, int32_t in_dtype, int32_t out_dtype, const void *O1,
+                           const float *L1, const void *O2, const float *L2, void *O, float *L, ba_stream_t stream) {
   if (rows < 0) return BA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return BA_ERR_UNSUPPORTED;
-  if (dtype != BA_DTYPE_F32 && dtype != BA_DTYPE_BF16) return BA_ERR_INVALID_ARG;
+  if ((in_dtype != BA_DTYPE_F32 && in_dtype != BA_DTYPE_BF16) ||
+      (out_dtype != BA_DTYPE_F32 && out_dtype != BA_DTYPE_BF16))
+    return BA_ERR_INVALID_ARG;
+  if (in_dtype == BA_DTYPE_BF16 && out_dtype == BA_DTYPE_F32) return BA_ERR_UNSUPPORTED;
   if (!O1 || !L1 || !O2 || !L2 || !O || !L) return BA_ERR_INVALID_ARG;
   if (!aligned16(O1) || !aligned16(O2) || !aligned16(O) || (reinterpret_cast<uintptr_t>(L1) & 3u) ||
       (reinterpret_cast<uintptr_t>(L2) & 3u) || (reinterpret_cast<uintptr_t>(L) & 3u))
@@ -275,19 +285,16 @@ ba_status ba_att_merge_lse(int64_t rows, int32_t d, int32_t dtype, const void *O
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   const int sms = num_sms_of_current_device();
   cudaError_t e;
-  if (dtype == BA_DTYPE_BF16) {
-    auto o1 = static_cast<const __nv_bfloat16 *>(O1);
-    auto o2 = static_cast<const __nv_bfloat16 *>(O2);
-    auto o = static_cast<__nv_bfloat16 *>(O);
-    e = d == 128 ? launch_merge<__nv_bfloat16, 128>(o1, L1, o2, L2, o, L, rows, sms, cs)
-                 : launch_merge<__nv_bfloat16, 64>(o1, L1, o2, L2, o, L, rows, sms, cs);
-  } else {
-    auto o1 = static_cast<const float *>(O1);
-    auto o2 = static_cast<const float *>(O2);
-    auto o = static_cast<float *>(O);
-    e = d == 128 ? launch_merge<float, 128>(o1, L1, o2, L2, o, L, rows, sms, cs)
-                 : launch_merge<float, 64>(o1, L1, o2, L2, o, L, rows, sms, cs);
-  }
+#define BA_MERGE(TI, TO, DD)                                                                                      \
+  launch_merge<TI, TO, DD>(static_cast<const TI *>(O1), L1, static_cast<const TI *>(O2), L2, static_cast<TO *>(O), \
+                           L, rows, sms, cs)
+  if (in_dtype == BA_DTYPE_BF16)
+    e = d == 128 ? BA_MERGE(__nv_bfloat16, __nv_bfloat16, 128) : BA_MERGE(__nv_bfloat16, __nv_bfloat16, 64);
+  else if (out_dtype == BA_DTYPE_BF16)
+    e = d == 128 ? BA_MERGE(float, __nv_bfloat16, 128) : BA_MERGE(float, __nv_bfloat16, 64);
+  else
+    e = d == 128 ? BA_MERGE(float, float, 128) : BA_MERGE(float, float, 64);
+#undef BA_MERGE
   return from_cuda(e);
 }
 

@@ -13,14 +13,29 @@ namespace baatt {
 
 constexpr int kMergeThreads = 256;
 
+// VEC consecutive elements as floats, read with 16-byte loads.
+template <typename T, int VEC>
+__device__ __forceinline__ void load_vec(const T *p, float (&f)[VEC]) {
+  constexpr int PER = Elem<T>::kVec;                  // elements per 16-byte load
+  static_assert(VEC % PER == 0, "vector width");
+#pragma unroll
+  for (int k = 0; k < VEC / PER; ++k) {
+    float g[PER];
+    Elem<T>::unpack(*reinterpret_cast<const uint4 *>(p + k * PER), g);
+#pragma unroll
+    for (int e = 0; e < PER; ++e) f[k * PER + e] = g[e];
+  }
+}
+
 // One 16-byte vector of a row per thread; rows are independent. HBM-bound:
 // reads O1, O2, L1, L2 once and writes O, L once.
-template <typename T, int D>
-__global__ void __launch_bounds__(kMergeThreads) merge_lse_kernel(const T *O1,
-                                                                  const float *L1, const T *O2,
-                                                                  const float *L2, T *O, float *L,
+// Each thread handles VEC consecutive elements of one row, VEC = the number of
+// output elements in 16 bytes; inputs are read as one or two 16-byte vectors.
+template <typename TI, typename TO, int D>
+__global__ void __launch_bounds__(kMergeThreads) merge_lse_kernel(const TI *O1, const float *L1, const TI *O2,
+                                                                  const float *L2, TO *O, float *L,
                                                                   long long rows) {
-  constexpr int VEC = Elem<T>::kVec;
+  constexpr int VEC = Elem<TO>::kVec;
   constexpr int VPR = D / VEC;                         // vectors per row
   const long long total = rows * VPR;
   const int lane = threadIdx.x & 31;
@@ -43,11 +58,9 @@ __global__ void __launch_bounds__(kMergeThreads) merge_lse_kernel(const T *O1,
       const float w2 = empty ? 0.f : expf(l2 - m);
       const float den = w1 + w2;
       const float inv = empty ? 0.f : 1.f / den;
-      const uint4 a = *(reinterpret_cast<const uint4 *>(O1 + r * D) + c);
-      const uint4 bb = *(reinterpret_cast<const uint4 *>(O2 + r * D) + c);
       float fa[VEC], fb[VEC];
-      Elem<T>::unpack(a, fa);
-      Elem<T>::unpack(bb, fb);
+      load_vec<TI, VEC>(O1 + r * D + c * VEC, fa);
+      load_vec<TI, VEC>(O2 + r * D + c * VEC, fb);
 #pragma unroll
       for (int e = 0; e < VEC; ++e) out[e] = (w1 * fa[e] + w2 * fb[e]) * inv;
       lse = empty ? -INFINITY : m + logf(den);
@@ -72,16 +85,16 @@ __global__ void __launch_bounds__(kMergeThreads) merge_lse_kernel(const T *O1,
   }
 }
 
-template <typename T, int D>
-cudaError_t launch_merge(const T *O1, const float *L1, const T *O2, const float *L2, T *O, float *L, long long rows,
+template <typename TI, typename TO, int D>
+cudaError_t launch_merge(const TI *O1, const float *L1, const TI *O2, const float *L2, TO *O, float *L, long long rows,
                          int num_sms, cudaStream_t stream) {
-  constexpr int VPR = D / Elem<T>::kVec;
+  constexpr int VPR = D / Elem<TO>::kVec;
   const long long total = rows * VPR;
   long long blocks = (total + kMergeThreads - 1) / kMergeThreads;
   const long long cap = static_cast<long long>(num_sms) * 8;     // 8 resident CTAs per SM
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
-  merge_lse_kernel<T, D><<<static_cast<unsigned>(blocks), kMergeThreads, 0, stream>>>(O1, L1, O2, L2, O, L, rows);
+  merge_lse_kernel<TI, TO, D><<<static_cast<unsigned>(blocks), kMergeThreads, 0, stream>>>(O1, L1, O2, L2, O, L, rows);
   return cudaGetLastError();
 }
 

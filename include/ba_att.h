@@ -73,7 +73,7 @@ typedef struct {
   int32_t N_alloc;  /* rows allocated per head                 >= N          */
   int32_t d;        /* head dimension: 64 or 128                             */
   int32_t block;    /* block size b: a multiple of 16 in [16, 256]           */
-  int32_t dtype;    /* ba_dtype of Q, K, V and O                             */
+  int32_t dtype;    /* ba_dtype of Q, K and V (and of O unless stated)      */
   float sm_scale;   /* softmax scale s; <= 0 selects d^-1/2                  */
 } ba_att_shape;
 
@@ -93,8 +93,8 @@ int32_t ba_att_keep_count(const ba_att_shape *shape, float keep);
 
 /*
  * ba_att_stats — stage one, block-wise pre-downsample statistics
- * (BA-Att abstract: "block-wise pre-downsampled operation"; diagonal Q/K
- * variances from "Core claim").
+ * (BA-Att abstract: Q and K are pooled per block before any scoring;
+ * "Core claim": the correction uses per-dimension Q/K variances).
  *
  * For every block i and head h, over the valid rows r of the block:
  *   mean[i, m] = (1/n_i) sum_r x[r, m]
@@ -172,7 +172,9 @@ ba_status ba_att_split_lists(const ba_att_shape *shape, int32_t split_block,
  * Q, K, V   device, shape->dtype, layouts as above.
  * kv_idx, kv_cnt, kmax   device int32 lists as written by ba_att_select
  *           (any strictly ascending lists in [0, nk) are accepted).
- * O         device [B, Hq, N_alloc, d] of shape->dtype (written).
+ * O         device [B, Hq, N_alloc, d] of o_dtype (written).
+ * o_dtype   shape->dtype, or BA_DTYPE_F32 to keep a partial output in fp32
+ *           (one rounding in total when partials are merged later).
  * LSE       device fp32 [B, Hq, N_alloc], natural log (written).
  * Paths: bf16 with d = 128 and block = 128 runs the tcgen05/TMEM tensor-core
  * kernel; every other supported shape runs an fp32 CUDA-core kernel.
@@ -180,7 +182,7 @@ ba_status ba_att_split_lists(const ba_att_shape *shape, int32_t split_block,
 ba_status ba_att_sparse_fwd(const ba_att_shape *shape,
                             const void *Q, const void *K, const void *V,
                             const int32_t *kv_idx, const int32_t *kv_cnt, int32_t kmax,
-                            void *O, float *LSE, ba_stream_t stream);
+                            void *O, int32_t o_dtype, float *LSE, ba_stream_t stream);
 
 /*
  * ba_att_merge_lse — log-space merge of two partial attentions over disjoint
@@ -190,10 +192,13 @@ ba_status ba_att_sparse_fwd(const ba_att_shape *shape,
  * both L = -inf gives O = 0, L = -inf.
  *
  * rows      number of rows (e.g. B*Hq*N_alloc); d in {64, 128}.
- * O1, O2, O device [rows, d] of dtype; L1, L2, L device fp32 [rows].
- * O may alias O1 or O2 and L may alias L1 or L2 (in-place merge).
+ * O1, O2    device [rows, d] of in_dtype; O device [rows, d] of out_dtype;
+ *           L1, L2, L device fp32 [rows]. Math in fp32, one rounding to
+ *           out_dtype.
+ * When in_dtype == out_dtype, O may alias O1 or O2 and L may alias L1 or L2
+ * (in-place merge).
  */
-ba_status ba_att_merge_lse(int64_t rows, int32_t d, int32_t dtype,
+ba_status ba_att_merge_lse(int64_t rows, int32_t d, int32_t in_dtype, int32_t out_dtype,
                            const void *O1, const float *L1,
                            const void *O2, const float *L2,
                            void *O, float *L, ba_stream_t stream);

@@ -77,7 +77,7 @@ MIS = ctypes.c_void_p(0x10008)
 def test_bad_shapes_rejected(lib, bad, status):
     s = shape(**bad)
     assert lib.ba_att_stats(ctypes.byref(s), P, P, P, P, P, P, None) == status
-    assert lib.ba_att_sparse_fwd(ctypes.byref(s), P, P, P, P, P, 4, P, P, None) == status
+    assert lib.ba_att_sparse_fwd(ctypes.byref(s), P, P, P, P, P, 4, P, 1, P, None) == status
     assert lib.ba_att_select(ctypes.byref(s), ctypes.c_float(0.5), P, P, P, P, P, P, 8, None, None) == status
     assert lib.ba_att_num_blocks(ctypes.byref(s)) == -1
 
@@ -87,11 +87,11 @@ def test_null_and_misaligned_pointers(lib):
     assert lib.ba_att_stats(None, P, P, P, P, P, P, None) == 1
     assert lib.ba_att_stats(ctypes.byref(s), None, P, P, P, P, P, None) == 1
     assert lib.ba_att_stats(ctypes.byref(s), MIS, P, P, P, P, P, None) == 3
-    assert lib.ba_att_sparse_fwd(ctypes.byref(s), P, P, P, P, P, 4, None, P, None) == 1
-    assert lib.ba_att_sparse_fwd(ctypes.byref(s), P, P, MIS, P, P, 4, P, P, None) == 3
+    assert lib.ba_att_sparse_fwd(ctypes.byref(s), P, P, P, P, P, 4, None, 1, P, None) == 1
+    assert lib.ba_att_sparse_fwd(ctypes.byref(s), P, P, MIS, P, P, 4, P, 1, P, None) == 3
     assert lib.ba_att_select(ctypes.byref(s), ctypes.c_float(0.5), P, P, P, P, P, MIS, 8, None, None) == 3
-    assert lib.ba_att_merge_lse(10, 128, 1, P, P, None, P, P, P, None) == 1
-    assert lib.ba_att_merge_lse(10, 128, 1, MIS, P, P, P, P, P, None) == 3
+    assert lib.ba_att_merge_lse(10, 128, 1, 1, P, P, None, P, P, P, None) == 1
+    assert lib.ba_att_merge_lse(10, 128, 1, 1, MIS, P, P, P, P, P, None) == 3
 
 
 def test_selection_arguments(lib):
@@ -107,13 +107,19 @@ def test_selection_arguments(lib):
     # split point outside [0, nb]
     assert lib.ba_att_split_lists(ctypes.byref(s), 9, P, P, 8, P, P, P, P, None) == 1
     assert lib.ba_att_split_lists(ctypes.byref(s), -1, P, P, 8, P, P, P, P, None) == 1
-    assert lib.ba_att_sparse_fwd(ctypes.byref(s), P, P, P, P, P, 0, P, P, None) == 1
+    assert lib.ba_att_sparse_fwd(ctypes.byref(s), P, P, P, P, P, 0, P, 1, P, None) == 1
 
 
 def test_merge_and_selftest_arguments(lib):
-    assert lib.ba_att_merge_lse(10, 96, 1, P, P, P, P, P, P, None) == 2
-    assert lib.ba_att_merge_lse(10, 128, 5, P, P, P, P, P, P, None) == 1
-    assert lib.ba_att_merge_lse(-1, 128, 1, P, P, P, P, P, P, None) == 1
-    assert lib.ba_att_merge_lse(0, 128, 1, P, P, P, P, P, P, None) == 0     # nothing to do
+    assert lib.ba_att_merge_lse(10, 96, 1, 1, P, P, P, P, P, P, None) == 2
+    assert lib.ba_att_merge_lse(10, 128, 5, 5, P, P, P, P, P, P, None) == 1
+    assert lib.ba_att_merge_lse(-1, 128, 1, 1, P, P, P, P, P, P, None) == 1
+    assert lib.ba_att_merge_lse(0, 128, 1, 1, P, P, P, P, P, P, None) == 0     # nothing to do
+    # bf16 partials cannot widen to an fp32 output; unknown dtypes are rejected
+    assert lib.ba_att_merge_lse(10, 128, 1, 0, P, P, P, P, P, P, None) == 2
+    assert lib.ba_att_merge_lse(10, 128, 0, 3, P, P, P, P, P, P, None) == 1
+    # sparse_fwd output dtype must be the input dtype or fp32
+    s = shape()
+    assert lib.ba_att_sparse_fwd(ctypes.byref(s), P, P, P, P, P, 4, P, 2, P, None) == 1
     assert lib.ba_att_selftest_bounded_wait(0, None) == 1
     assert lib.ba_att_selftest_bounded_wait(3_000_000, None) == 1
