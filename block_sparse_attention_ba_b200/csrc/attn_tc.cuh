@@ -197,16 +197,24 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
       for (int q = 0; q < 4; ++q) tmem_ld32(tS + q * 32, sr[q]);
       tmem_ld_wait();
-      float mx = -INFINITY;
+      if (n_keys < kTileRows) {                        // ragged last block or a skipped entry (rare)
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < 4; ++q) {
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const float x = (q * 32 + c < n_keys) ? __uint_as_float(sr[q][c]) * scale_log2 : -INFINITY;
-          sr[q][c] = __float_as_uint(x);
-          mx = fmaxf(mx, x);
+          for (int c = 0; c < 32; ++c)
+            if (q * 32 + c >= n_keys) sr[q][c] = __float_as_uint(-INFINITY);
         }
       }
+      // Row max of the raw scores: 4 independent chains of 3-input max.
+      float mxp[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        mxp[q] = fmaxf(__uint_as_float(sr[q][0]), __uint_as_float(sr[q][31]));
+#pragma unroll
+        for (int c = 1; c < 31; c += 2)
+          mxp[q] = fmax3(mxp[q], __uint_as_float(sr[q][c]), __uint_as_float(sr[q][c + 1]));
+      }
+      const float mx = fmaxf(fmax3(mxp[0], mxp[1], mxp[2]), mxp[3]) * scale_log2;   // scale > 0 keeps the order
       float alpha = 1.f;
       bool rescale = false;
       if (mx - m_used > kRescaleLog2) {                // false when both are -inf
@@ -215,22 +223,28 @@ __global__ void __launch_bounds__(kThreads, 2)
         rescale = true;
       }
       const float m_ref = (m_used == -INFINITY) ? 0.f : m_used;
-      float sum0 = 0.f, sum1 = 0.f;
-      uint32_t pk[2][32];
+      // p = 2^(s*scale_log2 - m): one packed FMA per pair, 8 independent
+      // packed partial sums.
+      const float negm = -m_ref;
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int half = 0; half < 2; ++half) {         // 64 keys -> 32 packed columns, stored at once
+        uint32_t pk[32];
 #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          const float p0 = ex2_approx(__uint_as_float(sr[q][c]) - m_ref);
-          const float p1 = ex2_approx(__uint_as_float(sr[q][c + 1]) - m_ref);
-          sum0 += p0;
-          sum1 += p1;
-          pk[q >> 1][(q & 1) * 16 + (c >> 1)] = pack_bf16x2(p0, p1);
+        for (int qq = 0; qq < 2; ++qq) {
+          const int q = 2 * half + qq;
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            const float p0 = ex2_approx(fmaf(__uint_as_float(sr[q][c]), scale_log2, negm));
+            const float p1 = ex2_approx(fmaf(__uint_as_float(sr[q][c + 1]), scale_log2, negm));
+            acc[c & 7] += p0;
+            acc[(c & 7) + 1] += p1;
+            pk[qq * 16 + (c >> 1)] = pack_bf16x2(p0, p1);
+          }
         }
+        tmem_st32(tS + half * 32, pk);
       }
-      l = l * alpha + (sum0 + sum1);
-      tmem_st32(tS + 0, pk[0]);
-      tmem_st32(tS + 32, pk[1]);
+      l = l * alpha + (((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7])));
       if (t > 0 && __any_sync(0xFFFFFFFFu, rescale)) {
         // O holds blocks 0..t-1 (their MMAs completed before S_t did)
 #pragma unroll
