@@ -59,6 +59,34 @@ __device__ __forceinline__ bool entry_ok(const int32_t *list, int t, int nb, int
   return true;
 }
 
+// P = 2^(s*scale_log2 - m) for one row: packed to bf16 pairs and stored
+// over the S columns 64 keys at a time; the fp32 values are summed into 8
+// independent partial sums. (Evaluating a share of the exponentials on the
+// FMA pipe instead of MUFU was measured slower here: issue slots, not MUFU
+// throughput, bound this loop.)
+__device__ __forceinline__ void exp_pack_store(const uint32_t (&sr)[4][32], float scale_log2, float negm,
+                                               float (&acc)[8], uint32_t tS) {
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    uint32_t pk[32];
+#pragma unroll
+    for (int qq = 0; qq < 2; ++qq) {
+      const int q = 2 * half + qq;
+#pragma unroll
+      for (int c = 0; c < 32; c += 2) {
+        const float x0 = fmaf(__uint_as_float(sr[q][c]), scale_log2, negm);
+        const float x1 = fmaf(__uint_as_float(sr[q][c + 1]), scale_log2, negm);
+        const float p0 = ex2_approx(x0);
+        const float p1 = ex2_approx(x1);
+        acc[c & 7] += p0;
+        acc[(c & 7) + 1] += p1;
+        pk[qq * 16 + (c >> 1)] = pack_bf16x2(p0, p1);
+      }
+    }
+    tmem_st32(tS + half * 32, pk);
+  }
+}
+
 // TO: output element type, bf16 (final output) or float (a partial that is
 // merged later, so the merged result is rounded only once).
 template <typename TO>
@@ -227,23 +255,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       // packed partial sums.
       const float negm = -m_ref;
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {         // 64 keys -> 32 packed columns, stored at once
-        uint32_t pk[32];
-#pragma unroll
-        for (int qq = 0; qq < 2; ++qq) {
-          const int q = 2 * half + qq;
-#pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            const float p0 = ex2_approx(fmaf(__uint_as_float(sr[q][c]), scale_log2, negm));
-            const float p1 = ex2_approx(fmaf(__uint_as_float(sr[q][c + 1]), scale_log2, negm));
-            acc[c & 7] += p0;
-            acc[(c & 7) + 1] += p1;
-            pk[qq * 16 + (c >> 1)] = pack_bf16x2(p0, p1);
-          }
-        }
-        tmem_st32(tS + half * 32, pk);
-      }
+      exp_pack_store(sr, scale_log2, negm, acc, tS);
       l = l * alpha + (((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7])));
       if (t > 0 && __any_sync(0xFFFFFFFFu, rescale)) {
         // O holds blocks 0..t-1 (their MMAs completed before S_t did)
