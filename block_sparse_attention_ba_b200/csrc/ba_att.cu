@@ -153,21 +153,22 @@ ba_status ba_att_stats(const ba_att_shape *s, const void *Q, const void *K, floa
       !aligned16(k_var))
     return BA_ERR_MISALIGNED;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  const int sms = num_sms_of_current_device();
   cudaError_t e;
   if (s->dtype == BA_DTYPE_BF16) {
     auto q = static_cast<const __nv_bfloat16 *>(Q);
     auto k = static_cast<const __nv_bfloat16 *>(K);
     e = s->d == 128 ? launch_stats<__nv_bfloat16, 128>(q, k, q_mean, q_var, k_mean, k_var, s->B, s->Hq, s->Hkv, s->N,
-                                                       s->N_alloc, s->block, cs)
+                                                       s->N_alloc, s->block, sms, cs)
                     : launch_stats<__nv_bfloat16, 64>(q, k, q_mean, q_var, k_mean, k_var, s->B, s->Hq, s->Hkv, s->N,
-                                                      s->N_alloc, s->block, cs);
+                                                      s->N_alloc, s->block, sms, cs);
   } else {
     auto q = static_cast<const float *>(Q);
     auto k = static_cast<const float *>(K);
     e = s->d == 128 ? launch_stats<float, 128>(q, k, q_mean, q_var, k_mean, k_var, s->B, s->Hq, s->Hkv, s->N,
-                                               s->N_alloc, s->block, cs)
+                                               s->N_alloc, s->block, sms, cs)
                     : launch_stats<float, 64>(q, k, q_mean, q_var, k_mean, k_var, s->B, s->Hq, s->Hkv, s->N,
-                                              s->N_alloc, s->block, cs);
+                                              s->N_alloc, s->block, sms, cs);
   }
   return from_cuda(e);
 }

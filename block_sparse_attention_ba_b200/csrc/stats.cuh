@@ -114,6 +114,159 @@ __global__ void __launch_bounds__(kStatsThreads) stats_kernel(const T *__restric
   }
 }
 
+// Streaming variant for blocks of at most 32 KB (every bf16 d=128 shape up to
+// block 128): a persistent CTA walks the (head, block) items with a stride of
+// the grid size; each item is one contiguous slab of rows, fetched with a
+// single bulk copy (cp.async.bulk) into a 3-stage shared-memory ring, so two
+// slabs per CTA are in flight while the current one is reduced. The reduction
+// is the same exact two-pass mean/variance as above, read from shared memory.
+constexpr int kStatsStages = 3;
+constexpr uint32_t kStatsStageBytes = 32768;
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kStatsThreads, 2)
+    stats_bulk_kernel(const T *__restrict__ Q, const T *__restrict__ K, float *__restrict__ q_mean,
+                      float *__restrict__ q_var, float *__restrict__ k_mean, float *__restrict__ k_var, int B,
+                      int Hq, int Hkv, int N, int N_alloc, int block, int nb) {
+  constexpr int VEC = Elem<T>::kVec;
+  constexpr int COLS = D / VEC;
+  constexpr int RPP = kStatsThreads / COLS;
+  constexpr int RPT = static_cast<int>(kStatsStageBytes / (D * sizeof(T))) / RPP;   // = 8
+  extern __shared__ __align__(128) uint8_t stage_mem[];
+  __shared__ float red[RPP][D];
+  __shared__ float mean_s[D];
+  __shared__ uint64_t full[kStatsStages];
+  __shared__ int abort_flag;
+
+  const long long n_q = static_cast<long long>(B) * Hq * nb;
+  const long long total = n_q + static_cast<long long>(B) * Hkv * nb;
+  const int tid = threadIdx.x, col = tid % COLS, rsub = tid / COLS;
+  const uint32_t ring = smem_u32(stage_mem);
+
+  // item w -> source slab, valid rows, output row offset, Q-or-K
+  auto locate = [&](long long w, const T *&src, int &n_rows, long long &orow, bool &is_q) {
+    is_q = w < n_q;
+    const long long c = is_q ? w : w - n_q;
+    const int blk = static_cast<int>(c % nb);
+    const long long bh = c / nb;
+    src = (is_q ? Q : K) + (bh * N_alloc + static_cast<long long>(blk) * block) * D;
+    n_rows = min(block, N - blk * block);
+    orow = (bh * nb + blk) * static_cast<long long>(D);
+  };
+  auto issue = [&](long long w, int s) {
+    const T *src;
+    int n_rows;
+    long long orow;
+    bool is_q;
+    locate(w, src, n_rows, orow, is_q);
+    const uint32_t bytes = static_cast<uint32_t>(n_rows) * D * sizeof(T);
+    mbar_arrive_expect_tx(smem_u32(&full[s]), bytes);
+    bulk_load(ring + s * kStatsStageBytes, src, bytes, smem_u32(&full[s]));
+  };
+
+  long long last_issued = -1;             // thread 0: newest item handed to the copy engine
+  if (tid == 0) {
+    for (int s = 0; s < kStatsStages; ++s) mbar_init(smem_u32(&full[s]), 1);
+    abort_flag = 0;
+    fence_mbar_init();
+    for (int s = 0; s < kStatsStages - 1; ++s) {
+      const long long w = blockIdx.x + static_cast<long long>(s) * gridDim.x;
+      if (w < total) {
+        issue(w, s);
+        last_issued = w;
+      }
+    }
+  }
+  __syncthreads();
+
+  int it = 0;
+  for (long long w = blockIdx.x; w < total; w += gridDim.x, ++it) {
+    const int s = it % kStatsStages;
+    if (tid == 0) {
+      const long long wn = w + static_cast<long long>(kStatsStages - 1) * gridDim.x;
+      if (wn < total) {
+        fence_proxy_async_smem();             // earlier reads of that stage before the bulk write
+        issue(wn, (it + kStatsStages - 1) % kStatsStages);
+        last_issued = wn;
+      }
+    }
+    const T *src;
+    int n_rows;
+    long long orow;
+    bool is_q;
+    locate(w, src, n_rows, orow, is_q);
+    const bool ok = mbar_wait_bounded(smem_u32(&full[s]), (it / kStatsStages) & 1, &abort_flag);
+    if (__syncthreads_or(!ok)) break;
+
+    const T *slab = reinterpret_cast<const T *>(stage_mem + s * kStatsStageBytes);
+    uint4 v[RPT];
+#pragma unroll
+    for (int k = 0; k < RPT; ++k) {
+      const int r = rsub + k * RPP;
+      v[k] = r < n_rows ? *reinterpret_cast<const uint4 *>(slab + r * D + col * VEC) : make_uint4(0, 0, 0, 0);
+    }
+    float acc[VEC];
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
+#pragma unroll
+    for (int k = 0; k < RPT; ++k) {
+      float f[VEC];
+      Elem<T>::unpack(v[k], f);
+#pragma unroll
+      for (int e = 0; e < VEC; ++e) acc[e] += f[e];
+    }
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) red[rsub][col * VEC + e] = acc[e];
+    __syncthreads();
+    const float inv_n = 1.f / static_cast<float>(n_rows);
+    if (tid < D) {
+      float sum = 0.f;
+#pragma unroll 8
+      for (int r = 0; r < RPP; ++r) sum += red[r][tid];
+      mean_s[tid] = sum * inv_n;
+    }
+    __syncthreads();
+    float mu[VEC];
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) {
+      mu[e] = mean_s[col * VEC + e];
+      acc[e] = 0.f;
+    }
+#pragma unroll
+    for (int k = 0; k < RPT; ++k) {
+      if (rsub + k * RPP < n_rows) {
+        float f[VEC];
+        Elem<T>::unpack(v[k], f);
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) {
+          const float dv = f[e] - mu[e];
+          acc[e] = fmaf(dv, dv, acc[e]);
+        }
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) red[rsub][col * VEC + e] = acc[e];
+    __syncthreads();
+    if (tid < D) {
+      float sum = 0.f;
+#pragma unroll 8
+      for (int r = 0; r < RPP; ++r) sum += red[r][tid];
+      (is_q ? q_mean : k_mean)[orow + tid] = mean_s[tid];
+      (is_q ? q_var : k_var)[orow + tid] = sum * inv_n;
+    }
+    __syncthreads();
+  }
+  // after an abandoned wait, let every issued copy land before exiting
+  // (the newest kStatsStages items issued, each in its own stage)
+  if (tid == 0 && abort_flag) {
+    for (long long w = last_issued; w >= blockIdx.x && w > last_issued - kStatsStages * static_cast<long long>(gridDim.x);
+         w -= gridDim.x) {
+      const long long idx = (w - blockIdx.x) / gridDim.x;
+      mbar_wait_bounded(smem_u32(&full[idx % kStatsStages]), (idx / kStatsStages) & 1, nullptr);
+    }
+  }
+}
+
 // Rows each thread holds for a given block size (power-of-two bucket).
 template <typename T, int D>
 inline int stats_rpt_needed(int block) {
@@ -123,9 +276,20 @@ inline int stats_rpt_needed(int block) {
 
 template <typename T, int D>
 cudaError_t launch_stats(const T *Q, const T *K, float *qm, float *qv, float *km, float *kv, int B, int Hq, int Hkv,
-                         int N, int N_alloc, int block, cudaStream_t stream) {
+                         int N, int N_alloc, int block, int num_sms, cudaStream_t stream) {
   const int nb = (N + block - 1) / block;
   const long long grid = static_cast<long long>(B) * (Hq + Hkv) * nb;
+  if (static_cast<size_t>(block) * D * sizeof(T) <= kStatsStageBytes) {
+    const size_t smem = static_cast<size_t>(kStatsStages) * kStatsStageBytes;
+    cudaError_t e = cudaFuncSetAttribute(stats_bulk_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    const long long persistent = static_cast<long long>(num_sms) * 2;
+    const unsigned g = static_cast<unsigned>(grid < persistent ? grid : persistent);
+    stats_bulk_kernel<T, D><<<g, kStatsThreads, smem, stream>>>(Q, K, qm, qv, km, kv, B, Hq, Hkv, N, N_alloc, block,
+                                                                 nb);
+    return cudaGetLastError();
+  }
   const int need = stats_rpt_needed<T, D>(block);
   dim3 g(static_cast<unsigned>(grid));
   if (need <= 2) {
