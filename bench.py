@@ -216,7 +216,8 @@ def run_ours(args):
                  torch.empty((w.B, w.Hkv, nb, w.d), device=dev), torch.empty((w.B, w.Hkv, nb, w.d), device=dev))
     idx = torch.empty((w.B, w.Hq, nb, k), device=dev, dtype=torch.int32)
     cnt = torch.empty((w.B, w.Hq, nb), device=dev, dtype=torch.int32)
-    lists = (torch.empty_like(idx), torch.empty_like(cnt), torch.empty_like(idx), torch.empty_like(cnt))
+    scores = torch.empty((w.B, w.Hq, nb, nb), device=dev, dtype=torch.float32)     # the block-score map
+    lists =(torch.empty_like(idx), torch.empty_like(cnt), torch.empty_like(idx), torch.empty_like(cnt))
     # span partials stay in fp32 so the merged output is rounded to bf16 once
     O1 = torch.empty(Qd.shape, device=dev, dtype=torch.float32)
     O2 = torch.empty(Qd.shape, device=dev, dtype=torch.float32)
@@ -233,7 +234,7 @@ def run_ours(args):
         mark(0)
         api.stats(Qd, Kd, shape, out=stats_buf)
         mark(1)
-        api.select(stats_buf, shape, keep, out=(idx, cnt, None))
+        api.select(stats_buf, shape, keep, out=(idx, cnt, scores))
         mark(2)
         api.split_lists(idx, cnt, shape, split_block, out=lists)
         mark(3)
@@ -375,7 +376,7 @@ def run_dense(ctx, steps=3):
     shape, dev = ctx["shape"], ctx["dev"]
     w = ctx["w"]
     st = api.stats(ctx["Qd"], ctx["Kd"], shape)
-    idx, cnt = api.select(st, shape, 1.0)
+    idx, cnt, sc1 = api.select(st, shape, 1.0, with_scores=True)
     O, L = api.sparse_fwd(ctx["Qd"], ctx["Kd"], ctx["Vd"], idx, cnt, shape)
     torch.cuda.synchronize()
     a, b, c = (torch.cuda.Event(enable_timing=True) for _ in range(3))
@@ -383,7 +384,7 @@ def run_dense(ctx, steps=3):
     a.record(stream)
     for _ in range(steps):
         api.stats(ctx["Qd"], ctx["Kd"], shape, out=st)
-        api.select(st, shape, 1.0, out=(idx, cnt, None))
+        api.select(st, shape, 1.0, out=(idx, cnt, sc1))
     b.record(stream)
     for _ in range(steps):
         api.sparse_fwd(ctx["Qd"], ctx["Kd"], ctx["Vd"], idx, cnt, shape, out=(O, L))

@@ -38,9 +38,9 @@ _SIGS = {
     "ba_att_version": (ctypes.c_char_p, []),
     "ba_att_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "ba_att_num_blocks": (_I32, [ctypes.POINTER(CShape)]),
-    "ba_att_keep_count": (_I32, [ctypes.POINTER(CShape), ctypes.c_float]),
+    "ba_att_keep_count": (_I32, [ctypes.POINTER(CShape), ctypes.c_double]),
     "ba_att_stats": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _P, _P, _P, _P, _P]),
-    "ba_att_select": (ctypes.c_int, [ctypes.POINTER(CShape), ctypes.c_float, _P, _P, _P, _P, _P, _P, _I32, _P, _P]),
+    "ba_att_select": (ctypes.c_int, [ctypes.POINTER(CShape), ctypes.c_double, _P, _P, _P, _P, _P, _P, _I32, _P, _P]),
     "ba_att_split_lists": (ctypes.c_int, [ctypes.POINTER(CShape), _I32, _P, _P, _I32, _P, _P, _P, _P, _P]),
     "ba_att_sparse_fwd": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _P, _P, _P, _I32, _P, _I32, _P, _P]),
     "ba_att_merge_lse": (ctypes.c_int, [ctypes.c_int64, _I32, _I32, _I32, _P, _P, _P, _P, _P, _P, _P]),
@@ -136,7 +136,7 @@ def num_blocks(shape: Shape) -> int:
 
 
 def keep_count(shape: Shape, keep: float) -> int:
-    return int(load_library().ba_att_keep_count(ctypes.byref(shape.c()), ctypes.c_float(keep)))
+    return int(load_library().ba_att_keep_count(ctypes.byref(shape.c()), ctypes.c_double(keep)))
 
 
 def stats(Q: torch.Tensor, K: torch.Tensor, shape: Shape, out=None):
@@ -155,7 +155,10 @@ def stats(Q: torch.Tensor, K: torch.Tensor, shape: Shape, out=None):
 
 
 def select(stats_out, shape: Shape, keep: float, kmax: int | None = None, with_scores: bool = False, out=None):
-    """Corrected block scores + top-k; returns (idx, cnt) or (idx, cnt, scores)."""
+    """Corrected block scores + top-k -> (idx, cnt), or (idx, cnt, scores) with with_scores.
+
+    The score map [B, Hq, nq, nk] fp32 is always written; out = (idx, cnt, scores) may pass
+    a preallocated one."""
     lib = load_library()
     qm, qv, km, kv = stats_out
     k = keep_count(shape, keep)
@@ -166,15 +169,16 @@ def select(stats_out, shape: Shape, keep: float, kmax: int | None = None, with_s
     if out is None:
         idx = torch.empty((shape.B, shape.Hq, shape.nb, kmax), device=dev, dtype=torch.int32)
         cnt = torch.empty((shape.B, shape.Hq, shape.nb), device=dev, dtype=torch.int32)
-        sc = torch.empty((shape.B, shape.Hq, shape.nb, shape.nb), device=dev, dtype=torch.float32) \
-            if with_scores else None
+        sc = None
     else:
         idx, cnt, sc = out
+    if sc is None:       # the score map is always written (the selection reads it back)
+        sc = torch.empty((shape.B, shape.Hq, shape.nb, shape.nb), device=dev, dtype=torch.float32)
     _check("ba_att_select", lib.ba_att_select(
-        ctypes.byref(shape.c()), ctypes.c_float(keep), _dev(qm, "q_mean"), _dev(qv, "q_var"), _dev(km, "k_mean"),
+        ctypes.byref(shape.c()), ctypes.c_double(keep), _dev(qm, "q_mean"), _dev(qv, "q_var"), _dev(km, "k_mean"),
         _dev(kv, "k_var"), _dev(idx, "kv_idx"), _dev(cnt, "kv_cnt"), idx.shape[-1],
-        _dev(sc, "block_scores") if sc is not None else None, _stream(qm)))
-    return (idx, cnt, sc) if sc is not None else (idx, cnt)
+        _dev(sc, "block_scores"), _stream(qm)))
+    return (idx, cnt, sc) if with_scores else (idx, cnt)
 
 
 def split_lists(idx: torch.Tensor, cnt: torch.Tensor, shape: Shape, split_block: int, out=None):

@@ -16,6 +16,7 @@
 #include "common.cuh"
 #include "stats.cuh"
 #include "select.cuh"
+#include "select_tc.cuh"
 #include "merge.cuh"
 #include "attn_simt.cuh"
 #include "attn_tc.cuh"
@@ -133,7 +134,7 @@ int32_t ba_att_num_blocks(const ba_att_shape *shape) {
   return nblocks(shape);
 }
 
-int32_t ba_att_keep_count(const ba_att_shape *shape, float keep) {
+int32_t ba_att_keep_count(const ba_att_shape *shape, double keep) {
   if (check_shape(shape) != BA_OK) return -1;
   if (!(keep > 0.f && keep <= 1.f)) return -1;
   const int nk = nblocks(shape);
@@ -173,14 +174,14 @@ ba_status ba_att_stats(const ba_att_shape *s, const void *Q, const void *K, floa
   return from_cuda(e);
 }
 
-ba_status ba_att_select(const ba_att_shape *s, float keep, const float *q_mean, const float *q_var,
+ba_status ba_att_select(const ba_att_shape *s, double keep, const float *q_mean, const float *q_var,
                         const float *k_mean, const float *k_var, int32_t *kv_idx, int32_t *kv_cnt, int32_t kmax,
                         float *block_scores, ba_stream_t stream) {
   ba_status st = check_shape(s);
   if (st != BA_OK) return st;
-  if (!q_mean || !q_var || !k_mean || !k_var || !kv_idx || !kv_cnt) return BA_ERR_INVALID_ARG;
+  if (!q_mean || !q_var || !k_mean || !k_var || !kv_idx || !kv_cnt || !block_scores) return BA_ERR_INVALID_ARG;
   if (!aligned16(q_mean) || !aligned16(q_var) || !aligned16(k_mean) || !aligned16(k_var) || !aligned16(kv_idx) ||
-      !aligned16(kv_cnt) || (block_scores && !aligned16(block_scores)))
+      !aligned16(kv_cnt) || !aligned16(block_scores))
     return BA_ERR_MISALIGNED;
   const int k = ba_att_keep_count(s, keep);
   if (k < 1) return BA_ERR_INVALID_ARG;
@@ -189,10 +190,18 @@ ba_status ba_att_select(const ba_att_shape *s, float keep, const float *q_mean, 
   if (nb > 4096) return BA_ERR_UNSUPPORTED;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   const float scale = effective_scale(s);
-  cudaError_t e = s->d == 128 ? launch_select<128>(q_mean, q_var, k_mean, k_var, kv_idx, kv_cnt, block_scores, s->B,
-                                                   s->Hq, s->Hkv, s->N, s->block, k, kmax, scale, cs)
-                              : launch_select<64>(q_mean, q_var, k_mean, k_var, kv_idx, kv_cnt, block_scores, s->B,
-                                                  s->Hq, s->Hkv, s->N, s->block, k, kmax, scale, cs);
+  cudaError_t e;
+  if (nb <= seltc::kMaxKeys) {    // the whole score row fits the TMEM columns: tensor-core path
+    e = s->d == 128 ? launch_select_tc<128>(q_mean, q_var, k_mean, k_var, kv_idx, kv_cnt, block_scores, s->B, s->Hq,
+                                            s->Hkv, s->N, s->block, k, kmax, scale, cs)
+                    : launch_select_tc<64>(q_mean, q_var, k_mean, k_var, kv_idx, kv_cnt, block_scores, s->B, s->Hq,
+                                           s->Hkv, s->N, s->block, k, kmax, scale, cs);
+  } else {
+    e = s->d == 128 ? launch_select<128>(q_mean, q_var, k_mean, k_var, kv_idx, kv_cnt, block_scores, s->B, s->Hq,
+                                         s->Hkv, s->N, s->block, k, kmax, scale, cs)
+                    : launch_select<64>(q_mean, q_var, k_mean, k_var, kv_idx, kv_cnt, block_scores, s->B, s->Hq,
+                                        s->Hkv, s->N, s->block, k, kmax, scale, cs);
+  }
   return from_cuda(e);
 }
 

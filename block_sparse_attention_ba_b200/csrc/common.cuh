@@ -10,7 +10,7 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
-#include "../../include/ba_att.h"
+#include "ba_att.h"   // found through -I include
 
 namespace baatt {
 
@@ -108,6 +108,12 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
       : "memory");
+}
+
+// Fire-and-forget add on a shared-memory word given by its shared-window
+// address (a shared-state atomic even when the C++ pointer was generic).
+__device__ __forceinline__ void red_shared_add(uint32_t saddr, uint32_t v) {
+  asm volatile("red.shared.add.u32 [%0], %1;" ::"r"(saddr), "r"(v) : "memory");
 }
 
 // Orders this thread's earlier generic-proxy shared-memory accesses before

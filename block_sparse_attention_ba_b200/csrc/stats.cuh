@@ -117,8 +117,9 @@ __global__ void __launch_bounds__(kStatsThreads) stats_kernel(const T *__restric
 // Streaming variant for blocks of at most 32 KB (every bf16 d=128 shape up to
 // block 128): a persistent CTA walks the (head, block) items with a stride of
 // the grid size; each item is one contiguous slab of rows, fetched with a
-// single bulk copy (cp.async.bulk) into a 3-stage shared-memory ring, so two
-// slabs per CTA are in flight while the current one is reduced. The reduction
+// single bulk copy (cp.async.bulk) into a 3-stage shared-memory ring. A stage
+// is refilled as soon as its rows sit in registers, so three slabs per CTA
+// are in flight while the current one is reduced. The reduction
 // is the same exact two-pass mean/variance as above, read from shared memory.
 constexpr int kStatsStages = 3;
 constexpr uint32_t kStatsStageBytes = 32768;
@@ -169,7 +170,7 @@ __global__ void __launch_bounds__(kStatsThreads, 2)
     for (int s = 0; s < kStatsStages; ++s) mbar_init(smem_u32(&full[s]), 1);
     abort_flag = 0;
     fence_mbar_init();
-    for (int s = 0; s < kStatsStages - 1; ++s) {
+    for (int s = 0; s < kStatsStages; ++s) {
       const long long w = blockIdx.x + static_cast<long long>(s) * gridDim.x;
       if (w < total) {
         issue(w, s);
@@ -182,14 +183,6 @@ __global__ void __launch_bounds__(kStatsThreads, 2)
   int it = 0;
   for (long long w = blockIdx.x; w < total; w += gridDim.x, ++it) {
     const int s = it % kStatsStages;
-    if (tid == 0) {
-      const long long wn = w + static_cast<long long>(kStatsStages - 1) * gridDim.x;
-      if (wn < total) {
-        fence_proxy_async_smem();             // earlier reads of that stage before the bulk write
-        issue(wn, (it + kStatsStages - 1) % kStatsStages);
-        last_issued = wn;
-      }
-    }
     const T *src;
     int n_rows;
     long long orow;
@@ -218,6 +211,16 @@ __global__ void __launch_bounds__(kStatsThreads, 2)
 #pragma unroll
     for (int e = 0; e < VEC; ++e) red[rsub][col * VEC + e] = acc[e];
     __syncthreads();
+    // every thread holds its rows in registers now: hand stage s straight
+    // back to the copy engine for the item kStatsStages ahead
+    if (tid == 0) {
+      const long long wn = w + static_cast<long long>(kStatsStages) * gridDim.x;
+      if (wn < total) {
+        fence_proxy_async_smem();             // the reads above before the bulk write
+        issue(wn, s);
+        last_issued = wn;
+      }
+    }
     const float inv_n = 1.f / static_cast<float>(n_rows);
     if (tid < D) {
       float sum = 0.f;

@@ -89,7 +89,7 @@ int32_t ba_att_num_blocks(const ba_att_shape *shape);
 /* Kept blocks per query block: max(1, ceil(keep * nk)) (the selector keeps
  * the top fraction of key blocks; "Core claim"). -1 if keep is outside (0,1]
  * or the shape is invalid. */
-int32_t ba_att_keep_count(const ba_att_shape *shape, float keep);
+int32_t ba_att_keep_count(const ba_att_shape *shape, double keep);
 
 /*
  * ba_att_stats — stage one, block-wise pre-downsample statistics
@@ -133,7 +133,7 @@ ba_status ba_att_stats(const ba_att_shape *shape, const void *Q, const void *K,
  *                 also written there.
  * Requires nk <= 4096.
  */
-ba_status ba_att_select(const ba_att_shape *shape, float keep,
+ba_status ba_att_select(const ba_att_shape *shape, double keep,
                         const float *q_mean, const float *q_var,
                         const float *k_mean, const float *k_var,
                         int32_t *kv_idx, int32_t *kv_cnt, int32_t kmax,

@@ -56,14 +56,14 @@ def shape(**kw):
 def test_num_blocks_and_keep_count(lib):
     s = shape()
     assert lib.ba_att_num_blocks(ctypes.byref(s)) == 8
-    assert lib.ba_att_keep_count(ctypes.byref(s), ctypes.c_float(0.5)) == 4
-    assert lib.ba_att_keep_count(ctypes.byref(s), ctypes.c_float(1.0)) == 8
-    assert lib.ba_att_keep_count(ctypes.byref(s), ctypes.c_float(1e-4)) == 1
-    assert lib.ba_att_keep_count(ctypes.byref(s), ctypes.c_float(0.0)) == -1
-    assert lib.ba_att_keep_count(ctypes.byref(s), ctypes.c_float(1.5)) == -1
+    assert lib.ba_att_keep_count(ctypes.byref(s), ctypes.c_double(0.5)) == 4
+    assert lib.ba_att_keep_count(ctypes.byref(s), ctypes.c_double(1.0)) == 8
+    assert lib.ba_att_keep_count(ctypes.byref(s), ctypes.c_double(1e-4)) == 1
+    assert lib.ba_att_keep_count(ctypes.byref(s), ctypes.c_double(0.0)) == -1
+    assert lib.ba_att_keep_count(ctypes.byref(s), ctypes.c_double(1.5)) == -1
     for n, keep, k in ((256, 0.5, 128), (256, 0.25, 64), (1024, 0.5, 512), (16, 0.5, 8)):
         s = shape(N=n * 128, N_alloc=n * 128)
-        assert lib.ba_att_keep_count(ctypes.byref(s), ctypes.c_float(keep)) == k
+        assert lib.ba_att_keep_count(ctypes.byref(s), ctypes.c_double(keep)) == k
 
 
 P = ctypes.c_void_p(0x10000)       # aligned, never dereferenced: every call below fails validation
@@ -78,7 +78,7 @@ def test_bad_shapes_rejected(lib, bad, status):
     s = shape(**bad)
     assert lib.ba_att_stats(ctypes.byref(s), P, P, P, P, P, P, None) == status
     assert lib.ba_att_sparse_fwd(ctypes.byref(s), P, P, P, P, P, 4, P, 1, P, None) == status
-    assert lib.ba_att_select(ctypes.byref(s), ctypes.c_float(0.5), P, P, P, P, P, P, 8, None, None) == status
+    assert lib.ba_att_select(ctypes.byref(s), ctypes.c_double(0.5), P, P, P, P, P, P, 8, None, None) == status
     assert lib.ba_att_num_blocks(ctypes.byref(s)) == -1
 
 
@@ -89,7 +89,8 @@ def test_null_and_misaligned_pointers(lib):
     assert lib.ba_att_stats(ctypes.byref(s), MIS, P, P, P, P, P, None) == 3
     assert lib.ba_att_sparse_fwd(ctypes.byref(s), P, P, P, P, P, 4, None, 1, P, None) == 1
     assert lib.ba_att_sparse_fwd(ctypes.byref(s), P, P, MIS, P, P, 4, P, 1, P, None) == 3
-    assert lib.ba_att_select(ctypes.byref(s), ctypes.c_float(0.5), P, P, P, P, P, MIS, 8, None, None) == 3
+    assert lib.ba_att_select(ctypes.byref(s), ctypes.c_double(0.5), P, P, P, P, P, MIS, 8, P, None) == 3
+    assert lib.ba_att_select(ctypes.byref(s), ctypes.c_double(0.5), P, P, P, P, P, P, 8, None, None) == 1
     assert lib.ba_att_merge_lse(10, 128, 1, 1, P, P, None, P, P, P, None) == 1
     assert lib.ba_att_merge_lse(10, 128, 1, 1, MIS, P, P, P, P, P, None) == 3
 
@@ -97,13 +98,13 @@ def test_null_and_misaligned_pointers(lib):
 def test_selection_arguments(lib):
     s = shape()
     # keep outside (0, 1]
-    assert lib.ba_att_select(ctypes.byref(s), ctypes.c_float(0.0), P, P, P, P, P, P, 8, None, None) == 1
-    assert lib.ba_att_select(ctypes.byref(s), ctypes.c_float(1.01), P, P, P, P, P, P, 8, None, None) == 1
+    assert lib.ba_att_select(ctypes.byref(s), ctypes.c_double(0.0), P, P, P, P, P, P, 8, None, None) == 1
+    assert lib.ba_att_select(ctypes.byref(s), ctypes.c_double(1.01), P, P, P, P, P, P, 8, None, None) == 1
     # kmax below the kept count (keep 0.5 of 8 blocks = 4)
-    assert lib.ba_att_select(ctypes.byref(s), ctypes.c_float(0.5), P, P, P, P, P, P, 3, None, None) == 1
+    assert lib.ba_att_select(ctypes.byref(s), ctypes.c_double(0.5), P, P, P, P, P, P, 3, None, None) == 1
     # too many blocks for the in-shared-memory selector
     big = shape(N=4097 * 16, N_alloc=4097 * 16, block=16)
-    assert lib.ba_att_select(ctypes.byref(big), ctypes.c_float(0.5), P, P, P, P, P, P, 4097, None, None) == 2
+    assert lib.ba_att_select(ctypes.byref(big), ctypes.c_double(0.5), P, P, P, P, P, P, 4097, P, None) == 2
     # split point outside [0, nb]
     assert lib.ba_att_split_lists(ctypes.byref(s), 9, P, P, 8, P, P, P, P, None) == 1
     assert lib.ba_att_split_lists(ctypes.byref(s), -1, P, P, 8, P, P, P, P, None) == 1

@@ -116,6 +116,9 @@ SMALL = [
     ("video_32k", dict(N=600, N_alloc=640, Hq=2, Hkv=2, grid=(3, 10, 20)), 0.5),
     ("dlm_16k", dict(N=1024, Hq=2, Hkv=1, d=64, block=64), 0.5),      # bf16 on the CUDA-core path
     ("tiny_fp32", dict(N=768, d=128, block=32), 0.3),                 # fp32 d=128, block 32
+    ("tiny_fp32", dict(N=9600 - 7, N_alloc=9600, block=16, Hq=2, Hkv=1), 0.5),   # 600 blocks: CUDA-core selector
+    ("dlm_16k", dict(N=64 * 128, Hq=2, Hkv=1), 0.5),                 # 512 blocks: widest tensor-core selector
+    ("dlm_16k", dict(N=300 * 128 - 5, Hq=2, Hkv=2), 0.3),             # 300 blocks: two score tiles, ragged
 ]
 
 
