@@ -57,6 +57,22 @@ def dist_env():
         int(os.environ.get("LOCAL_RANK", "0"))
 
 
+def max_over_ranks(x: float, device=None) -> float:
+    """The slowest rank's value (all ranks call it; identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(world: int, flops_per_rank_step: float, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank processes its own replica of the step."""
+    return world * flops_per_rank_step / (ms_per_step * 1e-3) / 1e12
+
+
 def kept_flops(cnt_total: int, block: int, d: int) -> float:
     """Two GEMMs (Q K^T and P V) per kept (query block, key block) pair."""
     return 4.0 * block * block * d * cnt_total
@@ -277,12 +293,9 @@ def run_ours(args):
     if st != 0:
         raise RuntimeError(f"device error word {word:#x} during timing")
 
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, dev)
     ms_per_step = elapsed_ms / args.steps
-    value = world * flops / (ms_per_step * 1e-3) / 1e12
+    value = job_tflops(world, flops, ms_per_step)
 
     result = None
     if rank == 0:
@@ -398,7 +411,7 @@ def run_dense(ctx, steps=3):
             "sparse_fwd_tflops": round(fl / (att_ms * 1e-3) / 1e12, 1)}
 
 
-def main():
+def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
@@ -407,7 +420,7 @@ def main():
     ap.add_argument("--workload", default="sweep_32k")
     ap.add_argument("--keep", type=float, default=0.5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    args = ap.parse_args()
+    args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     world, rank, _ = dist_env()

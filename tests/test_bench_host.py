@@ -1,0 +1,77 @@
+"""Host-side logic of bench.py for N > 1 ranks, on CPU with the gloo backend:
+the timed region is the slowest rank's, the value sums every rank's work,
+and the reference arm runs on rank 0 only."""
+
+import os
+import socket
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _rank_main(rank, world, port, q):
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        elapsed = 100.0 + 10.0 * rank              # rank r took 100 + 10 r ms
+        slowest = bench.max_over_ranks(elapsed)
+        q.put((rank, slowest, bench.job_tflops(world, 1e12, slowest / 10)))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_timing_is_the_slowest_rank_and_value_sums_ranks(world):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    got = sorted(q.get(timeout=10) for _ in range(world))
+    slowest = 100.0 + 10.0 * (world - 1)
+    for rank, s, v in got:
+        assert s == slowest
+        assert v == pytest.approx(world * 1e12 / (slowest / 10 * 1e-3) / 1e12)
+
+
+def test_without_a_process_group_the_value_is_local():
+    assert bench.max_over_ranks(12.5) == 12.5
+    assert bench.job_tflops(1, 4e12, 1000.0) == pytest.approx(4.0)
+
+
+def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    bench.main(["--impl", "reference", "--steps", "1", "--warmup", "3"])
+    assert capsys.readouterr().out == ""
+
+
+def test_algorithmic_work_formulas():
+    # two GEMMs of b x b x d per kept block pair
+    assert bench.kept_flops(10, 128, 128) == 4.0 * 128 * 128 * 128 * 10
+
+    class W:
+        B, Hq, Hkv, N, d, nb, dtype = 1, 4, 2, 1024, 128, 8, "bf16"
+    # Q and K read once (bf16), index lists (k + count) written once
+    assert bench.selector_bytes(W, 4) == (4 + 2) * 1024 * 128 * 2 + 4 * 8 * 5 * 4
