@@ -439,7 +439,7 @@ def main(argv=None):
         result["dense_keep1"] = dense
         if not args.no_cpu_baseline:
             per_step, desc, spent = oracle_sample(ctx["w"], ctx["Q"], ctx["K"], ctx["V"], ctx["keep"], 0,
-                                                  n_blocks=48, n_sel_heads=2)
+                                                  n_blocks=768, n_sel_heads=8)
             result["cpu_baseline"] = {"value": round(ctx["flops"] / per_step / 1e12, 6), "unit": UNIT,
                                       "cores": cpu_cores(), "kind": "oracle", "sample": desc,
                                       "sample_seconds": round(spent, 1)}
@@ -465,7 +465,7 @@ def run_reference(args):
     per = []
     t0 = time.perf_counter()
     for i in range(args.steps):
-        ps, desc, _ = oracle_sample(w, Q, K, V, args.keep, i, n_blocks=8, n_sel_heads=1)
+        ps, desc, _ = oracle_sample(w, Q, K, V, args.keep, i, n_blocks=192, n_sel_heads=2)
         per.append(ps)
     wall = time.perf_counter() - t0
     ms = float(np.mean(per)) * 1e3

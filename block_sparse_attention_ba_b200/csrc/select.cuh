@@ -12,10 +12,12 @@
 //   kt_j = [ kbar_j   , kbar_j^2 + vk_j , vk_j ]
 // so that S~ = qt_i . kt_j + ln m_j (fp32 FMA accumulation).
 //
-// One CTA handles R query blocks of one (batch, head): it scores them against
-// every key block (rows kept in shared memory), then each warp selects the
-// top k of its rows by an exact 4-pass radix select on order-preserving keys
-// of the fp32 scores; equal scores go to the lower block index, and the kept
+// Two launches. select_kernel (SIMT; the tensor-core variant for nk <= 512
+// lives in select_tc.cuh) writes the whole fp32 score map; topk_rows_kernel
+// then gives one warp to each (batch, head, query block) row and selects its
+// top k by an exact 4-pass radix select on order-preserving keys of the fp32
+// scores (taken relative to the row minimum so that the high bytes carry
+// information); equal scores go to the lower block index, and the kept
 // indices are emitted ascending.
 #pragma once
 

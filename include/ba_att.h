@@ -129,9 +129,12 @@ ba_status ba_att_stats(const ba_att_shape *shape, const void *Q, const void *K,
  *                 ascending; entries at positions >= count are set to -1.
  * kv_cnt          device int32 [B, Hq, nq]: number kept (= k).
  * kmax            row stride of kv_idx; must be >= k.
- * block_scores    nullable device fp32 [B, Hq, nq, nk]: if non-NULL, S~ is
- *                 also written there.
- * Requires nk <= 4096.
+ * block_scores    device fp32 [B, Hq, nq, nk], caller-owned, required: the
+ *                 full S~ map is written there first and the top-k pass
+ *                 reads it back, so on return it holds the score map.
+ *                 NULL -> BA_ERR_INVALID_ARG; misaligned (not 16 B) ->
+ *                 BA_ERR_MISALIGNED.
+ * Requires nk <= 4096 (BA_ERR_UNSUPPORTED above).
  */
 ba_status ba_att_select(const ba_att_shape *shape, double keep,
                         const float *q_mean, const float *q_var,
