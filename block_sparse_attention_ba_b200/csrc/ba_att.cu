@@ -191,17 +191,11 @@ ba_status ba_att_select(const ba_att_shape *s, double keep, const float *q_mean,
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   const float scale = effective_scale(s);
   cudaError_t e;
-  if (nb <= seltc::kMaxKeys) {    // the whole score row fits the TMEM columns: tensor-core path
-    e = s->d == 128 ? launch_select_tc<128>(q_mean, q_var, k_mean, k_var, kv_idx, kv_cnt, block_scores, s->B, s->Hq,
-                                            s->Hkv, s->N, s->block, k, kmax, scale, cs)
-                    : launch_select_tc<64>(q_mean, q_var, k_mean, k_var, kv_idx, kv_cnt, block_scores, s->B, s->Hq,
-                                           s->Hkv, s->N, s->block, k, kmax, scale, cs);
-  } else {
-    e = s->d == 128 ? launch_select<128>(q_mean, q_var, k_mean, k_var, kv_idx, kv_cnt, block_scores, s->B, s->Hq,
-                                         s->Hkv, s->N, s->block, k, kmax, scale, cs)
-                    : launch_select<64>(q_mean, q_var, k_mean, k_var, kv_idx, kv_cnt, block_scores, s->B, s->Hq,
-                                        s->Hkv, s->N, s->block, k, kmax, scale, cs);
-  }
+  const int sms = num_sms_of_current_device();
+  e = s->d == 128 ? launch_select_tc<128>(q_mean, q_var, k_mean, k_var, kv_idx, kv_cnt, block_scores, s->B, s->Hq,
+                                          s->Hkv, s->N, s->block, k, kmax, scale, sms, cs)
+                  : launch_select_tc<64>(q_mean, q_var, k_mean, k_var, kv_idx, kv_cnt, block_scores, s->B, s->Hq,
+                                         s->Hkv, s->N, s->block, k, kmax, scale, sms, cs);
   return from_cuda(e);
 }
 

@@ -277,6 +277,11 @@ struct Elem<float> {
     f[2] = __uint_as_float(v.z);
     f[3] = __uint_as_float(v.w);
   }
+  // the vector as (lo, hi) fp32 pairs for the packed .f32x2 instructions
+  __device__ static __forceinline__ void unpack2(const uint4 &v, uint64_t (&x)[2]) {
+    x[0] = pack_u32x2(v.x, v.y);
+    x[1] = pack_u32x2(v.z, v.w);
+  }
   __device__ static __forceinline__ float load(const float *p) { return __ldg(p); }
 };
 template <>
@@ -289,6 +294,12 @@ struct Elem<__nv_bfloat16> {
       f[2 * i] = __uint_as_float(w[i] << 16);
       f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
     }
+  }
+  // element pairs (2i, 2i+1) widened to (lo, hi) fp32 pairs, exactly
+  __device__ static __forceinline__ void unpack2(const uint4 &v, uint64_t (&x)[4]) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) x[i] = pack_u32x2(w[i] << 16, w[i] & 0xFFFF0000u);
   }
   __device__ static __forceinline__ float load(const __nv_bfloat16 *p) {
     return bf16_to_f32(__ldg(reinterpret_cast<const unsigned short *>(p)));

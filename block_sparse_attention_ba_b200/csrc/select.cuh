@@ -25,9 +25,6 @@
 
 namespace baatt {
 
-constexpr int kSelThreads = 256;
-constexpr int kSelKeyChunk = 32;
-
 __device__ __forceinline__ uint32_t order_key(float f) {
   if (f != f) return 0u;                       // NaN ranks last
   if (f == 0.f) f = 0.f;                       // -0 == +0
@@ -151,8 +148,24 @@ __device__ void topk_row_warp(const float *__restrict__ srow, int nk, int k, int
 
 // The same exact selection for a row held in registers: lane l holds the
 // order keys of columns c*32 + l, c < KPL (so column order is chunk-major).
-// Every radix pass reads registers only; the per-warp histogram lives in
-// shared memory at hist_s.
+// The per-warp histogram (256 counters) lives in shared memory at hist_s.
+//
+//  1. Bracket: 32 keys sampled across the chunks are sorted across the warp
+//     (bitonic), and the samples 8 ranks either side of the expected rank of
+//     the k-th key give a key window [lo, hi]. One histogram pass over the
+//     window at a bin width of 2^shift, (hi - lo) >> shift < 256, counts the
+//     keys above the window separately. When the k-th key falls inside the
+//     window its bin is the candidate range; otherwise (a poor sample) the
+//     candidate range is the whole row [min, max].
+//  2. While the candidate range holds more than 32 keys, 8-bit radix passes
+//     narrow it from its top bit.
+//  3. At most 32 candidates are ranked directly, one per lane, in the order
+//     (key descending, column ascending); the rank-(need-1) candidate is the
+//     exact cut. A range narrowed down to one key value instead keeps its
+//     equal keys in column order.
+// Scores of a row are concentrated in a narrow band with a long upper tail,
+// so a window placed by the sample spreads the band over many bins where the
+// row's full range would put most keys into one bin.
 template <int KPL>
 __device__ __forceinline__ void topk_row_regs(const uint32_t (&u)[KPL], int nk, int k, int32_t *__restrict__ out_idx,
                                               int kmax, int32_t *__restrict__ out_cnt, uint32_t hist_s, int lane) {
@@ -163,85 +176,197 @@ __device__ __forceinline__ void topk_row_regs(const uint32_t (&u)[KPL], int nk, 
     if (lane == 0) *out_cnt = nk;
     return;
   }
-  uint32_t umin = 0xFFFFFFFFu, umax = 0u;
-#pragma unroll
-  for (int c = 0; c < KPL; ++c) {
-    if (c * 32 + lane < nk) {
-      umin = min(umin, u[c]);
-      umax = max(umax, u[c]);
-    }
-  }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    umin = min(umin, __shfl_xor_sync(full, umin, off));
-    umax = max(umax, __shfl_xor_sync(full, umax, off));
-  }
-  const uint32_t range = umax - umin;
-  const int nbits = range == 0u ? 0 : ((32 - __clz(range) + 7) & ~7);
-  uint32_t prefix = 0u, mask = 0u;
-  int need = k;
-  for (int shift = nbits - 8; shift >= 0; shift -= 8) {
-#pragma unroll
-    for (int t = 0; t < 8; ++t) asm volatile("st.shared.u32 [%0], %1;" ::"r"(hist_s + 4u * (lane + 32 * t)), "r"(0u));
-    __syncwarp();
-#pragma unroll
-    for (int c = 0; c < KPL; ++c) {
-      const uint32_t v = u[c] - umin;
-      if (c * 32 + lane < nk && (v & mask) == prefix) red_shared_add(hist_s + 4u * ((v >> shift) & 255u), 1u);
-    }
-    __syncwarp();
-    int cnts[8];
+  auto hist_zero = [&]() {
+    asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(hist_s + 32u * lane), "r"(0u) : "memory");
+    asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(hist_s + 32u * lane + 16u), "r"(0u) : "memory");
+  };
+  // Bins in descending order: lane l reads bins 255-8l .. 248-8l; the bin
+  // where the running count first reaches `want` (0..255, or -1 if the bins
+  // hold fewer keys), the count of keys above it and its own count.
+  auto hist_find = [&](int want, int &digit, int &above, int &in_bin) {
+    uint32_t h[8];
+    const uint32_t a = hist_s + 4u * (248u - 8u * lane);
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3]) : "r"(a));
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(h[4]), "=r"(h[5]), "=r"(h[6]), "=r"(h[7])
+                 : "r"(a + 16u));
     int local = 0;
 #pragma unroll
-    for (int t = 0; t < 8; ++t) {
-      uint32_t x;
-      asm volatile("ld.shared.u32 %0, [%1];" : "=r"(x) : "r"(hist_s + 4u * (255 - 8 * lane - t)));
-      cnts[t] = static_cast<int>(x);
-      local += cnts[t];
-    }
+    for (int t = 0; t < 8; ++t) local += static_cast<int>(h[t]);
     int incl = local;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
       const int y = __shfl_up_sync(full, incl, off);
       if (lane >= off) incl += y;
     }
-    const int excl = incl - local;
-    const unsigned hit = __ballot_sync(full, incl >= need);
+    const unsigned hit = __ballot_sync(full, incl >= want);
+    digit = -1;
+    if (hit == 0u) return;
     const int src = __ffs(hit) - 1;
-    int digit = 0, above = 0;
+    int dg = 0, ab = 0, ib = 0;
     if (lane == src) {
-      int c = excl;
+      int c = incl - local;
 #pragma unroll
-      for (int t = 0; t < 8; ++t) {
-        if (c + cnts[t] >= need) {
-          digit = 255 - 8 * lane - t;
-          above = c;
-          break;
+      for (int t = 7; t >= 0; --t) {                   // h[7] is the highest bin of this lane
+        const int n = static_cast<int>(h[t]);
+        if (dg == 0 && c + n >= want) {
+          dg = 248 - 8 * lane + t + 1;                 // +1 so that 0 means "not yet"
+          ab = c;
+          ib = n;
         }
-        c += cnts[t];
+        c += n;
       }
     }
-    digit = __shfl_sync(full, digit, src);
-    above = __shfl_sync(full, above, src);
-    prefix |= static_cast<uint32_t>(digit) << shift;
-    mask |= 255u << shift;
-    need -= above;
+    digit = __shfl_sync(full, dg, src) - 1;
+    above = __shfl_sync(full, ab, src);
+    in_bin = __shfl_sync(full, ib, src);
+  };
+
+  // candidate range: keys in [base, base + 2^nbits) (nbits 32: every key >= base)
+  uint32_t base = 0u;
+  int nbits = 32, need = k, in_bin = nk;
+  bool bracketed = false;
+  if (KPL >= 2 && nk >= 64) {
+    const int cs = lane % KPL;
+    uint32_t smp = u[0];
+#pragma unroll
+    for (int c = 1; c < KPL; ++c)
+      if (c == cs && c * 32 + lane < nk) smp = u[c];
+#pragma unroll
+    for (int size = 2; size <= 32; size <<= 1) {       // bitonic sort, descending across lanes
+#pragma unroll
+      for (int stride = size >> 1; stride > 0; stride >>= 1) {
+        const uint32_t o = __shfl_xor_sync(full, smp, stride);
+        const bool take_max = ((lane & stride) == 0) == ((lane & size) == 0 || size == 32);
+        smp = take_max ? max(smp, o) : min(smp, o);
+      }
+    }
+    const int rq = min(31, static_cast<int>((static_cast<long long>(k) * 32) / nk));
+    const uint32_t hi = __shfl_sync(full, smp, max(rq - 8, 0));
+    const uint32_t lo = __shfl_sync(full, smp, min(rq + 8, 31));
+    const int shift = max(0, 24 - static_cast<int>(__clz(hi - lo)));
+    hist_zero();
+    __syncwarp();
+    int n_above = 0;
+#pragma unroll
+    for (int c = 0; c < KPL; ++c) {
+      if (c * 32 + lane < nk && u[c] >= lo) {
+        const uint32_t bin = (u[c] - lo) >> shift;
+        if (bin > 255u)
+          ++n_above;
+        else
+          red_shared_add(hist_s + 4u * bin, 1u);
+      }
+    }
+    n_above = __reduce_add_sync(full, n_above);
+    __syncwarp();
+    if (n_above < k) {
+      int digit, ab, ib;
+      hist_find(k - n_above, digit, ab, ib);
+      if (digit >= 0) {
+        bracketed = true;
+        base = lo + (static_cast<uint32_t>(digit) << shift);
+        nbits = shift;
+        need = k - n_above - ab;
+        in_bin = ib;
+      }
+    }
     __syncwarp();
   }
-  const uint32_t thr = prefix + umin;                   // the k-th largest key
-  int pos = 0, eq_seen = 0;
+  if (!bracketed) {
+    uint32_t umin = 0xFFFFFFFFu, umax = 0u;
 #pragma unroll
-  for (int c = 0; c < KPL; ++c) {
-    const int j = c * 32 + lane;
-    const bool in = j < nk;
-    const bool gt = in && u[c] > thr;
-    const bool eq = in && u[c] == thr;
-    const unsigned eqb = __ballot_sync(full, eq);
-    const bool kept = gt || (eq && eq_seen + __popc(eqb & lt_mask) < need);
-    const unsigned kb = __ballot_sync(full, kept);
-    if (kept) out_idx[pos + __popc(kb & lt_mask)] = j;
-    pos += __popc(kb);
-    eq_seen += __popc(eqb);
+    for (int c = 0; c < KPL; ++c) {
+      if (c * 32 + lane < nk) {
+        umin = min(umin, u[c]);
+        umax = max(umax, u[c]);
+      }
+    }
+    umin = __reduce_min_sync(full, umin);
+    umax = __reduce_max_sync(full, umax);
+    base = umin;
+    nbits = 32 - static_cast<int>(__clz(umax - umin));    // 0 when every key is equal
+    need = k;
+    in_bin = nk;
+  }
+  // in the range: nbits < 32 needs the offset below 2^nbits
+  auto in_range = [&](uint32_t x, int j) {
+    return j < nk && x >= base && (nbits >= 32 || ((x - base) >> nbits) == 0u);
+  };
+
+  uint32_t prefix = 0u, mask = 0u;                      // over the offset x - base
+  for (int shift = ((nbits + 7) & ~7) - 8; shift >= 0 && in_bin > 32; shift -= 8) {
+    hist_zero();
+    __syncwarp();
+#pragma unroll
+    for (int c = 0; c < KPL; ++c) {
+      const uint32_t v = u[c] - base;
+      if (in_range(u[c], c * 32 + lane) && (v & mask) == prefix)
+        red_shared_add(hist_s + 4u * ((v >> shift) & 255u), 1u);
+    }
+    __syncwarp();
+    int digit, ab, ib;
+    hist_find(need, digit, ab, ib);                     // the range holds >= need keys: always found
+    prefix |= static_cast<uint32_t>(digit) << shift;
+    mask |= 255u << shift;
+    need -= ab;
+    in_bin = ib;
+    __syncwarp();
+  }
+
+  int pos = 0;
+  if (in_bin <= 32) {
+    // gather the remaining candidates' (key, column) pairs, one per lane
+    int cnt = 0;
+#pragma unroll
+    for (int c = 0; c < KPL; ++c) {
+      const int j = c * 32 + lane;
+      const bool cand = in_range(u[c], j) && ((u[c] - base) & mask) == prefix;
+      const unsigned cb = __ballot_sync(full, cand);
+      if (cand) {
+        const uint32_t slot = hist_s + 8u * static_cast<uint32_t>(cnt + __popc(cb & lt_mask));
+        asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(slot), "r"(u[c]), "r"(j) : "memory");
+      }
+      cnt += __popc(cb);
+    }
+    __syncwarp();
+    uint32_t cv = 0u;
+    int cj = 0x7FFFFFFF;
+    if (lane < cnt)
+      asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(cv), "=r"(cj) : "r"(hist_s + 8u * lane));
+    int rank = 0;
+    for (int t = 0; t < cnt; ++t) {
+      const uint32_t tv = __shfl_sync(full, cv, t);
+      const int tj = __shfl_sync(full, cj, t);
+      rank += (tv > cv || (tv == cv && tj < cj)) ? 1 : 0;
+    }
+    const int cut = __ffs(__ballot_sync(full, lane < cnt && rank == need - 1)) - 1;
+    const uint32_t thr_u = __shfl_sync(full, cv, cut);
+    const int thr_j = __shfl_sync(full, cj, cut);
+#pragma unroll
+    for (int c = 0; c < KPL; ++c) {
+      const int j = c * 32 + lane;
+      const bool kept = j < nk && (u[c] > thr_u || (u[c] == thr_u && j <= thr_j));
+      const unsigned kb = __ballot_sync(full, kept);
+      if (kept) out_idx[pos + __popc(kb & lt_mask)] = j;
+      pos += __popc(kb);
+    }
+  } else {
+    const uint32_t thr = base + prefix;                 // the range is one key value: the k-th largest
+    int eq_seen = 0;
+#pragma unroll
+    for (int c = 0; c < KPL; ++c) {
+      const int j = c * 32 + lane;
+      const bool in = j < nk;
+      const bool gt = in && u[c] > thr;
+      const bool eq = in && u[c] == thr;
+      const unsigned eqb = __ballot_sync(full, eq);
+      const bool kept = gt || (eq && eq_seen + __popc(eqb & lt_mask) < need);
+      const unsigned kb = __ballot_sync(full, kept);
+      if (kept) out_idx[pos + __popc(kb & lt_mask)] = j;
+      pos += __popc(kb);
+      eq_seen += __popc(eqb);
+    }
   }
   for (int j = pos + lane; j < kmax; j += 32) out_idx[j] = -1;
   if (lane == 0) *out_cnt = pos;
@@ -251,159 +376,64 @@ __device__ __forceinline__ void topk_row_regs(const uint32_t (&u)[KPL], int nk, 
 // 32*KPL keys are held in registers, longer rows are re-read per pass.
 constexpr int kTopkWarps = 8;
 
+// Rows up to 32*KPL keys: persistent warps walk the rows with a stride of all
+// warps of the grid, and the next row's scores are loaded into registers
+// before the current row is selected, so the load latency overlaps the
+// selection. Longer rows: one warp per row, re-read from global memory.
 template <int KPL>
 __global__ void __launch_bounds__(kTopkWarps * 32) topk_rows_kernel(const float *__restrict__ scores, int nk, int k,
                                                                     int32_t *__restrict__ kv_idx, int kmax,
                                                                     int32_t *__restrict__ kv_cnt, long long rows) {
-  __shared__ unsigned hist[kTopkWarps][256];
+  __shared__ __align__(16) unsigned hist[kTopkWarps][256];   // also holds (key, column) pairs
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const long long row = blockIdx.x * static_cast<long long>(kTopkWarps) + warp;
-  if (row >= rows) return;
-  const float *srow = scores + row * nk;
+  long long row = blockIdx.x * static_cast<long long>(kTopkWarps) + warp;
   if constexpr (KPL > 0) {
-    uint32_t u[KPL];
+    const long long stride = static_cast<long long>(gridDim.x) * kTopkWarps;
+    float nxt[KPL];
+    auto fetch = [&](long long r) {
+      const float *srow = scores + r * nk;
 #pragma unroll
-    for (int c = 0; c < KPL; ++c) {
-      const int j = c * 32 + lane;
-      u[c] = j < nk ? order_key(__ldg(srow + j)) : 0u;
+      for (int c = 0; c < KPL; ++c) {
+        const int j = c * 32 + lane;
+        nxt[c] = (r < rows && j < nk) ? __ldg(srow + j) : 0.f;
+      }
+    };
+    fetch(row);
+    for (; row < rows; row += stride) {
+      uint32_t u[KPL];
+#pragma unroll
+      for (int c = 0; c < KPL; ++c) u[c] = order_key(nxt[c]);
+      fetch(row + stride);
+      topk_row_regs<KPL>(u, nk, k, kv_idx + row * kmax, kmax, kv_cnt + row, smem_u32(&hist[warp][0]), lane);
     }
-    topk_row_regs<KPL>(u, nk, k, kv_idx + row * kmax, kmax, kv_cnt + row, smem_u32(&hist[warp][0]), lane);
   } else {
-    topk_row_warp(srow, nk, k, kv_idx + row * kmax, kmax, kv_cnt + row, &hist[warp][0], lane);
+    if (row >= rows) return;
+    topk_row_warp(scores + row * nk, nk, k, kv_idx + row * kmax, kmax, kv_cnt + row, &hist[warp][0], lane);
   }
 }
 
-inline cudaError_t launch_topk(const float *scores, int nk, int k, int32_t *idx, int kmax, int32_t *cnt,
-                               long long rows, cudaStream_t stream) {
-  const unsigned grid = static_cast<unsigned>((rows + kTopkWarps - 1) / kTopkWarps);
+template <int KPL>
+inline cudaError_t launch_topk_kpl(const float *scores, int nk, int k, int32_t *idx, int kmax, int32_t *cnt,
+                                   long long rows, int num_sms, cudaStream_t stream) {
   const int threads = kTopkWarps * 32;
-  if (nk <= 256)
-    topk_rows_kernel<8><<<grid, threads, 0, stream>>>(scores, nk, k, idx, kmax, cnt, rows);
-  else if (nk <= 512)
-    topk_rows_kernel<16><<<grid, threads, 0, stream>>>(scores, nk, k, idx, kmax, cnt, rows);
-  else if (nk <= 1024)
-    topk_rows_kernel<32><<<grid, threads, 0, stream>>>(scores, nk, k, idx, kmax, cnt, rows);
-  else
-    topk_rows_kernel<0><<<grid, threads, 0, stream>>>(scores, nk, k, idx, kmax, cnt, rows);
+  long long grid = (rows + kTopkWarps - 1) / kTopkWarps;
+  if (KPL > 0) {                                    // persistent: every resident CTA slot once
+    int per_sm = 0;
+    const cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, topk_rows_kernel<KPL>, threads, 0);
+    if (e != cudaSuccess) return e;
+    const long long slots = static_cast<long long>(num_sms) * (per_sm > 0 ? per_sm : 1);
+    grid = grid < slots ? grid : slots;
+  }
+  topk_rows_kernel<KPL><<<static_cast<unsigned>(grid), threads, 0, stream>>>(scores, nk, k, idx, kmax, cnt, rows);
   return cudaGetLastError();
 }
 
-template <int D>
-__global__ void __launch_bounds__(kSelThreads) select_kernel(
-    const float *__restrict__ q_mean, const float *__restrict__ q_var, const float *__restrict__ k_mean,
-    const float *__restrict__ k_var, int32_t *__restrict__ kv_idx, int32_t *__restrict__ kv_cnt,
-    float *__restrict__ block_scores, int Hq, int Hkv, int N, int block, int nb, int R, int k, int kmax,
-    float sm_scale) {
-  constexpr int D3 = 3 * D;
-  constexpr int KT_STRIDE = D3 + 4;                  // floats; keeps float4 rows conflict-free
-  extern __shared__ __align__(16) float sel_smem[];
-  float *qt = sel_smem;                              // [R][D3]
-  float *kt = qt + R * D3;                           // [kSelKeyChunk][KT_STRIDE]
-  float *sc = kt + kSelKeyChunk * KT_STRIDE;         // [R][nb]
-
-  const int b = blockIdx.z, h = blockIdx.y;
-  const int g = h / (Hq / Hkv);
-  const int i0 = blockIdx.x * R;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const float s = sm_scale, hs2 = 0.5f * sm_scale * sm_scale;
-
-  const float *qm = q_mean + (static_cast<long long>(b) * Hq + h) * nb * D;
-  const float *qv = q_var + (static_cast<long long>(b) * Hq + h) * nb * D;
-  const float *km = k_mean + (static_cast<long long>(b) * Hkv + g) * nb * D;
-  const float *kv = k_var + (static_cast<long long>(b) * Hkv + g) * nb * D;
-
-  for (int e = tid; e < R * D; e += kSelThreads) {
-    const int r = e / D, m = e % D;
-    const int i = i0 + r;
-    float a = 0.f, bq = 0.f, cq = 0.f;
-    if (i < nb) {
-      const float mu = __ldg(qm + static_cast<long long>(i) * D + m);
-      const float va = __ldg(qv + static_cast<long long>(i) * D + m);
-      a = s * mu;
-      bq = hs2 * va;
-      cq = hs2 * mu * mu;
-    }
-    qt[r * D3 + m] = a;
-    qt[r * D3 + D + m] = bq;
-    qt[r * D3 + 2 * D + m] = cq;
-  }
-
-  for (int j0 = 0; j0 < nb; j0 += kSelKeyChunk) {
-    __syncthreads();
-    for (int e = tid; e < kSelKeyChunk * D; e += kSelThreads) {
-      const int c = e / D, m = e % D;
-      const int j = j0 + c;
-      float a = 0.f, bb = 0.f, cc = 0.f;
-      if (j < nb) {
-        const float mu = __ldg(km + static_cast<long long>(j) * D + m);
-        const float va = __ldg(kv + static_cast<long long>(j) * D + m);
-        a = mu;
-        bb = mu * mu + va;
-        cc = va;
-      }
-      kt[c * KT_STRIDE + m] = a;
-      kt[c * KT_STRIDE + D + m] = bb;
-      kt[c * KT_STRIDE + 2 * D + m] = cc;
-    }
-    __syncthreads();
-    const int j = j0 + lane;
-    const float4 *krow = reinterpret_cast<const float4 *>(kt + lane * KT_STRIDE);
-    for (int r = warp; r < R; r += kSelThreads / 32) {
-      const float4 *qrow = reinterpret_cast<const float4 *>(qt + r * D3);
-      float acc0 = 0.f, acc1 = 0.f;
-#pragma unroll 8
-      for (int m4 = 0; m4 < D3 / 4; ++m4) {
-        const float4 qv4 = qrow[m4];
-        const float4 kv4 = krow[m4];
-        acc0 = fmaf(qv4.x, kv4.x, acc0);
-        acc1 = fmaf(qv4.y, kv4.y, acc1);
-        acc0 = fmaf(qv4.z, kv4.z, acc0);
-        acc1 = fmaf(qv4.w, kv4.w, acc1);
-      }
-      if (j < nb) {
-        const int mj = min(block, N - j * block);
-        sc[r * nb + j] = (acc0 + acc1) + logf(static_cast<float>(mj));
-      }
-    }
-  }
-  __syncthreads();
-
-  for (int e = tid; e < R * nb; e += kSelThreads) {     // coalesced rows of the score map
-    const int r = e / nb, j = e % nb;
-    const int i = i0 + r;
-    if (i < nb) block_scores[((static_cast<long long>(b) * Hq + h) * nb + i) * nb + j] = sc[e];
-  }
-}
-
-inline int select_rows_per_cta(int nb) {
-  int R = 16384 / nb;
-  if (R > 16) R = 16;
-  if (R < 1) R = 1;
-  return R;
-}
-
-inline size_t select_smem_bytes(int D, int nb) {
-  const int R = select_rows_per_cta(nb);
-  return sizeof(float) * (static_cast<size_t>(R) * 3 * D + static_cast<size_t>(kSelKeyChunk) * (3 * D + 4) +
-                          static_cast<size_t>(R) * nb);
-}
-
-template <int D>
-cudaError_t launch_select(const float *qm, const float *qv, const float *km, const float *kv, int32_t *idx,
-                          int32_t *cnt, float *scores, int B, int Hq, int Hkv, int N, int block, int k, int kmax,
-                          float sm_scale, cudaStream_t stream) {
-  const int nb = (N + block - 1) / block;
-  const int R = select_rows_per_cta(nb);
-  const size_t smem = select_smem_bytes(D, nb);
-  cudaError_t e = cudaFuncSetAttribute(select_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  dim3 grid((nb + R - 1) / R, Hq, B);
-  select_kernel<D><<<grid, kSelThreads, smem, stream>>>(qm, qv, km, kv, idx, cnt, scores, Hq, Hkv, N, block, nb, R,
-                                                        k, kmax, sm_scale);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  return launch_topk(scores, nb, k, idx, kmax, cnt, static_cast<long long>(B) * Hq * nb, stream);
+inline cudaError_t launch_topk(const float *scores, int nk, int k, int32_t *idx, int kmax, int32_t *cnt,
+                               long long rows, int num_sms, cudaStream_t stream) {
+  if (nk <= 256) return launch_topk_kpl<8>(scores, nk, k, idx, kmax, cnt, rows, num_sms, stream);
+  if (nk <= 512) return launch_topk_kpl<16>(scores, nk, k, idx, kmax, cnt, rows, num_sms, stream);
+  if (nk <= 1024) return launch_topk_kpl<32>(scores, nk, k, idx, kmax, cnt, rows, num_sms, stream);
+  return launch_topk_kpl<0>(scores, nk, k, idx, kmax, cnt, rows, num_sms, stream);
 }
 
 }  // namespace baatt

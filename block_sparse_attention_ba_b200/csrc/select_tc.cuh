@@ -1,27 +1,30 @@
 // select_tc.cuh — K7 on the tensor cores: covariance-compensated block
-// scores as one tcgen05 GEMM, then an exact per-row top-k read from TMEM.
+// scores as a tiled tcgen05 GEMM; the exact per-row top-k follows as its own
+// launch (topk_rows_kernel in select.cuh).
 //
-// Same operator as select.cuh ("Efficient Long-Context Modeling in DLMs via
-// Block Approximate Sparse Attention": abstract; "Core claim"; Figure 2):
-//   S~[i,j] = qt_i . kt_j + ln m_j,
-//   qt_i = [ s qbar_i , (s^2/2) vq_i , (s^2/2) qbar_i^2 ],
-//   kt_j = [ kbar_j , kbar_j^2 + vk_j , vk_j ]            (3d = 384 wide)
+// Operator ("Efficient Long-Context Modeling in DLMs via Block Approximate
+// Sparse Attention": abstract; "Core claim"; Figure 2):
+//   S~[i,j] = qt_i . kt_j + ln m_j, summed over 3d augmented features
+//   qt_i = [ s qbar_i , (s^2/2) vq_i , (s^2/2) qbar_i^2 ]
+//   kt_j = [ kbar_j , kbar_j^2 + vk_j , vk_j ]
 // ranked per query block, ties to the lower key block, top k kept ascending.
 //
-// One CTA = 128 query blocks of one (batch, head) x every key block (nk <=
-// 512, so the fp32 score tile fits the 512 TMEM columns).
-//  1. GEMM: the augmented rows are built from the fp32 statistics straight
-//     into shared memory in the 128-byte-swizzled K-major layout, 64 of the
-//     384 dimensions at a time. For fp32-level accuracy every operand is split
-//     x = hi + lo (two bf16s, 16 significant bits) and S accumulates
-//     hi*hi + hi*lo + lo*hi in fp32 (the dropped lo*lo is ~2^-16 relative).
-//     One thread issues the tcgen05.mma (M=128, N<=256 per tile) and commits
-//     to an mbarrier that gates the next slice.
-//  2. The fp32 score rows are drained from TMEM through the (now free)
-//     operand buffer into the score map; the top-k then runs as its own
-//     launch with one warp per row over the whole GPU (topk_rows_kernel), as
-//     one CTA's 128 rows per SM leave most SMs idle and each row's radix
-//     select is latency-bound.
+// One CTA = one (batch, head) x 128 query blocks (MMA M, the TMEM lanes) x NT
+// key blocks (MMA N, 64 or 128 TMEM columns): grid (ceil(nb/128) *
+// ceil(nb/NT), Hq, B), which covers any nb up to the host limit.
+//  - The feature order inside the 3d-long dot product is free, so the
+//    features are taken in groups of 64 dimensions: one read of the fp32
+//    statistics for dimensions [64g, 64g+64) yields all three feature parts
+//    of that group, written as three 64-wide K slices.
+//  - fp32-level accuracy on bf16 tensor cores: every operand is split
+//    x = hi + lo (two bf16s, 16 significant bits) and S accumulates
+//    hi*hi + hi*lo + lo*hi in fp32 (the dropped lo*lo is ~2^-16 relative).
+//  - Operands go straight from registers into the 128-byte-swizzled K-major
+//    shared-memory layout; one thread issues the MMAs and commits to an
+//    mbarrier. The statistics of the next group are loaded into registers
+//    before that mbarrier is waited on, so the loads overlap the MMAs.
+//  - The fp32 scores are read from TMEM (warp w: lane quadrant w%4, a quarter
+//    of the columns) and stored straight to the score map, ln m_j added.
 #pragma once
 
 #include "common.cuh"
@@ -30,25 +33,27 @@
 namespace baatt {
 namespace seltc {
 
-constexpr int kThreads = 256;
-constexpr int kRows = 128;                       // query blocks per CTA (TMEM lanes)
-constexpr int kMaxKeys = 512;                    // TMEM columns
-constexpr uint32_t kSliceA = kRows * 128;        // 128 rows x 64 bf16 = 16 KB
-constexpr uint32_t kSliceB = kMaxKeys * 128;     // 512 rows x 64 bf16 = 64 KB
-constexpr uint32_t kOffAhi = 0, kOffAlo = kSliceA, kOffBhi = 2 * kSliceA, kOffBlo = 2 * kSliceA + kSliceB;
-constexpr uint32_t kOperandBytes = 2 * kSliceA + 2 * kSliceB;             // 160 KB
-constexpr uint32_t kScoreBytes = 152u * 1024u;                            // score rows (reuse the above)
-constexpr uint32_t kDynSmem = kOperandBytes + 1024;
+constexpr int kThreads = 512;
+constexpr int kRows = 128;                              // query blocks per tile
+constexpr uint32_t kABytes = kRows * 128;               // 128 rows x 64 bf16
+template <int NT>
+struct Tile {
+  static constexpr uint32_t kBBytes = NT * 128;         // NT rows x 64 bf16
+  static constexpr uint32_t kPart = 2 * kABytes + 2 * kBBytes;
+  static constexpr uint32_t kDynSmem = 3 * kPart + 1024;
+  static constexpr int kTasksPerThread = (kRows + NT) * 8 / kThreads;
+  static_assert((kRows + NT) * 8 % kThreads == 0, "tasks must split evenly over the threads");
+  static_assert((kRows * 8) % kThreads == 0, "A and B tasks must not share an iteration");
+};
 
-// 8 consecutive augmented values -> hi and lo bf16 vectors.
+// x = hi + lo for 8 consecutive values, hi = RN_bf16(x), lo = RN_bf16(x - hi).
 __device__ __forceinline__ void split8(const float (&x)[8], uint4 &hi, uint4 &lo) {
   uint32_t h[4], l[4];
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
-    const __nv_bfloat16 h0 = __float2bfloat16_rn(x[2 * e]), h1 = __float2bfloat16_rn(x[2 * e + 1]);
-    const float r0 = x[2 * e] - __bfloat162float(h0), r1 = x[2 * e + 1] - __bfloat162float(h1);
-    h[e] = pack_bf16x2(__bfloat162float(h0), __bfloat162float(h1));
-    l[e] = pack_bf16x2(r0, r1);
+    h[e] = pack_bf16x2(x[2 * e], x[2 * e + 1]);
+    const float h0 = __uint_as_float(h[e] << 16), h1 = __uint_as_float(h[e] & 0xFFFF0000u);
+    l[e] = pack_bf16x2(x[2 * e] - h0, x[2 * e + 1] - h1);
   }
   hi = make_uint4(h[0], h[1], h[2], h[3]);
   lo = make_uint4(l[0], l[1], l[2], l[3]);
@@ -59,222 +64,225 @@ __device__ __forceinline__ uint32_t sw128(int r, int c) {
   return static_cast<uint32_t>(r) * 128u + (static_cast<uint32_t>(c ^ (r & 7)) << 4);
 }
 
-// 8 consecutive fp32 statistics (read-only path, so loads of several chunks
-// can be in flight together).
-struct Raw8 {
-  float4 a, b;
+// The 8 fp32 means and 8 variances of one 8-dimension chunk.
+struct Raw {
+  float4 m0, m1, v0, v1;
 };
-__device__ __forceinline__ Raw8 ld8(const float *p) {
-  return {__ldg(reinterpret_cast<const float4 *>(p)), __ldg(reinterpret_cast<const float4 *>(p + 4))};
-}
-__device__ __forceinline__ void unpack8(const Raw8 &r, float (&x)[8]) {
-  x[0] = r.a.x; x[1] = r.a.y; x[2] = r.a.z; x[3] = r.a.w;
-  x[4] = r.b.x; x[5] = r.b.y; x[6] = r.b.z; x[7] = r.b.w;
-}
 
-// Augmented query features, part 0/1/2: s*qbar, (s^2/2)*vq, (s^2/2)*qbar^2.
-__device__ __forceinline__ void aug_q(const Raw8 &m, const Raw8 &v, int part, float s, float hs2, float (&x)[8]) {
-  float mm[8], vv[8];
-  unpack8(m, mm);
-  unpack8(v, vv);
-#pragma unroll
-  for (int e = 0; e < 8; ++e) x[e] = part == 0 ? s * mm[e] : (part == 1 ? hs2 * vv[e] : hs2 * mm[e] * mm[e]);
-}
-// Augmented key features, part 0/1/2: kbar, kbar^2 + vk, vk.
-__device__ __forceinline__ void aug_k(const Raw8 &m, const Raw8 &v, int part, float (&x)[8]) {
-  float mm[8], vv[8];
-  unpack8(m, mm);
-  unpack8(v, vv);
-#pragma unroll
-  for (int e = 0; e < 8; ++e) x[e] = part == 0 ? mm[e] : (part == 1 ? fmaf(mm[e], mm[e], vv[e]) : vv[e]);
-}
-
-template <int D>
+template <int D, int NT>
 __global__ void __launch_bounds__(kThreads, 1)
     select_tc_kernel(const float *__restrict__ q_mean, const float *__restrict__ q_var,
-                     const float *__restrict__ k_mean, const float *__restrict__ k_var, int32_t *__restrict__ kv_idx,
-                     int32_t *__restrict__ kv_cnt, float *__restrict__ block_scores, int Hq, int Hkv, int N,
-                     int block, int nb, int k, int kmax, float sm_scale) {
-  constexpr int SLICES = 3 * D / 64;
-  constexpr int SL_PER_PART = D / 64;
+                     const float *__restrict__ k_mean, const float *__restrict__ k_var,
+                     float *__restrict__ block_scores, int Hq, int Hkv, int N, int block, int nb, float sm_scale) {
+  using TL = Tile<NT>;
+  constexpr int GROUPS = D / 64;
+  constexpr int TPT = TL::kTasksPerThread;
+  constexpr int COLS_PER_WARP = NT / 4;
   extern __shared__ uint8_t dyn_smem[];
   __shared__ uint64_t mma_bar;
   __shared__ uint32_t tmem_base_s;
-  __shared__ float lnm[kMaxKeys];
   __shared__ int abort_flag;
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
 
-  const int tid = threadIdx.x, warp = tid >> 5;
-  const int b = blockIdx.z, h = blockIdx.y, g = h / (Hq / Hkv);
-  const int i0 = blockIdx.x * kRows;
-  const int nk_pad = (nb + 15) & ~15;
-  const int n_tiles = nk_pad > 256 ? 2 : 1;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int nk_tiles = (nb + NT - 1) / NT;
+  const int h = blockIdx.y, b = blockIdx.z, g_kv = h / (Hq / Hkv);
+  const long long bh = static_cast<long long>(b) * Hq + h;
+  const int i0 = static_cast<int>(blockIdx.x / nk_tiles) * kRows, j0 = static_cast<int>(blockIdx.x % nk_tiles) * NT;
   const float s = sm_scale, hs2 = 0.5f * sm_scale * sm_scale;
-  const float *qm = q_mean + (static_cast<long long>(b) * Hq + h) * nb * D;
-  const float *qv = q_var + (static_cast<long long>(b) * Hq + h) * nb * D;
-  const float *km = k_mean + (static_cast<long long>(b) * Hkv + g) * nb * D;
-  const float *kv = k_var + (static_cast<long long>(b) * Hkv + g) * nb * D;
+  const float *qm = q_mean + bh * nb * D;
+  const float *qv = q_var + bh * nb * D;
+  const float *km = k_mean + (static_cast<long long>(b) * Hkv + g_kv) * nb * D;
+  const float *kv = k_var + (static_cast<long long>(b) * Hkv + g_kv) * nb * D;
 
-  for (int j = tid; j < kMaxKeys; j += kThreads)
-    lnm[j] = j < nb ? logf(static_cast<float>(min(block, N - j * block))) : 0.f;
   if (tid == 0) {
     mbar_init(smem_u32(&mma_bar), 1);
     abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 0) {
-    tmem_alloc<kMaxKeys>(smem_u32(&tmem_base_s));
+    tmem_alloc<NT>(smem_u32(&tmem_base_s));
     tmem_relinquish();
   }
+
+  // task e = it * kThreads + tid: rows [0,128) are query blocks (A), the
+  // next NT rows key blocks (B); chunk e % 8 covers 8 of the group's 64 dims
+  auto load_group = [&](int grp, Raw (&raw)[TPT]) {
+#pragma unroll
+    for (int it = 0; it < TPT; ++it) {
+      const int e = it * kThreads + tid;
+      const int c = e & 7;
+      const bool is_a = e < kRows * 8;
+      const int r = is_a ? (e >> 3) : ((e - kRows * 8) >> 3);
+      const int blk = (is_a ? i0 : j0) + r;
+      raw[it].m0 = raw[it].m1 = raw[it].v0 = raw[it].v1 = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (blk < nb) {
+        const long long off = static_cast<long long>(blk) * D + grp * 64 + c * 8;
+        const float *pm = (is_a ? qm : km) + off;
+        const float *pv = (is_a ? qv : kv) + off;
+        raw[it].m0 = __ldg(reinterpret_cast<const float4 *>(pm));
+        raw[it].m1 = __ldg(reinterpret_cast<const float4 *>(pm + 4));
+        raw[it].v0 = __ldg(reinterpret_cast<const float4 *>(pv));
+        raw[it].v1 = __ldg(reinterpret_cast<const float4 *>(pv + 4));
+      }
+    }
+  };
+  auto store_group = [&](const Raw (&raw)[TPT]) {
+#pragma unroll
+    for (int it = 0; it < TPT; ++it) {
+      const int e = it * kThreads + tid;
+      const bool is_a = e < kRows * 8;
+      const int r = is_a ? (e >> 3) : ((e - kRows * 8) >> 3);
+      const uint32_t o = sw128(r, e & 7);
+      const float m[8] = {raw[it].m0.x, raw[it].m0.y, raw[it].m0.z, raw[it].m0.w,
+                          raw[it].m1.x, raw[it].m1.y, raw[it].m1.z, raw[it].m1.w};
+      const float v[8] = {raw[it].v0.x, raw[it].v0.y, raw[it].v0.z, raw[it].v0.w,
+                          raw[it].v1.x, raw[it].v1.y, raw[it].v1.z, raw[it].v1.w};
+#pragma unroll
+      for (int p = 0; p < 3; ++p) {
+        float x[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          if (is_a)
+            x[q] = p == 0 ? s * m[q] : (p == 1 ? hs2 * v[q] : hs2 * m[q] * m[q]);
+          else
+            x[q] = p == 0 ? m[q] : (p == 1 ? fmaf(m[q], m[q], v[q]) : v[q]);
+        }
+        uint4 hi, lo;
+        split8(x, hi, lo);
+        const uint32_t base = p * TL::kPart + (is_a ? 0u : 2u * kABytes);
+        const uint32_t step = is_a ? kABytes : TL::kBBytes;
+        *reinterpret_cast<uint4 *>(smem + base + o) = hi;
+        *reinterpret_cast<uint4 *>(smem + base + step + o) = lo;
+      }
+    }
+  };
+
+  Raw raw[TPT];
+  load_group(0, raw);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_s;
+  const uint32_t idesc = idesc_bf16_f32(128, NT, 0, 0);
 
-  // ---------------------------------------------------------------- GEMM
   bool ok = true;
-  for (int sl = 0; sl < SLICES && ok; ++sl) {
-    const int part = sl / SL_PER_PART;
-    const int d0 = (sl % SL_PER_PART) * 64;
-    // A: 128 rows x 8 chunks, then B: nk_pad rows x 8 chunks, 4 chunks per
-    // thread per batch with all their loads issued before any use.
-    const Raw8 zero8 = {make_float4(0.f, 0.f, 0.f, 0.f), make_float4(0.f, 0.f, 0.f, 0.f)};
-    for (int e0 = 0; e0 < (kRows + nk_pad) * 8; e0 += 4 * kThreads) {
-      Raw8 rm[4], rv[4];
-#pragma unroll
-      for (int it = 0; it < 4; ++it) {
-        const int e = e0 + it * kThreads + tid;
-        rm[it] = zero8;
-        rv[it] = zero8;
-        if (e < kRows * 8) {
-          const int i = i0 + (e >> 3);
-          if (i < nb) {
-            const long long off = static_cast<long long>(i) * D + d0 + 8 * (e & 7);
-            if (part != 1) rm[it] = ld8(qm + off);
-            if (part == 1) rv[it] = ld8(qv + off);
-          }
-        } else if (e < (kRows + nk_pad) * 8) {
-          const int r = (e - kRows * 8) >> 3;
-          if (r < nb) {
-            const long long off = static_cast<long long>(r) * D + d0 + 8 * (e & 7);
-            if (part != 2) rm[it] = ld8(km + off);
-            if (part != 0) rv[it] = ld8(kv + off);
-          }
-        }
-      }
-#pragma unroll
-      for (int it = 0; it < 4; ++it) {
-        const int e = e0 + it * kThreads + tid;
-        if (e >= (kRows + nk_pad) * 8) break;
-        float x[8];
-        uint4 hi, lo;
-        if (e < kRows * 8) {
-          aug_q(rm[it], rv[it], part, s, hs2, x);
-          split8(x, hi, lo);
-          const uint32_t o = sw128(e >> 3, e & 7);
-          *reinterpret_cast<uint4 *>(smem + kOffAhi + o) = hi;
-          *reinterpret_cast<uint4 *>(smem + kOffAlo + o) = lo;
-        } else {
-          aug_k(rm[it], rv[it], part, x);
-          split8(x, hi, lo);
-          const uint32_t o = sw128((e - kRows * 8) >> 3, e & 7);
-          *reinterpret_cast<uint4 *>(smem + kOffBhi + o) = hi;
-          *reinterpret_cast<uint4 *>(smem + kOffBlo + o) = lo;
-        }
+  for (int grp = 0; grp < GROUPS; ++grp) {
+    if (grp > 0) {
+      // the previous group's MMAs must be done reading the operand buffers
+      const bool w = mbar_wait_bounded(smem_u32(&mma_bar), (grp - 1) & 1, &abort_flag);
+      if (__syncthreads_or(!w)) {
+        ok = false;
+        break;
       }
     }
+    store_group(raw);
     fence_proxy_async_smem();
     __syncthreads();
     if (tid == 0) {
       tc_fence_after();
-      for (int nt = 0; nt < n_tiles; ++nt) {
-        const int n = (nt == 0) ? (nk_pad > 256 ? 256 : nk_pad) : nk_pad - 256;
-        const uint32_t idesc = idesc_bf16_f32(128, n, 0, 0);
-        const uint32_t d_tmem = tmem + nt * 256;
-        const uint32_t boff = nt * 256 * 128;
+#pragma unroll
+      for (int p = 0; p < 3; ++p) {
+        const uint32_t pa = sbase + p * TL::kPart;
+        const uint32_t pb = pa + 2 * kABytes;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t ah = smem_desc_sw128(sbase + kOffAhi + kk * 32, 16, 1024);
-          const uint64_t al = smem_desc_sw128(sbase + kOffAlo + kk * 32, 16, 1024);
-          const uint64_t bh = smem_desc_sw128(sbase + kOffBhi + boff + kk * 32, 16, 1024);
-          const uint64_t bl = smem_desc_sw128(sbase + kOffBlo + boff + kk * 32, 16, 1024);
-          mma_ss(d_tmem, ah, bh, idesc, (sl > 0 || kk > 0) ? 1u : 0u);
-          mma_ss(d_tmem, ah, bl, idesc, 1u);
-          mma_ss(d_tmem, al, bh, idesc, 1u);
+          const uint64_t ah = smem_desc_sw128(pa + kk * 32, 16, 1024);
+          const uint64_t al = smem_desc_sw128(pa + kABytes + kk * 32, 16, 1024);
+          const uint64_t bhd = smem_desc_sw128(pb + kk * 32, 16, 1024);
+          const uint64_t bld = smem_desc_sw128(pb + TL::kBBytes + kk * 32, 16, 1024);
+          mma_ss(tmem, ah, bhd, idesc, (grp > 0 || p > 0 || kk > 0) ? 1u : 0u);
+          mma_ss(tmem, ah, bld, idesc, 1u);
+          mma_ss(tmem, al, bhd, idesc, 1u);
         }
       }
       mma_commit(smem_u32(&mma_bar));
     }
-    // the operand buffers are rewritten by the next slice (and reused as
-    // histograms after the last): wait for these MMAs to finish reading them
-    const bool w = mbar_wait_bounded(smem_u32(&mma_bar), sl & 1, &abort_flag);
+    if (grp + 1 < GROUPS) load_group(grp + 1, raw);
+  }
+  if (ok) {
+    const bool w = mbar_wait_bounded(smem_u32(&mma_bar), (GROUPS - 1) & 1, &abort_flag);
     ok = !__syncthreads_or(!w);
   }
   tc_fence_after();
 
   // ---------------------------------------------------------------- scores out
-  // TMEM -> shared memory (row stride nk_pad + 1 keeps the per-row drain
-  // conflict-free), 128 rows at once when they fit, else two halves of 64,
-  // then coalesced row writes of S~ (ln m_j included) to the score map. Warps
-  // w and w + 4 drain the same TMEM lane quadrant, each half of the columns.
   if (ok) {
-    const int stride = nk_pad + 1;
-    float *sc = reinterpret_cast<float *>(smem);
-    const int rows_per_pass = (kRows * stride * 4 <= static_cast<int>(kScoreBytes)) ? kRows : kRows / 2;
-    for (int r0 = 0; r0 < kRows; r0 += rows_per_pass) {
-      const int quad = warp & 3;
-      if (quad * 32 >= r0 && quad * 32 < r0 + rows_per_pass) {
-        const uint32_t taddr = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-        const int r = quad * 32 + (tid & 31) - r0;          // row within this pass
-        const int half_cols = nk_pad / 2;                    // multiple of 8
-        const int cbeg = (warp < 4) ? 0 : half_cols, cend = (warp < 4) ? half_cols : nk_pad;
-        for (int c0 = cbeg; c0 < cend; c0 += 8) {
-          uint32_t v[8];
-          asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-                       : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
-                         "=r"(v[7])
-                       : "r"(taddr + c0));
-          tmem_ld_wait();
+    const int quad = warp & 3, cq = warp >> 2;
+    const int i = i0 + quad * 32 + lane;
+    const uint32_t taddr = tmem + (static_cast<uint32_t>(quad * 32) << 16) + cq * COLS_PER_WARP;
+    const float ln_full = logf(static_cast<float>(block));
+    const float ln_last = logf(static_cast<float>(N - (nb - 1) * block));
+    const bool vec = (nb & 3) == 0;
 #pragma unroll
-          for (int c = 0; c < 8; ++c) sc[r * stride + c0 + c] = __uint_as_float(v[c]) + lnm[c0 + c];
+    for (int c0 = 0; c0 < COLS_PER_WARP; c0 += 16) {
+      uint32_t r[16];
+      asm volatile(
+          "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+          : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+            "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+          : "r"(taddr + c0));
+      tmem_ld_wait();
+      if (i < nb) {
+        const int jb = j0 + cq * COLS_PER_WARP + c0;
+        float *dst = block_scores + (bh * nb + i) * nb + jb;
+        float val[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) val[c] = __uint_as_float(r[c]) + (jb + c == nb - 1 ? ln_last : ln_full);
+        if (vec && jb + 16 <= nb) {
+#pragma unroll
+          for (int c = 0; c < 16; c += 4)
+            *reinterpret_cast<float4 *>(dst + c) = make_float4(val[c], val[c + 1], val[c + 2], val[c + 3]);
+        } else {
+#pragma unroll
+          for (int c = 0; c < 16; ++c)
+            if (jb + c < nb) dst[c] = val[c];
         }
       }
-      __syncthreads();
-      for (int rr = warp; rr < rows_per_pass; rr += kThreads / 32) {   // coalesced row write-out
-        const int i = i0 + r0 + rr;
-        if (i >= nb) break;
-        const long long row = (static_cast<long long>(b) * Hq + h) * nb + i;
-        const float *srow = sc + rr * stride;
-        for (int j = tid & 31; j < nb; j += 32) block_scores[row * nb + j] = srow[j];
-      }
-      __syncthreads();
     }
   }
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc<kMaxKeys>(tmem);
+    tmem_dealloc<NT>(tmem);
   }
 }
 
 }  // namespace seltc
 
+// Scores with the widest key tile that still gives at least half the SMs a
+// CTA, then the top-k launch.
 template <int D>
 cudaError_t launch_select_tc(const float *qm, const float *qv, const float *km, const float *kv, int32_t *idx,
                              int32_t *cnt, float *scores, int B, int Hq, int Hkv, int N, int block, int k, int kmax,
-                             float sm_scale, cudaStream_t stream) {
+                             float sm_scale, int num_sms, cudaStream_t stream) {
   const int nb = (N + block - 1) / block;
-  cudaError_t e = cudaFuncSetAttribute(seltc::select_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(seltc::kDynSmem));
-  if (e != cudaSuccess) return e;
-  dim3 grid((nb + seltc::kRows - 1) / seltc::kRows, Hq, B);
-  seltc::select_tc_kernel<D><<<grid, seltc::kThreads, seltc::kDynSmem, stream>>>(qm, qv, km, kv, idx, cnt, scores, Hq,
-                                                                                Hkv, N, block, nb, k, kmax, sm_scale);
+  const long long bhs = static_cast<long long>(B) * Hq;
+  const int nq_tiles = (nb + seltc::kRows - 1) / seltc::kRows;
+  const bool wide = static_cast<long long>(nq_tiles) * ((nb + 127) / 128) * bhs >= num_sms / 2;
+  cudaError_t e;
+  if (wide) {
+    using TL = seltc::Tile<128>;
+    e = cudaFuncSetAttribute(seltc::select_tc_kernel<D, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(TL::kDynSmem));
+    if (e != cudaSuccess) return e;
+    dim3 grid(((nb + 127) / 128) * nq_tiles, Hq, B);
+    seltc::select_tc_kernel<D, 128><<<grid, seltc::kThreads, TL::kDynSmem, stream>>>(qm, qv, km, kv, scores, Hq, Hkv,
+                                                                                      N, block, nb, sm_scale);
+  } else {
+    using TL = seltc::Tile<64>;
+    e = cudaFuncSetAttribute(seltc::select_tc_kernel<D, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(TL::kDynSmem));
+    if (e != cudaSuccess) return e;
+    dim3 grid(((nb + 63) / 64) * nq_tiles, Hq, B);
+    seltc::select_tc_kernel<D, 64><<<grid, seltc::kThreads, TL::kDynSmem, stream>>>(qm, qv, km, kv, scores, Hq, Hkv,
+                                                                                     N, block, nb, sm_scale);
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  return launch_topk(scores, nb, k, idx, kmax, cnt, static_cast<long long>(B) * Hq * nb, stream);
+  return launch_topk(scores, nb, k, idx, kmax, cnt, bhs * nb, num_sms, stream);
 }
 
 }  // namespace baatt

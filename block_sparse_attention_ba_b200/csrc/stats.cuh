@@ -117,12 +117,128 @@ __global__ void __launch_bounds__(kStatsThreads) stats_kernel(const T *__restric
 // Streaming variant for blocks of at most 32 KB (every bf16 d=128 shape up to
 // block 128): a persistent CTA walks the (head, block) items with a stride of
 // the grid size; each item is one contiguous slab of rows, fetched with a
-// single bulk copy (cp.async.bulk) into a 3-stage shared-memory ring. A stage
-// is refilled as soon as its rows sit in registers, so three slabs per CTA
-// are in flight while the current one is reduced. The reduction
-// is the same exact two-pass mean/variance as above, read from shared memory.
+// single bulk copy (cp.async.bulk) into a 3-stage shared-memory ring, so that
+// three slabs per CTA are in flight while the current one is reduced.
+//
+// The reduction takes one CTA barrier per item. Each thread reduces its own
+// rows exactly (two passes over registers: local sum S_t, then the centred
+// second moment M2_t about S_t / n_t); the lanes of a warp that share columns
+// are merged with shuffles, and the 8 warp partials of a column are merged by
+// one thread after the barrier, using the pairwise update for centred moments
+// (Chan, Golub and LeVeque, "Algorithms for computing the sample variance"):
+//   n = na + nb,  S = Sa + Sb,  M2 = M2a + M2b + (Sa/na - Sb/nb)^2 na nb / n.
+// The partials are double-buffered, so the same barrier that publishes this
+// item's partials also frees the ring stage and the other partial buffer.
 constexpr int kStatsStages = 3;
 constexpr uint32_t kStatsStageBytes = 32768;
+constexpr int kStatsWarps = kStatsThreads / 32;
+
+// Valid rows among r = rsub + k*rpp (k < rpt) of a block with n_rows rows.
+__device__ __forceinline__ int stats_rows_of(int rsub, int rpp, int rpt, int n_rows) {
+  return n_rows > rsub ? min(rpt, (n_rows - rsub + rpp - 1) / rpp) : 0;
+}
+
+// Moments of this thread's rows (r = rsub + k*RPP) of a complete block, with
+// the packed .f32x2 instructions (two columns per instruction), then merged
+// over the lanes of the warp that hold the same columns. Every count is a
+// compile-time constant here.
+template <typename T, int D>
+__device__ __forceinline__ void stats_moments_full(const T *slab, int rsub, int col, float (&ps)[Elem<T>::kVec],
+                                                   float (&pm2)[Elem<T>::kVec]) {
+  constexpr int VEC = Elem<T>::kVec, P = VEC / 2;
+  constexpr int COLS = D / VEC, RPP = kStatsThreads / COLS;
+  constexpr int RPT = static_cast<int>(kStatsStageBytes / (D * sizeof(T))) / RPP;
+  uint64_t x[RPT][P];
+#pragma unroll
+  for (int k = 0; k < RPT; ++k)
+    Elem<T>::unpack2(*reinterpret_cast<const uint4 *>(slab + (rsub + k * RPP) * D + col * VEC), x[k]);
+  const float inv = 1.f / static_cast<float>(RPT);
+  const uint64_t neg_inv2 = pack_f32x2(-inv, -inv), zero2 = pack_f32x2(0.f, 0.f);
+#pragma unroll
+  for (int i = 0; i < P; ++i) {
+    uint64_t s2 = x[0][i];
+#pragma unroll
+    for (int k = 1; k < RPT; ++k) s2 = add_f32x2(s2, x[k][i]);
+    const uint64_t neg_mu = fma_f32x2(s2, neg_inv2, zero2);
+    uint64_t q2 = zero2;
+#pragma unroll
+    for (int k = 0; k < RPT; ++k) {
+      const uint64_t dv = add_f32x2(x[k][i], neg_mu);
+      q2 = fma_f32x2(dv, dv, q2);
+    }
+    ps[2 * i] = lo_f32(s2);
+    ps[2 * i + 1] = hi_f32(s2);
+    pm2[2 * i] = lo_f32(q2);
+    pm2[2 * i + 1] = hi_f32(q2);
+  }
+  int na = RPT;
+#pragma unroll
+  for (int off = COLS; off < 32; off <<= 1) {    // equal counts: M2 += (Sa - Sb)^2 / (2 na)
+    const float c = 0.5f / static_cast<float>(na);
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) {
+      const float sb = __shfl_xor_sync(0xFFFFFFFFu, ps[e], off);
+      const float mb = __shfl_xor_sync(0xFFFFFFFFu, pm2[e], off);
+      const float dm = ps[e] - sb;
+      pm2[e] = fmaf(dm * dm, c, pm2[e] + mb);
+      ps[e] += sb;
+    }
+    na *= 2;
+  }
+}
+
+// The same for the last, partly filled block of a head: rows at or beyond
+// n_rows are left out of every count.
+template <typename T, int D>
+__device__ __forceinline__ void stats_moments_ragged(const T *slab, int n_rows, int rsub, int col,
+                                                  float (&ps)[Elem<T>::kVec], float (&pm2)[Elem<T>::kVec]) {
+  constexpr int VEC = Elem<T>::kVec;
+  constexpr int COLS = D / VEC, RPP = kStatsThreads / COLS;
+  constexpr int RPT = static_cast<int>(kStatsStageBytes / (D * sizeof(T))) / RPP;
+  float f[RPT][VEC];
+#pragma unroll
+  for (int k = 0; k < RPT; ++k) {
+    const int r = rsub + k * RPP;
+    const uint4 v = r < n_rows ? *reinterpret_cast<const uint4 *>(slab + r * D + col * VEC) : make_uint4(0, 0, 0, 0);
+    Elem<T>::unpack(v, f[k]);
+  }
+  const int nt = stats_rows_of(rsub, RPP, RPT, n_rows);
+  const float inv_nt = nt > 0 ? 1.f / static_cast<float>(nt) : 0.f;
+#pragma unroll
+  for (int e = 0; e < VEC; ++e) {
+    float a = 0.f;
+#pragma unroll
+    for (int k = 0; k < RPT; ++k) a += f[k][e];              // padded rows hold 0
+    ps[e] = a;
+    const float mu = a * inv_nt;
+    float q = 0.f;
+#pragma unroll
+    for (int k = 0; k < RPT; ++k) {
+      const float dv = f[k][e] - mu;
+      q = (rsub + k * RPP < n_rows) ? fmaf(dv, dv, q) : q;
+    }
+    pm2[e] = q;
+  }
+  int na = nt;
+#pragma unroll
+  for (int off = COLS; off < 32; off <<= 1) {
+    const int nb_ = __shfl_xor_sync(0xFFFFFFFFu, na, off);
+    const int n = na + nb_;
+    const float ia = na > 0 ? 1.f / static_cast<float>(na) : 0.f;
+    const float ib = nb_ > 0 ? 1.f / static_cast<float>(nb_) : 0.f;
+    const float c = (na > 0 && nb_ > 0) ? static_cast<float>(na) * static_cast<float>(nb_) / static_cast<float>(n)
+                                        : 0.f;
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) {
+      const float sb = __shfl_xor_sync(0xFFFFFFFFu, ps[e], off);
+      const float mb = __shfl_xor_sync(0xFFFFFFFFu, pm2[e], off);
+      const float dm = ps[e] * ia - sb * ib;
+      pm2[e] = fmaf(dm * dm, c, pm2[e] + mb);
+      ps[e] += sb;
+    }
+    na = n;
+  }
+}
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kStatsThreads, 2)
@@ -130,18 +246,20 @@ __global__ void __launch_bounds__(kStatsThreads, 2)
                       float *__restrict__ q_var, float *__restrict__ k_mean, float *__restrict__ k_var, int B,
                       int Hq, int Hkv, int N, int N_alloc, int block, int nb) {
   constexpr int VEC = Elem<T>::kVec;
-  constexpr int COLS = D / VEC;
-  constexpr int RPP = kStatsThreads / COLS;
-  constexpr int RPT = static_cast<int>(kStatsStageBytes / (D * sizeof(T))) / RPP;   // = 8
+  constexpr int COLS = D / VEC;                     // threads per row (16-byte vectors)
+  constexpr int RPP = kStatsThreads / COLS;         // rows per pass of the CTA
+  constexpr int RPT = static_cast<int>(kStatsStageBytes / (D * sizeof(T))) / RPP;
+  constexpr int RPW = 32 / COLS;                    // row subsets (rsub values) per warp
+  static_assert(COLS <= 32 && 32 % COLS == 0, "a row must map onto whole lanes of a warp");
   extern __shared__ __align__(128) uint8_t stage_mem[];
-  __shared__ float red[RPP][D];
-  __shared__ float mean_s[D];
+  __shared__ float part_s[2][kStatsWarps][D];
+  __shared__ float part_m2[2][kStatsWarps][D];
   __shared__ uint64_t full[kStatsStages];
   __shared__ int abort_flag;
 
   const long long n_q = static_cast<long long>(B) * Hq * nb;
   const long long total = n_q + static_cast<long long>(B) * Hkv * nb;
-  const int tid = threadIdx.x, col = tid % COLS, rsub = tid / COLS;
+  const int tid = threadIdx.x, col = tid % COLS, rsub = tid / COLS, warp = tid >> 5;
   const uint32_t ring = smem_u32(stage_mem);
 
   // item w -> source slab, valid rows, output row offset, Q-or-K
@@ -182,37 +300,33 @@ __global__ void __launch_bounds__(kStatsThreads, 2)
 
   int it = 0;
   for (long long w = blockIdx.x; w < total; w += gridDim.x, ++it) {
-    const int s = it % kStatsStages;
+    const int s = it % kStatsStages, pb = it & 1;
     const T *src;
     int n_rows;
     long long orow;
     bool is_q;
     locate(w, src, n_rows, orow, is_q);
     const bool ok = mbar_wait_bounded(smem_u32(&full[s]), (it / kStatsStages) & 1, &abort_flag);
-    if (__syncthreads_or(!ok)) break;
 
+    // this thread's rows: exact local sum and centred second moment, merged
+    // over the lanes of the warp that hold the same columns
     const T *slab = reinterpret_cast<const T *>(stage_mem + s * kStatsStageBytes);
-    uint4 v[RPT];
-#pragma unroll
-    for (int k = 0; k < RPT; ++k) {
-      const int r = rsub + k * RPP;
-      v[k] = r < n_rows ? *reinterpret_cast<const uint4 *>(slab + r * D + col * VEC) : make_uint4(0, 0, 0, 0);
+    const bool full_block = n_rows == RPP * RPT;
+    float ps[VEC], pm2[VEC];
+    if (full_block) {
+      stats_moments_full<T, D>(slab, rsub, col, ps, pm2);
+    } else {
+      stats_moments_ragged<T, D>(slab, n_rows, rsub, col, ps, pm2);
     }
-    float acc[VEC];
+    if ((tid & 31) < COLS) {
 #pragma unroll
-    for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
-#pragma unroll
-    for (int k = 0; k < RPT; ++k) {
-      float f[VEC];
-      Elem<T>::unpack(v[k], f);
-#pragma unroll
-      for (int e = 0; e < VEC; ++e) acc[e] += f[e];
+      for (int e = 0; e < VEC; ++e) {
+        part_s[pb][warp][col * VEC + e] = ps[e];
+        part_m2[pb][warp][col * VEC + e] = pm2[e];
+      }
     }
-#pragma unroll
-    for (int e = 0; e < VEC; ++e) red[rsub][col * VEC + e] = acc[e];
-    __syncthreads();
-    // every thread holds its rows in registers now: hand stage s straight
-    // back to the copy engine for the item kStatsStages ahead
+    // one barrier: partials published, ring stage s consumed by every thread
+    if (__syncthreads_or(!ok)) break;
     if (tid == 0) {
       const long long wn = w + static_cast<long long>(kStatsStages) * gridDim.x;
       if (wn < total) {
@@ -221,43 +335,36 @@ __global__ void __launch_bounds__(kStatsThreads, 2)
         last_issued = wn;
       }
     }
-    const float inv_n = 1.f / static_cast<float>(n_rows);
     if (tid < D) {
-      float sum = 0.f;
-#pragma unroll 8
-      for (int r = 0; r < RPP; ++r) sum += red[r][tid];
-      mean_s[tid] = sum * inv_n;
-    }
-    __syncthreads();
-    float mu[VEC];
+      float S = 0.f;
 #pragma unroll
-    for (int e = 0; e < VEC; ++e) {
-      mu[e] = mean_s[col * VEC + e];
-      acc[e] = 0.f;
-    }
+      for (int q = 0; q < kStatsWarps; ++q) S += part_s[pb][q][tid];
+      float mean, M2 = 0.f;
+      if (full_block) {                       // every warp holds RPW * RPT rows
+        constexpr float kNw = static_cast<float>(RPW * RPT), kInvNw = 1.f / kNw;
+        constexpr float kInvN = 1.f / static_cast<float>(RPP * RPT);
+        mean = S * kInvN;
 #pragma unroll
-    for (int k = 0; k < RPT; ++k) {
-      if (rsub + k * RPP < n_rows) {
-        float f[VEC];
-        Elem<T>::unpack(v[k], f);
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) {
-          const float dv = f[e] - mu[e];
-          acc[e] = fmaf(dv, dv, acc[e]);
+        for (int q = 0; q < kStatsWarps; ++q) {
+          const float t = fmaf(-kNw, mean, part_s[pb][q][tid]);
+          M2 += fmaf(t * t, kInvNw, part_m2[pb][q][tid]);
         }
-      }
-    }
+        M2 *= kInvN;
+      } else {
+        mean = S / static_cast<float>(n_rows);
 #pragma unroll
-    for (int e = 0; e < VEC; ++e) red[rsub][col * VEC + e] = acc[e];
-    __syncthreads();
-    if (tid < D) {
-      float sum = 0.f;
-#pragma unroll 8
-      for (int r = 0; r < RPP; ++r) sum += red[r][tid];
-      (is_q ? q_mean : k_mean)[orow + tid] = mean_s[tid];
-      (is_q ? q_var : k_var)[orow + tid] = sum * inv_n;
+        for (int q = 0; q < kStatsWarps; ++q) {
+          int nq = 0;
+#pragma unroll
+          for (int u = 0; u < RPW; ++u) nq += stats_rows_of(q * RPW + u, RPP, RPT, n_rows);
+          const float t = fmaf(-static_cast<float>(nq), mean, part_s[pb][q][tid]);
+          M2 += part_m2[pb][q][tid] + (nq > 0 ? t * t / static_cast<float>(nq) : 0.f);
+        }
+        M2 /= static_cast<float>(n_rows);
+      }
+      (is_q ? q_mean : k_mean)[orow + tid] = mean;
+      (is_q ? q_var : k_var)[orow + tid] = M2;
     }
-    __syncthreads();
   }
   // after an abandoned wait, let every issued copy land before exiting
   // (the newest kStatsStages items issued, each in its own stage)
@@ -287,7 +394,10 @@ cudaError_t launch_stats(const T *Q, const T *K, float *qm, float *qv, float *km
     cudaError_t e = cudaFuncSetAttribute(stats_bulk_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    const long long persistent = static_cast<long long>(num_sms) * 2;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, stats_bulk_kernel<T, D>, kStatsThreads, smem);
+    if (e != cudaSuccess) return e;
+    const long long persistent = static_cast<long long>(num_sms) * (per_sm > 0 ? per_sm : 1);
     const unsigned g = static_cast<unsigned>(grid < persistent ? grid : persistent);
     stats_bulk_kernel<T, D><<<g, kStatsThreads, smem, stream>>>(Q, K, qm, qv, km, kv, B, Hq, Hkv, N, N_alloc, block,
                                                                  nb);
