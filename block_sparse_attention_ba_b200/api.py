@@ -19,6 +19,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 
 BA_OK = 0
+BA_ERR_INVALID_ARG = 1
 STATUS_NAMES = {0: "BA_OK", 1: "BA_ERR_INVALID_ARG", 2: "BA_ERR_UNSUPPORTED", 3: "BA_ERR_MISALIGNED",
                 4: "BA_ERR_CUDA", 5: "BA_ERR_DEVICE", 6: "BA_ERR_TIMEOUT"}
 DTYPE_F32, DTYPE_BF16 = 0, 1
@@ -46,6 +47,9 @@ _SIGS = {
     "ba_att_merge_lse": (ctypes.c_int, [ctypes.c_int64, _I32, _I32, _I32, _P, _P, _P, _P, _P, _P, _P]),
     "ba_att_get_device_error": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_uint32)]),
     "ba_att_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_uint32, _P]),
+    "ba_att_forward_host_workspace": (ctypes.c_int64, [ctypes.POINTER(CShape), ctypes.c_double, _I32, _I32]),
+    "ba_att_forward_host": (ctypes.c_int, [ctypes.POINTER(CShape), ctypes.c_double, _I32, _I32, _P, _P, _P, _P, _P,
+                                            _P, ctypes.c_int64, _P]),
 }
 
 _lib = None
@@ -237,6 +241,50 @@ def forward(Q, K, V, N: int, block: int, keep: float, sm_scale: float = 0.0):
     idx, cnt = select(st, shape, keep)
     O, LSE = sparse_fwd(Q, K, V, idx, cnt, shape)
     return O, LSE, idx, cnt
+
+
+def forward_host_workspace_bytes(shape: Shape, keep: float, split_block: int = -1, kv_heads_per_chunk: int = 0) -> int:
+    """Device workspace bytes ba_att_forward_host needs (raises on arguments it would reject)."""
+    n = load_library().ba_att_forward_host_workspace(ctypes.byref(shape.c()), float(keep), int(split_block),
+                                                     int(kv_heads_per_chunk))
+    if n < 0:
+        raise BaAttError("ba_att_forward_host_workspace", BA_ERR_INVALID_ARG)
+    return int(n)
+
+
+def _host(t: torch.Tensor, name: str) -> ctypes.c_void_p:
+    if t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous host (CPU) tensor")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def forward_host(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, N: int, block: int, keep: float,
+                 split_block: int = -1, kv_heads_per_chunk: int = 0, sm_scale: float = 0.0,
+                 workspace: torch.Tensor | None = None, out=None, device=None):
+    """Whole forward from host tensors to host tensors (ba_att_forward_host):
+    copies in, stats, select, sparse attention (split + merge when
+    split_block >= 0), copies out, pipelined per chunk of KV heads. Q, K, V,
+    and the outputs should be pinned for the copies to overlap compute.
+    Asynchronous on the current stream; synchronise before reading (O, LSE)."""
+    shape = Shape.of(Q, K, N, block, sm_scale)
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    need = forward_host_workspace_bytes(shape, keep, split_block, kv_heads_per_chunk)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+    if not workspace.is_cuda or workspace.numel() * workspace.element_size() < need:
+        raise ValueError(f"workspace must be a CUDA tensor of at least {need} bytes")
+    if out is None:
+        O = torch.empty(Q.shape, dtype=Q.dtype).pin_memory()
+        LSE = torch.empty(Q.shape[:3], dtype=torch.float32).pin_memory()
+    else:
+        O, LSE = out
+    lib = load_library()
+    _check("ba_att_forward_host",
+           lib.ba_att_forward_host(ctypes.byref(shape.c()), float(keep), int(split_block), int(kv_heads_per_chunk),
+                                   _host(Q, "Q"), _host(K, "K"), _host(V, "V"), _host(O, "O"), _host(LSE, "LSE"),
+                                   ctypes.c_void_p(workspace.data_ptr()), int(workspace.numel() * workspace.element_size()),
+                                   ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)))
+    return O, LSE
 
 
 def get_device_error(device=None):

@@ -3,8 +3,9 @@
 // Every entry point validates its arguments on the host first and launches
 // nothing on a bad argument. Launches are asynchronous on the caller's
 // stream; no call synchronises except ba_att_get_device_error. The library
-// allocates no device memory: its only global state is the device error word
-// (a __device__ variable) and a cache of per-device SM counts.
+// allocates no device memory: its global state is the device error word (a
+// __device__ variable), a cache of per-device SM counts, and per device the
+// two copy streams and events of the host-buffer pipeline.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -320,6 +321,222 @@ ba_status ba_att_selftest_bounded_wait(uint32_t timeout_us, ba_stream_t stream) 
   bounded_wait_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
       static_cast<unsigned long long>(timeout_us) * 1000ull);
   return from_cuda(cudaGetLastError());
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------- host-buffer pipeline
+namespace {
+
+constexpr size_t kWsAlign = 256;
+size_t round_up(size_t x) { return (x + kWsAlign - 1) / kWsAlign * kWsAlign; }
+
+// Workspace layout of ba_att_forward_host for chunks of C KV heads.
+struct PipeLayout {
+  int C = 0, G = 0, nb = 0, k = 0;
+  size_t q[2], kk[2], v[2], o[2], l[2];                 // double-buffered chunk inputs and outputs
+  size_t qm, qv, km, kv, idx, cnt, sc;                  // selector buffers of one chunk
+  size_t lo_idx, lo_cnt, hi_idx, hi_cnt, o1, o2, l1, l2;  // split + merge buffers of one chunk
+  size_t total = 0;
+};
+
+int auto_chunk(const ba_att_shape *s) { return s->Hkv >= 4 ? s->Hkv / 4 : 1; }
+
+bool pipe_layout(const ba_att_shape *s, double keep, int32_t split_block, int32_t chunk, PipeLayout *L) {
+  if (check_shape(s) != BA_OK) return false;
+  const int k = ba_att_keep_count(s, keep);
+  if (k < 1) return false;
+  const int nb = nblocks(s);
+  if (split_block > nb) return false;
+  L->C = chunk > 0 ? (chunk < s->Hkv ? chunk : s->Hkv) : auto_chunk(s);
+  L->G = s->Hq / s->Hkv;
+  L->nb = nb;
+  L->k = k;
+  const size_t e = s->dtype == BA_DTYPE_BF16 ? 2 : 4;
+  const size_t hq = static_cast<size_t>(L->C) * L->G, hk = static_cast<size_t>(L->C);
+  const size_t rows_q = hq * s->N_alloc, rows_k = hk * s->N_alloc;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off += round_up(bytes);
+    return at;
+  };
+  for (int b = 0; b < 2; ++b) {
+    L->q[b] = take(rows_q * s->d * e);
+    L->kk[b] = take(rows_k * s->d * e);
+    L->v[b] = take(rows_k * s->d * e);
+    L->o[b] = take(rows_q * s->d * e);
+    L->l[b] = take(rows_q * 4);
+  }
+  L->qm = take(hq * nb * s->d * 4);
+  L->qv = take(hq * nb * s->d * 4);
+  L->km = take(hk * nb * s->d * 4);
+  L->kv = take(hk * nb * s->d * 4);
+  L->idx = take(hq * nb * k * 4);
+  L->cnt = take(hq * nb * 4);
+  L->sc = take(hq * nb * static_cast<size_t>(nb) * 4);
+  if (split_block >= 0) {
+    L->lo_idx = take(hq * nb * k * 4);
+    L->lo_cnt = take(hq * nb * 4);
+    L->hi_idx = take(hq * nb * k * 4);
+    L->hi_cnt = take(hq * nb * 4);
+    L->o1 = take(rows_q * s->d * 4);
+    L->o2 = take(rows_q * s->d * 4);
+    L->l1 = take(rows_q * 4);
+    L->l2 = take(rows_q * 4);
+  }
+  L->total = off;
+  return true;
+}
+
+// Per-device copy streams and events, created on first use and kept for the
+// life of the process; `lock` serialises enqueueing calls on one device.
+struct PipeResources {
+  std::mutex lock;
+  bool ready = false;
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaEvent_t entry = nullptr, tail = nullptr;
+  cudaEvent_t in_ready[2] = {nullptr, nullptr}, in_free[2] = {nullptr, nullptr};
+  cudaEvent_t out_ready[2] = {nullptr, nullptr}, out_free[2] = {nullptr, nullptr};
+};
+
+PipeResources *pipe_resources(int dev) {
+  static PipeResources res[kMaxDevices];
+  return (dev >= 0 && dev < kMaxDevices) ? &res[dev] : nullptr;
+}
+
+cudaError_t pipe_init(PipeResources *r) {
+  if (r->ready) return cudaSuccess;
+  cudaError_t e = cudaStreamCreateWithFlags(&r->h2d, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&r->d2h, cudaStreamNonBlocking);
+  cudaEvent_t *evs[] = {&r->entry, &r->tail, &r->in_ready[0], &r->in_ready[1], &r->in_free[0], &r->in_free[1],
+                        &r->out_ready[0], &r->out_ready[1], &r->out_free[0], &r->out_free[1]};
+  for (cudaEvent_t *ev : evs)
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
+  if (e == cudaSuccess) r->ready = true;
+  return e;
+}
+
+}  // namespace
+
+extern "C" {
+
+int64_t ba_att_forward_host_workspace(const ba_att_shape *s, double keep, int32_t split_block,
+                                      int32_t kv_heads_per_chunk) {
+  PipeLayout L;
+  if (!pipe_layout(s, keep, split_block, kv_heads_per_chunk, &L)) return -1;
+  return static_cast<int64_t>(L.total);
+}
+
+ba_status ba_att_forward_host(const ba_att_shape *s, double keep, int32_t split_block, int32_t kv_heads_per_chunk,
+                              const void *Q, const void *K, const void *V, void *O, float *LSE, void *workspace,
+                              int64_t workspace_bytes, ba_stream_t stream) {
+  PipeLayout L;
+  ba_status st = check_shape(s);
+  if (st != BA_OK) return st;
+  if (!pipe_layout(s, keep, split_block, kv_heads_per_chunk, &L)) return BA_ERR_INVALID_ARG;
+  if (!Q || !K || !V || !O || !LSE || !workspace) return BA_ERR_INVALID_ARG;
+  if (workspace_bytes < static_cast<int64_t>(L.total)) return BA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(workspace) % kWsAlign != 0) return BA_ERR_MISALIGNED;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return BA_ERR_CUDA;
+  PipeResources *r = pipe_resources(dev);
+  if (r == nullptr) return BA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> guard(r->lock);
+  if (pipe_init(r) != cudaSuccess) return BA_ERR_CUDA;
+
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  const size_t e = s->dtype == BA_DTYPE_BF16 ? 2 : 4;
+  const size_t head_elems = static_cast<size_t>(s->N_alloc) * s->d;
+  const int chunks_per_b = (s->Hkv + L.C - 1) / L.C;
+  const int n_chunks = s->B * chunks_per_b;
+
+  // the copy streams start after whatever `stream` holds (e.g. an earlier
+  // call that used the same workspace)
+  cudaError_t ce = cudaEventRecord(r->entry, cs);
+  if (ce == cudaSuccess) ce = cudaStreamWaitEvent(r->h2d, r->entry, 0);
+  if (ce == cudaSuccess) ce = cudaStreamWaitEvent(r->d2h, r->entry, 0);
+  if (ce != cudaSuccess) return BA_ERR_CUDA;
+
+  for (int c = 0; c < n_chunks && st == BA_OK; ++c) {
+    const int sl = c & 1;
+    const int b = c / chunks_per_b, g0 = (c % chunks_per_b) * L.C;
+    const int gc = (s->Hkv - g0) < L.C ? (s->Hkv - g0) : L.C;
+    const int hq0 = g0 * L.G, hqc = gc * L.G;
+    const size_t q_off = (static_cast<size_t>(b) * s->Hq + hq0) * head_elems;
+    const size_t k_off = (static_cast<size_t>(b) * s->Hkv + g0) * head_elems;
+    void *Qc = ws + L.q[sl], *Kc = ws + L.kk[sl], *Vc = ws + L.v[sl], *Oc = ws + L.o[sl];
+    float *Lc = reinterpret_cast<float *>(ws + L.l[sl]);
+
+    // inputs of chunk c into slot sl, once chunk c-2 has finished reading it
+    if (c >= 2) ce = cudaStreamWaitEvent(r->h2d, r->in_free[sl], 0);
+    if (ce == cudaSuccess)
+      ce = cudaMemcpyAsync(Qc, static_cast<const uint8_t *>(Q) + q_off * e, hqc * head_elems * e,
+                           cudaMemcpyHostToDevice, r->h2d);
+    if (ce == cudaSuccess)
+      ce = cudaMemcpyAsync(Kc, static_cast<const uint8_t *>(K) + k_off * e, gc * head_elems * e,
+                           cudaMemcpyHostToDevice, r->h2d);
+    if (ce == cudaSuccess)
+      ce = cudaMemcpyAsync(Vc, static_cast<const uint8_t *>(V) + k_off * e, gc * head_elems * e,
+                           cudaMemcpyHostToDevice, r->h2d);
+    if (ce == cudaSuccess) ce = cudaEventRecord(r->in_ready[sl], r->h2d);
+    // compute on `stream`, into output slot sl once chunk c-2's outputs are out
+    if (ce == cudaSuccess) ce = cudaStreamWaitEvent(cs, r->in_ready[sl], 0);
+    if (ce == cudaSuccess && c >= 2) ce = cudaStreamWaitEvent(cs, r->out_free[sl], 0);
+    if (ce != cudaSuccess) {
+      st = BA_ERR_CUDA;
+      break;
+    }
+    ba_att_shape sc = *s;
+    sc.B = 1;
+    sc.Hq = hqc;
+    sc.Hkv = gc;
+    float *qm = reinterpret_cast<float *>(ws + L.qm), *qv = reinterpret_cast<float *>(ws + L.qv);
+    float *km = reinterpret_cast<float *>(ws + L.km), *kv = reinterpret_cast<float *>(ws + L.kv);
+    int32_t *idx = reinterpret_cast<int32_t *>(ws + L.idx), *cnt = reinterpret_cast<int32_t *>(ws + L.cnt);
+    st = ba_att_stats(&sc, Qc, Kc, qm, qv, km, kv, stream);
+    if (st == BA_OK)
+      st = ba_att_select(&sc, keep, qm, qv, km, kv, idx, cnt, L.k, reinterpret_cast<float *>(ws + L.sc), stream);
+    if (st == BA_OK && split_block >= 0) {
+      int32_t *lo_idx = reinterpret_cast<int32_t *>(ws + L.lo_idx), *lo_cnt = reinterpret_cast<int32_t *>(ws + L.lo_cnt);
+      int32_t *hi_idx = reinterpret_cast<int32_t *>(ws + L.hi_idx), *hi_cnt = reinterpret_cast<int32_t *>(ws + L.hi_cnt);
+      float *l1 = reinterpret_cast<float *>(ws + L.l1), *l2 = reinterpret_cast<float *>(ws + L.l2);
+      st = ba_att_split_lists(&sc, split_block, idx, cnt, L.k, lo_idx, lo_cnt, hi_idx, hi_cnt, stream);
+      if (st == BA_OK)
+        st = ba_att_sparse_fwd(&sc, Qc, Kc, Vc, lo_idx, lo_cnt, L.k, ws + L.o1, BA_DTYPE_F32, l1, stream);
+      if (st == BA_OK)
+        st = ba_att_sparse_fwd(&sc, Qc, Kc, Vc, hi_idx, hi_cnt, L.k, ws + L.o2, BA_DTYPE_F32, l2, stream);
+      if (st == BA_OK && cudaEventRecord(r->in_free[sl], cs) != cudaSuccess) st = BA_ERR_CUDA;
+      if (st == BA_OK)
+        st = ba_att_merge_lse(static_cast<int64_t>(hqc) * s->N_alloc, s->d, BA_DTYPE_F32, s->dtype, ws + L.o1, l1,
+                              ws + L.o2, l2, Oc, Lc, stream);
+    } else if (st == BA_OK) {
+      st = ba_att_sparse_fwd(&sc, Qc, Kc, Vc, idx, cnt, L.k, Oc, s->dtype, Lc, stream);
+      if (st == BA_OK && cudaEventRecord(r->in_free[sl], cs) != cudaSuccess) st = BA_ERR_CUDA;
+    }
+    if (st == BA_OK && cudaEventRecord(r->out_ready[sl], cs) != cudaSuccess) st = BA_ERR_CUDA;
+    if (st != BA_OK) break;
+    // outputs of chunk c: the N valid rows of each head
+    ce = cudaStreamWaitEvent(r->d2h, r->out_ready[sl], 0);
+    const size_t pitch_o = head_elems * e, row_o = static_cast<size_t>(s->N) * s->d * e;
+    if (ce == cudaSuccess)
+      ce = cudaMemcpy2DAsync(static_cast<uint8_t *>(O) + q_off * e, pitch_o, Oc, pitch_o, row_o, hqc,
+                             cudaMemcpyDeviceToHost, r->d2h);
+    const size_t pitch_l = static_cast<size_t>(s->N_alloc) * 4, row_l = static_cast<size_t>(s->N) * 4;
+    if (ce == cudaSuccess)
+      ce = cudaMemcpy2DAsync(LSE + (static_cast<size_t>(b) * s->Hq + hq0) * s->N_alloc, pitch_l, Lc, pitch_l, row_l,
+                             hqc, cudaMemcpyDeviceToHost, r->d2h);
+    if (ce == cudaSuccess) ce = cudaEventRecord(r->out_free[sl], r->d2h);
+    if (ce != cudaSuccess) st = BA_ERR_CUDA;
+  }
+  // `stream` passes this call only after both copy streams have drained
+  ce = cudaEventRecord(r->tail, r->h2d);
+  if (ce == cudaSuccess) ce = cudaStreamWaitEvent(cs, r->tail, 0);
+  if (ce == cudaSuccess) ce = cudaEventRecord(r->tail, r->d2h);
+  if (ce == cudaSuccess) ce = cudaStreamWaitEvent(cs, r->tail, 0);
+  if (st == BA_OK && ce != cudaSuccess) st = BA_ERR_CUDA;
+  return st;
 }
 
 }  // extern "C"

@@ -25,7 +25,8 @@
  *  - Grouped-query attention: query head h uses KV head h / (Hq / Hkv).
  *  - Memory: the caller allocates and owns every buffer. Device pointers are
  *    CUDA device (or managed) memory, 16-byte aligned. The library allocates
- *    no device memory; its only global state is one device-side error word.
+ *    no device memory; its global state is one device-side error word and,
+ *    per device, the two copy streams and events of ba_att_forward_host.
  *  - Streams: every call is asynchronous on `stream` (NULL = legacy default
  *    stream) and never synchronises, except ba_att_get_device_error.
  *  - Errors: arguments are checked on the host before anything is launched;
@@ -99,7 +100,8 @@ int32_t ba_att_keep_count(const ba_att_shape *shape, double keep);
  * For every block i and head h, over the valid rows r of the block:
  *   mean[i, m] = (1/n_i) sum_r x[r, m]
  *   var [i, m] = (1/n_i) sum_r (x[r, m] - mean[i, m])^2     (population)
- * computed in fp32 (two passes over register-resident data).
+ * computed in fp32: exact two-pass moments of each thread's register-resident
+ * rows, merged with the pairwise update for centred moments.
  *
  * Q, K      device, [B,Hq|Hkv,N_alloc,d] of shape->dtype; read once.
  * q_mean, q_var   device fp32 [B, Hq,  nq, d]  (written)
@@ -205,6 +207,50 @@ ba_status ba_att_merge_lse(int64_t rows, int32_t d, int32_t in_dtype, int32_t ou
                            const void *O1, const float *L1,
                            const void *O2, const float *L2,
                            void *O, float *L, ba_stream_t stream);
+
+/*
+ * ba_att_forward_host_workspace — device workspace bytes that
+ * ba_att_forward_host needs for this shape, keep, split and chunking; -1 for
+ * arguments ba_att_forward_host would reject.
+ */
+int64_t ba_att_forward_host_workspace(const ba_att_shape *shape, double keep, int32_t split_block,
+                                      int32_t kv_heads_per_chunk);
+
+/*
+ * ba_att_forward_host — the whole BA-Att forward from HOST buffers to HOST
+ * buffers: H2D of Q, K, V; ba_att_stats; ba_att_select; then either one
+ * ba_att_sparse_fwd (split_block < 0), or (split_block >= 0) the key set split
+ * at that key block (FlashBlock Eq. 5), one ba_att_sparse_fwd per span with
+ * fp32 partials, and ba_att_merge_lse (FlashBlock Eq. 9); D2H of O and LSE.
+ * The pages define the operator only; the pipelining is this library's.
+ *
+ * The work is cut into chunks of kv_heads_per_chunk KV heads (with their
+ * Hq/Hkv query heads each) of one batch entry; <= 0 picks about four chunks
+ * per batch entry. Chunk c+1's inputs are copied in, and chunk c-1's outputs
+ * copied out, on two internal non-blocking streams while chunk c computes
+ * on `stream`; every result equals that of the device-resident calls above
+ * bit for bit, as each chunk runs the same kernels on the same heads.
+ *
+ * Q, K, V   host [B, Hq|Hkv, N_alloc, d] of shape->dtype; pinned (page-locked)
+ *           memory lets the copies overlap compute, pageable memory works
+ *           but serialises them.
+ * O         host [B, Hq, N_alloc, d] of shape->dtype; LSE host fp32
+ *           [B, Hq, N_alloc]. Rows n < N of each head are written, padding
+ *           rows are left untouched.
+ * workspace device memory of at least ba_att_forward_host_workspace(...)
+ *           bytes, 256-byte aligned, owned by the caller and not used by
+ *           anything else until `stream` has passed this call.
+ * Returns once everything is enqueued; results are on the host when
+ * `stream` reaches the point of the call (e.g. after cudaStreamSynchronize).
+ * Calls for one device are enqueued one at a time (an internal lock), since
+ * they share the two copy streams. A status other than BA_OK may leave part
+ * of the work enqueued; `stream` still waits for all of it.
+ */
+ba_status ba_att_forward_host(const ba_att_shape *shape, double keep, int32_t split_block,
+                              int32_t kv_heads_per_chunk,
+                              const void *Q, const void *K, const void *V,
+                              void *O, float *LSE,
+                              void *workspace, int64_t workspace_bytes, ba_stream_t stream);
 
 /*
  * ba_att_get_device_error — synchronise `stream`, read the device error word

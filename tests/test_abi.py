@@ -124,3 +124,24 @@ def test_merge_and_selftest_arguments(lib):
     assert lib.ba_att_sparse_fwd(ctypes.byref(s), P, P, P, P, P, 4, P, 2, P, None) == 1
     assert lib.ba_att_selftest_bounded_wait(0, None) == 1
     assert lib.ba_att_selftest_bounded_wait(3_000_000, None) == 1
+
+
+def test_forward_host_arguments(lib):
+    s = shape(N=4096, N_alloc=4096, Hq=8, Hkv=4)
+    ws = lib.ba_att_forward_host_workspace(ctypes.byref(s), ctypes.c_double(0.5), 10, 0)
+    assert ws > 0
+    # split and smaller chunks change the size; bad keep, split past the end, bad shape -> -1
+    assert lib.ba_att_forward_host_workspace(ctypes.byref(s), ctypes.c_double(0.5), -1, 0) < ws
+    assert lib.ba_att_forward_host_workspace(ctypes.byref(s), ctypes.c_double(0.5), 10, 4) > ws
+    assert lib.ba_att_forward_host_workspace(ctypes.byref(s), ctypes.c_double(0.0), 10, 0) == -1
+    assert lib.ba_att_forward_host_workspace(ctypes.byref(s), ctypes.c_double(0.5), 33, 0) == -1
+    assert lib.ba_att_forward_host_workspace(ctypes.byref(shape(d=96)), ctypes.c_double(0.5), -1, 0) == -1
+    W = ctypes.c_void_p(0x100000)                      # 256-byte aligned, never dereferenced
+    call = lambda *a: lib.ba_att_forward_host(ctypes.byref(s), ctypes.c_double(0.5), 10, 0, *a, None)
+    assert call(None, P, P, P, P, W, ws) == 1
+    assert call(P, P, P, P, None, W, ws) == 1
+    assert call(P, P, P, P, P, None, ws) == 1
+    assert call(P, P, P, P, P, W, ws - 1) == 1                             # workspace too small
+    assert call(P, P, P, P, P, ctypes.c_void_p(0x100010), ws) == 3         # workspace not 256-byte aligned
+    assert lib.ba_att_forward_host(ctypes.byref(shape(d=96)), ctypes.c_double(0.5), -1, 0, P, P, P, P, P, W, ws,
+                                   None) == 2

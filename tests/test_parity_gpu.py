@@ -116,9 +116,9 @@ SMALL = [
     ("video_32k", dict(N=600, N_alloc=640, Hq=2, Hkv=2, grid=(3, 10, 20)), 0.5),
     ("dlm_16k", dict(N=1024, Hq=2, Hkv=1, d=64, block=64), 0.5),      # bf16 on the CUDA-core path
     ("tiny_fp32", dict(N=768, d=128, block=32), 0.3),                 # fp32 d=128, block 32
-    ("tiny_fp32", dict(N=9600 - 7, N_alloc=9600, block=16, Hq=2, Hkv=1), 0.5),   # 600 blocks: CUDA-core selector
-    ("dlm_16k", dict(N=64 * 128, Hq=2, Hkv=1), 0.5),                 # 512 blocks: widest tensor-core selector
-    ("dlm_16k", dict(N=300 * 128 - 5, Hq=2, Hkv=2), 0.3),             # 300 blocks: two score tiles, ragged
+    ("tiny_fp32", dict(N=9600 - 7, N_alloc=9600, block=16, Hq=2, Hkv=1), 0.5),   # 600 blocks: 5x5 score tiles
+    ("dlm_16k", dict(N=64 * 128, Hq=2, Hkv=1), 0.5),                 # 512 blocks: 16 keys per lane in the top-k
+    ("dlm_16k", dict(N=300 * 128 - 5, Hq=2, Hkv=2), 0.3),             # 300 blocks: ragged score tiles
 ]
 
 
@@ -180,6 +180,46 @@ def test_split_and_merge_equals_union():
         # against the single pass (its bf16 P and the spans' differ in rounding): the same bar
         assert max_abs(Om, r["O"]) <= tol["max_abs"] and rel_l2(Om, r["O"]) <= tol["rel_l2"]
         assert max_abs(Lm, r["L"]) <= tol["lse_abs"]
+
+
+@pytest.mark.parametrize("name,over,split,chunk", [
+    ("extreme_128k", dict(N=4096 - 50, N_alloc=4096, Hq=8, Hkv=4), True, 0),    # split + merge, 4 chunks of 1
+    ("extreme_128k", dict(N=4096, Hq=8, Hkv=4), False, 3),                      # chunks of 3 + 1 KV heads
+    ("dlm_16k", dict(N=2048, Hq=4, Hkv=2, B=2), True, 2),                       # one chunk per batch entry
+    ("tiny_fp32", dict(N=1000, N_alloc=1024), False, 1),                        # fp32, CUDA-core attention
+])
+def test_forward_host_pipeline(name, over, split, chunk):
+    # host buffers in and out, chunked and pipelined: bit-identical to the
+    # device-resident calls on the same heads, and at the parity bar
+    Q, K, V, meta = make_inputs(name, **over)
+    w = meta["workload"]
+    keep = 0.5
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    Qh, Kh, Vh = (torch.from_numpy(np.ascontiguousarray(x)).to(tdt).pin_memory() for x in (Q, K, V))
+    split_block = meta.get("split_block", w.nb // 2) if split else -1
+    Oh = torch.full(Qh.shape, 7.0, dtype=tdt).pin_memory()              # padding rows must stay untouched
+    Lh = torch.full(Qh.shape[:3], 7.0, dtype=torch.float32).pin_memory()
+    api.forward_host(Qh, Kh, Vh, w.N, w.block, keep, split_block=split_block, kv_heads_per_chunk=chunk, out=(Oh, Lh))
+    torch.cuda.synchronize()
+    # the same steps on device-resident buffers
+    r = run_gpu(Q, K, V, w, keep)
+    if split:
+        lo_i, lo_c, hi_i, hi_c = api.split_lists(r["idx_d"], r["cnt_d"], r["shape"], split_block)
+        O1, L1 = api.sparse_fwd(r["Qd"], r["Kd"], r["Vd"], lo_i, lo_c, r["shape"], out_dtype=torch.float32)
+        O2, L2 = api.sparse_fwd(r["Qd"], r["Kd"], r["Vd"], hi_i, hi_c, r["shape"], out_dtype=torch.float32)
+        Od, Ld = api.merge_lse(O1, L1, O2, L2, out_dtype=tdt)
+    else:
+        Od, Ld = api.sparse_fwd(r["Qd"], r["Kd"], r["Vd"], r["idx_d"], r["cnt_d"], r["shape"])
+    torch.cuda.synchronize()
+    n = w.N
+    assert torch.equal(Oh[:, :, :n], Od[:, :, :n].cpu()), "host pipeline differs from the device-resident calls"
+    assert torch.equal(Lh[:, :, :n], Ld[:, :, :n].cpu())
+    assert (Oh[:, :, n:] == 7.0).all() and (Lh[:, :, n:] == 7.0).all()
+    tol = TOL[w.dtype]
+    Oref, Lref = O.masked_attention(Q, K, V, r["idx"], r["cnt"], w.N, w.block, w.d ** -0.5)
+    got = Oh[:, :, :n].float().numpy()
+    assert max_abs(got, Oref[:, :, :n]) <= tol["max_abs"] and rel_l2(got, Oref[:, :, :n]) <= tol["rel_l2"]
+    assert max_abs(Lh[:, :, :n].numpy(), Lref[:, :, :n]) <= tol["lse_abs"]
 
 
 @pytest.mark.parametrize("dtype,out,d", [("bf16", "bf16", 128), ("f32", "f32", 64), ("bf16", "bf16", 64),
