@@ -50,7 +50,10 @@ _SIGS = {
     "ba_att_forward_host_workspace": (ctypes.c_int64, [ctypes.POINTER(CShape), ctypes.c_double, _I32, _I32]),
     "ba_att_forward_host": (ctypes.c_int, [ctypes.POINTER(CShape), ctypes.c_double, _I32, _I32, _P, _P, _P, _P, _P,
                                             _P, ctypes.c_int64, _P]),
+    "ba_att_forward_host_noalloc": (ctypes.c_int, [ctypes.POINTER(CShape), ctypes.c_double, _I32, _P, _P, _P, _P,
+                                                    _P, _P]),
 }
+STATIC_SCRATCH_BYTES = 512 << 20      # BA_ATT_STATIC_SCRATCH_BYTES
 
 _lib = None
 _lock = threading.Lock()
@@ -284,6 +287,25 @@ def forward_host(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, N: int, bloc
                                    _host(Q, "Q"), _host(K, "K"), _host(V, "V"), _host(O, "O"), _host(LSE, "LSE"),
                                    ctypes.c_void_p(workspace.data_ptr()), int(workspace.numel() * workspace.element_size()),
                                    ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)))
+    return O, LSE
+
+
+def forward_host_noalloc(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, N: int, block: int, keep: float,
+                         split_block: int = -1, sm_scale: float = 0.0, out=None, device=None):
+    """forward_host on the library's static device scratch (ba_att_forward_host_noalloc):
+    no workspace argument, nothing allocated on the device by this call."""
+    shape = Shape.of(Q, K, N, block, sm_scale)
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    if out is None:
+        O = torch.empty(Q.shape, dtype=Q.dtype).pin_memory()
+        LSE = torch.empty(Q.shape[:3], dtype=torch.float32).pin_memory()
+    else:
+        O, LSE = out
+    lib = load_library()
+    _check("ba_att_forward_host_noalloc",
+           lib.ba_att_forward_host_noalloc(ctypes.byref(shape.c()), float(keep), int(split_block), _host(Q, "Q"),
+                                           _host(K, "K"), _host(V, "V"), _host(O, "O"), _host(LSE, "LSE"),
+                                           ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)))
     return O, LSE
 
 

@@ -398,6 +398,8 @@ struct PipeResources {
   cudaEvent_t entry = nullptr, tail = nullptr;
   cudaEvent_t in_ready[2] = {nullptr, nullptr}, in_free[2] = {nullptr, nullptr};
   cudaEvent_t out_ready[2] = {nullptr, nullptr}, out_free[2] = {nullptr, nullptr};
+  cudaEvent_t scratch_free = nullptr;     // end of the last call on the static scratch
+  bool scratch_used = false;
 };
 
 PipeResources *pipe_resources(int dev) {
@@ -410,7 +412,7 @@ cudaError_t pipe_init(PipeResources *r) {
   cudaError_t e = cudaStreamCreateWithFlags(&r->h2d, cudaStreamNonBlocking);
   if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&r->d2h, cudaStreamNonBlocking);
   cudaEvent_t *evs[] = {&r->entry, &r->tail, &r->in_ready[0], &r->in_ready[1], &r->in_free[0], &r->in_free[1],
-                        &r->out_ready[0], &r->out_ready[1], &r->out_free[0], &r->out_free[1]};
+                        &r->out_ready[0], &r->out_ready[1], &r->out_free[0], &r->out_free[1], &r->scratch_free};
   for (cudaEvent_t *ev : evs)
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
   if (e == cudaSuccess) r->ready = true;
@@ -428,23 +430,15 @@ int64_t ba_att_forward_host_workspace(const ba_att_shape *s, double keep, int32_
   return static_cast<int64_t>(L.total);
 }
 
-ba_status ba_att_forward_host(const ba_att_shape *s, double keep, int32_t split_block, int32_t kv_heads_per_chunk,
-                              const void *Q, const void *K, const void *V, void *O, float *LSE, void *workspace,
-                              int64_t workspace_bytes, ba_stream_t stream) {
-  PipeLayout L;
-  ba_status st = check_shape(s);
-  if (st != BA_OK) return st;
-  if (!pipe_layout(s, keep, split_block, kv_heads_per_chunk, &L)) return BA_ERR_INVALID_ARG;
-  if (!Q || !K || !V || !O || !LSE || !workspace) return BA_ERR_INVALID_ARG;
-  if (workspace_bytes < static_cast<int64_t>(L.total)) return BA_ERR_INVALID_ARG;
-  if (reinterpret_cast<uintptr_t>(workspace) % kWsAlign != 0) return BA_ERR_MISALIGNED;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return BA_ERR_CUDA;
-  PipeResources *r = pipe_resources(dev);
-  if (r == nullptr) return BA_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> guard(r->lock);
-  if (pipe_init(r) != cudaSuccess) return BA_ERR_CUDA;
+}  // extern "C"
 
+namespace {
+
+// The pipeline proper; arguments already validated, r->lock held.
+ba_status forward_host_impl(PipeResources *r, const ba_att_shape *s, double keep, int32_t split_block,
+                            const PipeLayout &L, const void *Q, const void *K, const void *V, void *O, float *LSE,
+                            void *workspace, ba_stream_t stream) {
+  ba_status st = BA_OK;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   const size_t e = s->dtype == BA_DTYPE_BF16 ? 2 : 4;
@@ -536,6 +530,83 @@ ba_status ba_att_forward_host(const ba_att_shape *s, double keep, int32_t split_
   if (ce == cudaSuccess) ce = cudaEventRecord(r->tail, r->d2h);
   if (ce == cudaSuccess) ce = cudaStreamWaitEvent(cs, r->tail, 0);
   if (st == BA_OK && ce != cudaSuccess) st = BA_ERR_CUDA;
+  return st;
+}
+
+ba_status validate_host_call(const ba_att_shape *s, double keep, int32_t split_block, int32_t chunk, const void *Q,
+                             const void *K, const void *V, const void *O, const float *LSE, PipeLayout *L) {
+  ba_status st = check_shape(s);
+  if (st != BA_OK) return st;
+  if (!pipe_layout(s, keep, split_block, chunk, L)) return BA_ERR_INVALID_ARG;
+  if (!Q || !K || !V || !O || !LSE) return BA_ERR_INVALID_ARG;
+  return BA_OK;
+}
+
+PipeResources *lock_pipe(std::unique_lock<std::mutex> &guard, ba_status *st) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    *st = BA_ERR_CUDA;
+    return nullptr;
+  }
+  PipeResources *r = pipe_resources(dev);
+  if (r == nullptr) {
+    *st = BA_ERR_UNSUPPORTED;
+    return nullptr;
+  }
+  guard = std::unique_lock<std::mutex>(r->lock);
+  if (pipe_init(r) != cudaSuccess) {
+    *st = BA_ERR_CUDA;
+    return nullptr;
+  }
+  return r;
+}
+
+// Scratch of ba_att_forward_host_noalloc: static device memory of the
+// module, reserved when the module loads; nothing is allocated per call.
+__device__ __align__(256) uint8_t g_static_scratch[BA_ATT_STATIC_SCRATCH_BYTES];
+
+}  // namespace
+
+extern "C" {
+
+ba_status ba_att_forward_host(const ba_att_shape *s, double keep, int32_t split_block, int32_t kv_heads_per_chunk,
+                              const void *Q, const void *K, const void *V, void *O, float *LSE, void *workspace,
+                              int64_t workspace_bytes, ba_stream_t stream) {
+  PipeLayout L;
+  ba_status st = validate_host_call(s, keep, split_block, kv_heads_per_chunk, Q, K, V, O, LSE, &L);
+  if (st != BA_OK) return st;
+  if (!workspace || workspace_bytes < static_cast<int64_t>(L.total)) return BA_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(workspace) % kWsAlign != 0) return BA_ERR_MISALIGNED;
+  std::unique_lock<std::mutex> guard;
+  PipeResources *r = lock_pipe(guard, &st);
+  if (r == nullptr) return st;
+  return forward_host_impl(r, s, keep, split_block, L, Q, K, V, O, LSE, workspace, stream);
+}
+
+ba_status ba_att_forward_host_noalloc(const ba_att_shape *s, double keep, int32_t split_block, const void *Q,
+                                      const void *K, const void *V, void *O, float *LSE, ba_stream_t stream) {
+  PipeLayout L;
+  ba_status st = validate_host_call(s, keep, split_block, 0, Q, K, V, O, LSE, &L);
+  if (st != BA_OK) return st;
+  // the widest chunk whose workspace fits the static scratch
+  int chunk = s->Hkv;
+  for (; chunk >= 1; --chunk) {
+    if (!pipe_layout(s, keep, split_block, chunk, &L)) return BA_ERR_INVALID_ARG;
+    if (L.total <= static_cast<size_t>(BA_ATT_STATIC_SCRATCH_BYTES)) break;
+  }
+  if (chunk < 1) return BA_ERR_UNSUPPORTED;
+  std::unique_lock<std::mutex> guard;
+  PipeResources *r = lock_pipe(guard, &st);
+  if (r == nullptr) return st;
+  void *scratch = nullptr;
+  if (cudaGetSymbolAddress(&scratch, g_static_scratch) != cudaSuccess) return BA_ERR_CUDA;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  // one scratch per device: a call starts after the previous call on it ended,
+  // whatever stream that call used
+  if (r->scratch_used && cudaStreamWaitEvent(cs, r->scratch_free, 0) != cudaSuccess) return BA_ERR_CUDA;
+  st = forward_host_impl(r, s, keep, split_block, L, Q, K, V, O, LSE, scratch, stream);
+  if (cudaEventRecord(r->scratch_free, cs) != cudaSuccess && st == BA_OK) st = BA_ERR_CUDA;
+  r->scratch_used = true;
   return st;
 }
 

@@ -252,6 +252,29 @@ ba_status ba_att_forward_host(const ba_att_shape *shape, double keep, int32_t sp
                               void *O, float *LSE,
                               void *workspace, int64_t workspace_bytes, ba_stream_t stream);
 
+/* Size of the library's static device scratch (ba_att_forward_host_noalloc). */
+#define BA_ATT_STATIC_SCRATCH_BYTES (512ull << 20)
+
+/*
+ * ba_att_forward_host_noalloc — ba_att_forward_host without a workspace
+ * argument. The pages have no counterpart: this is a deployment variant of
+ * the same computation.
+ *
+ * The workspace is a static __device__ array of BA_ATT_STATIC_SCRATCH_BYTES
+ * inside the library (reserved once, when the library's device code is
+ * loaded; nothing is allocated at call time). The chunk is the largest number
+ * of KV heads whose workspace (ba_att_forward_host_workspace) fits it;
+ * BA_ERR_UNSUPPORTED when one KV head per chunk does not fit (e.g. 32 query
+ * heads per KV head at N = 128K with a split). Results are bit-identical to
+ * ba_att_forward_host. The scratch is shared by all calls on a device: each
+ * call starts on `stream` only after the previous call on the scratch has
+ * ended, whatever stream that call used.
+ * Arguments as for ba_att_forward_host.
+ */
+ba_status ba_att_forward_host_noalloc(const ba_att_shape *shape, double keep, int32_t split_block,
+                                      const void *Q, const void *K, const void *V,
+                                      void *O, float *LSE, ba_stream_t stream);
+
 /*
  * ba_att_get_device_error — synchronise `stream`, read the device error word
  * of the current device, clear it, and return BA_OK (word 0), BA_ERR_TIMEOUT
