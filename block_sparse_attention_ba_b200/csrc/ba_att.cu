@@ -340,7 +340,13 @@ struct PipeLayout {
   size_t total = 0;
 };
 
-int auto_chunk(const ba_att_shape *s) { return s->Hkv >= 4 ? s->Hkv / 4 : 1; }
+// Fewest KV heads per chunk that still give the attention kernel about 1024
+// (query head, query block) tiles, a few waves of the GPU's CTA slots.
+int auto_chunk(const ba_att_shape *s) {
+  const long long tiles_per_kv_head = static_cast<long long>(s->Hq / s->Hkv) * nblocks(s);
+  const long long c = (1024 + tiles_per_kv_head - 1) / tiles_per_kv_head;
+  return static_cast<int>(c < 1 ? 1 : (c > s->Hkv ? s->Hkv : c));
+}
 
 bool pipe_layout(const ba_att_shape *s, double keep, int32_t split_block, int32_t chunk, PipeLayout *L) {
   if (check_shape(s) != BA_OK) return false;

@@ -225,8 +225,8 @@ int64_t ba_att_forward_host_workspace(const ba_att_shape *shape, double keep, in
  * The pages define the operator only; the pipelining is this library's.
  *
  * The work is cut into chunks of kv_heads_per_chunk KV heads (with their
- * Hq/Hkv query heads each) of one batch entry; <= 0 picks about four chunks
- * per batch entry. Chunk c+1's inputs are copied in, and chunk c-1's outputs
+ * Hq/Hkv query heads each) of one batch entry; <= 0 picks the fewest KV heads
+ * that give about 1024 (query head, query block) tiles per chunk. Chunk c+1's inputs are copied in, and chunk c-1's outputs
  * copied out, on two internal non-blocking streams while chunk c computes
  * on `stream`; every result equals that of the device-resident calls above
  * bit for bit, as each chunk runs the same kernels on the same heads.

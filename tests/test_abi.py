@@ -130,9 +130,11 @@ def test_forward_host_arguments(lib):
     s = shape(N=4096, N_alloc=4096, Hq=8, Hkv=4)
     ws = lib.ba_att_forward_host_workspace(ctypes.byref(s), ctypes.c_double(0.5), 10, 0)
     assert ws > 0
-    # split and smaller chunks change the size; bad keep, split past the end, bad shape -> -1
+    # no split and smaller chunks need less (auto: every KV head in one chunk here, 64 tiles each);
+    # bad keep, split past the end, bad shape -> -1
     assert lib.ba_att_forward_host_workspace(ctypes.byref(s), ctypes.c_double(0.5), -1, 0) < ws
-    assert lib.ba_att_forward_host_workspace(ctypes.byref(s), ctypes.c_double(0.5), 10, 4) > ws
+    assert lib.ba_att_forward_host_workspace(ctypes.byref(s), ctypes.c_double(0.5), 10, 4) == ws
+    assert lib.ba_att_forward_host_workspace(ctypes.byref(s), ctypes.c_double(0.5), 10, 1) < ws
     assert lib.ba_att_forward_host_workspace(ctypes.byref(s), ctypes.c_double(0.0), 10, 0) == -1
     assert lib.ba_att_forward_host_workspace(ctypes.byref(s), ctypes.c_double(0.5), 33, 0) == -1
     assert lib.ba_att_forward_host_workspace(ctypes.byref(shape(d=96)), ctypes.c_double(0.5), -1, 0) == -1
