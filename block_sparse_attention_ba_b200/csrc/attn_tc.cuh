@@ -11,17 +11,22 @@
 // softmax overlaps the other CTA's MMAs. Roles (192 threads):
 //   warps 0-3  softmax + correction + epilogue; thread t owns query row t,
 //              i.e. TMEM lane t (a warp may only touch its own 32 lanes)
-//   warp 4     TMA producer (lane 0) and TMEM allocator (whole warp)
+//   warp 4     TMA producers (lane 0: Q and K, lane 1: V), TMEM allocator
 //   warp 5     MMA issuer (lane 0)
-// Per kept block j (list order):
-//   TMA:  K_j, V_j  -> shared memory, 128B-swizzled, one 2-D box per 64 dims
-//   MMA:  S = Q K_j^T               (SS form, fp32 accumulator in TMEM cols 0-127)
-//   SM :  P = exp2(s*log2e*S - m) as bf16, written back over S (cols 0-63);
-//         running max m only moves when it grows by more than 2^8, and only
-//         then is O (TMEM cols 128-255) rescaled
-//   MMA:  O += P V_j                (TS form: A = P from TMEM, B = V MN-major)
-// Because the key blocks are whole 128-row slabs of K and V, the "gather" of
-// the selected blocks is one tile load per block at the block's coordinate.
+// Each kept block j (list order) is taken as two 64-key halves, u = 2j + h,
+// with their own S columns (h*64 .. h*64+63), so the tensor cores compute
+// the next half's scores while the softmax warps work on this half:
+//   MMA:  S_u = Q K_u^T             (SS form, N = 64, fp32 in TMEM)
+//   SM :  P_u = exp2(s*log2e*S_u - m) as bf16, written back over S_u's first
+//         32 columns; the running max m only moves when it grows by more than
+//         2^8, and only then is O (TMEM cols 128-255) rescaled, after the
+//         MMA that last wrote O has completed
+//   MMA:  O += P_u V_u              (TS form: A = P from TMEM, B = V MN-major)
+// in the order S_0 S_1 PV_0 S_2 PV_1 S_3 ...: S_{u+2} reuses P_u's columns,
+// so it is issued after PV_u. K and V halves are loaded as separate 64-row
+// boxes with their own full/empty barriers. Because the key blocks are whole
+// 128-row slabs of K and V, the "gather" of the selected blocks is one tile
+// load per half block at the block's coordinate.
 // Every barrier wait is bounded; a stuck pipeline sets an error bit and the
 // CTA drains its copies and MMAs, frees TMEM and exits.
 #pragma once
@@ -41,8 +46,18 @@ constexpr uint32_t kDynSmem = 3 * kTileBytes + 1024; // + alignment slack
 constexpr int kTmemCols = 256;
 constexpr uint32_t kColS = 0, kColO = 128;
 constexpr float kRescaleLog2 = 8.0f;
+constexpr int kHalfKeys = 64;                        // keys per half block
+constexpr int kKvBoxRows = kHalfKeys;                // K/V tensor-map box: 64 dims x 64 rows
+constexpr uint32_t kHalfRowsBytes = kHalfKeys * 128; // 64 rows of one 64-dim span
 
-enum Bar { Q_FULL = 0, K_FULL, K_EMPTY, V_FULL, V_EMPTY, S_FULL, P_FULL, O_FINAL, DRAIN, NUM_BARS };
+// Barriers with a [2] suffix come in two, one per key half h.
+enum Bar {
+  Q_FULL = 0,
+  K_FULL0, K_FULL1, K_EMPTY0, K_EMPTY1,
+  V_FULL0, V_FULL1, V_EMPTY0, V_EMPTY1,
+  S_FULL0, S_FULL1, P_FULL0, P_FULL1, PV_DONE0, PV_DONE1,
+  O_FINAL, DRAIN, NUM_BARS
+};
 
 struct Ctl {
   uint64_t bar[NUM_BARS];
@@ -59,31 +74,33 @@ __device__ __forceinline__ bool entry_ok(const int32_t *list, int t, int nb, int
   return true;
 }
 
-// P = 2^(s*scale_log2 - m) for one row: packed to bf16 pairs and stored
-// over the S columns 64 keys at a time; the fp32 values are summed into 8
-// independent partial sums. (Evaluating a share of the exponentials on the
-// FMA pipe instead of MUFU was measured slower here: issue slots, not MUFU
-// throughput, bound this loop.)
-__device__ __forceinline__ void exp_pack_store(const uint32_t (&sr)[4][32], float scale_log2, float negm,
+// P = 2^(s*scale_log2 - m) for one row's 64 keys of a half block: packed to
+// bf16 pairs and stored over the first 32 of its S columns. The scale and
+// shift and the running sums use the packed .f32x2 instructions (two keys per
+// instruction, four packed partial sums); the exponentials run on MUFU.
+// (Evaluating a share of them on the FMA pipe instead was measured slower
+// here: issue slots, not MUFU throughput, bound this loop.)
+__device__ __forceinline__ void exp_pack_store(const uint32_t (&sr)[2][32], float scale_log2, float negm,
                                                float (&acc)[8], uint32_t tS) {
+  uint32_t pk[32];
+  const uint64_t sc2 = pack_f32x2(scale_log2, scale_log2), nm2 = pack_f32x2(negm, negm);
+  uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    uint32_t pk[32];
+  for (int q = 0; q < 2; ++q) {
 #pragma unroll
-    for (int qq = 0; qq < 2; ++qq) {
-      const int q = 2 * half + qq;
-#pragma unroll
-      for (int c = 0; c < 32; c += 2) {
-        const float x0 = fmaf(__uint_as_float(sr[q][c]), scale_log2, negm);
-        const float x1 = fmaf(__uint_as_float(sr[q][c + 1]), scale_log2, negm);
-        const float p0 = ex2_approx(x0);
-        const float p1 = ex2_approx(x1);
-        acc[c & 7] += p0;
-        acc[(c & 7) + 1] += p1;
-        pk[qq * 16 + (c >> 1)] = pack_bf16x2(p0, p1);
-      }
+    for (int c = 0; c < 32; c += 2) {
+      const uint64_t x2 = fma_f32x2(pack_u32x2(sr[q][c], sr[q][c + 1]), sc2, nm2);
+      const float p0 = ex2_approx(lo_f32(x2));
+      const float p1 = ex2_approx(hi_f32(x2));
+      acc2[(c >> 1) & 3] = add_f32x2(acc2[(c >> 1) & 3], pack_f32x2(p0, p1));
+      pk[q * 16 + (c >> 1)] = pack_bf16x2(p0, p1);
     }
-    tmem_st32(tS + half * 32, pk);
+  }
+  tmem_st32(tS, pk);
+#pragma unroll
+  for (int a = 0; a < 4; ++a) {
+    acc[2 * a] += lo_f32(acc2[a]);
+    acc[2 * a + 1] += hi_f32(acc2[a]);
   }
 }
 
@@ -122,7 +139,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
 
   if (threadIdx.x == 0) {
-    for (int k = 0; k < NUM_BARS; ++k) mbar_init(smem_u32(&ctl.bar[k]), k == P_FULL ? 128u : 1u);
+    for (int k = 0; k < NUM_BARS; ++k) mbar_init(smem_u32(&ctl.bar[k]), (k == P_FULL0 || k == P_FULL1) ? 128u : 1u);
     ctl.abort = 0;
     fence_mbar_init();
   }
@@ -140,15 +157,22 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int qz = b * Hq + h;          // row of the [B*H] head axis in the tensor maps
   const int kz = b * Hkv + g;
 
-  if (cnt > 0 && warp == 4 && lane == 0) {
-    // ------------------------------------------------------------ producer
-    tma_prefetch_desc(&tm_q);
-    tma_prefetch_desc(&tm_k);
-    tma_prefetch_desc(&tm_v);
-    mbar_arrive_expect_tx(bar(Q_FULL), kTileBytes);
-    tma_load_3d(&tm_q, sQ, bar(Q_FULL), 0, i * kTileRows, qz);
-    tma_load_3d(&tm_q, sQ + kHalfBytes, bar(Q_FULL), 64, i * kTileRows, qz);
-    int k_issued = -1, v_issued = -1;
+  if (cnt > 0 && warp == 4 && lane < 2) {
+    // ------------------------------------------------------------ producers
+    // lane 0: Q, then the K halves; lane 1: the V halves. Half h of block t
+    // reuses the slot rows of half h of block t-1 once its MMAs are done.
+    const bool is_k = lane == 0;
+    const CUtensorMap *tm = is_k ? &tm_k : &tm_v;
+    const uint32_t slot = is_k ? sK : sV;
+    const int full0 = is_k ? K_FULL0 : V_FULL0, empty0 = is_k ? K_EMPTY0 : V_EMPTY0;
+    tma_prefetch_desc(tm);
+    if (is_k) {
+      tma_prefetch_desc(&tm_q);
+      mbar_arrive_expect_tx(bar(Q_FULL), kTileBytes);
+      tma_load_3d(&tm_q, sQ, bar(Q_FULL), 0, i * kTileRows, qz);
+      tma_load_3d(&tm_q, sQ + kHalfBytes, bar(Q_FULL), 64, i * kTileRows, qz);
+    }
+    int issued = -1;                    // last half-block index u loaded
     bool bad_index = false, bad_order = false;
     for (int t = 0; t < cnt; ++t) {
       int j;
@@ -157,50 +181,65 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (raw < 0 || raw >= nb) bad_index = true; else bad_order = true;
         j = 0;                            // load a valid block; softmax masks it out
       }
-      if (t > 0 && !mbar_wait_bounded(bar(K_EMPTY), (t - 1) & 1, abort)) break;
-      mbar_arrive_expect_tx(bar(K_FULL), kTileBytes);
-      tma_load_3d(&tm_k, sK, bar(K_FULL), 0, j * kTileRows, kz);
-      tma_load_3d(&tm_k, sK + kHalfBytes, bar(K_FULL), 64, j * kTileRows, kz);
-      k_issued = t;
-      if (t > 0 && !mbar_wait_bounded(bar(V_EMPTY), (t - 1) & 1, abort)) break;
-      mbar_arrive_expect_tx(bar(V_FULL), kTileBytes);
-      tma_load_3d(&tm_v, sV, bar(V_FULL), 0, j * kTileRows, kz);
-      tma_load_3d(&tm_v, sV + kHalfBytes, bar(V_FULL), 64, j * kTileRows, kz);
-      v_issued = t;
+      bool stop = false;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        if (t > 0 && !mbar_wait_bounded(bar(empty0 + h), (t - 1) & 1, abort)) {
+          stop = true;
+          break;
+        }
+        mbar_arrive_expect_tx(bar(full0 + h), 2 * kHalfRowsBytes);
+        const int row = j * kTileRows + h * kHalfKeys;
+        tma_load_3d(tm, slot + h * kHalfRowsBytes, bar(full0 + h), 0, row, kz);
+        tma_load_3d(tm, slot + kHalfBytes + h * kHalfRowsBytes, bar(full0 + h), 64, row, kz);
+        issued = 2 * t + h;
+      }
+      if (stop) break;
     }
-    if (bad_index) raise_error(BA_DEVERR_BAD_INDEX);
-    if (bad_order) raise_error(BA_DEVERR_NOT_ASCENDING);
+    if (is_k && bad_index) raise_error(BA_DEVERR_BAD_INDEX);
+    if (is_k && bad_order) raise_error(BA_DEVERR_NOT_ASCENDING);
     if (*abort) {
       // let copies in flight land before the CTA's shared memory goes away
-      if (k_issued >= 0) mbar_wait_bounded(bar(K_FULL), k_issued & 1, nullptr);
-      if (v_issued >= 0) mbar_wait_bounded(bar(V_FULL), v_issued & 1, nullptr);
-      mbar_wait_bounded(bar(Q_FULL), 0, nullptr);
+      // (the newest load of each half)
+      for (int u = issued; u >= 0 && u > issued - 2; --u) mbar_wait_bounded(bar(full0 + (u & 1)), (u >> 1) & 1, nullptr);
+      if (is_k) mbar_wait_bounded(bar(Q_FULL), 0, nullptr);
     }
   } else if (cnt > 0 && warp == 5 && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
-    constexpr uint32_t idesc_qk = idesc_bf16_f32(128, 128, 0, 0);
+    constexpr uint32_t idesc_qk = idesc_bf16_f32(128, kHalfKeys, 0, 0);
     constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 128, 0, 1);
-    bool ok = mbar_wait_bounded(bar(Q_FULL), 0, abort);
-    for (int t = 0; ok && t < cnt; ++t) {
-      if (!mbar_wait_bounded(bar(K_FULL), t & 1, abort)) break;
+    const int n_half = 2 * cnt;
+    // S_u = Q K_u^T into S columns h*64..h*64+63
+    auto issue_s = [&](int u) -> bool {
+      const int h = u & 1;
+      if (!mbar_wait_bounded(bar(K_FULL0 + h), (u >> 1) & 1, abort)) return false;
       tc_fence_after();
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {            // K = 128 = 8 x 16
         const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
-        mma_ss(tmem + kColS, smem_desc_sw128(sQ + off, 16, 1024), smem_desc_sw128(sK + off, 16, 1024), idesc_qk,
-               kk > 0 ? 1u : 0u);
+        mma_ss(tmem + kColS + h * kHalfKeys, smem_desc_sw128(sQ + off, 16, 1024),
+               smem_desc_sw128(sK + off + h * kHalfRowsBytes, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
       }
-      mma_commit(bar(S_FULL));
-      mma_commit(bar(K_EMPTY));
-      if (!mbar_wait_bounded(bar(V_FULL), t & 1, abort)) break;
-      if (!mbar_wait_bounded(bar(P_FULL), t & 1, abort)) break;
+      mma_commit(bar(S_FULL0 + h));
+      mma_commit(bar(K_EMPTY0 + h));
+      return true;
+    };
+    bool ok = mbar_wait_bounded(bar(Q_FULL), 0, abort);
+    if (ok) ok = issue_s(0);
+    if (ok && n_half > 1) ok = issue_s(1);
+    for (int u = 0; ok && u < n_half; ++u) {
+      const int h = u & 1;
+      if (!mbar_wait_bounded(bar(V_FULL0 + h), (u >> 1) & 1, abort)) break;
+      if (!mbar_wait_bounded(bar(P_FULL0 + h), (u >> 1) & 1, abort)) break;
       tc_fence_after();
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {            // 128 keys = 8 x 16; P packs 2 keys per column
-        mma_ts(tmem + kColO, tmem + kColS + kk * 8, smem_desc_sw128(sV + kk * 2048, kHalfBytes, 1024), idesc_pv,
-               (t > 0 || kk > 0) ? 1u : 0u);
+      for (int kk = 0; kk < 4; ++kk) {            // 64 keys = 4 x 16; P packs 2 keys per column
+        mma_ts(tmem + kColO, tmem + kColS + h * kHalfKeys + kk * 8,
+               smem_desc_sw128(sV + (4 * h + kk) * 2048, kHalfBytes, 1024), idesc_pv, (u > 0 || kk > 0) ? 1u : 0u);
       }
-      mma_commit(bar(V_EMPTY));
+      mma_commit(bar(V_EMPTY0 + h));
+      mma_commit(bar(PV_DONE0 + h));
+      if (u + 2 < n_half && !issue_s(u + 2)) break;   // after PV_u: S_{u+2} overwrites P_u
     }
     mma_commit(bar(O_FINAL));
     mma_commit(bar(DRAIN));
@@ -214,35 +253,41 @@ __global__ void __launch_bounds__(kThreads, 2)
     const long long orow = static_cast<long long>(qz) * N_alloc + qrow;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int t = 0; t < cnt; ++t) {
-      int j;
-      const bool valid = entry_ok(list, t, nb, j);
-      const int n_keys = valid ? min(kTileRows, N - j * kTileRows) : 0;
-      bool w = mbar_wait_bounded(bar(S_FULL), t & 1, abort);
+    int n_keys = 0;
+    for (int u = 0; u < 2 * cnt; ++u) {
+      const int h = u & 1;
+      if (h == 0) {
+        int j;
+        const bool valid = entry_ok(list, u >> 1, nb, j);
+        n_keys = valid ? min(kTileRows, N - j * kTileRows) : 0;
+      }
+      const int n_half = min(max(n_keys - h * kHalfKeys, 0), kHalfKeys);
+      bool w = mbar_wait_bounded(bar(S_FULL0 + h), (u >> 1) & 1, abort);
       if (!__all_sync(0xFFFFFFFFu, w)) { ok = false; break; }
       tc_fence_after();
-      uint32_t sr[4][32];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) tmem_ld32(tS + q * 32, sr[q]);
+      const uint32_t tSu = tS + h * kHalfKeys;
+      uint32_t sr[2][32];
+      tmem_ld32(tSu, sr[0]);
+      tmem_ld32(tSu + 32, sr[1]);
       tmem_ld_wait();
-      if (n_keys < kTileRows) {                        // ragged last block or a skipped entry (rare)
+      if (n_half < kHalfKeys) {                        // ragged last block or a skipped entry (rare)
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < 2; ++q) {
 #pragma unroll
           for (int c = 0; c < 32; ++c)
-            if (q * 32 + c >= n_keys) sr[q][c] = __float_as_uint(-INFINITY);
+            if (q * 32 + c >= n_half) sr[q][c] = __float_as_uint(-INFINITY);
         }
       }
-      // Row max of the raw scores: 4 independent chains of 3-input max.
-      float mxp[4];
+      // Row max of the raw scores: 2 independent chains of 3-input max.
+      float mxp[2];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < 2; ++q) {
         mxp[q] = fmaxf(__uint_as_float(sr[q][0]), __uint_as_float(sr[q][31]));
 #pragma unroll
         for (int c = 1; c < 31; c += 2)
           mxp[q] = fmax3(mxp[q], __uint_as_float(sr[q][c]), __uint_as_float(sr[q][c + 1]));
       }
-      const float mx = fmaxf(fmax3(mxp[0], mxp[1], mxp[2]), mxp[3]) * scale_log2;   // scale > 0 keeps the order
+      const float mx = fmaxf(mxp[0], mxp[1]) * scale_log2;   // scale > 0 keeps the order
       float alpha = 1.f;
       bool rescale = false;
       if (mx - m_used > kRescaleLog2) {                // false when both are -inf
@@ -251,14 +296,17 @@ __global__ void __launch_bounds__(kThreads, 2)
         rescale = true;
       }
       const float m_ref = (m_used == -INFINITY) ? 0.f : m_used;
-      // p = 2^(s*scale_log2 - m): one packed FMA per pair, 8 independent
-      // packed partial sums.
       const float negm = -m_ref;
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      exp_pack_store(sr, scale_log2, negm, acc, tS);
+      exp_pack_store(sr, scale_log2, negm, acc, tSu);
       l = l * alpha + (((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7])));
-      if (t > 0 && __any_sync(0xFFFFFFFFu, rescale)) {
-        // O holds blocks 0..t-1 (their MMAs completed before S_t did)
+      if (u > 0 && __any_sync(0xFFFFFFFFu, rescale)) {
+        // O holds halves 0..u-1 once PV_{u-1} has completed (PV_{u-2} did
+        // before S_u was issued)
+        const int v = u - 1;
+        w = mbar_wait_bounded(bar(PV_DONE0 + (v & 1)), (v >> 1) & 1, abort);
+        if (!__all_sync(0xFFFFFFFFu, w)) { ok = false; break; }
+        tc_fence_after();
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           uint32_t orr[32];
@@ -271,7 +319,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(bar(P_FULL));
+      mbar_arrive(bar(P_FULL0 + h));
     }
     if (cnt == 0) {
       if (qrow < N) {

@@ -83,13 +83,14 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// [BH, rows, d] bf16 head-major tensor; rows >= N_valid read as zeros.
-bool make_head_map(CUtensorMap *map, const void *ptr, int d, int N_valid, int N_alloc, long long BH) {
+// [BH, rows, d] bf16 head-major tensor read in boxes of 64 dims x box_rows
+// rows; rows >= N_valid read as zeros.
+bool make_head_map(CUtensorMap *map, const void *ptr, int d, int N_valid, int N_alloc, long long BH, int box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N_valid), static_cast<cuuint64_t>(BH)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2u, static_cast<cuuint64_t>(N_alloc) * d * 2u};
-  cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(tc::kTileRows), 1u};
+  cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(box_rows), 1u};
   cuuint32_t estr[3] = {1u, 1u, 1u};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -233,9 +234,9 @@ ba_status ba_att_sparse_fwd(const ba_att_shape *s, const void *Q, const void *K,
   const bool out_f32 = (o_dtype == BA_DTYPE_F32);
   if (use_tensor_core_path(s)) {
     CUtensorMap mq, mk, mv;
-    if (!make_head_map(&mq, Q, s->d, s->N, s->N_alloc, static_cast<long long>(s->B) * s->Hq) ||
-        !make_head_map(&mk, K, s->d, s->N, s->N_alloc, static_cast<long long>(s->B) * s->Hkv) ||
-        !make_head_map(&mv, V, s->d, s->N, s->N_alloc, static_cast<long long>(s->B) * s->Hkv))
+    if (!make_head_map(&mq, Q, s->d, s->N, s->N_alloc, static_cast<long long>(s->B) * s->Hq, tc::kTileRows) ||
+        !make_head_map(&mk, K, s->d, s->N, s->N_alloc, static_cast<long long>(s->B) * s->Hkv, tc::kKvBoxRows) ||
+        !make_head_map(&mv, V, s->d, s->N, s->N_alloc, static_cast<long long>(s->B) * s->Hkv, tc::kKvBoxRows))
       return BA_ERR_CUDA;
     const long long tiles = static_cast<long long>(s->B) * s->Hq * nb;
     if (tiles > 0x7FFFFFFFLL) return BA_ERR_UNSUPPORTED;

@@ -177,9 +177,10 @@ def test_split_and_merge_equals_union():
         assert max_abs(Om, Oref) <= tol["max_abs"], max_abs(Om, Oref)
         assert rel_l2(Om, Oref) <= tol["rel_l2"]
         assert max_abs(Lm, Lref) <= tol["lse_abs"]
-        # against the single pass (its bf16 P and the spans' differ in rounding): the same bar
-        assert max_abs(Om, r["O"]) <= tol["max_abs"] and rel_l2(Om, r["O"]) <= tol["rel_l2"]
-        assert max_abs(Lm, r["L"]) <= tol["lse_abs"]
+        # against the single pass: both sit within the bar of the oracle, and
+        # their bf16 P roundings differ, so they agree within twice the bar
+        assert max_abs(Om, r["O"]) <= 2 * tol["max_abs"] and rel_l2(Om, r["O"]) <= 2 * tol["rel_l2"]
+        assert max_abs(Lm, r["L"]) <= 2 * tol["lse_abs"]
 
 
 @pytest.mark.parametrize("name,over,split,chunk", [
