@@ -86,6 +86,9 @@ def selector_bytes(w, k: int) -> int:
     return qk + lists
 
 
+LAUNCHES_PER_STEP = 7
+
+
 def kernel_sources_sha(files):
     h = hashlib.sha256()
     for f in files:
@@ -242,6 +245,7 @@ def run_ours(args):
     stream = torch.cuda.current_stream(dev)
 
     names = ("stats", "select", "split", "sparse_lo", "sparse_hi", "merge")
+    # kernels per step: stats_bulk, select_tc + topk_rows, split_lists, 2x attn_tc, merge_lse
 
     def step(events=None):
         def mark(i):
@@ -331,7 +335,7 @@ def run_ours(args):
                              f"126 MiB; no flush"},
             "roofline": roofline, "selector": selector,
             "stages_ms": {n: round(v, 4) for n, v in stage_ms.items()},
-            "gpu_launches": 6 * args.steps, "clocks": clk,
+            "gpu_launches": LAUNCHES_PER_STEP * args.steps, "clocks": clk,
         }
     return result, dict(Qd=Qd, Kd=Kd, Vd=Vd, shape=shape, keep=keep, w=w, Q=Q, K=K, V=V, split_block=split_block,
                         step=step, flops=flops, world=world, rank=rank, dev=dev,
