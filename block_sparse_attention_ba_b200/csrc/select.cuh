@@ -146,8 +146,9 @@ __device__ void topk_row_warp(const float *__restrict__ srow, int nk, int k, int
   if (lane == 0) *out_cnt = pos;
 }
 
-// The same exact selection for a row held in registers: lane l holds the
-// order keys of columns c*32 + l, c < KPL (so column order is chunk-major).
+// The same exact selection for a row of at most 32*KPL keys; key(c) is the
+// order key of column c*32 + l for lane l (so column order is chunk-major),
+// held in registers or in shared memory.
 // The per-warp histogram (256 counters) lives in shared memory at hist_s.
 //
 //  1. Bracket: 32 keys sampled across the chunks are sorted across the warp
@@ -166,8 +167,8 @@ __device__ void topk_row_warp(const float *__restrict__ srow, int nk, int k, int
 // Scores of a row are concentrated in a narrow band with a long upper tail,
 // so a window placed by the sample spreads the band over many bins where the
 // row's full range would put most keys into one bin.
-template <int KPL>
-__device__ __forceinline__ void topk_row_regs(const uint32_t (&u)[KPL], int nk, int k, int32_t *__restrict__ out_idx,
+template <int KPL, typename KeyAt>
+__device__ __forceinline__ void topk_row_keys(const KeyAt &key, int nk, int k, int32_t *__restrict__ out_idx,
                                               int kmax, int32_t *__restrict__ out_cnt, uint32_t hist_s, int lane) {
   const unsigned full = 0xFFFFFFFFu;
   const unsigned lt_mask = (1u << lane) - 1u;
@@ -228,10 +229,10 @@ __device__ __forceinline__ void topk_row_regs(const uint32_t (&u)[KPL], int nk, 
   bool bracketed = false;
   if (KPL >= 2 && nk >= 64) {
     const int cs = lane % KPL;
-    uint32_t smp = u[0];
+    uint32_t smp = key(0);
 #pragma unroll
     for (int c = 1; c < KPL; ++c)
-      if (c == cs && c * 32 + lane < nk) smp = u[c];
+      if (c == cs && c * 32 + lane < nk) smp = key(c);
 #pragma unroll
     for (int size = 2; size <= 32; size <<= 1) {       // bitonic sort, descending across lanes
 #pragma unroll
@@ -250,8 +251,8 @@ __device__ __forceinline__ void topk_row_regs(const uint32_t (&u)[KPL], int nk, 
     int n_above = 0;
 #pragma unroll
     for (int c = 0; c < KPL; ++c) {
-      if (c * 32 + lane < nk && u[c] >= lo) {
-        const uint32_t bin = (u[c] - lo) >> shift;
+      if (c * 32 + lane < nk && key(c) >= lo) {
+        const uint32_t bin = (key(c) - lo) >> shift;
         if (bin > 255u)
           ++n_above;
         else
@@ -278,8 +279,8 @@ __device__ __forceinline__ void topk_row_regs(const uint32_t (&u)[KPL], int nk, 
 #pragma unroll
     for (int c = 0; c < KPL; ++c) {
       if (c * 32 + lane < nk) {
-        umin = min(umin, u[c]);
-        umax = max(umax, u[c]);
+        umin = min(umin, key(c));
+        umax = max(umax, key(c));
       }
     }
     umin = __reduce_min_sync(full, umin);
@@ -300,8 +301,8 @@ __device__ __forceinline__ void topk_row_regs(const uint32_t (&u)[KPL], int nk, 
     __syncwarp();
 #pragma unroll
     for (int c = 0; c < KPL; ++c) {
-      const uint32_t v = u[c] - base;
-      if (in_range(u[c], c * 32 + lane) && (v & mask) == prefix)
+      const uint32_t v = key(c) - base;
+      if (in_range(key(c), c * 32 + lane) && (v & mask) == prefix)
         red_shared_add(hist_s + 4u * ((v >> shift) & 255u), 1u);
     }
     __syncwarp();
@@ -321,11 +322,11 @@ __device__ __forceinline__ void topk_row_regs(const uint32_t (&u)[KPL], int nk, 
 #pragma unroll
     for (int c = 0; c < KPL; ++c) {
       const int j = c * 32 + lane;
-      const bool cand = in_range(u[c], j) && ((u[c] - base) & mask) == prefix;
+      const bool cand = in_range(key(c), j) && ((key(c) - base) & mask) == prefix;
       const unsigned cb = __ballot_sync(full, cand);
       if (cand) {
         const uint32_t slot = hist_s + 8u * static_cast<uint32_t>(cnt + __popc(cb & lt_mask));
-        asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(slot), "r"(u[c]), "r"(j) : "memory");
+        asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(slot), "r"(key(c)), "r"(j) : "memory");
       }
       cnt += __popc(cb);
     }
@@ -346,7 +347,7 @@ __device__ __forceinline__ void topk_row_regs(const uint32_t (&u)[KPL], int nk, 
 #pragma unroll
     for (int c = 0; c < KPL; ++c) {
       const int j = c * 32 + lane;
-      const bool kept = j < nk && (u[c] > thr_u || (u[c] == thr_u && j <= thr_j));
+      const bool kept = j < nk && (key(c) > thr_u || (key(c) == thr_u && j <= thr_j));
       const unsigned kb = __ballot_sync(full, kept);
       if (kept) out_idx[pos + __popc(kb & lt_mask)] = j;
       pos += __popc(kb);
@@ -358,8 +359,8 @@ __device__ __forceinline__ void topk_row_regs(const uint32_t (&u)[KPL], int nk, 
     for (int c = 0; c < KPL; ++c) {
       const int j = c * 32 + lane;
       const bool in = j < nk;
-      const bool gt = in && u[c] > thr;
-      const bool eq = in && u[c] == thr;
+      const bool gt = in && key(c) > thr;
+      const bool eq = in && key(c) == thr;
       const unsigned eqb = __ballot_sync(full, eq);
       const bool kept = gt || (eq && eq_seen + __popc(eqb & lt_mask) < need);
       const unsigned kb = __ballot_sync(full, kept);
@@ -370,6 +371,13 @@ __device__ __forceinline__ void topk_row_regs(const uint32_t (&u)[KPL], int nk, 
   }
   for (int j = pos + lane; j < kmax; j += 32) out_idx[j] = -1;
   if (lane == 0) *out_cnt = pos;
+}
+
+// Row held in registers: lane l has the keys of columns c*32 + l in u[c].
+template <int KPL>
+__device__ __forceinline__ void topk_row_regs(const uint32_t (&u)[KPL], int nk, int k, int32_t *__restrict__ out_idx,
+                                              int kmax, int32_t *__restrict__ out_cnt, uint32_t hist_s, int lane) {
+  topk_row_keys<KPL>([&](int c) { return u[c]; }, nk, k, out_idx, kmax, out_cnt, hist_s, lane);
 }
 
 // One warp per (batch, head, query block) row of the score map; rows up to
@@ -412,9 +420,102 @@ __global__ void __launch_bounds__(kTopkWarps * 32) topk_rows_kernel(const float 
   }
 }
 
+// Rows staged in shared memory instead of registers (fewer registers, more
+// resident warps): each warp double-buffers its rows with cp.async (16-byte
+// copies when rows are 16-byte aligned, else 4-byte ones), converts its own
+// columns to order keys in place, and selects from there.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+template <int KPL>
+constexpr size_t topk_smem_bytes() {
+  return static_cast<size_t>(kTopkWarps) * (2 * KPL * 32 + 256) * sizeof(uint32_t);
+}
+
+template <int KPL>
+__global__ void __launch_bounds__(kTopkWarps * 32, KPL >= 32 ? 3 : 4) topk_rows_smem_kernel(const float *__restrict__ scores, int nk,
+                                                                         int k, int32_t *__restrict__ kv_idx,
+                                                                         int kmax, int32_t *__restrict__ kv_cnt,
+                                                                         long long rows) {
+  constexpr int ROW = KPL * 32;
+  extern __shared__ __align__(16) uint32_t tk_smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint32_t *buf = tk_smem + warp * (2 * ROW + 256);
+  const uint32_t hist_s = smem_u32(buf + 2 * ROW);
+  const long long stride = static_cast<long long>(gridDim.x) * kTopkWarps;
+  long long row = blockIdx.x * static_cast<long long>(kTopkWarps) + warp;
+  const bool vec = (nk & 3) == 0;
+  auto fetch = [&](long long r, int slot) {
+    if (r < rows) {
+      const float *src = scores + r * nk;
+      const uint32_t dst = smem_u32(buf + slot * ROW);
+      if (vec) {
+        for (int ch = lane; ch < (nk >> 2); ch += 32) cp_async16(dst + 16u * ch, src + 4 * ch);
+      } else {
+        for (int j = lane; j < nk; j += 32) cp_async4(dst + 4u * j, src + j);
+      }
+    }
+    cp_async_commit();                         // one group per row, empty past the end
+  };
+  fetch(row, 0);
+  for (int it = 0; row < rows; row += stride, ++it) {
+    const int slot = it & 1;
+    fetch(row + stride, slot ^ 1);
+    cp_async_wait<1>();                        // this row's group has landed (the newest may not)
+    __syncwarp();
+    uint32_t *keys = buf + slot * ROW;
+#pragma unroll
+    for (int c = 0; c < KPL; ++c) {
+      const int j = c * 32 + lane;
+      if (j < nk) keys[j] = order_key(__uint_as_float(keys[j]));
+    }
+    // volatile loads: re-read per use rather than held in registers
+    const uint32_t keys_s = smem_u32(keys) + 4u * lane;
+    auto key_at = [&](int c) {
+      uint32_t x;
+      asm volatile("ld.shared.u32 %0, [%1];" : "=r"(x) : "r"(keys_s + 128u * c));
+      return x;
+    };
+    topk_row_keys<KPL>(key_at, nk, k, kv_idx + row * kmax, kmax, kv_cnt + row, hist_s, lane);
+    __syncwarp();                              // the slot is refilled two rows later
+  }
+  cp_async_wait<0>();
+}
+
+#ifndef BA_TOPK_SMEM_MIN_KPL
+#define BA_TOPK_SMEM_MIN_KPL 16
+#endif
+
+template <int KPL>
+inline cudaError_t launch_topk_smem(const float *scores, int nk, int k, int32_t *idx, int kmax, int32_t *cnt,
+                                    long long rows, int num_sms, cudaStream_t stream) {
+  const int threads = kTopkWarps * 32;
+  constexpr size_t smem = topk_smem_bytes<KPL>();
+  cudaError_t e = cudaFuncSetAttribute(topk_rows_smem_kernel<KPL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, topk_rows_smem_kernel<KPL>, threads, smem);
+  if (e != cudaSuccess) return e;
+  long long grid = (rows + kTopkWarps - 1) / kTopkWarps;
+  const long long slots = static_cast<long long>(num_sms) * (per_sm > 0 ? per_sm : 1);
+  grid = grid < slots ? grid : slots;
+  topk_rows_smem_kernel<KPL><<<static_cast<unsigned>(grid), threads, smem, stream>>>(scores, nk, k, idx, kmax, cnt,
+                                                                                     rows);
+  return cudaGetLastError();
+}
+
 template <int KPL>
 inline cudaError_t launch_topk_kpl(const float *scores, int nk, int k, int32_t *idx, int kmax, int32_t *cnt,
                                    long long rows, int num_sms, cudaStream_t stream) {
+  if (KPL >= BA_TOPK_SMEM_MIN_KPL) return launch_topk_smem<(KPL > 0 ? KPL : 8)>(scores, nk, k, idx, kmax, cnt, rows, num_sms, stream);
   const int threads = kTopkWarps * 32;
   long long grid = (rows + kTopkWarps - 1) / kTopkWarps;
   if (KPL > 0) {                                    // persistent: every resident CTA slot once
