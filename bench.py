@@ -86,7 +86,7 @@ def selector_bytes(w, k: int) -> int:
     return qk + lists
 
 
-LAUNCHES_PER_STEP = 7
+LAUNCHES_PER_STEP = 6   # stats_bulk, select_tc + topk_rows, split_lists, attn_tc x2
 
 
 def kernel_sources_sha(files):
@@ -237,15 +237,13 @@ def run_ours(args):
     cnt = torch.empty((w.B, w.Hq, nb), device=dev, dtype=torch.int32)
     scores = torch.empty((w.B, w.Hq, nb, nb), device=dev, dtype=torch.float32)     # the block-score map
     lists =(torch.empty_like(idx), torch.empty_like(cnt), torch.empty_like(idx), torch.empty_like(cnt))
-    # span partials stay in fp32 so the merged output is rounded to bf16 once
+    # the first span's partial stays in fp32 so the merged output is rounded to bf16 once
     O1 = torch.empty(Qd.shape, device=dev, dtype=torch.float32)
-    O2 = torch.empty(Qd.shape, device=dev, dtype=torch.float32)
     Om = torch.empty_like(Qd)
-    L1, L2, Lm = (torch.empty((w.B, w.Hq, w.N_alloc), device=dev) for _ in range(3))
+    L1, Lm = (torch.empty((w.B, w.Hq, w.N_alloc), device=dev) for _ in range(2))
     stream = torch.cuda.current_stream(dev)
 
-    names = ("stats", "select", "split", "sparse_lo", "sparse_hi", "merge")
-    # kernels per step: stats_bulk, select_tc + topk_rows, split_lists, 2x attn_tc, merge_lse
+    names = ("stats", "select", "split", "sparse_lo", "sparse_hi_merge")
 
     def step(events=None):
         def mark(i):
@@ -260,10 +258,9 @@ def run_ours(args):
         mark(3)
         api.sparse_fwd(Qd, Kd, Vd, lists[0], lists[1], shape, out=(O1, L1))
         mark(4)
-        api.sparse_fwd(Qd, Kd, Vd, lists[2], lists[3], shape, out=(O2, L2))
+        # second span, merged with the first in its epilogue (FlashBlock Eq. 9)
+        api.sparse_fwd_merge(Qd, Kd, Vd, lists[2], lists[3], shape, O1, L1, out=(Om, Lm))
         mark(5)
-        api.merge_lse(O1, L1, O2, L2, out=(Om, Lm))
-        mark(6)
 
     for _ in range(args.warmup):
         step()
@@ -274,7 +271,7 @@ def run_ours(args):
     cnt_total = int(cnt.sum().item())
     flops = kept_flops(cnt_total, w.block, w.d)
 
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local)
     if world > 1:
@@ -304,11 +301,12 @@ def run_ours(args):
     result = None
     if rank == 0:
         peaks, peak_src = load_peaks()
-        sparse_ms = stage_ms["sparse_lo"] + stage_ms["sparse_hi"]
+        sparse_ms = stage_ms["sparse_lo"] + stage_ms["sparse_hi_merge"]
         achieved = flops / (sparse_ms * 1e-3) / 1e12
         sha = kernel_sources_sha(["attn_tc.cuh", "common.cuh"])
         traffic, prof = traffic_from_profile(sha)
-        roofline = {"bound": "tensor", "kernel": "attn_tc_kernel (both span launches of a step)",
+        roofline = {"bound": "tensor", "kernel": "attn_tc_kernel (both span launches of a step; the second "
+                                                  "also merges the first span's fp32 partial in its epilogue)",
                     "achieved": round(achieved, 1), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                     "frac": round(achieved / peaks["bf16_tflops"], 4),
                     "frac_vs_sustained": round(achieved / peaks["bf16_tflops_sustained"], 4),
@@ -328,7 +326,7 @@ def run_ours(args):
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": f"{w.name}: B={w.B} Hq={w.Hq} Hkv={w.Hkv} N={w.N} d={w.d} block={w.block} "
                                    f"bf16 keep={keep}; step = stats+select+split(block {split_block})"
-                                   f"+2x sparse_fwd+merge_lse",
+                                   f"+sparse_fwd+sparse_fwd_merge",
                        "keep": keep, "kept_blocks_per_query_block": k, "split_block": split_block,
                        "parallelism": f"{world} independent replica(s)",
                        "l2": f"inputs {(Qd.numel() + Kd.numel() + Vd.numel()) * 2 / 2**20:.0f} MiB > L2 "
@@ -339,7 +337,7 @@ def run_ours(args):
         }
     return result, dict(Qd=Qd, Kd=Kd, Vd=Vd, shape=shape, keep=keep, w=w, Q=Q, K=K, V=V, split_block=split_block,
                         step=step, flops=flops, world=world, rank=rank, dev=dev,
-                        bufs=(stats_buf, idx, cnt, lists, O1, O2, Om, L1, L2, Lm))
+                        bufs=(stats_buf, idx, cnt, lists, O1, Om, L1, Lm))
 
 
 def run_e2e(ctx, steps, warmup):
@@ -385,6 +383,32 @@ def run_e2e(ctx, steps, warmup):
     return {"value": round(ctx["world"] * ctx["flops"] / (ms * 1e-3) / 1e12, 2), "unit": UNIT,
             "ms_per_step": round(ms, 4), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
             "api": "ba_att_forward_host (pinned host buffers, copies pipelined per chunk of KV heads)"}
+
+
+def run_merge_standalone(ctx, steps=5):
+    """ba_att_merge_lse on its own (not part of the step, whose second span
+    merges in its epilogue): two fp32 span partials -> bf16, HBM-bound."""
+    import torch
+    from block_sparse_attention_ba_b200 import api
+
+    stats_buf, idx, cnt, lists, O1, Om, L1, Lm = ctx["bufs"]
+    shape = ctx["shape"]
+    O2, L2 = api.sparse_fwd(ctx["Qd"], ctx["Kd"], ctx["Vd"], lists[2], lists[3], shape, out_dtype=torch.float32)
+    Ox, Lx = torch.empty_like(Om), torch.empty_like(Lm)
+    api.merge_lse(O1, L1, O2, L2, out=(Ox, Lx))
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(ctx["dev"])
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        api.merge_lse(O1, L1, O2, L2, out=(Ox, Lx))
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    byts = (O1.numel() + O2.numel()) * 4 + (L1.numel() + L2.numel()) * 4 + Ox.numel() * 2 + Lx.numel() * 4
+    peaks, _ = load_peaks()
+    gbs = byts / (ms * 1e-3) / 1e9
+    return {"ms": round(ms, 4), "bytes": byts, "achieved_gbs": round(gbs, 1), "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4)}
 
 
 def run_dense(ctx, steps=3):
@@ -440,9 +464,11 @@ def main(argv=None):
     result, ctx = run_ours(args)
     e2e = run_e2e(ctx, max(3, args.steps // 2), 3)
     dense = run_dense(ctx)
+    merge_alone = run_merge_standalone(ctx)
     if rank == 0:
         result["e2e"] = e2e
         result["dense_keep1"] = dense
+        result["merge_lse_standalone"] = merge_alone
         if not args.no_cpu_baseline:
             per_step, desc, spent = oracle_sample(ctx["w"], ctx["Q"], ctx["K"], ctx["V"], ctx["keep"], 0,
                                                   n_blocks=768, n_sel_heads=8)

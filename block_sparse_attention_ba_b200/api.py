@@ -45,6 +45,8 @@ _SIGS = {
     "ba_att_split_lists": (ctypes.c_int, [ctypes.POINTER(CShape), _I32, _P, _P, _I32, _P, _P, _P, _P, _P]),
     "ba_att_sparse_fwd": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _P, _P, _P, _I32, _P, _I32, _P, _P]),
     "ba_att_merge_lse": (ctypes.c_int, [ctypes.c_int64, _I32, _I32, _I32, _P, _P, _P, _P, _P, _P, _P]),
+    "ba_att_sparse_fwd_merge": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _P, _P, _P, _I32, _P, _P, _P, _I32, _P,
+                                                _P]),
     "ba_att_get_device_error": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_uint32)]),
     "ba_att_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_uint32, _P]),
     "ba_att_forward_host_workspace": (ctypes.c_int64, [ctypes.POINTER(CShape), ctypes.c_double, _I32, _I32]),
@@ -216,6 +218,25 @@ def sparse_fwd(Q, K, V, idx, cnt, shape: Shape, out=None, out_dtype=None):
     _check("ba_att_sparse_fwd", lib.ba_att_sparse_fwd(
         ctypes.byref(shape.c()), _dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), _dev(idx, "kv_idx"), _dev(cnt, "kv_cnt"),
         idx.shape[-1], _dev(O, "O"), _TORCH_DT[O.dtype], _dev(LSE, "LSE"), _stream(Q)))
+    return out
+
+
+def sparse_fwd_merge(Q, K, V, idx, cnt, shape: Shape, O_prev, L_prev, out=None, out_dtype=None):
+    """Block-sparse attention over the kept blocks, merged in the epilogue with
+    an earlier fp32 partial (O_prev, L_prev) over a disjoint key set -> (O, LSE).
+    out may be (O_prev, L_prev) for an in-place fp32 merge."""
+    lib = load_library()
+    if O_prev.dtype != torch.float32 or L_prev.dtype != torch.float32:
+        raise TypeError("O_prev and L_prev must be float32")
+    if out is None:
+        odt = Q.dtype if out_dtype is None else out_dtype
+        out = (torch.empty(Q.shape, device=Q.device, dtype=odt),
+               torch.empty((shape.B, shape.Hq, shape.N_alloc), device=Q.device, dtype=torch.float32))
+    O, LSE = out
+    _check("ba_att_sparse_fwd_merge", lib.ba_att_sparse_fwd_merge(
+        ctypes.byref(shape.c()), _dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), _dev(idx, "kv_idx"), _dev(cnt, "kv_cnt"),
+        idx.shape[-1], _dev(O_prev, "O_prev"), _dev(L_prev, "L_prev"), _dev(O, "O"), _TORCH_DT[O.dtype],
+        _dev(LSE, "LSE"), _stream(Q)))
     return out
 
 

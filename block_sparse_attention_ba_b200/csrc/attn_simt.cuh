@@ -30,11 +30,13 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-template <typename T, typename TO, int D>
+// MERGE: merge with an earlier fp32 partial (O_prev, L_prev) before storing,
+// as in attn_tc.cuh (O, LSE may alias O_prev, L_prev when TO is float).
+template <typename T, typename TO, int D, bool MERGE>
 __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(
     const T *__restrict__ Q, const T *__restrict__ K, const T *__restrict__ V, const int32_t *__restrict__ kv_idx,
-    const int32_t *__restrict__ kv_cnt, int kmax, TO *__restrict__ O, float *__restrict__ LSE, int Hq, int Hkv, int N,
-    int N_alloc, int block, int nb, int subs, float scale_log2) {
+    const int32_t *__restrict__ kv_cnt, int kmax, TO *O, float *LSE, const float *O_prev, const float *L_prev, int Hq,
+    int Hkv, int N, int N_alloc, int block, int nb, int subs, float scale_log2) {
   constexpr int DPL = D / 32;
   constexpr int RPW = kSimtRows / (kSimtThreads / 32);      // rows per warp
   __shared__ float q_s[kSimtRows][D];
@@ -129,23 +131,32 @@ __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(
     if (r >= nrows) break;
     const bool has = lrow[rr] > 0.f;
     const float inv = has ? 1.f / lrow[rr] : 0.f;
-    TO *orow = O + (qhead + row0 + r) * D;
+    const long long grow = qhead + row0 + r;
+    const float lse_new = has ? (mrow[rr] + log2f(lrow[rr])) * kLn2 : -INFINITY;
+    MergeWeights mw{0.f, 0.f, 0.f, lse_new};
+    if constexpr (MERGE) mw = merge_weights(L_prev[grow], lse_new);
+    __syncwarp();                                      // every lane has read L_prev before lane 0 writes LSE
+    TO *orow = O + grow * D;
 #pragma unroll
-    for (int tt = 0; tt < DPL; ++tt) store_out(orow + lane + 32 * tt, o[rr][tt] * inv);
-    if (lane == 0) LSE[qhead + row0 + r] = has ? (mrow[rr] + log2f(lrow[rr])) * kLn2 : -INFINITY;
+    for (int tt = 0; tt < DPL; ++tt) {
+      float val = o[rr][tt] * inv;
+      if constexpr (MERGE) val = merge_value(mw, O_prev[grow * D + lane + 32 * tt], val);
+      store_out(orow + lane + 32 * tt, val);
+    }
+    if (lane == 0) LSE[grow] = mw.lse;
   }
 }
 
-template <typename T, typename TO, int D>
+template <typename T, typename TO, int D, bool MERGE = false>
 cudaError_t launch_attn_simt(const T *Q, const T *K, const T *V, const int32_t *idx, const int32_t *cnt, int kmax, TO *O,
                              float *LSE, int B, int Hq, int Hkv, int N, int N_alloc, int block, float sm_scale,
-                             cudaStream_t stream) {
+                             cudaStream_t stream, const float *O_prev = nullptr, const float *L_prev = nullptr) {
   const int nb = (N + block - 1) / block;
   const int subs = (block + kSimtRows - 1) / kSimtRows;
   dim3 grid(static_cast<unsigned>(nb * subs), Hq, B);
   const float scale_log2 = sm_scale * 1.4426950408889634f;
-  attn_simt_kernel<T, TO, D><<<grid, kSimtThreads, 0, stream>>>(Q, K, V, idx, cnt, kmax, O, LSE, Hq, Hkv, N, N_alloc,
-                                                             block, nb, subs, scale_log2);
+  attn_simt_kernel<T, TO, D, MERGE><<<grid, kSimtThreads, 0, stream>>>(Q, K, V, idx, cnt, kmax, O, LSE, O_prev, L_prev,
+                                                                    Hq, Hkv, N, N_alloc, block, nb, subs, scale_log2);
   return cudaGetLastError();
 }
 

@@ -106,12 +106,16 @@ __device__ __forceinline__ void exp_pack_store(const uint32_t (&sr)[2][32], floa
 
 // TO: output element type, bf16 (final output) or float (a partial that is
 // merged later, so the merged result is rounded only once).
-template <typename TO>
+// MERGE: the epilogue merges this span's result with an earlier fp32 partial
+// (O_prev, L_prev) over a disjoint key set before storing (O and LSE may
+// alias O_prev and L_prev when TO is float: each row is read before it is
+// written, by the same thread).
+template <typename TO, bool MERGE>
 __global__ void __launch_bounds__(kThreads, 2)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const int32_t *__restrict__ kv_idx,
-                   const int32_t *__restrict__ kv_cnt, int kmax, TO *__restrict__ O,
-                   float *__restrict__ LSE, int Hq, int Hkv, int N, int N_alloc, int nb, float scale_log2) {
+                   const int32_t *__restrict__ kv_cnt, int kmax, TO *O, float *LSE, const float *O_prev,
+                   const float *L_prev, int Hq, int Hkv, int N, int N_alloc, int nb, float scale_log2) {
   extern __shared__ uint8_t dyn_smem[];
   __shared__ Ctl ctl;
   const uint32_t smem_base = (smem_u32(dyn_smem) + 1023u) & ~1023u;
@@ -321,51 +325,61 @@ __global__ void __launch_bounds__(kThreads, 2)
       tc_fence_before();
       mbar_arrive(bar(P_FULL0 + h));
     }
-    if (cnt == 0) {
-      if (qrow < N) {
-        uint4 *dst = reinterpret_cast<uint4 *>(O + orow * kHeadDim);
-#pragma unroll
-        for (int v = 0; v < kHeadDim * static_cast<int>(sizeof(TO)) / 16; ++v) dst[v] = make_uint4(0, 0, 0, 0);
-        LSE[orow] = -INFINITY;
-      }
-    } else if (ok) {
+    // ------------------------------------------------------------ epilogue
+    // (cnt == 0: nothing was accumulated; this span contributes O = 0,
+    // LSE = -inf, and a merge passes the earlier partial through)
+    bool go = (cnt == 0);
+    if (cnt > 0 && ok) {
       const bool w = mbar_wait_bounded(bar(O_FINAL), 0, abort);
-      if (__all_sync(0xFFFFFFFFu, w)) {
-        tc_fence_after();
-        const bool has = l > 0.f;
-        const float inv = has ? 1.f / l : 0.f;
-        uint4 *dst = reinterpret_cast<uint4 *>(O + orow * kHeadDim);
+      go = __all_sync(0xFFFFFFFFu, w);
+      if (go) tc_fence_after();
+    }
+    if (go) {
+      const bool has = l > 0.f;
+      const float inv = has ? 1.f / l : 0.f;
+      const float lse_new = has ? (m_used + __log2f(l)) * 0.6931471805599453f : -INFINITY;
+      MergeWeights mw{0.f, 0.f, 0.f, lse_new};
+      if constexpr (MERGE) mw = merge_weights(qrow < N ? L_prev[orow] : -INFINITY, lse_new);
+      const float *prev = MERGE ? O_prev + orow * kHeadDim : nullptr;
+      uint4 *dst = reinterpret_cast<uint4 *>(O + orow * kHeadDim);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint32_t orr[32];
+      for (int q = 0; q < 4; ++q) {
+        uint32_t orr[32];
+        if (cnt > 0) {
           tmem_ld32(tO + q * 32, orr);
           tmem_ld_wait();
-          if (qrow < N) {
-            if constexpr (sizeof(TO) == 2) {
+        } else {
 #pragma unroll
-              for (int v = 0; v < 4; ++v) {
-                uint4 pkt;
-                pkt.x = pack_bf16x2(__uint_as_float(orr[8 * v + 0]) * inv, __uint_as_float(orr[8 * v + 1]) * inv);
-                pkt.y = pack_bf16x2(__uint_as_float(orr[8 * v + 2]) * inv, __uint_as_float(orr[8 * v + 3]) * inv);
-                pkt.z = pack_bf16x2(__uint_as_float(orr[8 * v + 4]) * inv, __uint_as_float(orr[8 * v + 5]) * inv);
-                pkt.w = pack_bf16x2(__uint_as_float(orr[8 * v + 6]) * inv, __uint_as_float(orr[8 * v + 7]) * inv);
-                dst[q * 4 + v] = pkt;
-              }
-            } else {
+          for (int c = 0; c < 32; ++c) orr[c] = 0u;
+        }
+        if (qrow < N) {
+          float o[32];
 #pragma unroll
-              for (int v = 0; v < 8; ++v) {
-                uint4 pkt;
-                pkt.x = __float_as_uint(__uint_as_float(orr[4 * v + 0]) * inv);
-                pkt.y = __float_as_uint(__uint_as_float(orr[4 * v + 1]) * inv);
-                pkt.z = __float_as_uint(__uint_as_float(orr[4 * v + 2]) * inv);
-                pkt.w = __float_as_uint(__uint_as_float(orr[4 * v + 3]) * inv);
-                dst[q * 8 + v] = pkt;
-              }
+          for (int c = 0; c < 32; ++c) o[c] = __uint_as_float(orr[c]) * inv;
+          if constexpr (MERGE) {
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+              const float4 pv = *reinterpret_cast<const float4 *>(prev + q * 32 + 4 * v);
+              o[4 * v + 0] = merge_value(mw, pv.x, o[4 * v + 0]);
+              o[4 * v + 1] = merge_value(mw, pv.y, o[4 * v + 1]);
+              o[4 * v + 2] = merge_value(mw, pv.z, o[4 * v + 2]);
+              o[4 * v + 3] = merge_value(mw, pv.w, o[4 * v + 3]);
             }
           }
+          if constexpr (sizeof(TO) == 2) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              dst[q * 4 + v] = make_uint4(pack_bf16x2(o[8 * v + 0], o[8 * v + 1]), pack_bf16x2(o[8 * v + 2], o[8 * v + 3]),
+                                          pack_bf16x2(o[8 * v + 4], o[8 * v + 5]), pack_bf16x2(o[8 * v + 6], o[8 * v + 7]));
+          } else {
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+              dst[q * 8 + v] = make_uint4(__float_as_uint(o[4 * v + 0]), __float_as_uint(o[4 * v + 1]),
+                                          __float_as_uint(o[4 * v + 2]), __float_as_uint(o[4 * v + 3]));
+          }
         }
-        if (qrow < N) LSE[orow] = has ? (m_used + __log2f(l)) * 0.6931471805599453f : -INFINITY;
       }
+      if (qrow < N) LSE[orow] = mw.lse;
     }
     tc_fence_before();
   }

@@ -217,9 +217,15 @@ ba_status ba_att_split_lists(const ba_att_shape *s, int32_t split_block, const i
                                 num_sms_of_current_device(), reinterpret_cast<cudaStream_t>(stream)));
 }
 
-ba_status ba_att_sparse_fwd(const ba_att_shape *s, const void *Q, const void *K, const void *V, const int32_t *kv_idx,
-                            const int32_t *kv_cnt, int32_t kmax, void *O, int32_t o_dtype, float *LSE,
-                            ba_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// Attention over the listed blocks; with O_prev/L_prev (both non-null) the
+// epilogue merges the result with that earlier fp32 partial.
+ba_status sparse_fwd_impl(const ba_att_shape *s, const void *Q, const void *K, const void *V, const int32_t *kv_idx,
+                          const int32_t *kv_cnt, int32_t kmax, void *O, int32_t o_dtype, float *LSE,
+                          const float *O_prev, const float *L_prev, ba_stream_t stream) {
   ba_status st = check_shape(s);
   if (st != BA_OK) return st;
   if (!Q || !K || !V || !kv_idx || !kv_cnt || !O || !LSE) return BA_ERR_INVALID_ARG;
@@ -227,6 +233,8 @@ ba_status ba_att_sparse_fwd(const ba_att_shape *s, const void *Q, const void *K,
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(kv_idx) || !aligned16(kv_cnt) || !aligned16(O) ||
       !aligned16(LSE))
     return BA_ERR_MISALIGNED;
+  const bool merge = O_prev != nullptr;
+  if (merge && (!aligned16(O_prev) || (reinterpret_cast<uintptr_t>(L_prev) & 3u))) return BA_ERR_MISALIGNED;
   if (kmax < 1) return BA_ERR_INVALID_ARG;
   const int nb = nblocks(s);
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
@@ -241,28 +249,28 @@ ba_status ba_att_sparse_fwd(const ba_att_shape *s, const void *Q, const void *K,
     const long long tiles = static_cast<long long>(s->B) * s->Hq * nb;
     if (tiles > 0x7FFFFFFFLL) return BA_ERR_UNSUPPORTED;
     const float sl2 = scale * 1.4426950408889634f;
-    cudaError_t e;
-    if (out_f32) {
-      e = cudaFuncSetAttribute(tc::attn_tc_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(tc::kDynSmem));
+    auto run = [&](auto kernel, auto *out) -> ba_status {
+      cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(tc::kDynSmem));
       if (e != cudaSuccess) return BA_ERR_CUDA;
-      tc::attn_tc_kernel<float><<<static_cast<unsigned>(tiles), tc::kThreads, tc::kDynSmem, cs>>>(
-          mq, mk, mv, kv_idx, kv_cnt, kmax, static_cast<float *>(O), LSE, s->Hq, s->Hkv, s->N, s->N_alloc, nb, sl2);
-    } else {
-      e = cudaFuncSetAttribute(tc::attn_tc_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(tc::kDynSmem));
-      if (e != cudaSuccess) return BA_ERR_CUDA;
-      tc::attn_tc_kernel<__nv_bfloat16><<<static_cast<unsigned>(tiles), tc::kThreads, tc::kDynSmem, cs>>>(
-          mq, mk, mv, kv_idx, kv_cnt, kmax, static_cast<__nv_bfloat16 *>(O), LSE, s->Hq, s->Hkv, s->N, s->N_alloc,
-          nb, sl2);
-    }
-    return from_cuda(cudaGetLastError());
+      kernel<<<static_cast<unsigned>(tiles), tc::kThreads, tc::kDynSmem, cs>>>(
+          mq, mk, mv, kv_idx, kv_cnt, kmax, out, LSE, O_prev, L_prev, s->Hq, s->Hkv, s->N, s->N_alloc, nb, sl2);
+      return from_cuda(cudaGetLastError());
+    };
+    float *of = static_cast<float *>(O);
+    __nv_bfloat16 *ob = static_cast<__nv_bfloat16 *>(O);
+    if (out_f32) return merge ? run(tc::attn_tc_kernel<float, true>, of) : run(tc::attn_tc_kernel<float, false>, of);
+    return merge ? run(tc::attn_tc_kernel<__nv_bfloat16, true>, ob) : run(tc::attn_tc_kernel<__nv_bfloat16, false>, ob);
   }
   cudaError_t e;
-#define BA_SIMT(T, TO, DD)                                                                                      \
-  launch_attn_simt<T, TO, DD>(static_cast<const T *>(Q), static_cast<const T *>(K), static_cast<const T *>(V), \
-                              kv_idx, kv_cnt, kmax, static_cast<TO *>(O), LSE, s->B, s->Hq, s->Hkv, s->N,       \
-                              s->N_alloc, s->block, scale, cs)
+#define BA_SIMT(T, TO, DD)                                                                                           \
+  (merge ? launch_attn_simt<T, TO, DD, true>(static_cast<const T *>(Q), static_cast<const T *>(K),                   \
+                                             static_cast<const T *>(V), kv_idx, kv_cnt, kmax, static_cast<TO *>(O), \
+                                             LSE, s->B, s->Hq, s->Hkv, s->N, s->N_alloc, s->block, scale, cs, O_prev, \
+                                             L_prev)                                                                 \
+         : launch_attn_simt<T, TO, DD, false>(static_cast<const T *>(Q), static_cast<const T *>(K),                  \
+                                              static_cast<const T *>(V), kv_idx, kv_cnt, kmax, static_cast<TO *>(O), \
+                                              LSE, s->B, s->Hq, s->Hkv, s->N, s->N_alloc, s->block, scale, cs))
   if (s->dtype == BA_DTYPE_BF16) {
     if (out_f32)
       e = s->d == 128 ? BA_SIMT(__nv_bfloat16, float, 128) : BA_SIMT(__nv_bfloat16, float, 64);
@@ -273,6 +281,23 @@ ba_status ba_att_sparse_fwd(const ba_att_shape *s, const void *Q, const void *K,
   }
 #undef BA_SIMT
   return from_cuda(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+ba_status ba_att_sparse_fwd(const ba_att_shape *s, const void *Q, const void *K, const void *V, const int32_t *kv_idx,
+                            const int32_t *kv_cnt, int32_t kmax, void *O, int32_t o_dtype, float *LSE,
+                            ba_stream_t stream) {
+  return sparse_fwd_impl(s, Q, K, V, kv_idx, kv_cnt, kmax, O, o_dtype, LSE, nullptr, nullptr, stream);
+}
+
+ba_status ba_att_sparse_fwd_merge(const ba_att_shape *s, const void *Q, const void *K, const void *V,
+                                  const int32_t *kv_idx, const int32_t *kv_cnt, int32_t kmax, const float *O_prev,
+                                  const float *LSE_prev, void *O, int32_t o_dtype, float *LSE, ba_stream_t stream) {
+  if (!O_prev || !LSE_prev) return BA_ERR_INVALID_ARG;
+  return sparse_fwd_impl(s, Q, K, V, kv_idx, kv_cnt, kmax, O, o_dtype, LSE, O_prev, LSE_prev, stream);
 }
 
 ba_status ba_att_merge_lse(int64_t rows, int32_t d, int32_t in_dtype, int32_t out_dtype, const void *O1,
@@ -337,7 +362,7 @@ struct PipeLayout {
   int C = 0, G = 0, nb = 0, k = 0;
   size_t q[2], kk[2], v[2], o[2], l[2];                 // double-buffered chunk inputs and outputs
   size_t qm, qv, km, kv, idx, cnt, sc;                  // selector buffers of one chunk
-  size_t lo_idx, lo_cnt, hi_idx, hi_cnt, o1, o2, l1, l2;  // split + merge buffers of one chunk
+  size_t lo_idx, lo_cnt, hi_idx, hi_cnt, o1, l1;         // split buffers and the first span's fp32 partial
   size_t total = 0;
 };
 
@@ -388,9 +413,7 @@ bool pipe_layout(const ba_att_shape *s, double keep, int32_t split_block, int32_
     L->hi_idx = take(hq * nb * k * 4);
     L->hi_cnt = take(hq * nb * 4);
     L->o1 = take(rows_q * s->d * 4);
-    L->o2 = take(rows_q * s->d * 4);
     L->l1 = take(rows_q * 4);
-    L->l2 = take(rows_q * 4);
   }
   L->total = off;
   return true;
@@ -502,16 +525,14 @@ ba_status forward_host_impl(PipeResources *r, const ba_att_shape *s, double keep
     if (st == BA_OK && split_block >= 0) {
       int32_t *lo_idx = reinterpret_cast<int32_t *>(ws + L.lo_idx), *lo_cnt = reinterpret_cast<int32_t *>(ws + L.lo_cnt);
       int32_t *hi_idx = reinterpret_cast<int32_t *>(ws + L.hi_idx), *hi_cnt = reinterpret_cast<int32_t *>(ws + L.hi_cnt);
-      float *l1 = reinterpret_cast<float *>(ws + L.l1), *l2 = reinterpret_cast<float *>(ws + L.l2);
+      float *l1 = reinterpret_cast<float *>(ws + L.l1);
       st = ba_att_split_lists(&sc, split_block, idx, cnt, L.k, lo_idx, lo_cnt, hi_idx, hi_cnt, stream);
       if (st == BA_OK)
         st = ba_att_sparse_fwd(&sc, Qc, Kc, Vc, lo_idx, lo_cnt, L.k, ws + L.o1, BA_DTYPE_F32, l1, stream);
-      if (st == BA_OK)
-        st = ba_att_sparse_fwd(&sc, Qc, Kc, Vc, hi_idx, hi_cnt, L.k, ws + L.o2, BA_DTYPE_F32, l2, stream);
+      if (st == BA_OK)   // the second span merges with the first in its epilogue
+        st = ba_att_sparse_fwd_merge(&sc, Qc, Kc, Vc, hi_idx, hi_cnt, L.k, reinterpret_cast<const float *>(ws + L.o1),
+                                     l1, Oc, s->dtype, Lc, stream);
       if (st == BA_OK && cudaEventRecord(r->in_free[sl], cs) != cudaSuccess) st = BA_ERR_CUDA;
-      if (st == BA_OK)
-        st = ba_att_merge_lse(static_cast<int64_t>(hqc) * s->N_alloc, s->d, BA_DTYPE_F32, s->dtype, ws + L.o1, l1,
-                              ws + L.o2, l2, Oc, Lc, stream);
     } else if (st == BA_OK) {
       st = ba_att_sparse_fwd(&sc, Qc, Kc, Vc, idx, cnt, L.k, Oc, s->dtype, Lc, stream);
       if (st == BA_OK && cudaEventRecord(r->in_free[sl], cs) != cudaSuccess) st = BA_ERR_CUDA;

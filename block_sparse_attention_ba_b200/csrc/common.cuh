@@ -306,6 +306,30 @@ struct Elem<__nv_bfloat16> {
   }
 };
 
+// Log-space merge of two partial attentions over disjoint key sets
+// ("FlashBlock", Eq. 9): with m = max(L1, L2) and w_k = exp(L_k - m),
+// O = (w1 O1 + w2 O2) / (w1 + w2) and L = m + ln(w1 + w2); both -inf gives
+// O = 0, L = -inf. Every merge in the library (the standalone kernel and the
+// attention epilogues) uses these two functions, with the rounding of each
+// step spelled out, so that fused and separate merges agree bit for bit.
+struct MergeWeights {
+  float w1, w2, inv, lse;
+};
+__device__ __forceinline__ MergeWeights merge_weights(float l1, float l2) {
+  const float m = fmaxf(l1, l2);
+  const bool empty = (m == -INFINITY);
+  MergeWeights w;
+  w.w1 = empty ? 0.f : expf(l1 - m);
+  w.w2 = empty ? 0.f : expf(l2 - m);
+  const float den = __fadd_rn(w.w1, w.w2);
+  w.inv = empty ? 0.f : __fdiv_rn(1.f, den);
+  w.lse = empty ? -INFINITY : m + logf(den);
+  return w;
+}
+__device__ __forceinline__ float merge_value(const MergeWeights &w, float o1, float o2) {
+  return __fmul_rn(__fmaf_rn(w.w1, o1, __fmul_rn(w.w2, o2)), w.inv);
+}
+
 __device__ __forceinline__ void store_out(float *p, float v) { *p = v; }
 __device__ __forceinline__ void store_out(__nv_bfloat16 *p, float v) { *p = __float2bfloat16_rn(v); }
 

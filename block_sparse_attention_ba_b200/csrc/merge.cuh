@@ -51,19 +51,13 @@ __global__ void __launch_bounds__(kMergeThreads) merge_lse_kernel(const TI *O1, 
     float out[VEC];
     float lse = 0.f;
     if (act) {
-      const float l1 = L1[r], l2 = L2[r];
-      const float m = fmaxf(l1, l2);
-      const bool empty = (m == -INFINITY);
-      const float w1 = empty ? 0.f : expf(l1 - m);
-      const float w2 = empty ? 0.f : expf(l2 - m);
-      const float den = w1 + w2;
-      const float inv = empty ? 0.f : 1.f / den;
+      const MergeWeights mw = merge_weights(L1[r], L2[r]);
       float fa[VEC], fb[VEC];
       load_vec<TI, VEC>(O1 + r * D + c * VEC, fa);
       load_vec<TI, VEC>(O2 + r * D + c * VEC, fb);
 #pragma unroll
-      for (int e = 0; e < VEC; ++e) out[e] = (w1 * fa[e] + w2 * fb[e]) * inv;
-      lse = empty ? -INFINITY : m + logf(den);
+      for (int e = 0; e < VEC; ++e) out[e] = merge_value(mw, fa[e], fb[e]);
+      lse = mw.lse;
     }
     __syncwarp();
     if (act) {

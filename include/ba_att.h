@@ -190,6 +190,28 @@ ba_status ba_att_sparse_fwd(const ba_att_shape *shape,
                             void *O, int32_t o_dtype, float *LSE, ba_stream_t stream);
 
 /*
+ * ba_att_sparse_fwd_merge — ba_att_sparse_fwd over the listed blocks, merged
+ * in the epilogue with an earlier partial over a disjoint key set
+ * (FlashBlock Eq. 5 and Eq. 9: attention over X u Y from the parts over X
+ * and Y). The result equals ba_att_sparse_fwd into an fp32 partial followed
+ * by ba_att_merge_lse(O_prev, LSE_prev, that partial) bit for bit (the same
+ * rounding steps), without writing or reading the second partial.
+ *
+ * O_prev    device fp32 [B, Hq, N_alloc, d]: the earlier partial, e.g. a
+ *           ba_att_sparse_fwd with o_dtype = BA_DTYPE_F32 over another span.
+ * LSE_prev  device fp32 [B, Hq, N_alloc]: its log-sum-exp.
+ * O, LSE    as for ba_att_sparse_fwd (o_dtype = shape dtype or fp32); with
+ *           fp32 output O may be O_prev and LSE may be LSE_prev (in place).
+ * Other arguments and paths as for ba_att_sparse_fwd. NULL O_prev or
+ * LSE_prev -> BA_ERR_INVALID_ARG.
+ */
+ba_status ba_att_sparse_fwd_merge(const ba_att_shape *shape,
+                                  const void *Q, const void *K, const void *V,
+                                  const int32_t *kv_idx, const int32_t *kv_cnt, int32_t kmax,
+                                  const float *O_prev, const float *LSE_prev,
+                                  void *O, int32_t o_dtype, float *LSE, ba_stream_t stream);
+
+/*
  * ba_att_merge_lse — log-space merge of two partial attentions over disjoint
  * key sets (FlashBlock Eq. 9, decomposition of Eq. 5):
  *   m = max(L1, L2), w_k = exp(L_k - m),
@@ -220,8 +242,9 @@ int64_t ba_att_forward_host_workspace(const ba_att_shape *shape, double keep, in
  * ba_att_forward_host — the whole BA-Att forward from HOST buffers to HOST
  * buffers: H2D of Q, K, V; ba_att_stats; ba_att_select; then either one
  * ba_att_sparse_fwd (split_block < 0), or (split_block >= 0) the key set split
- * at that key block (FlashBlock Eq. 5), one ba_att_sparse_fwd per span with
- * fp32 partials, and ba_att_merge_lse (FlashBlock Eq. 9); D2H of O and LSE.
+ * at that key block (FlashBlock Eq. 5), ba_att_sparse_fwd over the first span
+ * into an fp32 partial and ba_att_sparse_fwd_merge over the second (the
+ * FlashBlock Eq. 9 merge in its epilogue); D2H of O and LSE.
  * The pages define the operator only; the pipelining is this library's.
  *
  * The work is cut into chunks of kv_heads_per_chunk KV heads (with their

@@ -147,3 +147,12 @@ def test_forward_host_arguments(lib):
     assert call(P, P, P, P, P, ctypes.c_void_p(0x100010), ws) == 3         # workspace not 256-byte aligned
     assert lib.ba_att_forward_host(ctypes.byref(shape(d=96)), ctypes.c_double(0.5), -1, 0, P, P, P, P, P, W, ws,
                                    None) == 2
+
+
+def test_sparse_fwd_merge_arguments(lib):
+    s = shape()
+    # the earlier partial is required and must be aligned like every other buffer
+    assert lib.ba_att_sparse_fwd_merge(ctypes.byref(s), P, P, P, P, P, 4, None, P, P, 1, P, None) == 1
+    assert lib.ba_att_sparse_fwd_merge(ctypes.byref(s), P, P, P, P, P, 4, P, None, P, 1, P, None) == 1
+    assert lib.ba_att_sparse_fwd_merge(ctypes.byref(s), P, P, P, P, P, 4, MIS, P, P, 1, P, None) == 3
+    assert lib.ba_att_sparse_fwd_merge(ctypes.byref(shape(d=96)), P, P, P, P, P, 4, P, P, P, 1, P, None) == 2

@@ -183,6 +183,42 @@ def test_split_and_merge_equals_union():
         assert max_abs(Lm, r["L"]) <= 2 * tol["lse_abs"]
 
 
+@pytest.mark.parametrize("name,over", [
+    ("extreme_128k", dict(N=4096 - 50, N_alloc=4096, Hq=4, Hkv=2)),      # tensor-core path, ragged tail
+    ("tiny_fp32", dict(N=1000, N_alloc=1024)),                             # CUDA-core path, fp32
+    ("dlm_16k", dict(N=1024, Hq=2, Hkv=1, d=64, block=64)),                # CUDA-core path, bf16 inputs
+])
+def test_fused_merge_equals_separate_merge(name, over):
+    # attention over span B merged in the epilogue with the partial over span A
+    # equals the separate partial + ba_att_merge_lse bit for bit, and the
+    # oracle's attention over the union at the parity bar
+    Q, K, V, meta = make_inputs(name, **over)
+    w = meta["workload"]
+    r = run_gpu(Q, K, V, w, 0.5)
+    shape = r["shape"]
+    split = w.nb // 2
+    lo_i, lo_c, hi_i, hi_c = api.split_lists(r["idx_d"], r["cnt_d"], shape, split)
+    O1, L1 = api.sparse_fwd(r["Qd"], r["Kd"], r["Vd"], lo_i, lo_c, shape, out_dtype=torch.float32)
+    O2, L2 = api.sparse_fwd(r["Qd"], r["Kd"], r["Vd"], hi_i, hi_c, shape, out_dtype=torch.float32)
+    for odt in {r["Qd"].dtype, torch.float32}:
+        Om, Lm = api.merge_lse(O1, L1, O2, L2, out_dtype=odt)
+        Of, Lf = api.sparse_fwd_merge(r["Qd"], r["Kd"], r["Vd"], hi_i, hi_c, shape, O1, L1, out_dtype=odt)
+        torch.cuda.synchronize()
+        n = w.N
+        assert torch.equal(Of[:, :, :n], Om[:, :, :n]) and torch.equal(Lf[:, :, :n], Lm[:, :, :n])
+    # in place into the fp32 partial
+    O1c, L1c = O1.clone(), L1.clone()
+    api.sparse_fwd_merge(r["Qd"], r["Kd"], r["Vd"], hi_i, hi_c, shape, O1c, L1c, out=(O1c, L1c))
+    Om, Lm = api.merge_lse(O1, L1, O2, L2, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert torch.equal(O1c[:, :, :w.N], Om[:, :, :w.N]) and torch.equal(L1c[:, :, :w.N], Lm[:, :, :w.N])
+    tol = TOL[w.dtype]
+    Oref, Lref = O.masked_attention(Q, K, V, r["idx"], r["cnt"], w.N, w.block, w.d ** -0.5)
+    got = Of[:, :, :w.N].float().cpu().numpy()
+    assert max_abs(got, Oref[:, :, :w.N]) <= tol["max_abs"] and rel_l2(got, Oref[:, :, :w.N]) <= tol["rel_l2"]
+    assert max_abs(Lf[:, :, :w.N].cpu().numpy(), Lref[:, :, :w.N]) <= tol["lse_abs"]
+
+
 @pytest.mark.parametrize("name,over,split,chunk", [
     ("extreme_128k", dict(N=4096 - 50, N_alloc=4096, Hq=8, Hkv=4), True, 0),    # split + merge, 4 chunks of 1
     ("extreme_128k", dict(N=4096, Hq=8, Hkv=4), False, 3),                      # chunks of 3 + 1 KV heads
