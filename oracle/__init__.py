@@ -20,7 +20,8 @@ Sources (cited by page title and section throughout):
 The pages state the ingredients of the selector in prose only (block-wise
 pre-downsampling, per-dimension diagonal Q/K variances, a covariance-compensated
 correction, norm sorting keeping a top fraction). Every formula below is the
-plain reading of that prose; each reading is listed in the design doc.
+plain reading of that prose, stated in the docstring of the function that
+implements it.
 
 Parity status: every public function is pinned by tests in
 ``tests/test_oracle.py`` except the two diagnostics marked "parity unpinned"
@@ -42,6 +43,7 @@ from .ba_att_oracle import (  # noqa: F401
     dense_attention,
     merge_lse,
     split_lists,
+    complement_lists,
     post_downsample_map,
     block_mass_via_lse,
     spearman_vs_post,

@@ -325,6 +325,28 @@ def merge_lse(O1, L1, O2, L2, dtype=np.float64):
     return O.astype(dtype), L.astype(dtype)
 
 
+def complement_lists(idx, cnt, nk: int, ckmax: int | None = None):
+    """The key blocks each kept-block list leaves out, ascending, -1 padded.
+
+    [FlashBlock, review page: the "sparse + cached residual" form of Fig. 6]:
+    attention over the kept blocks and over the blocks the selector dropped
+    are two disjoint partial attentions whose log-space merge (``merge_lse``,
+    Eq. 9) is attention over every block. Entries outside [0, nk) in the
+    input are ignored. ckmax (default nk) is the row stride of the result.
+    """
+    idx = np.asarray(idx)
+    cnt = np.asarray(cnt)
+    ckmax = nk if ckmax is None else ckmax
+    cidx = np.full(cnt.shape + (ckmax,), -1, dtype=np.int32)
+    ccnt = np.zeros(cnt.shape, dtype=np.int32)
+    for pos in np.ndindex(cnt.shape):
+        kept = {int(j) for j in idx[pos][: int(cnt[pos])] if 0 <= int(j) < nk}
+        rest = [j for j in range(nk) if j not in kept]
+        cidx[pos][: len(rest)] = rest
+        ccnt[pos] = len(rest)
+    return cidx, ccnt
+
+
 def split_lists(idx, cnt, split_block: int):
     """Partition each kept-block list at a key-block boundary.
 

@@ -311,6 +311,36 @@ def test_merge_of_disjoint_spans_equals_union():
         np.testing.assert_allclose(Lm, Lu[:, :, :N], rtol=1e-12, atol=1e-12)
 
 
+def test_complement_lists_partition_and_kept_plus_rest_is_dense():
+    # the complement is the exact set difference (ascending, -1 padded), and
+    # merging attention over the kept blocks with attention over the rest
+    # gives dense attention (the "cached residual" identity)
+    Q, K, V = _qkv()
+    N, b, s = 200, 32, 16 ** -0.5
+    nb = O.num_blocks(N, b)
+    rng = np.random.default_rng(5)
+    S = rng.standard_normal((1, 4, nb, nb))
+    for k in (1, 3, nb):
+        idx, cnt = O.select_topk(S, k, kmax=nb)
+        cidx, ccnt = O.complement_lists(idx, cnt, nb)
+        assert ((cnt + ccnt) == nb).all()
+        for pos in np.ndindex(cnt.shape):
+            kept = list(idx[pos][: cnt[pos]])
+            rest = list(cidx[pos][: ccnt[pos]])
+            assert sorted(kept + rest) == list(range(nb)) and rest == sorted(rest)
+            assert (cidx[pos][ccnt[pos]:] == -1).all()
+        O1, L1 = O.masked_attention(Q, K, V, idx, cnt, N, b, s)
+        O2, L2 = O.masked_attention(Q, K, V, cidx, ccnt, N, b, s)
+        Od, Ld = O.dense_attention(Q, K, V, N, s)
+        Om, Lm = O.merge_lse(O1[:, :, :N], L1[:, :, :N], O2[:, :, :N], L2[:, :, :N])
+        np.testing.assert_allclose(Om, Od, rtol=1e-11, atol=1e-12)
+        np.testing.assert_allclose(Lm, Ld, rtol=1e-12, atol=1e-12)
+    # entries outside [0, nb) are ignored; a narrower stride truncates nothing that fits
+    idx = np.array([[[[0, 7, -1, 99]]]], dtype=np.int32)
+    cidx, ccnt = O.complement_lists(idx, np.array([[[4]]]), 8)
+    assert ccnt[0, 0, 0] == 6 and list(cidx[0, 0, 0]) == [1, 2, 3, 4, 5, 6, -1, -1]
+
+
 def test_merge_edge_cases():
     o1 = np.array([[1.0, 2.0], [3.0, 4.0]])
     o2 = np.array([[5.0, 6.0], [7.0, 8.0]])
