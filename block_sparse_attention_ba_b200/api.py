@@ -43,6 +43,7 @@ _SIGS = {
     "ba_att_stats": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _P, _P, _P, _P, _P]),
     "ba_att_select": (ctypes.c_int, [ctypes.POINTER(CShape), ctypes.c_double, _P, _P, _P, _P, _P, _P, _I32, _P, _P]),
     "ba_att_split_lists": (ctypes.c_int, [ctypes.POINTER(CShape), _I32, _P, _P, _I32, _P, _P, _P, _P, _P]),
+    "ba_att_complement_lists": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _I32, _P, _P, _I32, _P]),
     "ba_att_sparse_fwd": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _P, _P, _P, _I32, _P, _I32, _P, _P]),
     "ba_att_merge_lse": (ctypes.c_int, [ctypes.c_int64, _I32, _I32, _I32, _P, _P, _P, _P, _P, _P, _P]),
     "ba_att_sparse_fwd_merge": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _P, _P, _P, _I32, _P, _P, _P, _I32, _P,
@@ -203,6 +204,18 @@ def split_lists(idx: torch.Tensor, cnt: torch.Tensor, shape: Shape, split_block:
 
 
 _TORCH_DT = {torch.float32: DTYPE_F32, torch.bfloat16: DTYPE_BF16}
+
+
+def complement_lists(idx, cnt, shape: Shape, out=None):
+    """The key blocks each kept-block list leaves out -> (c_idx [.., nb], c_cnt)."""
+    lib = load_library()
+    if out is None:
+        out = (torch.empty(idx.shape[:-1] + (shape.nb,), device=idx.device, dtype=torch.int32), torch.empty_like(cnt))
+    c_idx, c_cnt = out
+    _check("ba_att_complement_lists", lib.ba_att_complement_lists(
+        ctypes.byref(shape.c()), _dev(idx, "kv_idx"), _dev(cnt, "kv_cnt"), idx.shape[-1], _dev(c_idx, "c_idx"),
+        _dev(c_cnt, "c_cnt"), c_idx.shape[-1], _stream(idx)))
+    return out
 
 
 def sparse_fwd(Q, K, V, idx, cnt, shape: Shape, out=None, out_dtype=None):

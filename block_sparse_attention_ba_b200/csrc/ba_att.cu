@@ -201,6 +201,20 @@ ba_status ba_att_select(const ba_att_shape *s, double keep, const float *q_mean,
   return from_cuda(e);
 }
 
+ba_status ba_att_complement_lists(const ba_att_shape *s, const int32_t *kv_idx, const int32_t *kv_cnt, int32_t kmax,
+                                  int32_t *c_idx, int32_t *c_cnt, int32_t c_kmax, ba_stream_t stream) {
+  ba_status st = check_shape(s);
+  if (st != BA_OK) return st;
+  if (!kv_idx || !kv_cnt || !c_idx || !c_cnt) return BA_ERR_INVALID_ARG;
+  if (!aligned16(kv_idx) || !aligned16(kv_cnt) || !aligned16(c_idx) || !aligned16(c_cnt)) return BA_ERR_MISALIGNED;
+  const int nb = nblocks(s);
+  if (nb > kComplMaxWords * 32) return BA_ERR_UNSUPPORTED;
+  if (kmax < 1 || c_kmax < nb) return BA_ERR_INVALID_ARG;
+  const long long n_lists = static_cast<long long>(s->B) * s->Hq * nb;
+  return from_cuda(launch_complement(kv_idx, kv_cnt, c_idx, c_cnt, n_lists, kmax, c_kmax, nb,
+                                     num_sms_of_current_device(), reinterpret_cast<cudaStream_t>(stream)));
+}
+
 ba_status ba_att_split_lists(const ba_att_shape *s, int32_t split_block, const int32_t *kv_idx, const int32_t *kv_cnt,
                              int32_t kmax, int32_t *lo_idx, int32_t *lo_cnt, int32_t *hi_idx, int32_t *hi_cnt,
                              ba_stream_t stream) {

@@ -148,4 +148,84 @@ inline cudaError_t launch_split(const int32_t *idx, const int32_t *cnt, int32_t 
   return cudaGetLastError();
 }
 
+// The complement of each list: the key blocks of [0, nk) it does not hold,
+// ascending, -1 padded to ckmax (attention over them, merged with attention
+// over the kept blocks, is dense attention: FlashBlock Eq. 5 and Eq. 9). One
+// warp per list marks its blocks in a shared-memory bitmap and emits the
+// clear bits 32 words at a time with a warp prefix sum over the popcounts.
+// Entries outside [0, nk) are ignored and flagged.
+constexpr int kComplWarps = 8;
+constexpr int kComplMaxWords = 4096 / 32;
+
+__global__ void __launch_bounds__(kComplWarps * 32)
+    complement_lists_kernel(const int32_t *__restrict__ idx, const int32_t *__restrict__ cnt,
+                            int32_t *__restrict__ c_idx, int32_t *__restrict__ c_cnt, long long n_lists, int kmax,
+                            int ckmax, int nk) {
+  __shared__ unsigned bits[kComplWarps][kComplMaxWords];
+  const unsigned full = 0xFFFFFFFFu;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int words = (nk + 31) >> 5;
+  unsigned *bw = bits[warp];
+  const long long warps_total = static_cast<long long>(gridDim.x) * kComplWarps;
+  for (long long row = blockIdx.x * static_cast<long long>(kComplWarps) + warp; row < n_lists; row += warps_total) {
+    for (int w = lane; w < words; w += 32) bw[w] = 0u;
+    __syncwarp();
+    int c = __ldg(cnt + row);
+    if (c < 0 || c > kmax) {
+      if (lane == 0) raise_error(BA_DEVERR_BAD_COUNT);
+      c = c < 0 ? 0 : kmax;
+    }
+    const int32_t *in = idx + row * kmax;
+    for (int t = lane; t < c; t += 32) {
+      const int j = __ldg(in + t);
+      if (j >= 0 && j < nk)
+        atomicOr(&bw[j >> 5], 1u << (j & 31));
+      else
+        raise_error(BA_DEVERR_BAD_INDEX);
+    }
+    __syncwarp();
+    int32_t *out = c_idx + row * ckmax;
+    int pos = 0;
+    for (int w0 = 0; w0 < words; w0 += 32) {
+      const int w = w0 + lane;
+      unsigned rest = 0u;
+      if (w < words) {
+        rest = ~bw[w];
+        const int valid = nk - (w << 5);                 // bits of this word inside [0, nk)
+        if (valid < 32) rest &= (1u << valid) - 1u;
+      }
+      const int n = __popc(rest);
+      int incl = n;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(full, incl, off);
+        if (lane >= off) incl += y;
+      }
+      int at = pos + incl - n;
+      while (rest) {                                     // this word's clear blocks, ascending
+        const int bit = __ffs(rest) - 1;
+        rest &= rest - 1u;
+        if (at < ckmax) out[at] = (w << 5) + bit;
+        ++at;
+      }
+      pos += __shfl_sync(full, incl, 31);
+    }
+    for (int t = pos + lane; t < ckmax; t += 32) out[t] = -1;
+    if (lane == 0) c_cnt[row] = pos < ckmax ? pos : ckmax;
+    __syncwarp();                                        // bitmap reused by the next list
+  }
+}
+
+inline cudaError_t launch_complement(const int32_t *idx, const int32_t *cnt, int32_t *c_idx, int32_t *c_cnt,
+                                     long long n_lists, int kmax, int ckmax, int nk, int num_sms,
+                                     cudaStream_t stream) {
+  long long blocks = (n_lists + kComplWarps - 1) / kComplWarps;
+  const long long cap = static_cast<long long>(num_sms) * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  complement_lists_kernel<<<static_cast<unsigned>(blocks), kComplWarps * 32, 0, stream>>>(idx, cnt, c_idx, c_cnt,
+                                                                                         n_lists, kmax, ckmax, nk);
+  return cudaGetLastError();
+}
+
 }  // namespace baatt

@@ -162,6 +162,25 @@ ba_status ba_att_split_lists(const ba_att_shape *shape, int32_t split_block,
                              int32_t *hi_idx, int32_t *hi_cnt, ba_stream_t stream);
 
 /*
+ * ba_att_complement_lists — for every kept-block list, the key blocks of
+ * [0, nk) it leaves out, ascending ("FlashBlock", review of Fig. 6: sparse
+ * attention plus a cached residual over the unselected blocks; by Eq. 5 and
+ * Eq. 9, attention over a list merged with attention over its complement is
+ * dense attention). Pairs with ba_att_sparse_fwd / ba_att_sparse_fwd_merge.
+ *
+ * kv_idx, kv_cnt, kmax   device int32 lists as written by ba_att_select;
+ *                        entries outside [0, nk) are ignored and flagged in
+ *                        the device error word.
+ * c_idx   device int32 [B, Hq, nq, c_kmax]: the complement, ascending,
+ *         -1 padded; c_kmax >= nk (BA_ERR_INVALID_ARG otherwise).
+ * c_cnt   device int32 [B, Hq, nq]: its length, nk minus the distinct valid
+ *         entries. Requires nk <= 4096 (BA_ERR_UNSUPPORTED above).
+ */
+ba_status ba_att_complement_lists(const ba_att_shape *shape, const int32_t *kv_idx, const int32_t *kv_cnt,
+                                  int32_t kmax, int32_t *c_idx, int32_t *c_cnt, int32_t c_kmax,
+                                  ba_stream_t stream);
+
+/*
  * ba_att_sparse_fwd — block-sparse bidirectional attention forward
  * (BA-Att abstract and Figure 4: attention evaluated only over the kept
  * blocks, no causal mask).

@@ -156,3 +156,13 @@ def test_sparse_fwd_merge_arguments(lib):
     assert lib.ba_att_sparse_fwd_merge(ctypes.byref(s), P, P, P, P, P, 4, P, None, P, 1, P, None) == 1
     assert lib.ba_att_sparse_fwd_merge(ctypes.byref(s), P, P, P, P, P, 4, MIS, P, P, 1, P, None) == 3
     assert lib.ba_att_sparse_fwd_merge(ctypes.byref(shape(d=96)), P, P, P, P, P, 4, P, P, P, 1, P, None) == 2
+
+
+def test_complement_lists_arguments(lib):
+    s = shape()                                          # nb = 8
+    assert lib.ba_att_complement_lists(ctypes.byref(s), P, P, 4, P, P, 7, None) == 1       # stride below nb
+    assert lib.ba_att_complement_lists(ctypes.byref(s), None, P, 4, P, P, 8, None) == 1
+    assert lib.ba_att_complement_lists(ctypes.byref(s), P, P, 0, P, P, 8, None) == 1
+    assert lib.ba_att_complement_lists(ctypes.byref(s), P, P, 4, MIS, P, 8, None) == 3
+    big = shape(N=4097 * 16, N_alloc=4097 * 16, block=16)
+    assert lib.ba_att_complement_lists(ctypes.byref(big), P, P, 4, P, P, 4097, None) == 2

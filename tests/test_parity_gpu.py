@@ -183,6 +183,66 @@ def test_split_and_merge_equals_union():
         assert max_abs(Lm, r["L"]) <= 2 * tol["lse_abs"]
 
 
+def test_complement_lists_long_rows_and_odd_entries():
+    # 2000 blocks (63 bitmap words, two rounds of 32), random kept sets of
+    # every size, duplicate and out-of-range entries (ignored and flagged)
+    B, H, nb, kmax = 1, 3, 2000, 64
+    N = nb * 16
+    rng = np.random.default_rng(9)
+    idx = np.full((B, H, nb, kmax), -1, dtype=np.int32)
+    cnt = np.zeros((B, H, nb), dtype=np.int32)
+    for pos in np.ndindex(cnt.shape):
+        c = int(rng.integers(0, kmax + 1))
+        idx[pos][:c] = np.sort(rng.choice(nb, size=c, replace=False))
+        cnt[pos] = c
+    idx[0, 0, 0, :3] = [5, 5, 7]                         # a duplicate
+    cnt[0, 0, 0] = 3
+    shape = api.Shape(B, H, H, N, N, 64, 16, api.DTYPE_F32)
+    c_idx, c_cnt = api.complement_lists(torch.from_numpy(idx).cuda(), torch.from_numpy(cnt).cuda(), shape)
+    torch.cuda.synchronize()
+    ref_idx, ref_cnt = O.complement_lists(idx, cnt, nb)
+    np.testing.assert_array_equal(c_cnt.cpu().numpy(), ref_cnt)
+    np.testing.assert_array_equal(c_idx.cpu().numpy(), ref_idx)
+    idx[0, 1, 0, 0] = nb + 3                              # out of range: ignored, flagged
+    cnt[0, 1, 0] = max(int(cnt[0, 1, 0]), 1)
+    c_idx, c_cnt = api.complement_lists(torch.from_numpy(idx).cuda(), torch.from_numpy(cnt).cuda(), shape)
+    st, word = api.get_device_error()
+    assert st == 5 and word & 0x1                          # BA_ERR_DEVICE, BA_DEVERR_BAD_INDEX
+    ref_idx, ref_cnt = O.complement_lists(idx, cnt, nb)
+    np.testing.assert_array_equal(c_idx.cpu().numpy(), ref_idx)
+
+
+@pytest.mark.parametrize("name,over,keep", [
+    ("dlm_16k", dict(N=2048 - 30, N_alloc=2048, Hq=4, Hkv=2), 0.25),    # tensor-core path, ragged tail
+    ("tiny_fp32", dict(N=1000, N_alloc=1024), 0.5),                      # CUDA-core path, fp32
+    ("tiny_fp32", dict(N=4800 - 7, N_alloc=4800, block=16, Hq=2, Hkv=1), 0.3),   # 300 blocks, 10 bitmap words
+])
+def test_complement_lists_and_cached_residual_is_dense(name, over, keep):
+    # the complement lists equal the oracle's exactly; attention over the kept
+    # blocks merged with attention over the rest is dense attention
+    Q, K, V, meta = make_inputs(name, **over)
+    w = meta["workload"]
+    r = run_gpu(Q, K, V, w, keep)
+    shape = r["shape"]
+    c_idx, c_cnt = api.complement_lists(r["idx_d"], r["cnt_d"], shape)
+    ref_idx, ref_cnt = O.complement_lists(r["idx"], r["cnt"], w.nb)
+    np.testing.assert_array_equal(c_cnt.cpu().numpy(), ref_cnt)
+    np.testing.assert_array_equal(c_idx.cpu().numpy(), ref_idx)
+    O1, L1 = api.sparse_fwd(r["Qd"], r["Kd"], r["Vd"], r["idx_d"], r["cnt_d"], shape, out_dtype=torch.float32)
+    Of, Lf = api.sparse_fwd_merge(r["Qd"], r["Kd"], r["Vd"], c_idx, c_cnt, shape, O1, L1)
+    torch.cuda.synchronize()
+    Od, Ld = O.dense_attention(Q, K, V, w.N, w.d ** -0.5)
+    tol = TOL[w.dtype]
+    got = Of[:, :, :w.N].float().cpu().numpy()
+    assert max_abs(got, Od) <= tol["max_abs"] and rel_l2(got, Od) <= tol["rel_l2"]
+    assert max_abs(Lf[:, :, :w.N].cpu().numpy(), Ld) <= tol["lse_abs"]
+    # keep = 1: nothing is left out
+    idx_all, cnt_all = api.select(api.stats(r["Qd"], r["Kd"], shape), shape, 1.0)
+    c_idx, c_cnt = api.complement_lists(idx_all, cnt_all, shape)
+    torch.cuda.synchronize()
+    assert int(c_cnt.max()) == 0 and bool((c_idx == -1).all())
+
+
 @pytest.mark.parametrize("name,over", [
     ("extreme_128k", dict(N=4096 - 50, N_alloc=4096, Hq=4, Hkv=2)),      # tensor-core path, ragged tail
     ("tiny_fp32", dict(N=1000, N_alloc=1024)),                             # CUDA-core path, fp32
