@@ -38,6 +38,7 @@ from .ba_att_oracle import (  # noqa: F401
     pooled_scores,
     pre_downsample_map,
     select_topk,
+    selection_scores,
     near_tie_mask,
     masked_attention,
     dense_attention,

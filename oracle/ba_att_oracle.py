@@ -87,7 +87,7 @@ def _kv_head(h: int, Hq: int, Hkv: int) -> int:
 
 
 def corrected_scores(q_mean, q_var, k_mean, k_var, k_counts, sm_scale: float,
-                     dtype=np.float64):
+                     dtype=np.float64, var_product: bool = True):
     """Covariance-compensated downsampled block scores S~[B, Hq, nq, nk].
 
     [BA-Att, abstract; "Core claim"]: blocks are scored in the compact
@@ -107,6 +107,9 @@ def corrected_scores(q_mean, q_var, k_mean, k_var, k_counts, sm_scale: float,
     A key block of m_j tokens contributes m_j such terms, hence + ln m_j:
         S~_ij = s * qbar_i.kbar_j + (s^2 / 2) * V_ij + ln m_j.
     Query head h reads the statistics of KV head g(h).
+
+    var_product=False drops the var_q * var_k term of V_ij (a selection
+    variant: the correction from the means' cross terms only).
     """
     q_mean = np.asarray(q_mean, dtype=dtype)
     q_var = np.asarray(q_var, dtype=dtype)
@@ -123,8 +126,9 @@ def corrected_scores(q_mean, q_var, k_mean, k_var, k_counts, sm_scale: float,
         km, kv = k_mean[:, g], k_var[:, g]          # [B, nk, d]
         mean_term = s * (qm @ km.transpose(0, 2, 1))
         V = (qv @ (km * km).transpose(0, 2, 1)
-             + (qm * qm) @ kv.transpose(0, 2, 1)
-             + qv @ kv.transpose(0, 2, 1))
+             + (qm * qm) @ kv.transpose(0, 2, 1))
+        if var_product:
+            V = V + qv @ kv.transpose(0, 2, 1)
         S[:, h] = mean_term + dtype(0.5) * s * s * V + log_m[None, None, :]
     return S
 
@@ -183,6 +187,27 @@ def select_topk(S, k: int, kmax: int | None = None):
     idx[..., :k] = kept
     cnt = np.full(S.shape[:-1], k, dtype=np.int32)
     return idx, cnt
+
+
+def selection_scores(S, Hkv: int, force_diagonal: bool = False, shared_gqa: bool = False):
+    """The scores a selection variant ranks, from the per-head S~ [B, Hq, nq, nk].
+
+    Variants of the norm sorting (the pages fix none of them; each is a plain
+    option around the ranking of "The pith"/"Core claim"):
+      shared_gqa      the query heads of one KV group share one selection,
+                      ranked by the mean of their S~ over the group;
+      force_diagonal  query block i always keeps key block i (ranked first).
+    ``select_topk`` of the result gives the lists.
+    """
+    R = np.array(S, dtype=np.float64, copy=True)
+    B, Hq, nq, nk = R.shape
+    if shared_gqa:
+        G = Hq // Hkv
+        R = np.repeat(R.reshape(B, Hkv, G, nq, nk).mean(axis=2), G, axis=1)
+    if force_diagonal:
+        n = min(nq, nk)
+        R[..., np.arange(n), np.arange(n)] = np.inf
+    return R
 
 
 def near_tie_mask(S, k: int, rel: float = 1e-3):

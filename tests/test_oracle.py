@@ -341,6 +341,42 @@ def test_complement_lists_partition_and_kept_plus_rest_is_dense():
     assert ccnt[0, 0, 0] == 6 and list(cidx[0, 0, 0]) == [1, 2, 3, 4, 5, 6, -1, -1]
 
 
+def test_selection_variants():
+    rng = np.random.default_rng(11)
+    B, Hq, Hkv, nb, d = 2, 4, 2, 9, 8
+    qm, qv = rng.standard_normal((B, Hq, nb, d)), rng.random((B, Hq, nb, d))
+    km, kv = rng.standard_normal((B, Hkv, nb, d)), rng.random((B, Hkv, nb, d))
+    counts = np.full(nb, 16.0)
+    s = 0.3
+    full = O.corrected_scores(qm, qv, km, kv, counts, s)
+    novar = O.corrected_scores(qm, qv, km, kv, counts, s, var_product=False)
+    # the dropped term is (s^2/2) var_q . var_k, a plain matrix product per head
+    G = Hq // Hkv
+    for h in range(Hq):
+        np.testing.assert_allclose(full[:, h] - novar[:, h],
+                                   0.5 * s * s * np.einsum("bid,bjd->bij", qv[:, h], kv[:, h // G]), rtol=1e-12)
+    assert (full >= novar - 1e-12).all()
+    np.testing.assert_allclose(O.corrected_scores(qm, qv, km, 0 * kv, counts, s),
+                               O.corrected_scores(qm, qv, km, 0 * kv, counts, s, var_product=False), rtol=0)
+    k = 3
+    # forced diagonal: block i always kept, plus the best k-1 of the others
+    idx, cnt = O.select_topk(O.selection_scores(full, Hkv, force_diagonal=True), k)
+    for pos in np.ndindex(cnt.shape):
+        i = pos[-1]
+        row = full[pos]
+        others = sorted((j for j in range(nb) if j != i), key=lambda j: (-row[j], j))[: k - 1]
+        assert sorted(idx[pos][:k]) == sorted(others + [i])
+    # shared GQA selection: one list per KV group, the top k of the group mean
+    idx, cnt = O.select_topk(O.selection_scores(full, Hkv, shared_gqa=True), k)
+    for b in range(B):
+        for g in range(Hkv):
+            mean = full[b, g * G:(g + 1) * G].mean(axis=0)
+            for i in range(nb):
+                best = sorted(range(nb), key=lambda j: (-mean[i, j], j))[:k]
+                for hh in range(G):
+                    assert list(idx[b, g * G + hh, i, :k]) == sorted(best)
+
+
 def test_merge_edge_cases():
     o1 = np.array([[1.0, 2.0], [3.0, 4.0]])
     o2 = np.array([[5.0, 6.0], [7.0, 8.0]])
