@@ -23,6 +23,7 @@ BA_ERR_INVALID_ARG = 1
 STATUS_NAMES = {0: "BA_OK", 1: "BA_ERR_INVALID_ARG", 2: "BA_ERR_UNSUPPORTED", 3: "BA_ERR_MISALIGNED",
                 4: "BA_ERR_CUDA", 5: "BA_ERR_DEVICE", 6: "BA_ERR_TIMEOUT"}
 DTYPE_F32, DTYPE_BF16 = 0, 1
+SELECT_NO_VAR_PRODUCT, SELECT_FORCE_DIAGONAL, SELECT_SHARED_GQA = 0x1, 0x2, 0x4    # ba_att_select_ex flags
 
 # Entry points declared in include/ba_att.h: name -> (restype, argtypes)
 _P = ctypes.c_void_p
@@ -42,6 +43,8 @@ _SIGS = {
     "ba_att_keep_count": (_I32, [ctypes.POINTER(CShape), ctypes.c_double]),
     "ba_att_stats": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _P, _P, _P, _P, _P]),
     "ba_att_select": (ctypes.c_int, [ctypes.POINTER(CShape), ctypes.c_double, _P, _P, _P, _P, _P, _P, _I32, _P, _P]),
+    "ba_att_select_ex": (ctypes.c_int, [ctypes.POINTER(CShape), ctypes.c_double, ctypes.c_uint32, _P, _P, _P, _P, _P,
+                                         _P, _I32, _P, _P]),
     "ba_att_split_lists": (ctypes.c_int, [ctypes.POINTER(CShape), _I32, _P, _P, _I32, _P, _P, _P, _P, _P]),
     "ba_att_complement_lists": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _I32, _P, _P, _I32, _P]),
     "ba_att_sparse_fwd": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _P, _P, _P, _I32, _P, _I32, _P, _P]),
@@ -164,11 +167,12 @@ def stats(Q: torch.Tensor, K: torch.Tensor, shape: Shape, out=None):
     return out
 
 
-def select(stats_out, shape: Shape, keep: float, kmax: int | None = None, with_scores: bool = False, out=None):
+def select(stats_out, shape: Shape, keep: float, kmax: int | None = None, with_scores: bool = False, out=None,
+           flags: int = 0):
     """Corrected block scores + top-k -> (idx, cnt), or (idx, cnt, scores) with with_scores.
 
     The score map [B, Hq, nq, nk] fp32 is always written; out = (idx, cnt, scores) may pass
-    a preallocated one."""
+    a preallocated one. flags: SELECT_* variants (ba_att_select_ex)."""
     lib = load_library()
     qm, qv, km, kv = stats_out
     k = keep_count(shape, keep)
@@ -184,10 +188,10 @@ def select(stats_out, shape: Shape, keep: float, kmax: int | None = None, with_s
         idx, cnt, sc = out
     if sc is None:       # the score map is always written (the selection reads it back)
         sc = torch.empty((shape.B, shape.Hq, shape.nb, shape.nb), device=dev, dtype=torch.float32)
-    _check("ba_att_select", lib.ba_att_select(
-        ctypes.byref(shape.c()), ctypes.c_double(keep), _dev(qm, "q_mean"), _dev(qv, "q_var"), _dev(km, "k_mean"),
-        _dev(kv, "k_var"), _dev(idx, "kv_idx"), _dev(cnt, "kv_cnt"), idx.shape[-1],
-        _dev(sc, "block_scores"), _stream(qm)))
+    _check("ba_att_select_ex", lib.ba_att_select_ex(
+        ctypes.byref(shape.c()), ctypes.c_double(keep), ctypes.c_uint32(flags), _dev(qm, "q_mean"),
+        _dev(qv, "q_var"), _dev(km, "k_mean"), _dev(kv, "k_var"), _dev(idx, "kv_idx"), _dev(cnt, "kv_cnt"),
+        idx.shape[-1], _dev(sc, "block_scores"), _stream(qm)))
     return (idx, cnt, sc) if with_scores else (idx, cnt)
 
 

@@ -176,11 +176,13 @@ ba_status ba_att_stats(const ba_att_shape *s, const void *Q, const void *K, floa
   return from_cuda(e);
 }
 
-ba_status ba_att_select(const ba_att_shape *s, double keep, const float *q_mean, const float *q_var,
-                        const float *k_mean, const float *k_var, int32_t *kv_idx, int32_t *kv_cnt, int32_t kmax,
-                        float *block_scores, ba_stream_t stream) {
+ba_status ba_att_select_ex(const ba_att_shape *s, double keep, uint32_t flags, const float *q_mean,
+                           const float *q_var, const float *k_mean, const float *k_var, int32_t *kv_idx,
+                           int32_t *kv_cnt, int32_t kmax, float *block_scores, ba_stream_t stream) {
   ba_status st = check_shape(s);
   if (st != BA_OK) return st;
+  constexpr uint32_t kKnown = BA_SELECT_NO_VAR_PRODUCT | BA_SELECT_FORCE_DIAGONAL | BA_SELECT_SHARED_GQA;
+  if (flags & ~kKnown) return BA_ERR_INVALID_ARG;
   if (!q_mean || !q_var || !k_mean || !k_var || !kv_idx || !kv_cnt || !block_scores) return BA_ERR_INVALID_ARG;
   if (!aligned16(q_mean) || !aligned16(q_var) || !aligned16(k_mean) || !aligned16(k_var) || !aligned16(kv_idx) ||
       !aligned16(kv_cnt) || !aligned16(block_scores))
@@ -190,15 +192,21 @@ ba_status ba_att_select(const ba_att_shape *s, double keep, const float *q_mean,
   if (kmax < k) return BA_ERR_INVALID_ARG;
   const int nb = nblocks(s);
   if (nb > 4096) return BA_ERR_UNSUPPORTED;
+  if ((flags & (BA_SELECT_FORCE_DIAGONAL | BA_SELECT_SHARED_GQA)) && nb > 1024) return BA_ERR_UNSUPPORTED;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   const float scale = effective_scale(s);
-  cudaError_t e;
   const int sms = num_sms_of_current_device();
-  e = s->d == 128 ? launch_select_tc<128>(q_mean, q_var, k_mean, k_var, kv_idx, kv_cnt, block_scores, s->B, s->Hq,
-                                          s->Hkv, s->N, s->block, k, kmax, scale, sms, cs)
-                  : launch_select_tc<64>(q_mean, q_var, k_mean, k_var, kv_idx, kv_cnt, block_scores, s->B, s->Hq,
-                                         s->Hkv, s->N, s->block, k, kmax, scale, sms, cs);
+  cudaError_t e = s->d == 128 ? launch_select_tc<128>(q_mean, q_var, k_mean, k_var, kv_idx, kv_cnt, block_scores, s->B,
+                                                      s->Hq, s->Hkv, s->N, s->block, k, kmax, scale, flags, sms, cs)
+                              : launch_select_tc<64>(q_mean, q_var, k_mean, k_var, kv_idx, kv_cnt, block_scores, s->B,
+                                                     s->Hq, s->Hkv, s->N, s->block, k, kmax, scale, flags, sms, cs);
   return from_cuda(e);
+}
+
+ba_status ba_att_select(const ba_att_shape *s, double keep, const float *q_mean, const float *q_var,
+                        const float *k_mean, const float *k_var, int32_t *kv_idx, int32_t *kv_cnt, int32_t kmax,
+                        float *block_scores, ba_stream_t stream) {
+  return ba_att_select_ex(s, keep, 0u, q_mean, q_var, k_mean, k_var, kv_idx, kv_cnt, kmax, block_scores, stream);
 }
 
 ba_status ba_att_complement_lists(const ba_att_shape *s, const int32_t *kv_idx, const int32_t *kv_cnt, int32_t kmax,

@@ -529,6 +529,89 @@ inline cudaError_t launch_topk_kpl(const float *scores, int nk, int k, int32_t *
   return cudaGetLastError();
 }
 
+// Selection variants (the plain top-k above is the default):
+//   group > 1       the `group` query heads of a KV group share one selection,
+//                   ranked by the mean of their scores (one warp per
+//                   (batch, KV head, query block); the list is written to
+//                   every head of the group);
+//   force_diagonal  key block i always ranks first for query block i.
+// Rows of at most 1024 keys, held in registers.
+struct TopkVariant {
+  int group;            // query heads per selection (1: none shared)
+  int heads;            // Hq
+  int nq;               // query blocks per head (= nk)
+  bool force_diagonal;
+};
+
+template <int KPL>
+__global__ void __launch_bounds__(kTopkWarps * 32) topk_variant_kernel(const float *__restrict__ scores, int nk, int k,
+                                                                       int32_t *__restrict__ kv_idx, int kmax,
+                                                                       int32_t *__restrict__ kv_cnt, long long sel_rows,
+                                                                       TopkVariant var) {
+  __shared__ __align__(16) unsigned hist[kTopkWarps][256];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long stride = static_cast<long long>(gridDim.x) * kTopkWarps;
+  const int kv_heads = var.heads / var.group;
+  const float inv_group = 1.f / static_cast<float>(var.group);
+  for (long long r = blockIdx.x * static_cast<long long>(kTopkWarps) + warp; r < sel_rows; r += stride) {
+    const int i = static_cast<int>(r % var.nq);
+    const long long bg = r / var.nq;                   // b*Hkv + g (shared) or b*Hq + h
+    const long long first_row = var.group > 1
+                                    ? ((bg / kv_heads) * var.heads + (bg % kv_heads) * var.group) * var.nq + i
+                                    : r;
+    float acc[KPL];
+#pragma unroll
+    for (int c = 0; c < KPL; ++c) acc[c] = 0.f;
+    for (int hh = 0; hh < var.group; ++hh) {           // heads of the group are consecutive score rows nq apart
+      const float *srow = scores + (first_row + static_cast<long long>(hh) * var.nq) * nk;
+#pragma unroll
+      for (int c = 0; c < KPL; ++c) {
+        const int j = c * 32 + lane;
+        if (j < nk) acc[c] += __ldg(srow + j);
+      }
+    }
+    uint32_t u[KPL];
+#pragma unroll
+    for (int c = 0; c < KPL; ++c) {
+      const int j = c * 32 + lane;
+      u[c] = order_key(var.group > 1 ? acc[c] * inv_group : acc[c]);
+      if (var.force_diagonal && j == i) u[c] = 0xFFFFFFFFu;
+    }
+    int32_t *out = kv_idx + first_row * kmax;
+    topk_row_regs<KPL>(u, nk, k, out, kmax, kv_cnt + first_row, smem_u32(&hist[warp][0]), lane);
+    __syncwarp();
+    for (int hh = 1; hh < var.group; ++hh) {           // the same list for the other heads of the group
+      const long long orow = first_row + static_cast<long long>(hh) * var.nq;
+      for (int t = lane; t < kmax; t += 32) kv_idx[orow * kmax + t] = out[t];
+      if (lane == 0) kv_cnt[orow] = kv_cnt[first_row];
+    }
+  }
+}
+
+template <int KPL>
+inline cudaError_t launch_topk_variant_kpl(const float *scores, int nk, int k, int32_t *idx, int kmax, int32_t *cnt,
+                                           long long sel_rows, const TopkVariant &var, int num_sms,
+                                           cudaStream_t stream) {
+  const int threads = kTopkWarps * 32;
+  int per_sm = 0;
+  const cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, topk_variant_kernel<KPL>, threads, 0);
+  if (e != cudaSuccess) return e;
+  long long grid = (sel_rows + kTopkWarps - 1) / kTopkWarps;
+  const long long slots = static_cast<long long>(num_sms) * (per_sm > 0 ? per_sm : 1);
+  grid = grid < slots ? grid : slots;
+  topk_variant_kernel<KPL><<<static_cast<unsigned>(grid), threads, 0, stream>>>(scores, nk, k, idx, kmax, cnt,
+                                                                                sel_rows, var);
+  return cudaGetLastError();
+}
+
+// sel_rows = B * (Hq / group) * nq
+inline cudaError_t launch_topk_variant(const float *scores, int nk, int k, int32_t *idx, int kmax, int32_t *cnt,
+                                       long long sel_rows, const TopkVariant &var, int num_sms, cudaStream_t stream) {
+  if (nk <= 256) return launch_topk_variant_kpl<8>(scores, nk, k, idx, kmax, cnt, sel_rows, var, num_sms, stream);
+  if (nk <= 512) return launch_topk_variant_kpl<16>(scores, nk, k, idx, kmax, cnt, sel_rows, var, num_sms, stream);
+  return launch_topk_variant_kpl<32>(scores, nk, k, idx, kmax, cnt, sel_rows, var, num_sms, stream);
+}
+
 inline cudaError_t launch_topk(const float *scores, int nk, int k, int32_t *idx, int kmax, int32_t *cnt,
                                long long rows, int num_sms, cudaStream_t stream) {
   if (nk <= 256) return launch_topk_kpl<8>(scores, nk, k, idx, kmax, cnt, rows, num_sms, stream);

@@ -73,7 +73,8 @@ template <int D, int NT>
 __global__ void __launch_bounds__(kThreads, 1)
     select_tc_kernel(const float *__restrict__ q_mean, const float *__restrict__ q_var,
                      const float *__restrict__ k_mean, const float *__restrict__ k_var,
-                     float *__restrict__ block_scores, int Hq, int Hkv, int N, int block, int nb, float sm_scale) {
+                     float *__restrict__ block_scores, int Hq, int Hkv, int N, int block, int nb, float sm_scale,
+                     int var_product) {
   using TL = Tile<NT>;
   constexpr int GROUPS = D / 64;
   constexpr int TPT = TL::kTasksPerThread;
@@ -147,7 +148,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (is_a)
             x[q] = p == 0 ? s * m[q] : (p == 1 ? hs2 * v[q] : hs2 * m[q] * m[q]);
           else
-            x[q] = p == 0 ? m[q] : (p == 1 ? fmaf(m[q], m[q], v[q]) : v[q]);
+            x[q] = p == 0 ? m[q] : (p == 1 ? (var_product ? fmaf(m[q], m[q], v[q]) : m[q] * m[q]) : v[q]);
         }
         uint4 hi, lo;
         split8(x, hi, lo);
@@ -254,10 +255,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // Scores with the widest key tile that still gives at least half the SMs a
 // CTA, then the top-k launch.
+// flags: the ba_att_select_ex bits (BA_SELECT_*).
 template <int D>
 cudaError_t launch_select_tc(const float *qm, const float *qv, const float *km, const float *kv, int32_t *idx,
                              int32_t *cnt, float *scores, int B, int Hq, int Hkv, int N, int block, int k, int kmax,
-                             float sm_scale, int num_sms, cudaStream_t stream) {
+                             float sm_scale, uint32_t flags, int num_sms, cudaStream_t stream) {
+  const int var_product = (flags & BA_SELECT_NO_VAR_PRODUCT) ? 0 : 1;
   const int nb = (N + block - 1) / block;
   const long long bhs = static_cast<long long>(B) * Hq;
   const int nq_tiles = (nb + seltc::kRows - 1) / seltc::kRows;
@@ -270,7 +273,8 @@ cudaError_t launch_select_tc(const float *qm, const float *qv, const float *km, 
     if (e != cudaSuccess) return e;
     dim3 grid(((nb + 127) / 128) * nq_tiles, Hq, B);
     seltc::select_tc_kernel<D, 128><<<grid, seltc::kThreads, TL::kDynSmem, stream>>>(qm, qv, km, kv, scores, Hq, Hkv,
-                                                                                      N, block, nb, sm_scale);
+                                                                                      N, block, nb, sm_scale,
+                                                                                      var_product);
   } else {
     using TL = seltc::Tile<64>;
     e = cudaFuncSetAttribute(seltc::select_tc_kernel<D, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -278,11 +282,16 @@ cudaError_t launch_select_tc(const float *qm, const float *qv, const float *km, 
     if (e != cudaSuccess) return e;
     dim3 grid(((nb + 63) / 64) * nq_tiles, Hq, B);
     seltc::select_tc_kernel<D, 64><<<grid, seltc::kThreads, TL::kDynSmem, stream>>>(qm, qv, km, kv, scores, Hq, Hkv,
-                                                                                     N, block, nb, sm_scale);
+                                                                                     N, block, nb, sm_scale,
+                                                                                     var_product);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  return launch_topk(scores, nb, k, idx, kmax, cnt, bhs * nb, num_sms, stream);
+  const bool shared = (flags & BA_SELECT_SHARED_GQA) != 0, diag = (flags & BA_SELECT_FORCE_DIAGONAL) != 0;
+  if (!shared && !diag) return launch_topk(scores, nb, k, idx, kmax, cnt, bhs * nb, num_sms, stream);
+  const TopkVariant var{shared ? Hq / Hkv : 1, Hq, nb, diag};
+  return launch_topk_variant(scores, nb, k, idx, kmax, cnt, static_cast<long long>(B) * (Hq / var.group) * nb, var,
+                             num_sms, stream);
 }
 
 }  // namespace baatt

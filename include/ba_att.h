@@ -161,6 +161,31 @@ ba_status ba_att_split_lists(const ba_att_shape *shape, int32_t split_block,
                              int32_t *lo_idx, int32_t *lo_cnt,
                              int32_t *hi_idx, int32_t *hi_cnt, ba_stream_t stream);
 
+/* Selection variants for ba_att_select_ex (bit flags; the pages fix none of
+ * them, they are options around the ranking of "The pith" / "Core claim"). */
+#define BA_SELECT_NO_VAR_PRODUCT  0x1u  /* drop the var_q * var_k term of the correction   */
+#define BA_SELECT_FORCE_DIAGONAL  0x2u  /* query block i always keeps key block i           */
+#define BA_SELECT_SHARED_GQA      0x4u  /* one selection per KV group: mean S~ of its heads */
+
+/*
+ * ba_att_select_ex — ba_att_select with selection variants (flags, above).
+ *  - NO_VAR_PRODUCT: S~ without the (s^2/2) sum_m vq_i,m vk_j,m term; the
+ *    score map holds this S~.
+ *  - FORCE_DIAGONAL: block i of every query block i is kept and ranked
+ *    first; the other k-1 follow the usual ranking.
+ *  - SHARED_GQA: the Hq/Hkv query heads of each KV group rank key blocks by
+ *    the mean of their S~ (fp32, summed in head order) and all receive the
+ *    same list; the score map still holds each head's own S~.
+ * flags = 0 is ba_att_select. FORCE_DIAGONAL and SHARED_GQA require
+ * nk <= 1024 (BA_ERR_UNSUPPORTED above); unknown bits -> BA_ERR_INVALID_ARG.
+ * Other arguments as for ba_att_select.
+ */
+ba_status ba_att_select_ex(const ba_att_shape *shape, double keep, uint32_t flags,
+                           const float *q_mean, const float *q_var,
+                           const float *k_mean, const float *k_var,
+                           int32_t *kv_idx, int32_t *kv_cnt, int32_t kmax,
+                           float *block_scores, ba_stream_t stream);
+
 /*
  * ba_att_complement_lists — for every kept-block list, the key blocks of
  * [0, nk) it leaves out, ascending ("FlashBlock", review of Fig. 6: sparse

@@ -166,3 +166,16 @@ def test_complement_lists_arguments(lib):
     assert lib.ba_att_complement_lists(ctypes.byref(s), P, P, 4, MIS, P, 8, None) == 3
     big = shape(N=4097 * 16, N_alloc=4097 * 16, block=16)
     assert lib.ba_att_complement_lists(ctypes.byref(big), P, P, 4, P, P, 4097, None) == 2
+
+
+def test_select_variant_arguments(lib):
+    s = shape()
+    args = (P, P, P, P, P, P, 8, P, None)
+    assert lib.ba_att_select_ex(ctypes.byref(s), ctypes.c_double(0.5), ctypes.c_uint32(0x8), *args) == 1
+    big = shape(N=1025 * 16, N_alloc=1025 * 16, block=16)
+    bigargs = (P, P, P, P, P, P, 1025, P, None)
+    for flag in (api.SELECT_FORCE_DIAGONAL, api.SELECT_SHARED_GQA):
+        assert lib.ba_att_select_ex(ctypes.byref(big), ctypes.c_double(0.5), ctypes.c_uint32(flag), *bigargs) == 2
+    # the plain variant-free flag set of ba_att_select still reaches the same checks
+    assert lib.ba_att_select_ex(ctypes.byref(s), ctypes.c_double(0.5), ctypes.c_uint32(0), P, P, P, P, P, P, 3,
+                                P, None) == 1

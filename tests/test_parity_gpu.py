@@ -183,6 +183,42 @@ def test_split_and_merge_equals_union():
         assert max_abs(Lm, r["L"]) <= 2 * tol["lse_abs"]
 
 
+@pytest.mark.parametrize("flags", [api.SELECT_NO_VAR_PRODUCT, api.SELECT_FORCE_DIAGONAL, api.SELECT_SHARED_GQA,
+                                   api.SELECT_NO_VAR_PRODUCT | api.SELECT_FORCE_DIAGONAL | api.SELECT_SHARED_GQA])
+@pytest.mark.parametrize("name,over,keep", [
+    ("dlm_16k", dict(N=2048 - 40, N_alloc=2048, Hq=8, Hkv=2), 0.25),       # 16 blocks, 4 heads per group
+    ("tiny_fp32", dict(N=1000, N_alloc=1024, Hq=4, Hkv=2), 0.5),            # d = 64
+    ("dlm_16k", dict(N=300 * 128 - 5, Hq=2, Hkv=1), 0.3),                   # 300 blocks, 16 keys per lane
+])
+def test_selection_variants(name, over, keep, flags):
+    Q, K, V, meta = make_inputs(name, **over)
+    w = meta["workload"]
+    Qd, Kd = to_dev(Q, w.dtype), to_dev(K, w.dtype)
+    shape = api.Shape.of(Qd, Kd, w.N, w.block)
+    st = api.stats(Qd, Kd, shape)
+    idx, cnt, sc = api.select(st, shape, keep, with_scores=True, flags=flags)
+    torch.cuda.synchronize()
+    qm, qv, _ = O.block_stats(Q, w.N, w.block)
+    km, kv, kc = O.block_stats(K, w.N, w.block)
+    S = O.corrected_scores(qm, qv, km, kv, kc, w.d ** -0.5, var_product=not (flags & api.SELECT_NO_VAR_PRODUCT))
+    err = np.abs(sc.cpu().numpy() - S)
+    assert np.all(err <= 1e-5 * np.abs(S) + 5e-5), err.max()
+    R = O.selection_scores(S, w.Hkv, force_diagonal=bool(flags & api.SELECT_FORCE_DIAGONAL),
+                           shared_gqa=bool(flags & api.SELECT_SHARED_GQA))
+    k = O.keep_count(keep, w.nb)
+    idx_ref, cnt_ref = O.select_topk(R, k)
+    got = mask_of(idx.cpu().numpy(), cnt.cpu().numpy(), w.nb)
+    ref = mask_of(idx_ref, cnt_ref, w.nb)
+    near = O.near_tie_mask(R, k, NEAR_TIE_REL)
+    assert not ((got != ref) & ~near).any()
+    if flags & api.SELECT_FORCE_DIAGONAL:
+        assert got[..., np.arange(w.nb), np.arange(w.nb)].all()
+    if flags & api.SELECT_SHARED_GQA:
+        G = w.Hq // w.Hkv
+        g_idx = idx.cpu().numpy().reshape(w.B, w.Hkv, G, w.nb, -1)
+        assert (g_idx == g_idx[:, :, :1]).all()
+
+
 def test_complement_lists_long_rows_and_odd_entries():
     # 2000 blocks (63 bitmap words, two rounds of 32), random kept sets of
     # every size, duplicate and out-of-range entries (ignored and flagged)
