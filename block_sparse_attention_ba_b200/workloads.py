@@ -186,5 +186,7 @@ def make_inputs(w: Workload | str, **overrides):
     gen = {"iid_planted": _gen_iid_planted, "shared_dir": _gen_shared_dir,
            "video_field": _gen_video_field}[w.kind]
     Q, K, V, meta = gen(w)
+    if w.split and "split_block" not in meta:      # generators without their own split point
+        meta["split_block"] = int(np.random.default_rng([w.seed, 2]).integers(1, w.nb))
     meta["workload"] = w
     return round_to(Q, w.dtype), round_to(K, w.dtype), round_to(V, w.dtype), meta
