@@ -1,5 +1,5 @@
 // attn_tc.cuh — K8: block-sparse attention forward on the 5th-generation
-// tensor cores (tcgen05 + TMEM), bf16 inputs, d = 128, block = 128.
+// tensor cores (tcgen05 + TMEM), bf16 inputs, d = 64 or 128, block = 128.
 //
 // Operator: "Efficient Long-Context Modeling in DLMs via Block Approximate
 // Sparse Attention" (abstract; Figure 4) — bidirectional attention over the
@@ -7,7 +7,7 @@
 // softmax over blocks is the FlashAttention recurrence the pages compare to.
 //
 // One CTA = one 128-row query block of one (batch, head) = one tile. Two CTAs
-// share an SM (96 KB shared memory and 256 TMEM columns each), so one CTA's
+// share an SM (up to 96 KB shared memory and 256 TMEM columns each), so one CTA's
 // softmax overlaps the other CTA's MMAs. Roles (192 threads):
 //   warps 0-3  softmax + correction + epilogue; thread t owns query row t,
 //              i.e. TMEM lane t (a warp may only touch its own 32 lanes)
@@ -38,12 +38,18 @@ namespace tc {
 
 constexpr int kThreads = 192;
 constexpr int kTileRows = 128;
-constexpr int kHeadDim = 128;
 constexpr uint32_t kHalfBytes = 128 * 64 * 2;        // 128 rows x 64 bf16 (one 128-byte swizzle span)
-constexpr uint32_t kTileBytes = 2 * kHalfBytes;      // 128 x 128 bf16
-constexpr uint32_t kSmemQ = 0, kSmemK = kTileBytes, kSmemV = 2 * kTileBytes;
-constexpr uint32_t kDynSmem = 3 * kTileBytes + 1024; // + alignment slack
-constexpr int kTmemCols = 256;
+// Per head dimension D (64 or 128): D/64 swizzle spans per 128-row tile.
+template <int D>
+struct Dims {
+  static_assert(D == 64 || D == 128, "head dimension");
+  static constexpr int kSpans = D / 64;
+  static constexpr uint32_t kTileBytes = kSpans * kHalfBytes;    // 128 x D bf16
+  static constexpr uint32_t kSmemQ = 0, kSmemK = kTileBytes, kSmemV = 2 * kTileBytes;
+  static constexpr uint32_t kDynSmem = 3 * kTileBytes + 1024;   // + alignment slack
+};
+constexpr uint32_t dyn_smem_bytes(int d) { return d == 64 ? Dims<64>::kDynSmem : Dims<128>::kDynSmem; }
+constexpr int kTmemCols = 256;                       // S (128) + O (D <= 128), a power of two
 constexpr uint32_t kColS = 0, kColO = 128;
 constexpr float kRescaleLog2 = 8.0f;
 constexpr int kHalfKeys = 64;                        // keys per half block
@@ -110,7 +116,7 @@ __device__ __forceinline__ void exp_pack_store(const uint32_t (&sr)[2][32], floa
 // (O_prev, L_prev) over a disjoint key set before storing (O and LSE may
 // alias O_prev and L_prev when TO is float: each row is read before it is
 // written, by the same thread).
-template <typename TO, bool MERGE>
+template <typename TO, bool MERGE, int D>
 __global__ void __launch_bounds__(kThreads, 2)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const int32_t *__restrict__ kv_idx,
@@ -119,7 +125,8 @@ __global__ void __launch_bounds__(kThreads, 2)
   extern __shared__ uint8_t dyn_smem[];
   __shared__ Ctl ctl;
   const uint32_t smem_base = (smem_u32(dyn_smem) + 1023u) & ~1023u;
-  const uint32_t sQ = smem_base + kSmemQ, sK = smem_base + kSmemK, sV = smem_base + kSmemV;
+  using DM = Dims<D>;
+  const uint32_t sQ = smem_base + DM::kSmemQ, sK = smem_base + DM::kSmemK, sV = smem_base + DM::kSmemV;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -172,9 +179,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     tma_prefetch_desc(tm);
     if (is_k) {
       tma_prefetch_desc(&tm_q);
-      mbar_arrive_expect_tx(bar(Q_FULL), kTileBytes);
-      tma_load_3d(&tm_q, sQ, bar(Q_FULL), 0, i * kTileRows, qz);
-      tma_load_3d(&tm_q, sQ + kHalfBytes, bar(Q_FULL), 64, i * kTileRows, qz);
+      mbar_arrive_expect_tx(bar(Q_FULL), DM::kTileBytes);
+#pragma unroll
+      for (int sp = 0; sp < DM::kSpans; ++sp) tma_load_3d(&tm_q, sQ + sp * kHalfBytes, bar(Q_FULL), 64 * sp, i * kTileRows, qz);
     }
     int issued = -1;                    // last half-block index u loaded
     bool bad_index = false, bad_order = false;
@@ -192,10 +199,11 @@ __global__ void __launch_bounds__(kThreads, 2)
           stop = true;
           break;
         }
-        mbar_arrive_expect_tx(bar(full0 + h), 2 * kHalfRowsBytes);
+        mbar_arrive_expect_tx(bar(full0 + h), DM::kSpans * kHalfRowsBytes);
         const int row = j * kTileRows + h * kHalfKeys;
-        tma_load_3d(tm, slot + h * kHalfRowsBytes, bar(full0 + h), 0, row, kz);
-        tma_load_3d(tm, slot + kHalfBytes + h * kHalfRowsBytes, bar(full0 + h), 64, row, kz);
+#pragma unroll
+        for (int sp = 0; sp < DM::kSpans; ++sp)
+          tma_load_3d(tm, slot + sp * kHalfBytes + h * kHalfRowsBytes, bar(full0 + h), 64 * sp, row, kz);
         issued = 2 * t + h;
       }
       if (stop) break;
@@ -211,7 +219,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   } else if (cnt > 0 && warp == 5 && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
     constexpr uint32_t idesc_qk = idesc_bf16_f32(128, kHalfKeys, 0, 0);
-    constexpr uint32_t idesc_pv = idesc_bf16_f32(128, 128, 0, 1);
+    constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
     const int n_half = 2 * cnt;
     // S_u = Q K_u^T into S columns h*64..h*64+63
     auto issue_s = [&](int u) -> bool {
@@ -219,7 +227,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       if (!mbar_wait_bounded(bar(K_FULL0 + h), (u >> 1) & 1, abort)) return false;
       tc_fence_after();
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {            // K = 128 = 8 x 16
+      for (int kk = 0; kk < D / 16; ++kk) {       // K = D in steps of 16
         const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32;
         mma_ss(tmem + kColS + h * kHalfKeys, smem_desc_sw128(sQ + off, 16, 1024),
                smem_desc_sw128(sK + off + h * kHalfRowsBytes, 16, 1024), idesc_qk, kk > 0 ? 1u : 0u);
@@ -312,7 +320,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         if (!__all_sync(0xFFFFFFFFu, w)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < D / 32; ++q) {
           uint32_t orr[32];
           tmem_ld32(tO + q * 32, orr);
           tmem_ld_wait();
@@ -340,10 +348,10 @@ __global__ void __launch_bounds__(kThreads, 2)
       const float lse_new = has ? (m_used + __log2f(l)) * 0.6931471805599453f : -INFINITY;
       MergeWeights mw{0.f, 0.f, 0.f, lse_new};
       if constexpr (MERGE) mw = merge_weights(qrow < N ? L_prev[orow] : -INFINITY, lse_new);
-      const float *prev = MERGE ? O_prev + orow * kHeadDim : nullptr;
-      uint4 *dst = reinterpret_cast<uint4 *>(O + orow * kHeadDim);
+      const float *prev = MERGE ? O_prev + orow * D : nullptr;
+      uint4 *dst = reinterpret_cast<uint4 *>(O + orow * D);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < D / 32; ++q) {
         uint32_t orr[32];
         if (cnt > 0) {
           tmem_ld32(tO + q * 32, orr);

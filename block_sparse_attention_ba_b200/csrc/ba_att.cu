@@ -99,7 +99,7 @@ bool make_head_map(CUtensorMap *map, const void *ptr, int d, int N_valid, int N_
 }
 
 bool use_tensor_core_path(const ba_att_shape *s) {
-  return s->dtype == BA_DTYPE_BF16 && s->d == 128 && s->block == 128;
+  return s->dtype == BA_DTYPE_BF16 && (s->d == 128 || s->d == 64) && s->block == 128;
 }
 
 __global__ void bounded_wait_selftest_kernel(unsigned long long limit_ns) {
@@ -271,18 +271,26 @@ ba_status sparse_fwd_impl(const ba_att_shape *s, const void *Q, const void *K, c
     const long long tiles = static_cast<long long>(s->B) * s->Hq * nb;
     if (tiles > 0x7FFFFFFFLL) return BA_ERR_UNSUPPORTED;
     const float sl2 = scale * 1.4426950408889634f;
+    const uint32_t smem = tc::dyn_smem_bytes(s->d);
     auto run = [&](auto kernel, auto *out) -> ba_status {
-      cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           static_cast<int>(tc::kDynSmem));
+      cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
       if (e != cudaSuccess) return BA_ERR_CUDA;
-      kernel<<<static_cast<unsigned>(tiles), tc::kThreads, tc::kDynSmem, cs>>>(
+      kernel<<<static_cast<unsigned>(tiles), tc::kThreads, smem, cs>>>(
           mq, mk, mv, kv_idx, kv_cnt, kmax, out, LSE, O_prev, L_prev, s->Hq, s->Hkv, s->N, s->N_alloc, nb, sl2);
       return from_cuda(cudaGetLastError());
     };
     float *of = static_cast<float *>(O);
     __nv_bfloat16 *ob = static_cast<__nv_bfloat16 *>(O);
-    if (out_f32) return merge ? run(tc::attn_tc_kernel<float, true>, of) : run(tc::attn_tc_kernel<float, false>, of);
-    return merge ? run(tc::attn_tc_kernel<__nv_bfloat16, true>, ob) : run(tc::attn_tc_kernel<__nv_bfloat16, false>, ob);
+    if (s->d == 128) {
+      if (out_f32)
+        return merge ? run(tc::attn_tc_kernel<float, true, 128>, of) : run(tc::attn_tc_kernel<float, false, 128>, of);
+      return merge ? run(tc::attn_tc_kernel<__nv_bfloat16, true, 128>, ob)
+                   : run(tc::attn_tc_kernel<__nv_bfloat16, false, 128>, ob);
+    }
+    if (out_f32)
+      return merge ? run(tc::attn_tc_kernel<float, true, 64>, of) : run(tc::attn_tc_kernel<float, false, 64>, of);
+    return merge ? run(tc::attn_tc_kernel<__nv_bfloat16, true, 64>, ob)
+                 : run(tc::attn_tc_kernel<__nv_bfloat16, false, 64>, ob);
   }
   cudaError_t e;
 #define BA_SIMT(T, TO, DD)                                                                                           \

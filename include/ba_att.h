@@ -225,7 +225,7 @@ ba_status ba_att_complement_lists(const ba_att_shape *shape, const int32_t *kv_i
  * o_dtype   shape->dtype, or BA_DTYPE_F32 to keep a partial output in fp32
  *           (one rounding in total when partials are merged later).
  * LSE       device fp32 [B, Hq, N_alloc], natural log (written).
- * Paths: bf16 with d = 128 and block = 128 runs the tcgen05/TMEM tensor-core
+ * Paths: bf16 with d = 64 or 128 and block = 128 runs the tcgen05/TMEM tensor-core
  * kernel; every other supported shape runs an fp32 CUDA-core kernel.
  */
 ba_status ba_att_sparse_fwd(const ba_att_shape *shape,

@@ -119,6 +119,8 @@ SMALL = [
     ("tiny_fp32", dict(N=9600 - 7, N_alloc=9600, block=16, Hq=2, Hkv=1), 0.5),   # 600 blocks: 5x5 score tiles
     ("dlm_16k", dict(N=64 * 128, Hq=2, Hkv=1), 0.5),                 # 512 blocks: 16 keys per lane in the top-k
     ("dlm_16k", dict(N=300 * 128 - 5, Hq=2, Hkv=2), 0.3),             # 300 blocks: ragged score tiles
+    ("dlm_16k", dict(N=2048 - 17, N_alloc=2048, Hq=4, Hkv=2, d=64), 0.5),   # tcgen05 path with d = 64, ragged
+    ("sweep_32k", dict(N=4096, Hq=4, Hkv=1, d=64), 0.25),            # d = 64, needle generator
 ]
 
 
@@ -139,6 +141,7 @@ def test_small_full_parity(name, over, keep):
 
 
 @pytest.mark.parametrize("name,over", [("tiny_fp32", {}), ("dlm_16k", dict(N=1536, Hq=4, Hkv=2)),
+                                       ("dlm_16k", dict(N=1536 - 9, N_alloc=1536, Hq=4, Hkv=2, d=64)),
                                        ("video_32k", dict(N=600, N_alloc=640, Hq=2, Hkv=2, grid=(3, 10, 20)))])
 def test_keep_all_equals_dense(name, over):
     # check (1): keep = 1.0 selects every block and equals dense attention
@@ -283,6 +286,7 @@ def test_complement_lists_and_cached_residual_is_dense(name, over, keep):
     ("extreme_128k", dict(N=4096 - 50, N_alloc=4096, Hq=4, Hkv=2)),      # tensor-core path, ragged tail
     ("tiny_fp32", dict(N=1000, N_alloc=1024)),                             # CUDA-core path, fp32
     ("dlm_16k", dict(N=1024, Hq=2, Hkv=1, d=64, block=64)),                # CUDA-core path, bf16 inputs
+    ("dlm_16k", dict(N=2048 - 40, N_alloc=2048, Hq=4, Hkv=2, d=64)),       # tensor-core path, d = 64
 ])
 def test_fused_merge_equals_separate_merge(name, over):
     # attention over span B merged in the epilogue with the partial over span A
