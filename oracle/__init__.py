@@ -39,6 +39,8 @@ from .ba_att_oracle import (  # noqa: F401
     pre_downsample_map,
     select_topk,
     selection_scores,
+    select_by_mass,
+    mass_share_before,
     near_tie_mask,
     masked_attention,
     dense_attention,

@@ -210,6 +210,51 @@ def selection_scores(S, Hkv: int, force_diagonal: bool = False, shared_gqa: bool
     return R
 
 
+def select_by_mass(R, tau: float, kmax: int | None = None):
+    """Keep, per row, the fewest top-ranked key blocks whose share of the
+    softmax-normalised block probability reaches tau.
+
+    A selection variant (the pages keep a fixed top fraction; this keeps a
+    fixed share of the pre-downsample map A^ = softmax_j S~ instead): rank
+    as ``select_topk`` does (R descending, ties to the lower index), take
+    the shortest prefix whose A^ sum is >= tau (at least one block), emit it
+    ascending. Returns (idx [..., kmax] -1 padded, cnt).
+    """
+    R = np.asarray(R, dtype=np.float64)
+    nk = R.shape[-1]
+    kmax = nk if kmax is None else kmax
+    idx = np.full(R.shape[:-1] + (kmax,), -1, dtype=np.int32)
+    cnt = np.zeros(R.shape[:-1], dtype=np.int32)
+    for pos in np.ndindex(R.shape[:-1]):
+        row = R[pos]
+        order = np.argsort(-row, kind="stable")
+        e = np.exp(row - row.max())
+        share = np.cumsum(e[order]) / e.sum()
+        m = int(np.searchsorted(share, tau, side="left")) + 1
+        m = min(max(m, 1), nk)
+        kept = np.sort(order[:m])
+        idx[pos][:m] = kept
+        cnt[pos] = m
+    return idx, cnt
+
+
+def mass_share_before(R, idx, cnt):
+    """For each row, the A^ share of its kept blocks without the lowest-ranked
+    one, and with it (the two sides of the tau cut); used to tell cuts that
+    rounding may move (the share sits within a relative band of tau)."""
+    R = np.asarray(R, dtype=np.float64)
+    lo = np.zeros(cnt.shape)
+    hi = np.zeros(cnt.shape)
+    for pos in np.ndindex(cnt.shape):
+        row = R[pos]
+        e = np.exp(row - row.max())
+        kept = idx[pos][: cnt[pos]]
+        vals = np.sort(e[kept])                       # ascending: vals[0] is the lowest-ranked kept block
+        hi[pos] = vals.sum() / e.sum()
+        lo[pos] = (vals.sum() - vals[0]) / e.sum()
+    return lo, hi
+
+
 def near_tie_mask(S, k: int, rel: float = 1e-3):
     """Blocks whose score lies within ``rel`` of the selection threshold.
 

@@ -377,6 +377,29 @@ def test_selection_variants():
                     assert list(idx[b, g * G + hh, i, :k]) == sorted(best)
 
 
+def test_select_by_mass():
+    rng = np.random.default_rng(13)
+    R = rng.standard_normal((2, 3, 5, 11)) * 2
+    for tau in (1e-9, 0.3, 0.5, 0.9, 0.999, 1.0):
+        idx, cnt = O.select_by_mass(R, tau)
+        lo, hi = O.mass_share_before(R, idx, cnt)
+        for pos in np.ndindex(cnt.shape):
+            m = int(cnt[pos])
+            row = R[pos]
+            # brute force: the shortest prefix of the ranking whose softmax share reaches tau
+            order = sorted(range(row.size), key=lambda j: (-row[j], j))
+            p = np.exp(row - row.max()) / np.exp(row - row.max()).sum()
+            shares = np.cumsum([p[j] for j in order])
+            want = next((i + 1 for i, v in enumerate(shares) if v >= tau - 1e-15), row.size)
+            assert m == max(1, want), (tau, pos, m, want)
+            assert list(idx[pos][:m]) == sorted(order[:m]) and (idx[pos][m:] == -1).all()
+            assert hi[pos] >= min(tau, 1.0) - 1e-12 and (m == 1 or lo[pos] < tau)
+    # tau -> 0 keeps the single best block; tau = 1 keeps every block
+    idx, cnt = O.select_by_mass(R, 1e-12)
+    assert (cnt == 1).all() and (idx[..., 0] == R.argmax(-1)).all()
+    assert (O.select_by_mass(R, 1.0)[1] == R.shape[-1]).all()
+
+
 def test_merge_edge_cases():
     o1 = np.array([[1.0, 2.0], [3.0, 4.0]])
     o2 = np.array([[5.0, 6.0], [7.0, 8.0]])
