@@ -23,7 +23,7 @@ BA_ERR_INVALID_ARG = 1
 STATUS_NAMES = {0: "BA_OK", 1: "BA_ERR_INVALID_ARG", 2: "BA_ERR_UNSUPPORTED", 3: "BA_ERR_MISALIGNED",
                 4: "BA_ERR_CUDA", 5: "BA_ERR_DEVICE", 6: "BA_ERR_TIMEOUT"}
 DTYPE_F32, DTYPE_BF16 = 0, 1
-SELECT_NO_VAR_PRODUCT, SELECT_FORCE_DIAGONAL, SELECT_SHARED_GQA = 0x1, 0x2, 0x4    # ba_att_select_ex flags
+SELECT_NO_VAR_PRODUCT, SELECT_FORCE_DIAGONAL, SELECT_SHARED_GQA, SELECT_BY_MASS = 0x1, 0x2, 0x4, 0x8   # select_ex flags
 
 # Entry points declared in include/ba_att.h: name -> (restype, argtypes)
 _P = ctypes.c_void_p
@@ -178,7 +178,8 @@ def select(stats_out, shape: Shape, keep: float, kmax: int | None = None, with_s
     k = keep_count(shape, keep)
     if k < 1:
         raise BaAttError("ba_att_keep_count", 1)
-    kmax = k if kmax is None else kmax
+    if kmax is None:                     # by-mass counts vary per row, up to nk
+        kmax = shape.nb if flags & SELECT_BY_MASS else k
     dev = qm.device
     if out is None:
         idx = torch.empty((shape.B, shape.Hq, shape.nb, kmax), device=dev, dtype=torch.int32)

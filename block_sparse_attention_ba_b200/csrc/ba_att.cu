@@ -181,7 +181,8 @@ ba_status ba_att_select_ex(const ba_att_shape *s, double keep, uint32_t flags, c
                            int32_t *kv_cnt, int32_t kmax, float *block_scores, ba_stream_t stream) {
   ba_status st = check_shape(s);
   if (st != BA_OK) return st;
-  constexpr uint32_t kKnown = BA_SELECT_NO_VAR_PRODUCT | BA_SELECT_FORCE_DIAGONAL | BA_SELECT_SHARED_GQA;
+  constexpr uint32_t kKnown =
+      BA_SELECT_NO_VAR_PRODUCT | BA_SELECT_FORCE_DIAGONAL | BA_SELECT_SHARED_GQA | BA_SELECT_BY_MASS;
   if (flags & ~kKnown) return BA_ERR_INVALID_ARG;
   if (!q_mean || !q_var || !k_mean || !k_var || !kv_idx || !kv_cnt || !block_scores) return BA_ERR_INVALID_ARG;
   if (!aligned16(q_mean) || !aligned16(q_var) || !aligned16(k_mean) || !aligned16(k_var) || !aligned16(kv_idx) ||
@@ -192,14 +193,22 @@ ba_status ba_att_select_ex(const ba_att_shape *s, double keep, uint32_t flags, c
   if (kmax < k) return BA_ERR_INVALID_ARG;
   const int nb = nblocks(s);
   if (nb > 4096) return BA_ERR_UNSUPPORTED;
-  if ((flags & (BA_SELECT_FORCE_DIAGONAL | BA_SELECT_SHARED_GQA)) && nb > 1024) return BA_ERR_UNSUPPORTED;
+  if ((flags & (BA_SELECT_FORCE_DIAGONAL | BA_SELECT_SHARED_GQA | BA_SELECT_BY_MASS)) && nb > 1024)
+    return BA_ERR_UNSUPPORTED;
+  if (flags & BA_SELECT_BY_MASS) {
+    if (flags & BA_SELECT_FORCE_DIAGONAL) return BA_ERR_UNSUPPORTED;
+    if (kmax < nb) return BA_ERR_INVALID_ARG;
+  }
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   const float scale = effective_scale(s);
   const int sms = num_sms_of_current_device();
+  const float tau = static_cast<float>(keep);
   cudaError_t e = s->d == 128 ? launch_select_tc<128>(q_mean, q_var, k_mean, k_var, kv_idx, kv_cnt, block_scores, s->B,
-                                                      s->Hq, s->Hkv, s->N, s->block, k, kmax, scale, flags, sms, cs)
+                                                      s->Hq, s->Hkv, s->N, s->block, k, kmax, scale, flags, tau, sms,
+                                                      cs)
                               : launch_select_tc<64>(q_mean, q_var, k_mean, k_var, kv_idx, kv_cnt, block_scores, s->B,
-                                                     s->Hq, s->Hkv, s->N, s->block, k, kmax, scale, flags, sms, cs);
+                                                     s->Hq, s->Hkv, s->N, s->block, k, kmax, scale, flags, tau, sms,
+                                                     cs);
   return from_cuda(e);
 }
 

@@ -529,18 +529,113 @@ inline cudaError_t launch_topk_kpl(const float *scores, int nk, int k, int32_t *
   return cudaGetLastError();
 }
 
+// Selection by cumulative share: keep the shortest prefix of the ranking
+// (key descending, column ascending) whose softmax share
+// exp(x_j - max) / sum_j exp(x_j - max) reaches tau (at least one block).
+// e_j and their sum are fp32; the cut key t* is the largest key whose
+// mass of keys >= t* still reaches tau*Z, found by bisection over the
+// 32-bit key space with warp-wide sums; of the keys equal to t* (equal x,
+// hence equal e) the first ones in column order are taken until the share
+// is reached. All lanes hold identical sums (xor-butterfly), so every lane
+// takes the same branch.
+template <int KPL>
+__device__ __forceinline__ void topk_row_mass(const float (&x)[KPL], const uint32_t (&u)[KPL], int nk, float tau,
+                                              int32_t *__restrict__ out_idx, int kmax, int32_t *__restrict__ out_cnt,
+                                              int lane) {
+  const unsigned full = 0xFFFFFFFFu;
+  const unsigned lt_mask = (1u << lane) - 1u;
+  auto wsum = [&](float v) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(full, v, off);
+    return v;
+  };
+  float mx = -INFINITY;
+  uint32_t umin = 0xFFFFFFFFu, umax = 0u;
+#pragma unroll
+  for (int c = 0; c < KPL; ++c) {
+    if (c * 32 + lane < nk) {
+      mx = fmaxf(mx, x[c]);
+      umin = min(umin, u[c]);
+      umax = max(umax, u[c]);
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(full, mx, off));
+  umin = __reduce_min_sync(full, umin);
+  umax = __reduce_max_sync(full, umax);
+  float e[KPL];
+  float part = 0.f;
+#pragma unroll
+  for (int c = 0; c < KPL; ++c) {
+    e[c] = (c * 32 + lane < nk) ? expf(x[c] - mx) : 0.f;
+    part += e[c];
+  }
+  const float Z = wsum(part);
+  const float target = tau * Z;
+  // largest t with mass(keys >= t) >= target: invariant mass(>= lo) >= target > mass(>= hi)
+  uint64_t lo = umin, hi = static_cast<uint64_t>(umax) + 1u;
+  while (hi - lo > 1u) {
+    const uint64_t mid = lo + ((hi - lo) >> 1);
+    float m = 0.f;
+#pragma unroll
+    for (int c = 0; c < KPL; ++c) m += (c * 32 + lane < nk && u[c] >= mid) ? e[c] : 0.f;
+    if (wsum(m) >= target) lo = mid; else hi = mid;
+  }
+  const uint32_t thr = static_cast<uint32_t>(lo);
+  float above = 0.f, e_eq = 0.f;
+  int n_eq = 0;
+#pragma unroll
+  for (int c = 0; c < KPL; ++c) {
+    const bool in = c * 32 + lane < nk;
+    if (in && u[c] > thr) above += e[c];
+    if (in && u[c] == thr) {
+      e_eq = e[c];
+      ++n_eq;
+    }
+  }
+  above = wsum(above);
+  e_eq = __shfl_sync(full, e_eq, __ffs(__ballot_sync(full, e_eq > 0.f || n_eq > 0)) - 1);
+  n_eq = __reduce_add_sync(full, n_eq);
+  int take = n_eq;                                      // equal keys needed, in column order
+  if (e_eq > 0.f) {
+    const float need = target - above;
+    take = static_cast<int>(ceilf(need / e_eq));
+    take = take < 1 ? 1 : (take > n_eq ? n_eq : take);
+  }
+  int pos = 0, eq_seen = 0;
+#pragma unroll
+  for (int c = 0; c < KPL; ++c) {
+    const int j = c * 32 + lane;
+    const bool in = j < nk;
+    const bool gt = in && u[c] > thr;
+    const bool eq = in && u[c] == thr;
+    const unsigned eqb = __ballot_sync(full, eq);
+    const bool kept = gt || (eq && eq_seen + __popc(eqb & lt_mask) < take);
+    const unsigned kb = __ballot_sync(full, kept);
+    if (kept && pos + __popc(kb & lt_mask) < kmax) out_idx[pos + __popc(kb & lt_mask)] = j;
+    pos += __popc(kb);
+    eq_seen += __popc(eqb);
+  }
+  for (int j = pos + lane; j < kmax; j += 32) out_idx[j] = -1;
+  if (lane == 0) *out_cnt = pos < kmax ? pos : kmax;
+}
+
 // Selection variants (the plain top-k above is the default):
 //   group > 1       the `group` query heads of a KV group share one selection,
 //                   ranked by the mean of their scores (one warp per
 //                   (batch, KV head, query block); the list is written to
 //                   every head of the group);
-//   force_diagonal  key block i always ranks first for query block i.
+//   force_diagonal  key block i always ranks first for query block i;
+//   by_mass         keep the shortest top-ranked prefix whose softmax share
+//                   reaches tau (topk_row_mass) instead of k blocks.
 // Rows of at most 1024 keys, held in registers.
 struct TopkVariant {
   int group;            // query heads per selection (1: none shared)
   int heads;            // Hq
   int nq;               // query blocks per head (= nk)
   bool force_diagonal;
+  bool by_mass;         // keep the shortest prefix reaching the share tau (instead of k blocks)
+  float tau;
 };
 
 template <int KPL>
@@ -574,11 +669,15 @@ __global__ void __launch_bounds__(kTopkWarps * 32) topk_variant_kernel(const flo
 #pragma unroll
     for (int c = 0; c < KPL; ++c) {
       const int j = c * 32 + lane;
-      u[c] = order_key(var.group > 1 ? acc[c] * inv_group : acc[c]);
+      if (var.group > 1) acc[c] *= inv_group;
+      u[c] = order_key(acc[c]);
       if (var.force_diagonal && j == i) u[c] = 0xFFFFFFFFu;
     }
     int32_t *out = kv_idx + first_row * kmax;
-    topk_row_regs<KPL>(u, nk, k, out, kmax, kv_cnt + first_row, smem_u32(&hist[warp][0]), lane);
+    if (var.by_mass)
+      topk_row_mass<KPL>(acc, u, nk, var.tau, out, kmax, kv_cnt + first_row, lane);
+    else
+      topk_row_regs<KPL>(u, nk, k, out, kmax, kv_cnt + first_row, smem_u32(&hist[warp][0]), lane);
     __syncwarp();
     for (int hh = 1; hh < var.group; ++hh) {           // the same list for the other heads of the group
       const long long orow = first_row + static_cast<long long>(hh) * var.nq;

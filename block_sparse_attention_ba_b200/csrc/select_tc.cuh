@@ -259,7 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int D>
 cudaError_t launch_select_tc(const float *qm, const float *qv, const float *km, const float *kv, int32_t *idx,
                              int32_t *cnt, float *scores, int B, int Hq, int Hkv, int N, int block, int k, int kmax,
-                             float sm_scale, uint32_t flags, int num_sms, cudaStream_t stream) {
+                             float sm_scale, uint32_t flags, float tau, int num_sms, cudaStream_t stream) {
   const int var_product = (flags & BA_SELECT_NO_VAR_PRODUCT) ? 0 : 1;
   const int nb = (N + block - 1) / block;
   const long long bhs = static_cast<long long>(B) * Hq;
@@ -288,8 +288,9 @@ cudaError_t launch_select_tc(const float *qm, const float *qv, const float *km, 
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const bool shared = (flags & BA_SELECT_SHARED_GQA) != 0, diag = (flags & BA_SELECT_FORCE_DIAGONAL) != 0;
-  if (!shared && !diag) return launch_topk(scores, nb, k, idx, kmax, cnt, bhs * nb, num_sms, stream);
-  const TopkVariant var{shared ? Hq / Hkv : 1, Hq, nb, diag};
+  const bool mass = (flags & BA_SELECT_BY_MASS) != 0;
+  if (!shared && !diag && !mass) return launch_topk(scores, nb, k, idx, kmax, cnt, bhs * nb, num_sms, stream);
+  const TopkVariant var{shared ? Hq / Hkv : 1, Hq, nb, diag, mass, tau};
   return launch_topk_variant(scores, nb, k, idx, kmax, cnt, static_cast<long long>(B) * (Hq / var.group) * nb, var,
                              num_sms, stream);
 }

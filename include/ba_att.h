@@ -166,6 +166,7 @@ ba_status ba_att_split_lists(const ba_att_shape *shape, int32_t split_block,
 #define BA_SELECT_NO_VAR_PRODUCT  0x1u  /* drop the var_q * var_k term of the correction   */
 #define BA_SELECT_FORCE_DIAGONAL  0x2u  /* query block i always keeps key block i           */
 #define BA_SELECT_SHARED_GQA      0x4u  /* one selection per KV group: mean S~ of its heads */
+#define BA_SELECT_BY_MASS         0x8u  /* keep the shortest top prefix with softmax share >= keep */
 
 /*
  * ba_att_select_ex — ba_att_select with selection variants (flags, above).
@@ -176,7 +177,12 @@ ba_status ba_att_split_lists(const ba_att_shape *shape, int32_t split_block,
  *  - SHARED_GQA: the Hq/Hkv query heads of each KV group rank key blocks by
  *    the mean of their S~ (fp32, summed in head order) and all receive the
  *    same list; the score map still holds each head's own S~.
- * flags = 0 is ba_att_select. FORCE_DIAGONAL and SHARED_GQA require
+ *  - BY_MASS: keep is a target share tau in (0, 1]: per query block, the
+ *    shortest prefix of the ranking (S~ descending, ties to the lower j)
+ *    whose share of softmax_j S~ (fp32) reaches tau, at least one block;
+ *    counts vary per row, so kmax must be >= nk (BA_ERR_INVALID_ARG
+ *    otherwise). Not combined with FORCE_DIAGONAL (BA_ERR_UNSUPPORTED).
+ * flags = 0 is ba_att_select. FORCE_DIAGONAL, SHARED_GQA and BY_MASS require
  * nk <= 1024 (BA_ERR_UNSUPPORTED above); unknown bits -> BA_ERR_INVALID_ARG.
  * Other arguments as for ba_att_select.
  */

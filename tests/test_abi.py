@@ -171,10 +171,15 @@ def test_complement_lists_arguments(lib):
 def test_select_variant_arguments(lib):
     s = shape()
     args = (P, P, P, P, P, P, 8, P, None)
-    assert lib.ba_att_select_ex(ctypes.byref(s), ctypes.c_double(0.5), ctypes.c_uint32(0x8), *args) == 1
+    assert lib.ba_att_select_ex(ctypes.byref(s), ctypes.c_double(0.5), ctypes.c_uint32(0x10), *args) == 1
+    # by-mass lists need room for every block, and do not combine with the forced diagonal
+    assert lib.ba_att_select_ex(ctypes.byref(s), ctypes.c_double(0.5), ctypes.c_uint32(api.SELECT_BY_MASS),
+                                P, P, P, P, P, P, 7, P, None) == 1
+    assert lib.ba_att_select_ex(ctypes.byref(s), ctypes.c_double(0.5),
+                                ctypes.c_uint32(api.SELECT_BY_MASS | api.SELECT_FORCE_DIAGONAL), *args) == 2
     big = shape(N=1025 * 16, N_alloc=1025 * 16, block=16)
     bigargs = (P, P, P, P, P, P, 1025, P, None)
-    for flag in (api.SELECT_FORCE_DIAGONAL, api.SELECT_SHARED_GQA):
+    for flag in (api.SELECT_FORCE_DIAGONAL, api.SELECT_SHARED_GQA, api.SELECT_BY_MASS):
         assert lib.ba_att_select_ex(ctypes.byref(big), ctypes.c_double(0.5), ctypes.c_uint32(flag), *bigargs) == 2
     # the plain variant-free flag set of ba_att_select still reaches the same checks
     assert lib.ba_att_select_ex(ctypes.byref(s), ctypes.c_double(0.5), ctypes.c_uint32(0), P, P, P, P, P, P, 3,

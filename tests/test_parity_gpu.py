@@ -222,6 +222,52 @@ def test_selection_variants(name, over, keep, flags):
         assert (g_idx == g_idx[:, :, :1]).all()
 
 
+@pytest.mark.parametrize("tau", [0.3, 0.7, 0.95])
+@pytest.mark.parametrize("shared", [False, True])
+@pytest.mark.parametrize("name,over", [
+    ("dlm_16k", dict(N=2048 - 40, N_alloc=2048, Hq=8, Hkv=2)),     # 16 blocks
+    ("video_32k", dict(N=600, N_alloc=640, Hq=2, Hkv=2, grid=(3, 10, 20))),
+    ("dlm_16k", dict(N=300 * 128 - 5, Hq=2, Hkv=1)),               # 300 blocks
+])
+def test_selection_by_mass(name, over, tau, shared):
+    # the shortest top-ranked prefix reaching the softmax share tau; the GPU
+    # sums in fp32, so where its cut differs from the oracle's the oracle's
+    # shares must put that cut within 1e-4 of tau, and the kept set must be
+    # the top m of the ranking outside near-ties
+    Q, K, V, meta = make_inputs(name, **over)
+    w = meta["workload"]
+    Qd, Kd = to_dev(Q, w.dtype), to_dev(K, w.dtype)
+    shape = api.Shape.of(Qd, Kd, w.N, w.block)
+    flags = api.SELECT_BY_MASS | (api.SELECT_SHARED_GQA if shared else 0)
+    idx, cnt = api.select(api.stats(Qd, Kd, shape), shape, tau, flags=flags)
+    torch.cuda.synchronize()
+    idx, cnt = idx.cpu().numpy(), cnt.cpu().numpy()
+    qm, qv, _ = O.block_stats(Q, w.N, w.block)
+    km, kv, kc = O.block_stats(K, w.N, w.block)
+    R = O.selection_scores(O.corrected_scores(qm, qv, km, kv, kc, w.d ** -0.5), w.Hkv, shared_gqa=shared)
+    idx_ref, cnt_ref = O.select_by_mass(R, tau)
+    band = 1e-4
+    moved = 0
+    for pos in np.ndindex(cnt.shape):
+        m = int(cnt[pos])
+        assert 1 <= m <= w.nb and (idx[pos][m:] == -1).all() and (np.diff(idx[pos][:m]) > 0).all()
+        if m == cnt_ref[pos] and (idx[pos][:m] == idx_ref[pos][:m]).all():
+            continue
+        moved += 1
+        row = R[pos]
+        order = np.argsort(-row, kind="stable")
+        e = np.exp(row - row.max())
+        share = np.cumsum(e[order]) / e.sum()
+        assert share[m - 1] >= tau - band and (m == 1 or share[m - 2] < tau + band), (pos, m, cnt_ref[pos])
+        got = np.zeros(w.nb, bool)
+        got[idx[pos][:m]] = True
+        top = np.zeros(w.nb, bool)
+        top[order[:m]] = True
+        near = O.near_tie_mask(row[None], m, NEAR_TIE_REL)[0]
+        assert not ((got != top) & ~near).any()
+    assert moved <= max(2, cnt.size // 50), moved
+
+
 def test_complement_lists_long_rows_and_odd_entries():
     # 2000 blocks (63 bitmap words, two rounds of 32), random kept sets of
     # every size, duplicate and out-of-range entries (ignored and flagged)
