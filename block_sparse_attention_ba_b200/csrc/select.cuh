@@ -1,24 +1,21 @@
-// select.cuh — K7: covariance-compensated block scores + norm sorting.
+// select.cuh — K7: norm sorting, the per-row exact top-k of the block scores.
 //
 // "Efficient Long-Context Modeling in DLMs via Block Approximate Sparse
 // Attention" (abstract; "Core claim"; Figure 2): key blocks are scored in
 // the downsampled block space, the pooled score is corrected with diagonal
 // Q/K variances, blocks are sorted and the top fraction is kept.
 //
-//   S~[i,j] = s qbar_i.kbar_j + (s^2/2) sum_m (vq kbar^2 + qbar^2 vk + vq vk) + ln m_j
-//
-// written as one 3d-long dot product of augmented rows
-//   qt_i = [ s qbar_i , (s^2/2) vq_i , (s^2/2) qbar_i^2 ]
-//   kt_j = [ kbar_j   , kbar_j^2 + vk_j , vk_j ]
-// so that S~ = qt_i . kt_j + ln m_j (fp32 FMA accumulation).
-//
-// Two launches. select_kernel (SIMT; the tensor-core variant for nk <= 512
-// lives in select_tc.cuh) writes the whole fp32 score map; topk_rows_kernel
-// then gives one warp to each (batch, head, query block) row and selects its
-// top k by an exact 4-pass radix select on order-preserving keys of the fp32
-// scores (taken relative to the row minimum so that the high bytes carry
-// information); equal scores go to the lower block index, and the kept
-// indices are emitted ascending.
+// The scores S~[i,j] are written by select_tc_kernel (select_tc.cuh, tensor
+// cores); this file ranks each (batch, head, query block) row of that map.
+// One warp per row selects the top k exactly on order-preserving 32-bit keys
+// of the fp32 scores (topk_row_keys: a sampled key window, 8-bit radix
+// passes, then direct ranking of at most 32 candidates); equal scores go to
+// the lower block index, and the kept indices are emitted ascending. Rows of
+// up to 256 keys are held in registers (topk_rows_kernel), up to 1024 in
+// shared memory (topk_rows_smem_kernel), longer ones are re-read from global
+// memory (topk_row_warp). topk_variant_kernel serves the selection variants
+// of ba_att_select_ex (shared per GQA group, forced diagonal, cumulative
+// softmax share: topk_row_mass).
 #pragma once
 
 #include "common.cuh"
