@@ -71,13 +71,39 @@ struct Ctl {
   int abort;
 };
 
-// Validity of list entry t, computed identically by every role from the raw
-// list: inside [0, nb) and strictly above the previous raw entry.
-__device__ __forceinline__ bool entry_ok(const int32_t *list, int t, int nb, int &j) {
-  j = __ldg(list + t);
-  if (j < 0 || j >= nb) return false;
-  if (t > 0 && j <= __ldg(list + t - 1)) return false;
-  return true;
+// Validity of list entries, computed identically by every role from the raw
+// list: entry t is valid when it lies in [0, nb) and strictly above the
+// previous raw entry. Walks the list in order, with the next entry's load
+// issued one step ahead so that its latency hides behind the current block.
+struct ListCursor {
+  const int32_t *list;
+  int cnt, nb, prev, next;
+  __device__ __forceinline__ ListCursor(const int32_t *l, int c, int n) : list(l), cnt(c), nb(n), prev(-1), next(0) {
+    if (cnt > 0) next = __ldg(list);
+  }
+  // entry t (called for t = 0, 1, 2, ... in order); returns its validity
+  __device__ __forceinline__ bool step(int t, int &j) {
+    j = next;
+    if (t + 1 < cnt) next = __ldg(list + t + 1);
+    const bool ok = j >= 0 && j < nb && (t == 0 || j > prev);
+    prev = j;
+    return ok;
+  }
+};
+
+// Row max of 64 raw scores held as two 32-column halves: four independent
+// chains of 3-input max.
+__device__ __forceinline__ float row_max64(const uint32_t (&sr)[2][32]) {
+  float m4[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint32_t *v = &sr[k >> 1][(k & 1) * 16];
+    float m = fmaxf(__uint_as_float(v[0]), __uint_as_float(v[1]));
+#pragma unroll
+    for (int c = 2; c < 16; c += 2) m = fmax3(m, __uint_as_float(v[c]), __uint_as_float(v[c + 1]));
+    m4[k] = m;
+  }
+  return fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]);
 }
 
 // P = 2^(s*scale_log2 - m) for one row's 64 keys of a half block: packed to
@@ -185,11 +211,11 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     int issued = -1;                    // last half-block index u loaded
     bool bad_index = false, bad_order = false;
+    ListCursor cur(list, cnt, nb);
     for (int t = 0; t < cnt; ++t) {
       int j;
-      if (!entry_ok(list, t, nb, j)) {
-        const int raw = __ldg(list + t);
-        if (raw < 0 || raw >= nb) bad_index = true; else bad_order = true;
+      if (!cur.step(t, j)) {
+        if (j < 0 || j >= nb) bad_index = true; else bad_order = true;
         j = 0;                            // load a valid block; softmax masks it out
       }
       bool stop = false;
@@ -266,11 +292,12 @@ __global__ void __launch_bounds__(kThreads, 2)
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     int n_keys = 0;
+    ListCursor cur(list, cnt, nb);
     for (int u = 0; u < 2 * cnt; ++u) {
       const int h = u & 1;
       if (h == 0) {
         int j;
-        const bool valid = entry_ok(list, u >> 1, nb, j);
+        const bool valid = cur.step(u >> 1, j);
         n_keys = valid ? min(kTileRows, N - j * kTileRows) : 0;
       }
       const int n_half = min(max(n_keys - h * kHalfKeys, 0), kHalfKeys);
@@ -290,16 +317,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             if (q * 32 + c >= n_half) sr[q][c] = __float_as_uint(-INFINITY);
         }
       }
-      // Row max of the raw scores: 2 independent chains of 3-input max.
-      float mxp[2];
-#pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        mxp[q] = fmaxf(__uint_as_float(sr[q][0]), __uint_as_float(sr[q][31]));
-#pragma unroll
-        for (int c = 1; c < 31; c += 2)
-          mxp[q] = fmax3(mxp[q], __uint_as_float(sr[q][c]), __uint_as_float(sr[q][c + 1]));
-      }
-      const float mx = fmaxf(mxp[0], mxp[1]) * scale_log2;   // scale > 0 keeps the order
+      const float mx = row_max64(sr) * scale_log2;   // scale > 0 keeps the order
       float alpha = 1.f;
       bool rescale = false;
       if (mx - m_used > kRescaleLog2) {                // false when both are -inf
@@ -398,6 +416,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     tmem_dealloc<kTmemCols>(tmem);
   }
 }
+
 
 }  // namespace tc
 }  // namespace baatt
