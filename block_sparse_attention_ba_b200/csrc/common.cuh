@@ -113,6 +113,24 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void *src, uint32_
       : "memory");
 }
 
+// The same copy with an L2 eviction-priority hint (a policy from
+// l2_evict_first_policy): for data read exactly once, so that streaming it
+// through L2 displaces its own lines first instead of other resident (and
+// possibly dirty) lines.
+__device__ __forceinline__ void bulk_load_hint(uint32_t dst, const void *src, uint32_t bytes, uint32_t bar,
+                                               uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar), "l"(policy)
+      : "memory");
+}
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
 // Fire-and-forget add on a shared-memory word given by its shared-window
 // address (a shared-state atomic even when the C++ pointer was generic).
 __device__ __forceinline__ void red_shared_add(uint32_t saddr, uint32_t v) {

@@ -14,6 +14,10 @@
 
 #include "common.cuh"
 
+#ifndef BA_STATS_EVICT_FIRST
+#define BA_STATS_EVICT_FIRST 1
+#endif
+
 namespace baatt {
 
 constexpr int kStatsThreads = 256;
@@ -280,7 +284,14 @@ __global__ void __launch_bounds__(kStatsThreads, 2)
     locate(w, src, n_rows, orow, is_q);
     const uint32_t bytes = static_cast<uint32_t>(n_rows) * D * sizeof(T);
     mbar_arrive_expect_tx(smem_u32(&full[s]), bytes);
+#if BA_STATS_EVICT_FIRST
+    // Q and K are read exactly once here: stream them through L2 at evict-first
+    // priority so that lines still resident from earlier kernels (for example
+    // an attention output not yet written back) are not displaced by them
+    bulk_load_hint(ring + s * kStatsStageBytes, src, bytes, smem_u32(&full[s]), l2_evict_first_policy());
+#else
     bulk_load(ring + s * kStatsStageBytes, src, bytes, smem_u32(&full[s]));
+#endif
   };
 
   long long last_issued = -1;             // thread 0: newest item handed to the copy engine
