@@ -45,6 +45,9 @@ _SIGS = {
     "ba_att_select": (ctypes.c_int, [ctypes.POINTER(CShape), ctypes.c_double, _P, _P, _P, _P, _P, _P, _I32, _P, _P]),
     "ba_att_select_ex": (ctypes.c_int, [ctypes.POINTER(CShape), ctypes.c_double, ctypes.c_uint32, _P, _P, _P, _P, _P,
                                          _P, _I32, _P, _P]),
+    "ba_att_selector_workspace": (ctypes.c_int64, [ctypes.POINTER(CShape)]),
+    "ba_att_selector": (ctypes.c_int, [ctypes.POINTER(CShape), ctypes.c_double, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                        _P, _I32, _P]),
     "ba_att_split_lists": (ctypes.c_int, [ctypes.POINTER(CShape), _I32, _P, _P, _I32, _P, _P, _P, _P, _P]),
     "ba_att_complement_lists": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _I32, _P, _P, _I32, _P]),
     "ba_att_sparse_fwd": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _P, _P, _P, _I32, _P, _I32, _P, _P]),
@@ -194,6 +197,47 @@ def select(stats_out, shape: Shape, keep: float, kmax: int | None = None, with_s
         _dev(qv, "q_var"), _dev(km, "k_mean"), _dev(kv, "k_var"), _dev(idx, "kv_idx"), _dev(cnt, "kv_cnt"),
         idx.shape[-1], _dev(sc, "block_scores"), _stream(qm)))
     return (idx, cnt, sc) if with_scores else (idx, cnt)
+
+
+def selector_workspace_bytes(shape: Shape) -> int:
+    """Device workspace bytes of ba_att_selector for this shape."""
+    n = int(load_library().ba_att_selector_workspace(ctypes.byref(shape.c())))
+    if n < 0:
+        raise BaAttError("ba_att_selector_workspace", 1)
+    return n
+
+
+def selector(Q: torch.Tensor, K: torch.Tensor, shape: Shape, keep: float, kmax: int | None = None, out=None,
+             workspace: torch.Tensor | None = None):
+    """The whole selector in one call (ba_att_selector): stats, scores and top-k.
+
+    Returns (stats, idx, cnt, scores) with stats = (q_mean, q_var, k_mean, k_var); out may
+    pass the same tuple preallocated, workspace a uint8 device tensor of at least
+    selector_workspace_bytes(shape)."""
+    lib = load_library()
+    k = keep_count(shape, keep)
+    if k < 1:
+        raise BaAttError("ba_att_keep_count", 1)
+    kmax = k if kmax is None else kmax
+    dev = Q.device
+    if out is None:
+        st = (torch.empty((shape.B, shape.Hq, shape.nb, shape.d), device=dev, dtype=torch.float32),
+              torch.empty((shape.B, shape.Hq, shape.nb, shape.d), device=dev, dtype=torch.float32),
+              torch.empty((shape.B, shape.Hkv, shape.nb, shape.d), device=dev, dtype=torch.float32),
+              torch.empty((shape.B, shape.Hkv, shape.nb, shape.d), device=dev, dtype=torch.float32))
+        idx = torch.empty((shape.B, shape.Hq, shape.nb, kmax), device=dev, dtype=torch.int32)
+        cnt = torch.empty((shape.B, shape.Hq, shape.nb), device=dev, dtype=torch.int32)
+        sc = torch.empty((shape.B, shape.Hq, shape.nb, shape.nb), device=dev, dtype=torch.float32)
+    else:
+        st, idx, cnt, sc = out
+    if workspace is None:
+        workspace = torch.empty(selector_workspace_bytes(shape), device=dev, dtype=torch.uint8)
+    qm, qv, km, kv = st
+    _check("ba_att_selector", lib.ba_att_selector(
+        ctypes.byref(shape.c()), ctypes.c_double(keep), _dev(Q, "Q"), _dev(K, "K"), _dev(qm, "q_mean"),
+        _dev(qv, "q_var"), _dev(km, "k_mean"), _dev(kv, "k_var"), _dev(workspace, "workspace"),
+        _dev(sc, "block_scores"), _dev(idx, "kv_idx"), _dev(cnt, "kv_cnt"), idx.shape[-1], _stream(Q)))
+    return st, idx, cnt, sc
 
 
 def split_lists(idx: torch.Tensor, cnt: torch.Tensor, shape: Shape, split_block: int, out=None):

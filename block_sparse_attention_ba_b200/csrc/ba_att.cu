@@ -218,6 +218,115 @@ ba_status ba_att_select(const ba_att_shape *s, double keep, const float *q_mean,
   return ba_att_select_ex(s, keep, 0u, q_mean, q_var, k_mean, k_var, kv_idx, kv_cnt, kmax, block_scores, stream);
 }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------- one-call selector
+
+namespace {
+// [6 planes][rows][d] bf16 feature array read in boxes of 64 dims x 128 rows.
+bool make_feat_map(CUtensorMap *map, const void *ptr, int d, long long rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows), 6u};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2u, static_cast<cuuint64_t>(rows) * d * 2u};
+  cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(selft::kTile), 1u};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+long long feat_rows_q(const ba_att_shape *s) { return static_cast<long long>(s->B) * s->Hq * nblocks(s); }
+long long feat_rows_k(const ba_att_shape *s) { return static_cast<long long>(s->B) * s->Hkv * nblocks(s); }
+
+// Whether the shape takes the feature path (else the selector is the plain
+// ba_att_stats + ba_att_select sequence).
+bool selector_feature_path(const ba_att_shape *s) {
+  const bool bulk = s->dtype == BA_DTYPE_BF16
+                        ? (s->d == 128 ? stats_bulk_fits<__nv_bfloat16, 128>(s->block)
+                                       : stats_bulk_fits<__nv_bfloat16, 64>(s->block))
+                        : (s->d == 128 ? stats_bulk_fits<float, 128>(s->block) : stats_bulk_fits<float, 64>(s->block));
+  return bulk && feat_rows_q(s) + selft::kTile < 0x7FFFFFFFLL;
+}
+
+template <int D>
+cudaError_t launch_select_feat(const CUtensorMap &mq, const CUtensorMap &mk, float *scores, const ba_att_shape *s,
+                               int nb, int sms, cudaStream_t cs) {
+  const int n_tq = (nb + selft::kTile - 1) / selft::kTile;
+  const long long n_tiles = static_cast<long long>(s->B) * s->Hq * n_tq * n_tq;
+  cudaError_t e = cudaFuncSetAttribute(selft::select_feat_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(selft::kDynSmem));
+  if (e != cudaSuccess) return e;
+  const unsigned grid = static_cast<unsigned>(n_tiles < sms ? n_tiles : sms);
+  selft::select_feat_kernel<D><<<grid, selft::kThreads, selft::kDynSmem, cs>>>(mq, mk, scores, s->Hq, s->Hkv, s->N,
+                                                                              s->block, nb, n_tiles, n_tq);
+  return cudaGetLastError();
+}
+}  // namespace
+
+extern "C" {
+
+int64_t ba_att_selector_workspace(const ba_att_shape *s) {
+  if (check_shape(s) != BA_OK) return -1;
+  const long long bytes = 6LL * (feat_rows_q(s) + feat_rows_k(s)) * s->d * 2;
+  return (bytes + 255) & ~255LL;
+}
+
+ba_status ba_att_selector(const ba_att_shape *s, double keep, const void *Q, const void *K, float *q_mean,
+                          float *q_var, float *k_mean, float *k_var, void *workspace, float *block_scores,
+                          int32_t *kv_idx, int32_t *kv_cnt, int32_t kmax, ba_stream_t stream) {
+  ba_status st = check_shape(s);
+  if (st != BA_OK) return st;
+  if (!Q || !K || !q_mean || !q_var || !k_mean || !k_var || !workspace || !block_scores || !kv_idx || !kv_cnt)
+    return BA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(q_mean) || !aligned16(q_var) || !aligned16(k_mean) ||
+      !aligned16(k_var) || !aligned16(workspace) || !aligned16(block_scores) || !aligned16(kv_idx) ||
+      !aligned16(kv_cnt))
+    return BA_ERR_MISALIGNED;
+  const int k = ba_att_keep_count(s, keep);
+  if (k < 1 || kmax < k) return BA_ERR_INVALID_ARG;
+  const int nb = nblocks(s);
+  if (nb > 4096) return BA_ERR_UNSUPPORTED;
+  if (!selector_feature_path(s)) {
+    st = ba_att_stats(s, Q, K, q_mean, q_var, k_mean, k_var, stream);
+    return st == BA_OK ? ba_att_select(s, keep, q_mean, q_var, k_mean, k_var, kv_idx, kv_cnt, kmax, block_scores,
+                                       stream)
+                       : st;
+  }
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  const int sms = num_sms_of_current_device();
+  const float scale = effective_scale(s);
+  auto *fq = static_cast<__nv_bfloat16 *>(workspace);
+  auto *fk = fq + 6 * feat_rows_q(s) * s->d;
+  const FeatOut feat{fq, fk, scale, 0.5f * scale * scale, feat_rows_q(s), feat_rows_k(s)};
+  cudaError_t e;
+  if (s->dtype == BA_DTYPE_BF16) {
+    auto q = static_cast<const __nv_bfloat16 *>(Q);
+    auto kk = static_cast<const __nv_bfloat16 *>(K);
+    e = s->d == 128 ? launch_stats<__nv_bfloat16, 128>(q, kk, q_mean, q_var, k_mean, k_var, s->B, s->Hq, s->Hkv, s->N,
+                                                       s->N_alloc, s->block, sms, cs, feat)
+                    : launch_stats<__nv_bfloat16, 64>(q, kk, q_mean, q_var, k_mean, k_var, s->B, s->Hq, s->Hkv, s->N,
+                                                      s->N_alloc, s->block, sms, cs, feat);
+  } else {
+    auto q = static_cast<const float *>(Q);
+    auto kk = static_cast<const float *>(K);
+    e = s->d == 128 ? launch_stats<float, 128>(q, kk, q_mean, q_var, k_mean, k_var, s->B, s->Hq, s->Hkv, s->N,
+                                               s->N_alloc, s->block, sms, cs, feat)
+                    : launch_stats<float, 64>(q, kk, q_mean, q_var, k_mean, k_var, s->B, s->Hq, s->Hkv, s->N,
+                                              s->N_alloc, s->block, sms, cs, feat);
+  }
+  if (e != cudaSuccess) return from_cuda(e);
+  CUtensorMap mq, mk;
+  if (!make_feat_map(&mq, fq, s->d, feat_rows_q(s)) || !make_feat_map(&mk, fk, s->d, feat_rows_k(s)))
+    return BA_ERR_CUDA;
+  e = s->d == 128 ? launch_select_feat<128>(mq, mk, block_scores, s, nb, sms, cs)
+                  : launch_select_feat<64>(mq, mk, block_scores, s, nb, sms, cs);
+  if (e != cudaSuccess) return from_cuda(e);
+  return from_cuda(launch_topk(block_scores, nb, k, kv_idx, kmax, kv_cnt, static_cast<long long>(s->B) * s->Hq * nb,
+                               sms, cs));
+}
+
 ba_status ba_att_complement_lists(const ba_att_shape *s, const int32_t *kv_idx, const int32_t *kv_cnt, int32_t kmax,
                                   int32_t *c_idx, int32_t *c_cnt, int32_t c_kmax, ba_stream_t stream) {
   ba_status st = check_shape(s);

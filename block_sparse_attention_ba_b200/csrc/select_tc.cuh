@@ -253,6 +253,188 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace seltc
 
+// ---------------------------------------------------------------- feature-fed scores
+// The same score map from augmented features that the statistics pass wrote
+// once per block (FeatOut in stats.cuh: planes [part, hi/lo][rows][D] bf16),
+// so no tile re-derives them. Persistent CTAs walk 128 x 128 tiles ordered
+// (batch and head, query tile, key tile); roles (192 threads):
+//   warp 4 lane 0  TMA producer: per (64-dim group, part) stage the A hi/lo
+//                  and B hi/lo operand tiles (4 x 16 KB) into a 3-stage ring;
+//                  warp 4 also allocates TMEM
+//   warp 5 lane 0  MMA issuer: per stage, for each 16-dim step, hi*hi, hi*lo
+//                  and lo*hi into one of two 128-column TMEM accumulators
+//   warps 0-3      epilogue: drain an accumulator (lane = query block), add
+//                  ln m_j and store the rows while the next tile accumulates
+// The MMA sequence per tile is the one select_tc_kernel issues (groups, then
+// parts, then 16-dim steps; hh, hl, lh), so the scores are bit-identical.
+namespace selft {
+constexpr int kThreads = 192;
+constexpr int kStages = 3;
+constexpr uint32_t kOp = 128 * 128;              // 128 rows x 64 bf16, one swizzle span
+constexpr uint32_t kStageBytes = 4 * kOp;        // A hi, A lo, B hi, B lo
+constexpr uint32_t kDynSmem = kStages * kStageBytes + 1024;
+constexpr int kTile = 128;
+enum Bar : int { FULL = 0, EMPTY = FULL + kStages, ACC_FULL = EMPTY + kStages, ACC_EMPTY = ACC_FULL + 2,
+                 DRAIN = ACC_EMPTY + 2, NUM_BARS };
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    select_feat_kernel(const __grid_constant__ CUtensorMap tm_fq, const __grid_constant__ CUtensorMap tm_fk,
+                       float *__restrict__ block_scores, int Hq, int Hkv, int N, int block, int nb,
+                       long long n_tiles, int n_tq) {
+  constexpr int GROUPS = D / 64;
+  extern __shared__ uint8_t dyn_smem[];
+  __shared__ uint64_t bars[NUM_BARS];
+  __shared__ uint32_t tmem_base_s;
+  __shared__ int abort_flag;
+  const uint32_t sbase = (smem_u32(dyn_smem) + 1023u) & ~1023u;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  auto bar = [&](int k) { return smem_u32(&bars[k]); };
+  const int G = Hq / Hkv;
+  // tile t -> (bh, query tile, key tile)
+  auto decode = [&](long long t, long long &bh, int &tq, int &tk) {
+    tk = static_cast<int>(t % n_tq);
+    const long long r = t / n_tq;
+    tq = static_cast<int>(r % n_tq);
+    bh = r / n_tq;
+  };
+  if (threadIdx.x == 0) {
+    for (int k = 0; k < NUM_BARS; ++k) mbar_init(bar(k), (k >= ACC_EMPTY && k < ACC_EMPTY + 2) ? 128u : 1u);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 4) {
+    tmem_alloc<256>(smem_u32(&tmem_base_s));
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_s;
+  volatile int *abort = &abort_flag;
+
+  if (warp == 4 && lane == 0) {
+    // ------------------------------------------------------------ producer
+    tma_prefetch_desc(&tm_fq);
+    tma_prefetch_desc(&tm_fk);
+    long long it = 0;
+    bool stop = false;
+    for (long long t = blockIdx.x; t < n_tiles && !stop; t += gridDim.x) {
+      long long bh;
+      int tq, tk;
+      decode(t, bh, tq, tk);
+      const int b = static_cast<int>(bh / Hq), h = static_cast<int>(bh % Hq);
+      const int qrow = static_cast<int>(bh * nb) + tq * kTile;
+      const int krow = (b * Hkv + h / G) * nb + tk * kTile;
+      for (int g = 0; g < GROUPS && !stop; ++g) {
+        for (int p = 0; p < 3; ++p, ++it) {
+          const int st = static_cast<int>(it % kStages);
+          const long long use = it / kStages;
+          if (use > 0 && !mbar_wait_bounded(bar(EMPTY + st), static_cast<uint32_t>((use - 1) & 1), abort)) {
+            stop = true;
+            break;
+          }
+          const uint32_t dst = sbase + st * kStageBytes;
+          mbar_arrive_expect_tx(bar(FULL + st), kStageBytes);
+          tma_load_3d(&tm_fq, dst, bar(FULL + st), 64 * g, qrow, 2 * p);
+          tma_load_3d(&tm_fq, dst + kOp, bar(FULL + st), 64 * g, qrow, 2 * p + 1);
+          tma_load_3d(&tm_fk, dst + 2 * kOp, bar(FULL + st), 64 * g, krow, 2 * p);
+          tma_load_3d(&tm_fk, dst + 3 * kOp, bar(FULL + st), 64 * g, krow, 2 * p + 1);
+        }
+      }
+    }
+    if (*abort) {
+      // let the copies in flight land before the CTA's shared memory goes away
+      for (long long u = it - 1; u >= 0 && u >= it - kStages; --u)
+        mbar_wait_bounded(bar(FULL + static_cast<int>(u % kStages)), static_cast<uint32_t>((u / kStages) & 1), nullptr);
+    }
+  } else if (warp == 5 && lane == 0) {
+    // ------------------------------------------------------------ MMA issuer
+    constexpr uint32_t idesc = idesc_bf16_f32(128, kTile, 0, 0);
+    const uint64_t d0 = smem_desc_sw128(sbase, 16, 1024);
+    long long it = 0;
+    int tl = 0;
+    bool ok = true;
+    for (long long t = blockIdx.x; t < n_tiles && ok; t += gridDim.x, ++tl) {
+      const int acc = tl & 1, use = tl >> 1;
+      if (use > 0 && !mbar_wait_bounded(bar(ACC_EMPTY + acc), static_cast<uint32_t>((use - 1) & 1), abort)) break;
+      tc_fence_after();
+      const uint32_t dt = tmem + acc * kTile;
+      for (int sidx = 0; sidx < 3 * GROUPS; ++sidx, ++it) {
+        const int st = static_cast<int>(it % kStages);
+        if (!mbar_wait_bounded(bar(FULL + st), static_cast<uint32_t>((it / kStages) & 1), abort)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        // start-address field in 16-byte units (no carry: shared addresses < 256 KB)
+        const uint64_t ah = d0 + ((st * kStageBytes) >> 4), al = ah + (kOp >> 4);
+        const uint64_t bhd = ah + ((2 * kOp) >> 4), bld = ah + ((3 * kOp) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          mma_ss(dt, ah + 2 * kk, bhd + 2 * kk, idesc, (sidx > 0 || kk > 0) ? 1u : 0u);
+          mma_ss(dt, ah + 2 * kk, bld + 2 * kk, idesc, 1u);
+          mma_ss(dt, al + 2 * kk, bhd + 2 * kk, idesc, 1u);
+        }
+        mma_commit(bar(EMPTY + st));
+      }
+      if (!ok) break;
+      mma_commit(bar(ACC_FULL + acc));
+    }
+    mma_commit(bar(DRAIN));
+    mbar_wait_bounded(bar(DRAIN), 0, nullptr);
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ epilogue
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const float ln_full = logf(static_cast<float>(block));
+    const float ln_last = logf(static_cast<float>(N - (nb - 1) * block));
+    const bool vec = (nb & 3) == 0;
+    int tl = 0;
+    for (long long t = blockIdx.x; t < n_tiles; t += gridDim.x, ++tl) {
+      const int acc = tl & 1, use = tl >> 1;
+      const bool w = mbar_wait_bounded(bar(ACC_FULL + acc), static_cast<uint32_t>(use & 1), abort);
+      if (!__all_sync(0xFFFFFFFFu, w)) break;
+      tc_fence_after();
+      long long bh;
+      int tq, tk;
+      decode(t, bh, tq, tk);
+      const int i = tq * kTile + warp * 32 + lane;
+      const int j0 = tk * kTile;
+#pragma unroll
+      for (int c0 = 0; c0 < kTile; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_off + acc * kTile + c0, r);
+        tmem_ld_wait();
+        if (i < nb) {
+          const int jb = j0 + c0;
+          float *dst = block_scores + (bh * nb + i) * nb + jb;
+          float val[32];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) val[c] = __uint_as_float(r[c]) + (jb + c == nb - 1 ? ln_last : ln_full);
+          if (vec && jb + 32 <= nb) {
+#pragma unroll
+            for (int c = 0; c < 32; c += 4)
+              *reinterpret_cast<float4 *>(dst + c) = make_float4(val[c], val[c + 1], val[c + 2], val[c + 3]);
+          } else {
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+              if (jb + c < nb) dst[c] = val[c];
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(ACC_EMPTY + acc));
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc<256>(tmem);
+  }
+}
+}  // namespace selft
+
 // Scores with the widest key tile that still gives at least half the SMs a
 // CTA, then the top-k launch.
 // flags: the ba_att_select_ex bits (BA_SELECT_*).

@@ -244,11 +244,36 @@ __device__ __forceinline__ void stats_moments_ragged(const T *slab, int n_rows, 
   }
 }
 
+// Optional output of the statistics pass: the augmented score features of
+// every block, so that the score GEMM reads them instead of deriving them per
+// tile. Plane p2 = 2p + h holds part p (0..2) as bf16, h = 0 the high and
+// h = 1 the low half of x = hi + lo (hi = RN(x), lo = RN(x - hi)); a plane is
+// [rows][D] with rows = B*H*nb, Q and K in separate arrays:
+//   Q parts: s*mean, (s^2/2)*var, (s^2/2)*mean*mean
+//   K parts: mean, mean*mean + var, var
+struct FeatOut {
+  __nv_bfloat16 *q, *k;        // nullptr: no feature output
+  float s, hs2;                // sm_scale and 0.5 * sm_scale * sm_scale
+  long long q_rows, k_rows;    // rows per plane
+};
+
+__device__ __forceinline__ void store_feat(__nv_bfloat16 *base, long long plane_elems, long long at, float x0, float x1,
+                                           float x2) {
+  const float x[3] = {x0, x1, x2};
+#pragma unroll
+  for (int p = 0; p < 3; ++p) {
+    const __nv_bfloat16 hi = __float2bfloat16_rn(x[p]);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(x[p] - __bfloat162float(hi));
+    base[(2 * p) * plane_elems + at] = hi;
+    base[(2 * p + 1) * plane_elems + at] = lo;
+  }
+}
+
 template <typename T, int D>
 __global__ void __launch_bounds__(kStatsThreads, 2)
     stats_bulk_kernel(const T *__restrict__ Q, const T *__restrict__ K, float *__restrict__ q_mean,
                       float *__restrict__ q_var, float *__restrict__ k_mean, float *__restrict__ k_var, int B,
-                      int Hq, int Hkv, int N, int N_alloc, int block, int nb) {
+                      int Hq, int Hkv, int N, int N_alloc, int block, int nb, FeatOut feat) {
   constexpr int VEC = Elem<T>::kVec;
   constexpr int COLS = D / VEC;                     // threads per row (16-byte vectors)
   constexpr int RPP = kStatsThreads / COLS;         // rows per pass of the CTA
@@ -260,6 +285,10 @@ __global__ void __launch_bounds__(kStatsThreads, 2)
   __shared__ float part_m2[2][kStatsWarps][D];
   __shared__ uint64_t full[kStatsStages];
   __shared__ int abort_flag;
+  // the decoded item of each ring stage, written by the issuing thread before
+  // its expect_tx arrive (release) and read after the full wait (acquire)
+  __shared__ long long meta_orow[kStatsStages];
+  __shared__ int meta_rows[kStatsStages];
 
   const long long n_q = static_cast<long long>(B) * Hq * nb;
   const long long total = n_q + static_cast<long long>(B) * Hkv * nb;
@@ -283,6 +312,8 @@ __global__ void __launch_bounds__(kStatsThreads, 2)
     bool is_q;
     locate(w, src, n_rows, orow, is_q);
     const uint32_t bytes = static_cast<uint32_t>(n_rows) * D * sizeof(T);
+    meta_orow[s] = is_q ? orow : -1 - orow;             // sign carries Q-or-K
+    meta_rows[s] = n_rows;
     mbar_arrive_expect_tx(smem_u32(&full[s]), bytes);
 #if BA_STATS_EVICT_FIRST
     // Q and K are read exactly once here: stream them through L2 at evict-first
@@ -312,12 +343,11 @@ __global__ void __launch_bounds__(kStatsThreads, 2)
   int it = 0;
   for (long long w = blockIdx.x; w < total; w += gridDim.x, ++it) {
     const int s = it % kStatsStages, pb = it & 1;
-    const T *src;
-    int n_rows;
-    long long orow;
-    bool is_q;
-    locate(w, src, n_rows, orow, is_q);
     const bool ok = mbar_wait_bounded(smem_u32(&full[s]), (it / kStatsStages) & 1, &abort_flag);
+    const long long mo = meta_orow[s];
+    const int n_rows = meta_rows[s];
+    const bool is_q = mo >= 0;
+    const long long orow = is_q ? mo : -1 - mo;
 
     // this thread's rows: exact local sum and centred second moment, merged
     // over the lanes of the warp that hold the same columns
@@ -375,6 +405,13 @@ __global__ void __launch_bounds__(kStatsThreads, 2)
       }
       (is_q ? q_mean : k_mean)[orow + tid] = mean;
       (is_q ? q_var : k_var)[orow + tid] = M2;
+      if (feat.q != nullptr) {
+        if (is_q)
+          store_feat(feat.q, feat.q_rows * D, orow + tid, __fmul_rn(feat.s, mean), __fmul_rn(feat.hs2, M2),
+                     __fmul_rn(__fmul_rn(feat.hs2, mean), mean));
+        else
+          store_feat(feat.k, feat.k_rows * D, orow + tid, mean, __fmaf_rn(mean, mean, M2), M2);
+      }
     }
   }
   // after an abandoned wait, let every issued copy land before exiting
@@ -395,12 +432,20 @@ inline int stats_rpt_needed(int block) {
   return (block + RPP - 1) / RPP;
 }
 
+// Whether the one-copy-per-block kernel (the one that can also write the
+// score features) serves this block size.
+template <typename T, int D>
+constexpr bool stats_bulk_fits(int block) {
+  return static_cast<size_t>(block) * D * sizeof(T) <= kStatsStageBytes;
+}
+
 template <typename T, int D>
 cudaError_t launch_stats(const T *Q, const T *K, float *qm, float *qv, float *km, float *kv, int B, int Hq, int Hkv,
-                         int N, int N_alloc, int block, int num_sms, cudaStream_t stream) {
+                         int N, int N_alloc, int block, int num_sms, cudaStream_t stream,
+                         FeatOut feat = FeatOut{nullptr, nullptr, 0.f, 0.f, 0, 0}) {
   const int nb = (N + block - 1) / block;
   const long long grid = static_cast<long long>(B) * (Hq + Hkv) * nb;
-  if (static_cast<size_t>(block) * D * sizeof(T) <= kStatsStageBytes) {
+  if (stats_bulk_fits<T, D>(block)) {
     const size_t smem = static_cast<size_t>(kStatsStages) * kStatsStageBytes;
     cudaError_t e = cudaFuncSetAttribute(stats_bulk_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
@@ -411,9 +456,10 @@ cudaError_t launch_stats(const T *Q, const T *K, float *qm, float *qv, float *km
     const long long persistent = static_cast<long long>(num_sms) * (per_sm > 0 ? per_sm : 1);
     const unsigned g = static_cast<unsigned>(grid < persistent ? grid : persistent);
     stats_bulk_kernel<T, D><<<g, kStatsThreads, smem, stream>>>(Q, K, qm, qv, km, kv, B, Hq, Hkv, N, N_alloc, block,
-                                                                 nb);
+                                                                 nb, feat);
     return cudaGetLastError();
   }
+  if (feat.q != nullptr) return cudaErrorInvalidValue;    // features only from the one-copy kernel
   const int need = stats_rpt_needed<T, D>(block);
   dim3 g(static_cast<unsigned>(grid));
   if (need <= 2) {

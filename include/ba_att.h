@@ -145,6 +145,46 @@ ba_status ba_att_select(const ba_att_shape *shape, double keep,
                         float *block_scores, ba_stream_t stream);
 
 /*
+ * ba_att_selector_workspace — device workspace bytes that ba_att_selector
+ * needs for this shape: the augmented score features of every block,
+ * 6 planes (3 parts x {hi, lo}) x (B*Hq*nq + B*Hkv*nk) rows x d bf16, rounded
+ * up to 256. -1 for an invalid shape.
+ */
+int64_t ba_att_selector_workspace(const ba_att_shape *shape);
+
+/*
+ * ba_att_selector — the whole selector stage in one call: ba_att_stats,
+ * then the scores and norm sorting of ba_att_select (default ranking, no
+ * variant flags). The pages give the two steps as one stage (BA-Att
+ * abstract, "Core claim": pooled means and diagonal variances, the corrected
+ * block score, sort and keep); there is no separate counterpart for the
+ * feature workspace, which is a layout of this implementation.
+ *
+ * The statistics pass also writes, per block, the augmented features of the
+ * score dot product (S~ = sum over parts p of q~_p . k~_p + ln m_j):
+ *   q~ = [ s*qbar, (s^2/2)*vq, (s^2/2)*qbar^2 ],  k~ = [ kbar, kbar^2 + vk, vk ]
+ * each split x = hi + lo into two bf16s (hi = RN(x), lo = RN(x - hi)), into
+ * `workspace`; the score GEMM reads them instead of deriving them per tile.
+ * Outputs are bit-identical to ba_att_stats followed by ba_att_select.
+ *
+ * Q, K, q_mean..k_var, kv_idx, kv_cnt, kmax, block_scores: as for
+ * ba_att_stats and ba_att_select (block_scores holds the score map on return).
+ * workspace   device, caller-owned, >= ba_att_selector_workspace(shape)
+ *             bytes, 16-byte aligned; its contents on return are unspecified.
+ * Shapes whose block of d values does not fit one 32 KB copy (bf16 with
+ * block * d > 16384, fp32 with block * d > 8192) run ba_att_stats and
+ * ba_att_select instead, leaving the workspace unused. NULL pointers ->
+ * BA_ERR_INVALID_ARG; misaligned -> BA_ERR_MISALIGNED; nk > 4096 ->
+ * BA_ERR_UNSUPPORTED.
+ */
+ba_status ba_att_selector(const ba_att_shape *shape, double keep,
+                          const void *Q, const void *K,
+                          float *q_mean, float *q_var, float *k_mean, float *k_var,
+                          void *workspace, float *block_scores,
+                          int32_t *kv_idx, int32_t *kv_cnt, int32_t kmax,
+                          ba_stream_t stream);
+
+/*
  * ba_att_split_lists — partition every kept-block list at a key-block
  * boundary into a block-external span (blocks < split_block) and a
  * block-internal span (blocks >= split_block) (FlashBlock Eq. 5: the two

@@ -184,3 +184,24 @@ def test_select_variant_arguments(lib):
     # the plain variant-free flag set of ba_att_select still reaches the same checks
     assert lib.ba_att_select_ex(ctypes.byref(s), ctypes.c_double(0.5), ctypes.c_uint32(0), P, P, P, P, P, P, 3,
                                 P, None) == 1
+
+
+def test_selector_workspace_and_arguments(lib):
+    s = shape()
+    nb = lib.ba_att_num_blocks(ctypes.byref(s))
+    want = 6 * s.B * (s.Hq + s.Hkv) * nb * s.d * 2
+    assert lib.ba_att_selector_workspace(ctypes.byref(s)) == (want + 255) // 256 * 256
+    assert lib.ba_att_selector_workspace(ctypes.byref(shape(d=96))) == -1
+    call = lambda sh, keep, *ptrs, kmax=8: lib.ba_att_selector(ctypes.byref(sh), ctypes.c_double(keep), *ptrs[:9],
+                                                               ptrs[9], kmax, None)
+    ptrs = [P] * 10
+    for i in range(10):                        # every pointer is required
+        bad = list(ptrs)
+        bad[i] = None
+        assert call(s, 0.5, *bad) == 1
+        bad[i] = MIS
+        assert call(s, 0.5, *bad) == 3
+    assert call(s, 0.0, *ptrs) == 1            # keep outside (0, 1]
+    assert call(s, 0.5, *ptrs, kmax=3) == 1    # kmax below the keep count
+    big = shape(N=4097 * 16, N_alloc=4097 * 16, block=16)
+    assert call(big, 0.5, *ptrs, kmax=4097) == 2
