@@ -243,24 +243,24 @@ def run_ours(args):
     L1, Lm = (torch.empty((w.B, w.Hq, w.N_alloc), device=dev) for _ in range(2))
     stream = torch.cuda.current_stream(dev)
 
-    names = ("stats", "select", "split", "sparse_lo", "sparse_hi_merge")
+    names = ("selector", "split", "sparse_lo", "sparse_hi_merge")
+    sel_ws = torch.empty(api.selector_workspace_bytes(shape), device=dev, dtype=torch.uint8)
 
     def step(events=None):
         def mark(i):
             if events is not None:
                 events[i].record(stream)
         mark(0)
-        api.stats(Qd, Kd, shape, out=stats_buf)
+        # stats, scores and top-k in one call (ba_att_selector)
+        api.selector(Qd, Kd, shape, keep, kmax=k, out=(stats_buf, idx, cnt, scores), workspace=sel_ws)
         mark(1)
-        api.select(stats_buf, shape, keep, out=(idx, cnt, scores))
-        mark(2)
         api.split_lists(idx, cnt, shape, split_block, out=lists)
-        mark(3)
+        mark(2)
         api.sparse_fwd(Qd, Kd, Vd, lists[0], lists[1], shape, out=(O1, L1))
-        mark(4)
+        mark(3)
         # second span, merged with the first in its epilogue (FlashBlock Eq. 9)
         api.sparse_fwd_merge(Qd, Kd, Vd, lists[2], lists[3], shape, O1, L1, out=(Om, Lm))
-        mark(5)
+        mark(4)
 
     for _ in range(args.warmup):
         step()
@@ -317,14 +317,13 @@ def run_ours(args):
                     "peak_source": f"{peak_src} (dense bf16 burst)", "traffic": traffic,
                     "units": f"{cnt_total} kept (query block, key block) pairs x 4*b^2*d FLOP"}
         sel_bytes = selector_bytes(w, k)
-        stats_bytes = sel_bytes - w.B * w.Hq * nb * (k + 1) * 4
-        sel_ms = stage_ms_median["stats"] + stage_ms_median["select"]
-        sel_ms_mean = stage_ms["stats"] + stage_ms["select"]
+        sel_ms = stage_ms_median["selector"]
+        sel_ms_mean = stage_ms["selector"]
         frac = lambda byts, ms: round(byts / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)
-        selector = {"bound": "hbm", "achieved": round(sel_bytes / (sel_ms * 1e-3) / 1e9, 1),
+        selector = {"bound": "hbm", "call": "ba_att_selector (stats, scores, top-k)",
+                    "achieved": round(sel_bytes / (sel_ms * 1e-3) / 1e9, 1),
                     "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": frac(sel_bytes, sel_ms),
                     "bytes": sel_bytes, "ms": round(sel_ms, 4), "timing": "in the step, median over steps",
-                    "stats_frac": frac(stats_bytes, stage_ms_median["stats"]),
                     "frac_mean_over_steps": frac(sel_bytes, sel_ms_mean)}
         result = {
             "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -402,30 +401,38 @@ def run_selector_isolated(ctx, reps=20):
     stats_buf, idx, cnt, lists, O1, Om, L1, Lm = ctx["bufs"]
     shape, keep, w, dev = ctx["shape"], ctx["keep"], ctx["w"], ctx["dev"]
     scores = torch.empty((w.B, w.Hq, w.nb, w.nb), device=dev, dtype=torch.float32)
+    ws = torch.empty(api.selector_workspace_bytes(shape), device=dev, dtype=torch.uint8)
     stream = torch.cuda.current_stream(dev)
+    k = idx.shape[-1]
+    one_call = lambda: api.selector(ctx["Qd"], ctx["Kd"], shape, keep, kmax=k, out=(stats_buf, idx, cnt, scores),
+                                    workspace=ws)
+    one_call()
     api.stats(ctx["Qd"], ctx["Kd"], shape, out=stats_buf)
     api.select(stats_buf, shape, keep, out=(idx, cnt, scores))
     torch.cuda.synchronize()
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(reps)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(reps)]
     torch.cuda._sleep(100_000_000)                 # ~50 ms of GPU time while the host queues the reps
     for r in range(reps):
         ev[r][0].record(stream)
-        api.stats(ctx["Qd"], ctx["Kd"], shape, out=stats_buf)
+        one_call()
         ev[r][1].record(stream)
-        api.select(stats_buf, shape, keep, out=(idx, cnt, scores))
+        api.stats(ctx["Qd"], ctx["Kd"], shape, out=stats_buf)
         ev[r][2].record(stream)
+        api.select(stats_buf, shape, keep, out=(idx, cnt, scores))
+        ev[r][3].record(stream)
     torch.cuda.synchronize()
-    s_ms = float(np.median([e[0].elapsed_time(e[1]) for e in ev]))
-    l_ms = float(np.median([e[1].elapsed_time(e[2]) for e in ev]))
-    k = idx.shape[-1]
+    med = lambda a, b: float(np.median([e[a].elapsed_time(e[b]) for e in ev]))
+    o_ms, s_ms, l_ms = med(0, 1), med(1, 2), med(2, 3)
     byts = selector_bytes(w, k)
     stats_bytes = byts - w.B * w.Hq * w.nb * (k + 1) * 4
     peaks, _ = load_peaks()
-    return {"stats_ms": round(s_ms, 4), "select_ms": round(l_ms, 4), "bytes": byts,
-            "achieved_gbs": round(byts / ((s_ms + l_ms) * 1e-3) / 1e9, 1),
-            "frac": round(byts / ((s_ms + l_ms) * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
-            "stats_frac": round(stats_bytes / (s_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
-            "timing": f"stats + select back to back, median of {reps}, launches queued ahead"}
+    fr = lambda b, ms: round(b / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)
+    return {"ms": round(o_ms, 4), "bytes": byts, "achieved_gbs": round(byts / (o_ms * 1e-3) / 1e9, 1),
+            "frac": fr(byts, o_ms),
+            "two_calls": {"stats_ms": round(s_ms, 4), "select_ms": round(l_ms, 4), "frac": fr(byts, s_ms + l_ms),
+                          "stats_frac": fr(stats_bytes, s_ms)},
+            "timing": f"ba_att_selector, then ba_att_stats + ba_att_select, back to back, median of {reps}, "
+                      "launches queued ahead"}
 
 
 def run_merge_standalone(ctx, steps=5):
