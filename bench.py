@@ -330,7 +330,7 @@ def run_ours(args):
             "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": f"{w.name}: B={w.B} Hq={w.Hq} Hkv={w.Hkv} N={w.N} d={w.d} block={w.block} "
-                                   f"bf16 keep={keep}; step = stats+select+split(block {split_block})"
+                                   f"bf16 keep={keep}; step = selector(stats+scores+top-k)+split(block {split_block})"
                                    f"+sparse_fwd+sparse_fwd_merge",
                        "keep": keep, "kept_blocks_per_query_block": k, "split_block": split_block,
                        "parallelism": f"{world} independent replica(s)",

@@ -509,7 +509,7 @@ size_t round_up(size_t x) { return (x + kWsAlign - 1) / kWsAlign * kWsAlign; }
 struct PipeLayout {
   int C = 0, G = 0, nb = 0, k = 0;
   size_t q[2], kk[2], v[2], o[2], l[2];                 // double-buffered chunk inputs and outputs
-  size_t qm, qv, km, kv, idx, cnt, sc;                  // selector buffers of one chunk
+  size_t qm, qv, km, kv, idx, cnt, sc, feat;            // selector buffers of one chunk
   size_t lo_idx, lo_cnt, hi_idx, hi_cnt, o1, l1;         // split buffers and the first span's fp32 partial
   size_t total = 0;
 };
@@ -555,6 +555,7 @@ bool pipe_layout(const ba_att_shape *s, double keep, int32_t split_block, int32_
   L->idx = take(hq * nb * k * 4);
   L->cnt = take(hq * nb * 4);
   L->sc = take(hq * nb * static_cast<size_t>(nb) * 4);
+  L->feat = take(6 * (hq + hk) * nb * s->d * 2);          // ba_att_selector's feature workspace
   if (split_block >= 0) {
     L->lo_idx = take(hq * nb * k * 4);
     L->lo_cnt = take(hq * nb * 4);
@@ -667,9 +668,8 @@ ba_status forward_host_impl(PipeResources *r, const ba_att_shape *s, double keep
     float *qm = reinterpret_cast<float *>(ws + L.qm), *qv = reinterpret_cast<float *>(ws + L.qv);
     float *km = reinterpret_cast<float *>(ws + L.km), *kv = reinterpret_cast<float *>(ws + L.kv);
     int32_t *idx = reinterpret_cast<int32_t *>(ws + L.idx), *cnt = reinterpret_cast<int32_t *>(ws + L.cnt);
-    st = ba_att_stats(&sc, Qc, Kc, qm, qv, km, kv, stream);
-    if (st == BA_OK)
-      st = ba_att_select(&sc, keep, qm, qv, km, kv, idx, cnt, L.k, reinterpret_cast<float *>(ws + L.sc), stream);
+    st = ba_att_selector(&sc, keep, Qc, Kc, qm, qv, km, kv, ws + L.feat, reinterpret_cast<float *>(ws + L.sc), idx,
+                         cnt, L.k, stream);
     if (st == BA_OK && split_block >= 0) {
       int32_t *lo_idx = reinterpret_cast<int32_t *>(ws + L.lo_idx), *lo_cnt = reinterpret_cast<int32_t *>(ws + L.lo_cnt);
       int32_t *hi_idx = reinterpret_cast<int32_t *>(ws + L.hi_idx), *hi_cnt = reinterpret_cast<int32_t *>(ws + L.hi_cnt);
