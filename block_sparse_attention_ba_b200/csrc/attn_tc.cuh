@@ -147,7 +147,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const int32_t *__restrict__ kv_idx,
                    const int32_t *__restrict__ kv_cnt, int kmax, TO *O, float *LSE, const float *O_prev,
-                   const float *L_prev, int Hq, int Hkv, int N, int N_alloc, int nb, float scale_log2) {
+                   const float *L_prev, int Hq, int Hkv, int N, int N_alloc, int nb, int block,
+                   float scale_log2) {
   extern __shared__ uint8_t dyn_smem[];
   __shared__ Ctl ctl;
   const uint32_t smem_base = (smem_u32(dyn_smem) + 1023u) & ~1023u;
@@ -156,14 +157,18 @@ __global__ void __launch_bounds__(kThreads, 2)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // tile -> (b, kv head, query block, head within group): consecutive CTAs
-  // share a KV head, so its K/V stay hot in L2.
+  // tile -> (b, kv head, 128-row query tile, head within group): consecutive
+  // CTAs share a KV head, so its K/V stay hot in L2. A block of `block` rows
+  // (128 or 256) is block/128 query tiles (which share its list) and
+  // block/64 key halves.
   const int G = Hq / Hkv;
+  const int qpb = block >> 7, hpe = block >> 6;
   long long tile = blockIdx.x;
   const int hg = static_cast<int>(tile % G);
   tile /= G;
-  const int i = static_cast<int>(tile % nb);
-  tile /= nb;
+  const int it = static_cast<int>(tile % (static_cast<long long>(nb) * qpb));   // query tile within the head
+  const int i = it / qpb;                                                        // its query block
+  tile /= static_cast<long long>(nb) * qpb;
   const int g = static_cast<int>(tile % Hkv);
   const int b = static_cast<int>(tile / Hkv);
   const int h = g * G + hg;
@@ -207,7 +212,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       tma_prefetch_desc(&tm_q);
       mbar_arrive_expect_tx(bar(Q_FULL), DM::kTileBytes);
 #pragma unroll
-      for (int sp = 0; sp < DM::kSpans; ++sp) tma_load_3d(&tm_q, sQ + sp * kHalfBytes, bar(Q_FULL), 64 * sp, i * kTileRows, qz);
+      for (int sp = 0; sp < DM::kSpans; ++sp) tma_load_3d(&tm_q, sQ + sp * kHalfBytes, bar(Q_FULL), 64 * sp, it * kTileRows, qz);
     }
     int issued = -1;                    // last half-block index u loaded
     bool bad_index = false, bad_order = false;
@@ -219,18 +224,18 @@ __global__ void __launch_bounds__(kThreads, 2)
         j = 0;                            // load a valid block; softmax masks it out
       }
       bool stop = false;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        if (t > 0 && !mbar_wait_bounded(bar(empty0 + h), (t - 1) & 1, abort)) {
+      for (int hh = 0; hh < hpe; ++hh) {
+        const int u = t * hpe + hh, h = u & 1;          // half index; halves alternate the two slots
+        if (u >= 2 && !mbar_wait_bounded(bar(empty0 + h), ((u >> 1) - 1) & 1, abort)) {
           stop = true;
           break;
         }
         mbar_arrive_expect_tx(bar(full0 + h), DM::kSpans * kHalfRowsBytes);
-        const int row = j * kTileRows + h * kHalfKeys;
+        const int row = j * block + hh * kHalfKeys;
 #pragma unroll
         for (int sp = 0; sp < DM::kSpans; ++sp)
           tma_load_3d(tm, slot + sp * kHalfBytes + h * kHalfRowsBytes, bar(full0 + h), 64 * sp, row, kz);
-        issued = 2 * t + h;
+        issued = u;
       }
       if (stop) break;
     }
@@ -246,7 +251,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     // ------------------------------------------------------------ MMA issuer
     constexpr uint32_t idesc_qk = idesc_bf16_f32(128, kHalfKeys, 0, 0);
     constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
-    const int n_half = 2 * cnt;
+    const int n_half = hpe * cnt;
     // S_u = Q K_u^T into S columns h*64..h*64+63
     auto issue_s = [&](int u) -> bool {
       const int h = u & 1;
@@ -287,20 +292,20 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int row = threadIdx.x;                       // TMEM lane = query row in tile
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
     const uint32_t tS = tmem + lane_off + kColS, tO = tmem + lane_off + kColO;
-    const int qrow = i * kTileRows + row;
+    const int qrow = it * kTileRows + row;
     const long long orow = static_cast<long long>(qz) * N_alloc + qrow;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     int n_keys = 0;
     ListCursor cur(list, cnt, nb);
-    for (int u = 0; u < 2 * cnt; ++u) {
-      const int h = u & 1;
-      if (h == 0) {
+    for (int u = 0; u < hpe * cnt; ++u) {
+      const int h = u & 1, hh = u % hpe;                // S slot; half within the key block
+      if (hh == 0) {
         int j;
-        const bool valid = cur.step(u >> 1, j);
-        n_keys = valid ? min(kTileRows, N - j * kTileRows) : 0;
+        const bool valid = cur.step(u / hpe, j);
+        n_keys = valid ? min(block, N - j * block) : 0;
       }
-      const int n_half = min(max(n_keys - h * kHalfKeys, 0), kHalfKeys);
+      const int n_half = min(max(n_keys - hh * kHalfKeys, 0), kHalfKeys);
       bool w = mbar_wait_bounded(bar(S_FULL0 + h), (u >> 1) & 1, abort);
       if (!__all_sync(0xFFFFFFFFu, w)) { ok = false; break; }
       tc_fence_after();

@@ -99,7 +99,7 @@ bool make_head_map(CUtensorMap *map, const void *ptr, int d, int N_valid, int N_
 }
 
 bool use_tensor_core_path(const ba_att_shape *s) {
-  return s->dtype == BA_DTYPE_BF16 && (s->d == 128 || s->d == 64) && s->block == 128;
+  return s->dtype == BA_DTYPE_BF16 && (s->d == 128 || s->d == 64) && (s->block == 128 || s->block == 256);
 }
 
 __global__ void bounded_wait_selftest_kernel(unsigned long long limit_ns) {
@@ -386,7 +386,8 @@ ba_status sparse_fwd_impl(const ba_att_shape *s, const void *Q, const void *K, c
         !make_head_map(&mk, K, s->d, s->N, s->N_alloc, static_cast<long long>(s->B) * s->Hkv, tc::kKvBoxRows) ||
         !make_head_map(&mv, V, s->d, s->N, s->N_alloc, static_cast<long long>(s->B) * s->Hkv, tc::kKvBoxRows))
       return BA_ERR_CUDA;
-    const long long tiles = static_cast<long long>(s->B) * s->Hq * nb;
+    // one CTA per 128-row query tile (a 256-row block is two tiles sharing its list)
+    const long long tiles = static_cast<long long>(s->B) * s->Hq * nb * (s->block / tc::kTileRows);
     if (tiles > 0x7FFFFFFFLL) return BA_ERR_UNSUPPORTED;
     const float sl2 = scale * 1.4426950408889634f;
     const uint32_t smem = tc::dyn_smem_bytes(s->d);
@@ -394,7 +395,8 @@ ba_status sparse_fwd_impl(const ba_att_shape *s, const void *Q, const void *K, c
       cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
       if (e != cudaSuccess) return BA_ERR_CUDA;
       kernel<<<static_cast<unsigned>(tiles), tc::kThreads, smem, cs>>>(
-          mq, mk, mv, kv_idx, kv_cnt, kmax, out, LSE, O_prev, L_prev, s->Hq, s->Hkv, s->N, s->N_alloc, nb, sl2);
+          mq, mk, mv, kv_idx, kv_cnt, kmax, out, LSE, O_prev, L_prev, s->Hq, s->Hkv, s->N, s->N_alloc, nb, s->block,
+          sl2);
       return from_cuda(cudaGetLastError());
     };
     float *of = static_cast<float *>(O);

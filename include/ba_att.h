@@ -271,8 +271,10 @@ ba_status ba_att_complement_lists(const ba_att_shape *shape, const int32_t *kv_i
  * o_dtype   shape->dtype, or BA_DTYPE_F32 to keep a partial output in fp32
  *           (one rounding in total when partials are merged later).
  * LSE       device fp32 [B, Hq, N_alloc], natural log (written).
- * Paths: bf16 with d = 64 or 128 and block = 128 runs the tcgen05/TMEM tensor-core
- * kernel; every other supported shape runs an fp32 CUDA-core kernel.
+ * Paths: bf16 with d = 64 or 128 and block = 128 or 256 runs the tcgen05/TMEM
+ * tensor-core kernel (a 256-row block is two 128-row query tiles sharing its
+ * list, its key blocks four 64-key halves); every other supported shape runs
+ * an fp32 CUDA-core kernel.
  */
 ba_status ba_att_sparse_fwd(const ba_att_shape *shape,
                             const void *Q, const void *K, const void *V,

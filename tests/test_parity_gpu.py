@@ -121,6 +121,9 @@ SMALL = [
     ("dlm_16k", dict(N=300 * 128 - 5, Hq=2, Hkv=2), 0.3),             # 300 blocks: ragged score tiles
     ("dlm_16k", dict(N=2048 - 17, N_alloc=2048, Hq=4, Hkv=2, d=64), 0.5),   # tcgen05 path with d = 64, ragged
     ("sweep_32k", dict(N=4096, Hq=4, Hkv=1, d=64), 0.25),            # d = 64, needle generator
+    ("dlm_16k", dict(N=4096, Hq=4, Hkv=2, block=256), 0.5),          # tcgen05 path, 256-row blocks
+    ("dlm_16k", dict(N=3 * 256 + 200, N_alloc=1024, Hq=2, Hkv=1, block=256), 0.5),   # 256-row blocks, ragged
+    ("dlm_16k", dict(N=2048 - 40, N_alloc=2048, Hq=4, Hkv=2, d=64, block=256), 0.5),  # 256-row blocks, d = 64
 ]
 
 
@@ -142,6 +145,7 @@ def test_small_full_parity(name, over, keep):
 
 @pytest.mark.parametrize("name,over", [("tiny_fp32", {}), ("dlm_16k", dict(N=1536, Hq=4, Hkv=2)),
                                        ("dlm_16k", dict(N=1536 - 9, N_alloc=1536, Hq=4, Hkv=2, d=64)),
+                                       ("dlm_16k", dict(N=1536, Hq=4, Hkv=2, block=256)),
                                        ("video_32k", dict(N=600, N_alloc=640, Hq=2, Hkv=2, grid=(3, 10, 20)))])
 def test_keep_all_equals_dense(name, over):
     # check (1): keep = 1.0 selects every block and equals dense attention

@@ -22,6 +22,7 @@ CASES = [
     ("dlm_16k", dict(N=2048 - 17, N_alloc=2048, Hq=4, Hkv=2, d=64), 0.5),   # d 64
     ("dlm_16k", dict(N=1024, Hq=2, Hkv=1, d=64, block=64), 0.5),       # bf16 block 64
     ("dlm_16k", dict(N=1024, B=2, Hq=4, Hkv=2), 0.5),                  # two batches
+    ("dlm_16k", dict(N=2048 - 40, N_alloc=2048, Hq=4, Hkv=2, d=64, block=256), 0.5),   # 256-row blocks, d 64
     ("tiny_fp32", dict(N=2048, d=128, block=128), 0.5),                # 64 KB blocks: plain stats + select
 ]
 
