@@ -162,7 +162,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   // (128 or 256) is block/128 query tiles (which share its list) and
   // block/64 key halves.
   const int G = Hq / Hkv;
-  const int qpb = block >> 7, hpe = block >> 6;
+  const int qpb = block >> 7, hpe_log2 = block == 256 ? 2 : 1, hpe = 1 << hpe_log2;
   long long tile = blockIdx.x;
   const int hg = static_cast<int>(tile % G);
   tile /= G;
@@ -299,10 +299,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     int n_keys = 0;
     ListCursor cur(list, cnt, nb);
     for (int u = 0; u < hpe * cnt; ++u) {
-      const int h = u & 1, hh = u % hpe;                // S slot; half within the key block
+      const int h = u & 1, hh = u & (hpe - 1);          // S slot; half within the key block
       if (hh == 0) {
         int j;
-        const bool valid = cur.step(u / hpe, j);
+        const bool valid = cur.step(u >> hpe_log2, j);
         n_keys = valid ? min(block, N - j * block) : 0;
       }
       const int n_half = min(max(n_keys - hh * kHalfKeys, 0), kHalfKeys);

@@ -5,8 +5,11 @@ passes float32). Inputs are arrays shaped [B, H, N_alloc, d]; only the first
 ``N`` rows of each head are tokens, the rest is padding and is never read.
 
 Notation (used in every docstring below):
-  b      block size, equal for queries and keys
-  nq=nk  number of blocks, ceil(N / b); block i covers rows [i*b, min(N, (i+1)*b))
+  b      block size; queries and keys share it unless a key block size b_k
+         is given (asymmetric blocks), then query blocks have b rows and key
+         blocks b_k rows
+  nq, nk number of query / key blocks, ceil(N / b) and ceil(N / b_k); block i
+         covers rows [i*b, min(N, (i+1)*b)) (b_k for key blocks)
   n_i    valid rows of query block i,  m_j  valid rows of key block j
   s      softmax scale (default d**-0.5)
   g(h)   KV head of query head h: h // (Hq // Hkv)  (grouped-query attention)
@@ -292,7 +295,7 @@ def _attend(q, keys, vals, s, dtype):
 
 
 def masked_attention(Q, K, V, idx, cnt, N: int, b: int, sm_scale: float,
-                     query_blocks=None, dtype=np.float64):
+                     query_blocks=None, dtype=np.float64, b_k: int | None = None):
     """Block-sparse bidirectional attention over the kept key blocks.
 
     [BA-Att, abstract; Figure 4]: attention is computed only over the selected
@@ -304,7 +307,9 @@ def masked_attention(Q, K, V, idx, cnt, N: int, b: int, sm_scale: float,
     probability matrix per query block; no online rescaling.
 
     query_blocks: optional iterable of (batch, head, i) to evaluate; rows of
-    other blocks are left as NaN. Returns O [B, Hq, N_alloc, d], LSE [B, Hq, N_alloc].
+    other blocks are left as NaN. b_k: key block size when it differs from the
+    query block size b (the lists then index blocks of b_k keys).
+    Returns O [B, Hq, N_alloc, d], LSE [B, Hq, N_alloc].
     """
     Q = np.asarray(Q)
     K = np.asarray(K)
@@ -320,7 +325,8 @@ def masked_attention(Q, K, V, idx, cnt, N: int, b: int, sm_scale: float,
         g = _kv_head(h, Hq, Hkv)
         rows = _block_rows(N, b, i)
         blocks = [int(j) for j in idx[bb, h, i, : int(cnt[bb, h, i])]]
-        keys = np.concatenate([_block_rows(N, b, j) for j in blocks]) if blocks else np.zeros(0, dtype=np.int64)
+        bk = b if b_k is None else b_k
+        keys = np.concatenate([_block_rows(N, bk, j) for j in blocks]) if blocks else np.zeros(0, dtype=np.int64)
         q = Q[bb, h, rows].astype(dtype)
         kk = K[bb, g, keys].astype(dtype)
         vv = V[bb, g, keys].astype(dtype)
@@ -448,8 +454,8 @@ def split_lists(idx, cnt, split_block: int):
 # The oracle post-downsample map and diagnostics
 # ---------------------------------------------------------------------------
 
-def post_downsample_map(Q, K, N: int, b: int, sm_scale: float, dtype=np.float64):
-    """Exact post-downsample block map A[B, Hq, nq, nk].
+def post_downsample_map(Q, K, N: int, b: int, sm_scale: float, dtype=np.float64, b_k: int | None = None):
+    """Exact post-downsample block map A[B, Hq, nq, nk] (key blocks of b_k rows if given).
 
     [BA-Att, "Core claim"; abstract]: the reference the selector approximates
     is the full softmax attention map aggregated to blocks after the softmax:
@@ -462,8 +468,10 @@ def post_downsample_map(Q, K, N: int, b: int, sm_scale: float, dtype=np.float64)
     B, Hq, _, _ = Q.shape
     Hkv = K.shape[1]
     counts = block_counts(N, b)
-    nb = len(counts)
-    A = np.zeros((B, Hq, nb, nb), dtype=dtype)
+    bk = b if b_k is None else b_k
+    kcounts = block_counts(N, bk)
+    nb, nk = len(counts), len(kcounts)
+    A = np.zeros((B, Hq, nb, nk), dtype=dtype)
     for bb in range(B):
         for h in range(Hq):
             g = _kv_head(h, Hq, Hkv)
@@ -472,8 +480,8 @@ def post_downsample_map(Q, K, N: int, b: int, sm_scale: float, dtype=np.float64)
             P /= P.sum(axis=1, keepdims=True)
             for i in range(nb):
                 ri = slice(i * b, i * b + counts[i])
-                for j in range(nb):
-                    cj = slice(j * b, j * b + counts[j])
+                for j in range(nk):
+                    cj = slice(j * bk, j * bk + kcounts[j])
                     A[bb, h, i, j] = P[ri, cj].sum() / counts[i]
     return A
 

@@ -458,3 +458,58 @@ def test_correction_improves_rank_agreement_on_planted_blocks():
     A = O.post_downsample_map(Q, K, w.N, w.block, s)
     assert O.spearman_vs_post(S, A) >= O.spearman_vs_post(P, A) - 1e-9
     assert 0.0 <= O.topk_recall_vs_post(S, A, 4) <= 1.0
+
+
+# ------------------------------------------------- asymmetric blocks (query block b, key block b_k)
+
+def test_asymmetric_keep_all_equals_dense():
+    # every key block kept is dense attention whatever the two block sizes
+    Q, K, V = _qkv()
+    N, s = 200, 16 ** -0.5
+    for b, bk in ((32, 16), (16, 64), (64, 24)):
+        nq, nk = O.num_blocks(N, b), O.num_blocks(N, bk)
+        idx = np.tile(np.arange(nk, dtype=np.int32), (1, 4, nq, 1))
+        cnt = np.full((1, 4, nq), nk, dtype=np.int32)
+        Om, Lm = O.masked_attention(Q, K, V, idx, cnt, N, b, s, b_k=bk)
+        Od, Ld = O.dense_attention(Q, K, V, N, s)
+        np.testing.assert_allclose(Om[:, :, :N], Od, rtol=1e-11, atol=1e-12)
+        np.testing.assert_allclose(Lm[:, :, :N], Ld, rtol=1e-12, atol=1e-12)
+
+
+def test_asymmetric_lists_equal_their_refinement():
+    # a key block of 2c rows is the union of two blocks of c rows: lists over
+    # b_k = 32 equal, row by row, lists over b_k = 16 naming both halves
+    Q, K, V = _qkv()
+    N, b, s = 200, 32, 16 ** -0.5                 # ragged last blocks: 200 = 6*32 + 8
+    nq, nk = O.num_blocks(N, b), O.num_blocks(N, 32)
+    rng = np.random.default_rng(7)
+    idx = np.full((1, 4, nq, nk), -1, dtype=np.int32)
+    cnt = np.zeros((1, 4, nq), dtype=np.int32)
+    fine_idx = np.full((1, 4, nq, 2 * nk), -1, dtype=np.int32)
+    fine_cnt = np.zeros((1, 4, nq), dtype=np.int32)
+    for h in range(4):
+        for i in range(nq):
+            sel = np.sort(rng.choice(nk, size=int(rng.integers(1, nk + 1)), replace=False))
+            idx[0, h, i, : len(sel)] = sel
+            cnt[0, h, i] = len(sel)
+            fine = [f for j in sel for f in (2 * j, 2 * j + 1) if f < O.num_blocks(N, 16)]
+            fine_idx[0, h, i, : len(fine)] = fine
+            fine_cnt[0, h, i] = len(fine)
+    Oa, La = O.masked_attention(Q, K, V, idx, cnt, N, b, s, b_k=32)
+    Of, Lf = O.masked_attention(Q, K, V, fine_idx, fine_cnt, N, b, s, b_k=16)
+    np.testing.assert_allclose(Oa[:, :, :N], Of[:, :, :N], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(La[:, :, :N], Lf[:, :, :N], rtol=1e-13, atol=1e-13)
+
+
+def test_asymmetric_post_downsample_map():
+    # rows sum to 1; merging adjacent key columns gives the map at twice the key block
+    rng = np.random.default_rng(13)
+    N, d = 90, 8
+    Q = rng.standard_normal((1, 2, N, d))
+    K = rng.standard_normal((1, 1, N, d))
+    s = d ** -0.5
+    A16 = O.post_downsample_map(Q, K, N, 32, s, b_k=16)       # 3 query blocks x 6 key blocks
+    A32 = O.post_downsample_map(Q, K, N, 32, s)
+    assert A16.shape == (1, 2, 3, 6) and A32.shape == (1, 2, 3, 3)
+    np.testing.assert_allclose(A16.sum(-1), 1.0, rtol=1e-13)
+    np.testing.assert_allclose(A16[..., 0::2] + A16[..., 1::2], A32, rtol=1e-12, atol=1e-15)
