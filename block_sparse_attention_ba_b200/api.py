@@ -33,13 +33,14 @@ _I32 = ctypes.c_int32
 class CShape(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32), ("N", ctypes.c_int32),
                 ("N_alloc", ctypes.c_int32), ("d", ctypes.c_int32), ("block", ctypes.c_int32),
-                ("dtype", ctypes.c_int32), ("sm_scale", ctypes.c_float)]
+                ("dtype", ctypes.c_int32), ("sm_scale", ctypes.c_float), ("block_k", ctypes.c_int32)]
 
 
 _SIGS = {
     "ba_att_version": (ctypes.c_char_p, []),
     "ba_att_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "ba_att_num_blocks": (_I32, [ctypes.POINTER(CShape)]),
+    "ba_att_num_key_blocks": (_I32, [ctypes.POINTER(CShape)]),
     "ba_att_keep_count": (_I32, [ctypes.POINTER(CShape), ctypes.c_double]),
     "ba_att_stats": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _P, _P, _P, _P, _P]),
     "ba_att_select": (ctypes.c_int, [ctypes.POINTER(CShape), ctypes.c_double, _P, _P, _P, _P, _P, _P, _I32, _P, _P]),
@@ -111,10 +112,22 @@ class Shape:
     block: int
     dtype: int
     sm_scale: float = 0.0
+    block_k: int = 0          # key block size when it differs from block (0: equal)
 
     @property
     def nb(self) -> int:
+        """Query blocks, ceil(N / block)."""
         return -(-self.N // self.block)
+
+    @property
+    def kb(self) -> int:
+        """Key block size."""
+        return self.block_k if self.block_k > 0 else self.block
+
+    @property
+    def nk(self) -> int:
+        """Key blocks, ceil(N / key block size)."""
+        return -(-self.N // self.kb)
 
     @property
     def scale(self) -> float:
@@ -122,16 +135,16 @@ class Shape:
 
     def c(self) -> CShape:
         return CShape(self.B, self.Hq, self.Hkv, self.N, self.N_alloc, self.d, self.block, self.dtype,
-                      float(self.sm_scale))
+                      float(self.sm_scale), self.block_k)
 
     @staticmethod
     def of(Q: torch.Tensor, K: torch.Tensor, N: int | None = None, block: int = 128,
-           sm_scale: float = 0.0) -> "Shape":
+           sm_scale: float = 0.0, block_k: int = 0) -> "Shape":
         B, Hq, N_alloc, d = Q.shape
         dt = {torch.float32: DTYPE_F32, torch.bfloat16: DTYPE_BF16}.get(Q.dtype)
         if dt is None:
             raise TypeError(f"unsupported dtype {Q.dtype}")
-        return Shape(B, Hq, K.shape[1], N_alloc if N is None else N, N_alloc, d, block, dt, sm_scale)
+        return Shape(B, Hq, K.shape[1], N_alloc if N is None else N, N_alloc, d, block, dt, sm_scale, block_k)
 
 
 def _stream(t: torch.Tensor | None = None):
@@ -162,8 +175,8 @@ def stats(Q: torch.Tensor, K: torch.Tensor, shape: Shape, out=None):
     if out is None:
         out = (torch.empty((shape.B, shape.Hq, shape.nb, shape.d), device=dev, dtype=torch.float32),
                torch.empty((shape.B, shape.Hq, shape.nb, shape.d), device=dev, dtype=torch.float32),
-               torch.empty((shape.B, shape.Hkv, shape.nb, shape.d), device=dev, dtype=torch.float32),
-               torch.empty((shape.B, shape.Hkv, shape.nb, shape.d), device=dev, dtype=torch.float32))
+               torch.empty((shape.B, shape.Hkv, shape.nk, shape.d), device=dev, dtype=torch.float32),
+               torch.empty((shape.B, shape.Hkv, shape.nk, shape.d), device=dev, dtype=torch.float32))
     qm, qv, km, kv = out
     _check("ba_att_stats", lib.ba_att_stats(ctypes.byref(shape.c()), _dev(Q, "Q"), _dev(K, "K"), _dev(qm, "q_mean"),
                                             _dev(qv, "q_var"), _dev(km, "k_mean"), _dev(kv, "k_var"), _stream(Q)))
@@ -182,7 +195,7 @@ def select(stats_out, shape: Shape, keep: float, kmax: int | None = None, with_s
     if k < 1:
         raise BaAttError("ba_att_keep_count", 1)
     if kmax is None:                     # by-mass counts vary per row, up to nk
-        kmax = shape.nb if flags & SELECT_BY_MASS else k
+        kmax = shape.nk if flags & SELECT_BY_MASS else k
     dev = qm.device
     if out is None:
         idx = torch.empty((shape.B, shape.Hq, shape.nb, kmax), device=dev, dtype=torch.int32)
@@ -191,7 +204,7 @@ def select(stats_out, shape: Shape, keep: float, kmax: int | None = None, with_s
     else:
         idx, cnt, sc = out
     if sc is None:       # the score map is always written (the selection reads it back)
-        sc = torch.empty((shape.B, shape.Hq, shape.nb, shape.nb), device=dev, dtype=torch.float32)
+        sc = torch.empty((shape.B, shape.Hq, shape.nb, shape.nk), device=dev, dtype=torch.float32)
     _check("ba_att_select_ex", lib.ba_att_select_ex(
         ctypes.byref(shape.c()), ctypes.c_double(keep), ctypes.c_uint32(flags), _dev(qm, "q_mean"),
         _dev(qv, "q_var"), _dev(km, "k_mean"), _dev(kv, "k_var"), _dev(idx, "kv_idx"), _dev(cnt, "kv_cnt"),
@@ -223,11 +236,11 @@ def selector(Q: torch.Tensor, K: torch.Tensor, shape: Shape, keep: float, kmax: 
     if out is None:
         st = (torch.empty((shape.B, shape.Hq, shape.nb, shape.d), device=dev, dtype=torch.float32),
               torch.empty((shape.B, shape.Hq, shape.nb, shape.d), device=dev, dtype=torch.float32),
-              torch.empty((shape.B, shape.Hkv, shape.nb, shape.d), device=dev, dtype=torch.float32),
-              torch.empty((shape.B, shape.Hkv, shape.nb, shape.d), device=dev, dtype=torch.float32))
+              torch.empty((shape.B, shape.Hkv, shape.nk, shape.d), device=dev, dtype=torch.float32),
+              torch.empty((shape.B, shape.Hkv, shape.nk, shape.d), device=dev, dtype=torch.float32))
         idx = torch.empty((shape.B, shape.Hq, shape.nb, kmax), device=dev, dtype=torch.int32)
         cnt = torch.empty((shape.B, shape.Hq, shape.nb), device=dev, dtype=torch.int32)
-        sc = torch.empty((shape.B, shape.Hq, shape.nb, shape.nb), device=dev, dtype=torch.float32)
+        sc = torch.empty((shape.B, shape.Hq, shape.nb, shape.nk), device=dev, dtype=torch.float32)
     else:
         st, idx, cnt, sc = out
     if workspace is None:
@@ -259,7 +272,7 @@ def complement_lists(idx, cnt, shape: Shape, out=None):
     """The key blocks each kept-block list leaves out -> (c_idx [.., nb], c_cnt)."""
     lib = load_library()
     if out is None:
-        out = (torch.empty(idx.shape[:-1] + (shape.nb,), device=idx.device, dtype=torch.int32), torch.empty_like(cnt))
+        out = (torch.empty(idx.shape[:-1] + (shape.nk,), device=idx.device, dtype=torch.int32), torch.empty_like(cnt))
     c_idx, c_cnt = out
     _check("ba_att_complement_lists", lib.ba_att_complement_lists(
         ctypes.byref(shape.c()), _dev(idx, "kv_idx"), _dev(cnt, "kv_cnt"), idx.shape[-1], _dev(c_idx, "c_idx"),
@@ -320,9 +333,9 @@ def merge_lse(O1, L1, O2, L2, out=None, out_dtype=None):
     return out
 
 
-def forward(Q, K, V, N: int, block: int, keep: float, sm_scale: float = 0.0):
+def forward(Q, K, V, N: int, block: int, keep: float, sm_scale: float = 0.0, block_k: int = 0):
     """Full BA-Att forward: stats -> select -> sparse attention. Returns (O, LSE, idx, cnt)."""
-    shape = Shape.of(Q, K, N, block, sm_scale)
+    shape = Shape.of(Q, K, N, block, sm_scale, block_k)
     st = stats(Q, K, shape)
     idx, cnt = select(st, shape, keep)
     O, LSE = sparse_fwd(Q, K, V, idx, cnt, shape)
@@ -346,13 +359,13 @@ def _host(t: torch.Tensor, name: str) -> ctypes.c_void_p:
 
 def forward_host(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, N: int, block: int, keep: float,
                  split_block: int = -1, kv_heads_per_chunk: int = 0, sm_scale: float = 0.0,
-                 workspace: torch.Tensor | None = None, out=None, device=None):
+                 workspace: torch.Tensor | None = None, out=None, device=None, block_k: int = 0):
     """Whole forward from host tensors to host tensors (ba_att_forward_host):
     copies in, stats, select, sparse attention (split + merge when
     split_block >= 0), copies out, pipelined per chunk of KV heads. Q, K, V,
     and the outputs should be pinned for the copies to overlap compute.
     Asynchronous on the current stream; synchronise before reading (O, LSE)."""
-    shape = Shape.of(Q, K, N, block, sm_scale)
+    shape = Shape.of(Q, K, N, block, sm_scale, block_k)
     dev = torch.device("cuda") if device is None else torch.device(device)
     need = forward_host_workspace_bytes(shape, keep, split_block, kv_heads_per_chunk)
     if workspace is None:
@@ -374,10 +387,10 @@ def forward_host(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, N: int, bloc
 
 
 def forward_host_noalloc(Q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, N: int, block: int, keep: float,
-                         split_block: int = -1, sm_scale: float = 0.0, out=None, device=None):
+                         split_block: int = -1, sm_scale: float = 0.0, out=None, device=None, block_k: int = 0):
     """forward_host on the library's static device scratch (ba_att_forward_host_noalloc):
     no workspace argument, nothing allocated on the device by this call."""
-    shape = Shape.of(Q, K, N, block, sm_scale)
+    shape = Shape.of(Q, K, N, block, sm_scale, block_k)
     dev = torch.device("cuda") if device is None else torch.device(device)
     if out is None:
         O = torch.empty(Q.shape, dtype=Q.dtype).pin_memory()

@@ -36,7 +36,7 @@ template <typename T, typename TO, int D, bool MERGE>
 __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(
     const T *__restrict__ Q, const T *__restrict__ K, const T *__restrict__ V, const int32_t *__restrict__ kv_idx,
     const int32_t *__restrict__ kv_cnt, int kmax, TO *O, float *LSE, const float *O_prev, const float *L_prev, int Hq,
-    int Hkv, int N, int N_alloc, int block, int nb, int subs, float scale_log2) {
+    int Hkv, int N, int N_alloc, int block, int nb, int kblock, int nk, int subs, float scale_log2) {
   constexpr int DPL = D / 32;
   constexpr int RPW = kSimtRows / (kSimtThreads / 32);      // rows per warp
   __shared__ float q_s[kSimtRows][D];
@@ -78,7 +78,7 @@ __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(
 
   for (int t = 0; t < c; ++t) {
     const int j = __ldg(list + t);
-    if (j < 0 || j >= nb) {
+    if (j < 0 || j >= nk) {
       if (tid == 0 && sub == 0) raise_error(BA_DEVERR_BAD_INDEX);
       continue;
     }
@@ -86,8 +86,8 @@ __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(
       if (tid == 0 && sub == 0) raise_error(BA_DEVERR_NOT_ASCENDING);
       continue;
     }
-    const int key0 = j * block;
-    const int mj = min(block, N - key0);
+    const int key0 = j * kblock;
+    const int mj = min(kblock, N - key0);
     for (int c0 = 0; c0 < mj; c0 += 32) {
       __syncthreads();
       for (int e = tid; e < 32 * D; e += kSimtThreads) {
@@ -149,14 +149,16 @@ __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(
 
 template <typename T, typename TO, int D, bool MERGE = false>
 cudaError_t launch_attn_simt(const T *Q, const T *K, const T *V, const int32_t *idx, const int32_t *cnt, int kmax, TO *O,
-                             float *LSE, int B, int Hq, int Hkv, int N, int N_alloc, int block, float sm_scale,
-                             cudaStream_t stream, const float *O_prev = nullptr, const float *L_prev = nullptr) {
-  const int nb = (N + block - 1) / block;
+                             float *LSE, int B, int Hq, int Hkv, int N, int N_alloc, int block, int kblock,
+                             float sm_scale, cudaStream_t stream, const float *O_prev = nullptr,
+                             const float *L_prev = nullptr) {
+  const int nb = (N + block - 1) / block, nk = (N + kblock - 1) / kblock;
   const int subs = (block + kSimtRows - 1) / kSimtRows;
   dim3 grid(static_cast<unsigned>(nb * subs), Hq, B);
   const float scale_log2 = sm_scale * 1.4426950408889634f;
   attn_simt_kernel<T, TO, D, MERGE><<<grid, kSimtThreads, 0, stream>>>(Q, K, V, idx, cnt, kmax, O, LSE, O_prev, L_prev,
-                                                                    Hq, Hkv, N, N_alloc, block, nb, subs, scale_log2);
+                                                                    Hq, Hkv, N, N_alloc, block, nb, kblock, nk, subs,
+                                                                    scale_log2);
   return cudaGetLastError();
 }
 

@@ -147,8 +147,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const int32_t *__restrict__ kv_idx,
                    const int32_t *__restrict__ kv_cnt, int kmax, TO *O, float *LSE, const float *O_prev,
-                   const float *L_prev, int Hq, int Hkv, int N, int N_alloc, int nb, int block,
-                   float scale_log2) {
+                   const float *L_prev, int Hq, int Hkv, int N, int N_alloc, int nq, int block, int nk,
+                   int kblock, float scale_log2) {
   extern __shared__ uint8_t dyn_smem[];
   __shared__ Ctl ctl;
   const uint32_t smem_base = (smem_u32(dyn_smem) + 1023u) & ~1023u;
@@ -158,21 +158,21 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   // tile -> (b, kv head, 128-row query tile, head within group): consecutive
-  // CTAs share a KV head, so its K/V stay hot in L2. A block of `block` rows
-  // (128 or 256) is block/128 query tiles (which share its list) and
-  // block/64 key halves.
+  // CTAs share a KV head, so its K/V stay hot in L2. A query block of `block`
+  // rows (128 or 256) is block/128 query tiles, which share its list; a key
+  // block of `kblock` rows (64, 128 or 256) is kblock/64 key halves.
   const int G = Hq / Hkv;
-  const int qpb = block >> 7, hpe_log2 = block == 256 ? 2 : 1, hpe = 1 << hpe_log2;
+  const int qpb = block >> 7, hpe_log2 = kblock == 256 ? 2 : (kblock == 128 ? 1 : 0), hpe = 1 << hpe_log2;
   long long tile = blockIdx.x;
   const int hg = static_cast<int>(tile % G);
   tile /= G;
-  const int it = static_cast<int>(tile % (static_cast<long long>(nb) * qpb));   // query tile within the head
+  const int it = static_cast<int>(tile % (static_cast<long long>(nq) * qpb));   // query tile within the head
   const int i = it / qpb;                                                        // its query block
-  tile /= static_cast<long long>(nb) * qpb;
+  tile /= static_cast<long long>(nq) * qpb;
   const int g = static_cast<int>(tile % Hkv);
   const int b = static_cast<int>(tile / Hkv);
   const int h = g * G + hg;
-  const long long list_row = (static_cast<long long>(b) * Hq + h) * nb + i;
+  const long long list_row = (static_cast<long long>(b) * Hq + h) * nq + i;
   const int32_t *list = kv_idx + list_row * kmax;
   int cnt = __ldg(kv_cnt + list_row);
   if (cnt < 0 || cnt > kmax) {
@@ -216,11 +216,11 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     int issued = -1;                    // last half-block index u loaded
     bool bad_index = false, bad_order = false;
-    ListCursor cur(list, cnt, nb);
+    ListCursor cur(list, cnt, nk);
     for (int t = 0; t < cnt; ++t) {
       int j;
       if (!cur.step(t, j)) {
-        if (j < 0 || j >= nb) bad_index = true; else bad_order = true;
+        if (j < 0 || j >= nk) bad_index = true; else bad_order = true;
         j = 0;                            // load a valid block; softmax masks it out
       }
       bool stop = false;
@@ -231,7 +231,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           break;
         }
         mbar_arrive_expect_tx(bar(full0 + h), DM::kSpans * kHalfRowsBytes);
-        const int row = j * block + hh * kHalfKeys;
+        const int row = j * kblock + hh * kHalfKeys;
 #pragma unroll
         for (int sp = 0; sp < DM::kSpans; ++sp)
           tma_load_3d(tm, slot + sp * kHalfBytes + h * kHalfRowsBytes, bar(full0 + h), 64 * sp, row, kz);
@@ -297,13 +297,13 @@ __global__ void __launch_bounds__(kThreads, 2)
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     int n_keys = 0;
-    ListCursor cur(list, cnt, nb);
+    ListCursor cur(list, cnt, nk);
     for (int u = 0; u < hpe * cnt; ++u) {
       const int h = u & 1, hh = u & (hpe - 1);          // S slot; half within the key block
       if (hh == 0) {
         int j;
         const bool valid = cur.step(u >> hpe_log2, j);
-        n_keys = valid ? min(block, N - j * block) : 0;
+        n_keys = valid ? min(kblock, N - j * kblock) : 0;
       }
       const int n_half = min(max(n_keys - hh * kHalfKeys, 0), kHalfKeys);
       bool w = mbar_wait_bounded(bar(S_FULL0 + h), (u >> 1) & 1, abort);

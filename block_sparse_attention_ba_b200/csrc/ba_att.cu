@@ -50,13 +50,17 @@ ba_status check_shape(const ba_att_shape *s) {
   if (s->dtype != BA_DTYPE_F32 && s->dtype != BA_DTYPE_BF16) return BA_ERR_INVALID_ARG;
   if (s->d != 64 && s->d != 128) return BA_ERR_UNSUPPORTED;
   if (s->block < 16 || s->block > 256 || s->block % 16 != 0) return BA_ERR_UNSUPPORTED;
+  if (s->block_k != 0 && (s->block_k < 16 || s->block_k > 256 || s->block_k % 16 != 0)) return BA_ERR_UNSUPPORTED;
   if (std::isnan(s->sm_scale) || std::isinf(s->sm_scale)) return BA_ERR_INVALID_ARG;
   const long long rows = static_cast<long long>(s->B) * (s->Hq > s->Hkv ? s->Hq : s->Hkv) * s->N_alloc;
   if (rows > (1LL << 36)) return BA_ERR_UNSUPPORTED;
   return BA_OK;
 }
 
+// query blocks (block rows) and key blocks (kblock rows)
 int nblocks(const ba_att_shape *s) { return (s->N + s->block - 1) / s->block; }
+int kblock(const ba_att_shape *s) { return s->block_k > 0 ? s->block_k : s->block; }
+int nkblocks(const ba_att_shape *s) { return (s->N + kblock(s) - 1) / kblock(s); }
 
 float effective_scale(const ba_att_shape *s) {
   return s->sm_scale > 0.f ? s->sm_scale : 1.0f / std::sqrt(static_cast<float>(s->d));
@@ -99,7 +103,9 @@ bool make_head_map(CUtensorMap *map, const void *ptr, int d, int N_valid, int N_
 }
 
 bool use_tensor_core_path(const ba_att_shape *s) {
-  return s->dtype == BA_DTYPE_BF16 && (s->d == 128 || s->d == 64) && (s->block == 128 || s->block == 256);
+  const int kb = s->block_k > 0 ? s->block_k : s->block;
+  return s->dtype == BA_DTYPE_BF16 && (s->d == 128 || s->d == 64) && (s->block == 128 || s->block == 256) &&
+         (kb == 64 || kb == 128 || kb == 256);
 }
 
 __global__ void bounded_wait_selftest_kernel(unsigned long long limit_ns) {
@@ -136,10 +142,15 @@ int32_t ba_att_num_blocks(const ba_att_shape *shape) {
   return nblocks(shape);
 }
 
+int32_t ba_att_num_key_blocks(const ba_att_shape *shape) {
+  if (check_shape(shape) != BA_OK) return -1;
+  return nkblocks(shape);
+}
+
 int32_t ba_att_keep_count(const ba_att_shape *shape, double keep) {
   if (check_shape(shape) != BA_OK) return -1;
   if (!(keep > 0.f && keep <= 1.f)) return -1;
-  const int nk = nblocks(shape);
+  const int nk = nkblocks(shape);
   const double kk = std::ceil(static_cast<double>(keep) * nk - 1e-9);
   int k = static_cast<int>(kk);
   if (k < 1) k = 1;
@@ -162,16 +173,16 @@ ba_status ba_att_stats(const ba_att_shape *s, const void *Q, const void *K, floa
     auto q = static_cast<const __nv_bfloat16 *>(Q);
     auto k = static_cast<const __nv_bfloat16 *>(K);
     e = s->d == 128 ? launch_stats<__nv_bfloat16, 128>(q, k, q_mean, q_var, k_mean, k_var, s->B, s->Hq, s->Hkv, s->N,
-                                                       s->N_alloc, s->block, sms, cs)
+                                                       s->N_alloc, s->block, kblock(s), sms, cs)
                     : launch_stats<__nv_bfloat16, 64>(q, k, q_mean, q_var, k_mean, k_var, s->B, s->Hq, s->Hkv, s->N,
-                                                      s->N_alloc, s->block, sms, cs);
+                                                      s->N_alloc, s->block, kblock(s), sms, cs);
   } else {
     auto q = static_cast<const float *>(Q);
     auto k = static_cast<const float *>(K);
     e = s->d == 128 ? launch_stats<float, 128>(q, k, q_mean, q_var, k_mean, k_var, s->B, s->Hq, s->Hkv, s->N,
-                                               s->N_alloc, s->block, sms, cs)
+                                               s->N_alloc, s->block, kblock(s), sms, cs)
                     : launch_stats<float, 64>(q, k, q_mean, q_var, k_mean, k_var, s->B, s->Hq, s->Hkv, s->N,
-                                              s->N_alloc, s->block, sms, cs);
+                                              s->N_alloc, s->block, kblock(s), sms, cs);
   }
   return from_cuda(e);
 }
@@ -191,8 +202,10 @@ ba_status ba_att_select_ex(const ba_att_shape *s, double keep, uint32_t flags, c
   const int k = ba_att_keep_count(s, keep);
   if (k < 1) return BA_ERR_INVALID_ARG;
   if (kmax < k) return BA_ERR_INVALID_ARG;
-  const int nb = nblocks(s);
-  if (nb > 4096) return BA_ERR_UNSUPPORTED;
+  const int nb = nkblocks(s);                     // score row length
+  if (nb > 4096 || nblocks(s) > 1048576) return BA_ERR_UNSUPPORTED;
+  // the forced diagonal pairs query block i with key block i: equal block sizes only
+  if ((flags & BA_SELECT_FORCE_DIAGONAL) && kblock(s) != s->block) return BA_ERR_UNSUPPORTED;
   if ((flags & (BA_SELECT_FORCE_DIAGONAL | BA_SELECT_SHARED_GQA | BA_SELECT_BY_MASS)) && nb > 1024)
     return BA_ERR_UNSUPPORTED;
   if (flags & BA_SELECT_BY_MASS) {
@@ -204,10 +217,10 @@ ba_status ba_att_select_ex(const ba_att_shape *s, double keep, uint32_t flags, c
   const int sms = num_sms_of_current_device();
   const float tau = static_cast<float>(keep);
   cudaError_t e = s->d == 128 ? launch_select_tc<128>(q_mean, q_var, k_mean, k_var, kv_idx, kv_cnt, block_scores, s->B,
-                                                      s->Hq, s->Hkv, s->N, s->block, k, kmax, scale, flags, tau, sms,
+                                                      s->Hq, s->Hkv, s->N, s->block, kblock(s), k, kmax, scale, flags, tau, sms,
                                                       cs)
                               : launch_select_tc<64>(q_mean, q_var, k_mean, k_var, kv_idx, kv_cnt, block_scores, s->B,
-                                                     s->Hq, s->Hkv, s->N, s->block, k, kmax, scale, flags, tau, sms,
+                                                     s->Hq, s->Hkv, s->N, s->block, kblock(s), k, kmax, scale, flags, tau, sms,
                                                      cs);
   return from_cuda(e);
 }
@@ -238,29 +251,31 @@ bool make_feat_map(CUtensorMap *map, const void *ptr, int d, long long rows) {
 }
 
 long long feat_rows_q(const ba_att_shape *s) { return static_cast<long long>(s->B) * s->Hq * nblocks(s); }
-long long feat_rows_k(const ba_att_shape *s) { return static_cast<long long>(s->B) * s->Hkv * nblocks(s); }
+long long feat_rows_k(const ba_att_shape *s) { return static_cast<long long>(s->B) * s->Hkv * nkblocks(s); }
 
 // Whether the shape takes the feature path (else the selector is the plain
 // ba_att_stats + ba_att_select sequence).
 bool selector_feature_path(const ba_att_shape *s) {
+  const int bmax = s->block > kblock(s) ? s->block : kblock(s);
   const bool bulk = s->dtype == BA_DTYPE_BF16
-                        ? (s->d == 128 ? stats_bulk_fits<__nv_bfloat16, 128>(s->block)
-                                       : stats_bulk_fits<__nv_bfloat16, 64>(s->block))
-                        : (s->d == 128 ? stats_bulk_fits<float, 128>(s->block) : stats_bulk_fits<float, 64>(s->block));
+                        ? (s->d == 128 ? stats_bulk_fits<__nv_bfloat16, 128>(bmax)
+                                       : stats_bulk_fits<__nv_bfloat16, 64>(bmax))
+                        : (s->d == 128 ? stats_bulk_fits<float, 128>(bmax) : stats_bulk_fits<float, 64>(bmax));
   return bulk && feat_rows_q(s) + selft::kTile < 0x7FFFFFFFLL;
 }
 
 template <int D>
 cudaError_t launch_select_feat(const CUtensorMap &mq, const CUtensorMap &mk, float *scores, const ba_att_shape *s,
-                               int nb, int sms, cudaStream_t cs) {
-  const int n_tq = (nb + selft::kTile - 1) / selft::kTile;
-  const long long n_tiles = static_cast<long long>(s->B) * s->Hq * n_tq * n_tq;
+                               int nq, int nk, int sms, cudaStream_t cs) {
+  const int n_tq = (nq + selft::kTile - 1) / selft::kTile, n_tk = (nk + selft::kTile - 1) / selft::kTile;
+  const long long n_tiles = static_cast<long long>(s->B) * s->Hq * n_tq * n_tk;
   cudaError_t e = cudaFuncSetAttribute(selft::select_feat_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(selft::kDynSmem));
   if (e != cudaSuccess) return e;
   const unsigned grid = static_cast<unsigned>(n_tiles < sms ? n_tiles : sms);
   selft::select_feat_kernel<D><<<grid, selft::kThreads, selft::kDynSmem, cs>>>(mq, mk, scores, s->Hq, s->Hkv, s->N,
-                                                                              s->block, nb, n_tiles, n_tq);
+                                                                              kblock(s), nq, nk, n_tiles, n_tq,
+                                                                              n_tk);
   return cudaGetLastError();
 }
 }  // namespace
@@ -286,8 +301,8 @@ ba_status ba_att_selector(const ba_att_shape *s, double keep, const void *Q, con
     return BA_ERR_MISALIGNED;
   const int k = ba_att_keep_count(s, keep);
   if (k < 1 || kmax < k) return BA_ERR_INVALID_ARG;
-  const int nb = nblocks(s);
-  if (nb > 4096) return BA_ERR_UNSUPPORTED;
+  const int nq = nblocks(s), nk = nkblocks(s);
+  if (nk > 4096 || nq > 1048576) return BA_ERR_UNSUPPORTED;
   if (!selector_feature_path(s)) {
     st = ba_att_stats(s, Q, K, q_mean, q_var, k_mean, k_var, stream);
     return st == BA_OK ? ba_att_select(s, keep, q_mean, q_var, k_mean, k_var, kv_idx, kv_cnt, kmax, block_scores,
@@ -305,25 +320,25 @@ ba_status ba_att_selector(const ba_att_shape *s, double keep, const void *Q, con
     auto q = static_cast<const __nv_bfloat16 *>(Q);
     auto kk = static_cast<const __nv_bfloat16 *>(K);
     e = s->d == 128 ? launch_stats<__nv_bfloat16, 128>(q, kk, q_mean, q_var, k_mean, k_var, s->B, s->Hq, s->Hkv, s->N,
-                                                       s->N_alloc, s->block, sms, cs, feat)
+                                                       s->N_alloc, s->block, kblock(s), sms, cs, feat)
                     : launch_stats<__nv_bfloat16, 64>(q, kk, q_mean, q_var, k_mean, k_var, s->B, s->Hq, s->Hkv, s->N,
-                                                      s->N_alloc, s->block, sms, cs, feat);
+                                                      s->N_alloc, s->block, kblock(s), sms, cs, feat);
   } else {
     auto q = static_cast<const float *>(Q);
     auto kk = static_cast<const float *>(K);
     e = s->d == 128 ? launch_stats<float, 128>(q, kk, q_mean, q_var, k_mean, k_var, s->B, s->Hq, s->Hkv, s->N,
-                                               s->N_alloc, s->block, sms, cs, feat)
+                                               s->N_alloc, s->block, kblock(s), sms, cs, feat)
                     : launch_stats<float, 64>(q, kk, q_mean, q_var, k_mean, k_var, s->B, s->Hq, s->Hkv, s->N,
-                                              s->N_alloc, s->block, sms, cs, feat);
+                                              s->N_alloc, s->block, kblock(s), sms, cs, feat);
   }
   if (e != cudaSuccess) return from_cuda(e);
   CUtensorMap mq, mk;
   if (!make_feat_map(&mq, fq, s->d, feat_rows_q(s)) || !make_feat_map(&mk, fk, s->d, feat_rows_k(s)))
     return BA_ERR_CUDA;
-  e = s->d == 128 ? launch_select_feat<128>(mq, mk, block_scores, s, nb, sms, cs)
-                  : launch_select_feat<64>(mq, mk, block_scores, s, nb, sms, cs);
+  e = s->d == 128 ? launch_select_feat<128>(mq, mk, block_scores, s, nq, nk, sms, cs)
+                  : launch_select_feat<64>(mq, mk, block_scores, s, nq, nk, sms, cs);
   if (e != cudaSuccess) return from_cuda(e);
-  return from_cuda(launch_topk(block_scores, nb, k, kv_idx, kmax, kv_cnt, static_cast<long long>(s->B) * s->Hq * nb,
+  return from_cuda(launch_topk(block_scores, nk, k, kv_idx, kmax, kv_cnt, static_cast<long long>(s->B) * s->Hq * nq,
                                sms, cs));
 }
 
@@ -333,10 +348,10 @@ ba_status ba_att_complement_lists(const ba_att_shape *s, const int32_t *kv_idx, 
   if (st != BA_OK) return st;
   if (!kv_idx || !kv_cnt || !c_idx || !c_cnt) return BA_ERR_INVALID_ARG;
   if (!aligned16(kv_idx) || !aligned16(kv_cnt) || !aligned16(c_idx) || !aligned16(c_cnt)) return BA_ERR_MISALIGNED;
-  const int nb = nblocks(s);
+  const int nb = nkblocks(s);
   if (nb > kComplMaxWords * 32) return BA_ERR_UNSUPPORTED;
   if (kmax < 1 || c_kmax < nb) return BA_ERR_INVALID_ARG;
-  const long long n_lists = static_cast<long long>(s->B) * s->Hq * nb;
+  const long long n_lists = static_cast<long long>(s->B) * s->Hq * nblocks(s);
   return from_cuda(launch_complement(kv_idx, kv_cnt, c_idx, c_cnt, n_lists, kmax, c_kmax, nb,
                                      num_sms_of_current_device(), reinterpret_cast<cudaStream_t>(stream)));
 }
@@ -350,9 +365,9 @@ ba_status ba_att_split_lists(const ba_att_shape *s, int32_t split_block, const i
   if (!aligned16(kv_idx) || !aligned16(kv_cnt) || !aligned16(lo_idx) || !aligned16(lo_cnt) || !aligned16(hi_idx) ||
       !aligned16(hi_cnt))
     return BA_ERR_MISALIGNED;
-  const int nb = nblocks(s);
+  const int nb = nkblocks(s);                     // split_block counts key blocks
   if (kmax < 1 || split_block < 0 || split_block > nb) return BA_ERR_INVALID_ARG;
-  const long long n_lists = static_cast<long long>(s->B) * s->Hq * nb;
+  const long long n_lists = static_cast<long long>(s->B) * s->Hq * nblocks(s);
   return from_cuda(launch_split(kv_idx, kv_cnt, lo_idx, lo_cnt, hi_idx, hi_cnt, n_lists, kmax, nb, split_block,
                                 num_sms_of_current_device(), reinterpret_cast<cudaStream_t>(stream)));
 }
@@ -396,7 +411,7 @@ ba_status sparse_fwd_impl(const ba_att_shape *s, const void *Q, const void *K, c
       if (e != cudaSuccess) return BA_ERR_CUDA;
       kernel<<<static_cast<unsigned>(tiles), tc::kThreads, smem, cs>>>(
           mq, mk, mv, kv_idx, kv_cnt, kmax, out, LSE, O_prev, L_prev, s->Hq, s->Hkv, s->N, s->N_alloc, nb, s->block,
-          sl2);
+          nkblocks(s), kblock(s), sl2);
       return from_cuda(cudaGetLastError());
     };
     float *of = static_cast<float *>(O);
@@ -416,11 +431,12 @@ ba_status sparse_fwd_impl(const ba_att_shape *s, const void *Q, const void *K, c
 #define BA_SIMT(T, TO, DD)                                                                                           \
   (merge ? launch_attn_simt<T, TO, DD, true>(static_cast<const T *>(Q), static_cast<const T *>(K),                   \
                                              static_cast<const T *>(V), kv_idx, kv_cnt, kmax, static_cast<TO *>(O), \
-                                             LSE, s->B, s->Hq, s->Hkv, s->N, s->N_alloc, s->block, scale, cs, O_prev, \
-                                             L_prev)                                                                 \
+                                             LSE, s->B, s->Hq, s->Hkv, s->N, s->N_alloc, s->block, kblock(s), scale, \
+                                             cs, O_prev, L_prev)                                                      \
          : launch_attn_simt<T, TO, DD, false>(static_cast<const T *>(Q), static_cast<const T *>(K),                  \
                                               static_cast<const T *>(V), kv_idx, kv_cnt, kmax, static_cast<TO *>(O), \
-                                              LSE, s->B, s->Hq, s->Hkv, s->N, s->N_alloc, s->block, scale, cs))
+                                              LSE, s->B, s->Hq, s->Hkv, s->N, s->N_alloc, s->block, kblock(s), scale, \
+                                              cs))
   if (s->dtype == BA_DTYPE_BF16) {
     if (out_f32)
       e = s->d == 128 ? BA_SIMT(__nv_bfloat16, float, 128) : BA_SIMT(__nv_bfloat16, float, 64);
@@ -519,7 +535,7 @@ struct PipeLayout {
 // Fewest KV heads per chunk that still give the attention kernel about 1024
 // (query head, query block) tiles, a few waves of the GPU's CTA slots.
 int auto_chunk(const ba_att_shape *s) {
-  const long long tiles_per_kv_head = static_cast<long long>(s->Hq / s->Hkv) * nblocks(s);
+  const long long tiles_per_kv_head = static_cast<long long>(s->Hq / s->Hkv) * nblocks(s);   // query blocks
   const long long c = (1024 + tiles_per_kv_head - 1) / tiles_per_kv_head;
   return static_cast<int>(c < 1 ? 1 : (c > s->Hkv ? s->Hkv : c));
 }
@@ -528,8 +544,8 @@ bool pipe_layout(const ba_att_shape *s, double keep, int32_t split_block, int32_
   if (check_shape(s) != BA_OK) return false;
   const int k = ba_att_keep_count(s, keep);
   if (k < 1) return false;
-  const int nb = nblocks(s);
-  if (split_block > nb) return false;
+  const int nb = nblocks(s), nk = nkblocks(s);
+  if (split_block > nk) return false;
   L->C = chunk > 0 ? (chunk < s->Hkv ? chunk : s->Hkv) : auto_chunk(s);
   L->G = s->Hq / s->Hkv;
   L->nb = nb;
@@ -552,12 +568,12 @@ bool pipe_layout(const ba_att_shape *s, double keep, int32_t split_block, int32_
   }
   L->qm = take(hq * nb * s->d * 4);
   L->qv = take(hq * nb * s->d * 4);
-  L->km = take(hk * nb * s->d * 4);
-  L->kv = take(hk * nb * s->d * 4);
+  L->km = take(hk * nk * s->d * 4);
+  L->kv = take(hk * nk * s->d * 4);
   L->idx = take(hq * nb * k * 4);
   L->cnt = take(hq * nb * 4);
-  L->sc = take(hq * nb * static_cast<size_t>(nb) * 4);
-  L->feat = take(6 * (hq + hk) * nb * s->d * 2);          // ba_att_selector's feature workspace
+  L->sc = take(hq * nb * static_cast<size_t>(nk) * 4);
+  L->feat = take(6 * (hq * nb + hk * nk) * s->d * 2);     // ba_att_selector's feature workspace
   if (split_block >= 0) {
     L->lo_idx = take(hq * nb * k * 4);
     L->lo_cnt = take(hq * nb * 4);

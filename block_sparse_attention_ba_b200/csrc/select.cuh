@@ -629,7 +629,7 @@ __device__ __forceinline__ void topk_row_mass(const float (&x)[KPL], const uint3
 struct TopkVariant {
   int group;            // query heads per selection (1: none shared)
   int heads;            // Hq
-  int nq;               // query blocks per head (= nk)
+  int nq;               // query blocks per head
   bool force_diagonal;
   bool by_mass;         // keep the shortest prefix reaching the share tau (instead of k blocks)
   float tau;

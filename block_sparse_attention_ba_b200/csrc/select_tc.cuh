@@ -10,8 +10,8 @@
 // ranked per query block, ties to the lower key block, top k kept ascending.
 //
 // One CTA = one (batch, head) x 128 query blocks (MMA M, the TMEM lanes) x NT
-// key blocks (MMA N, 64 or 128 TMEM columns): grid (ceil(nb/128) *
-// ceil(nb/NT), Hq, B), which covers any nb up to the host limit.
+// key blocks (MMA N, 64 or 128 TMEM columns): grid (ceil(nq/128) *
+// ceil(nk/NT), Hq, B), which covers any nq, nk up to the host limit.
 //  - The feature order inside the 3d-long dot product is free, so the
 //    features are taken in groups of 64 dimensions: one read of the fp32
 //    statistics for dimensions [64g, 64g+64) yields all three feature parts
@@ -73,8 +73,8 @@ template <int D, int NT>
 __global__ void __launch_bounds__(kThreads, 1)
     select_tc_kernel(const float *__restrict__ q_mean, const float *__restrict__ q_var,
                      const float *__restrict__ k_mean, const float *__restrict__ k_var,
-                     float *__restrict__ block_scores, int Hq, int Hkv, int N, int block, int nb, float sm_scale,
-                     int var_product) {
+                     float *__restrict__ block_scores, int Hq, int Hkv, int N, int kblock, int nq, int nk,
+                     float sm_scale, int var_product) {
   using TL = Tile<NT>;
   constexpr int GROUPS = D / 64;
   constexpr int TPT = TL::kTasksPerThread;
@@ -87,15 +87,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t sbase = smem_u32(smem);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int nk_tiles = (nb + NT - 1) / NT;
+  const int nk_tiles = (nk + NT - 1) / NT;
   const int h = blockIdx.y, b = blockIdx.z, g_kv = h / (Hq / Hkv);
   const long long bh = static_cast<long long>(b) * Hq + h;
   const int i0 = static_cast<int>(blockIdx.x / nk_tiles) * kRows, j0 = static_cast<int>(blockIdx.x % nk_tiles) * NT;
   const float s = sm_scale, hs2 = 0.5f * sm_scale * sm_scale;
-  const float *qm = q_mean + bh * nb * D;
-  const float *qv = q_var + bh * nb * D;
-  const float *km = k_mean + (static_cast<long long>(b) * Hkv + g_kv) * nb * D;
-  const float *kv = k_var + (static_cast<long long>(b) * Hkv + g_kv) * nb * D;
+  const float *qm = q_mean + bh * nq * D;
+  const float *qv = q_var + bh * nq * D;
+  const float *km = k_mean + (static_cast<long long>(b) * Hkv + g_kv) * nk * D;
+  const float *kv = k_var + (static_cast<long long>(b) * Hkv + g_kv) * nk * D;
 
   if (tid == 0) {
     mbar_init(smem_u32(&mma_bar), 1);
@@ -118,7 +118,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int r = is_a ? (e >> 3) : ((e - kRows * 8) >> 3);
       const int blk = (is_a ? i0 : j0) + r;
       raw[it].m0 = raw[it].m1 = raw[it].v0 = raw[it].v1 = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (blk < nb) {
+      if (blk < (is_a ? nq : nk)) {
         const long long off = static_cast<long long>(blk) * D + grp * 64 + c * 8;
         const float *pm = (is_a ? qm : km) + off;
         const float *pv = (is_a ? qv : kv) + off;
@@ -213,9 +213,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int quad = warp & 3, cq = warp >> 2;
     const int i = i0 + quad * 32 + lane;
     const uint32_t taddr = tmem + (static_cast<uint32_t>(quad * 32) << 16) + cq * COLS_PER_WARP;
-    const float ln_full = logf(static_cast<float>(block));
-    const float ln_last = logf(static_cast<float>(N - (nb - 1) * block));
-    const bool vec = (nb & 3) == 0;
+    const float ln_full = logf(static_cast<float>(kblock));
+    const float ln_last = logf(static_cast<float>(N - (nk - 1) * kblock));
+    const bool vec = (nk & 3) == 0;
 #pragma unroll
     for (int c0 = 0; c0 < COLS_PER_WARP; c0 += 16) {
       uint32_t r[16];
@@ -225,20 +225,20 @@ __global__ void __launch_bounds__(kThreads, 1)
             "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
           : "r"(taddr + c0));
       tmem_ld_wait();
-      if (i < nb) {
+      if (i < nq) {
         const int jb = j0 + cq * COLS_PER_WARP + c0;
-        float *dst = block_scores + (bh * nb + i) * nb + jb;
+        float *dst = block_scores + (bh * nq + i) * nk + jb;
         float val[16];
 #pragma unroll
-        for (int c = 0; c < 16; ++c) val[c] = __uint_as_float(r[c]) + (jb + c == nb - 1 ? ln_last : ln_full);
-        if (vec && jb + 16 <= nb) {
+        for (int c = 0; c < 16; ++c) val[c] = __uint_as_float(r[c]) + (jb + c == nk - 1 ? ln_last : ln_full);
+        if (vec && jb + 16 <= nk) {
 #pragma unroll
           for (int c = 0; c < 16; c += 4)
             *reinterpret_cast<float4 *>(dst + c) = make_float4(val[c], val[c + 1], val[c + 2], val[c + 3]);
         } else {
 #pragma unroll
           for (int c = 0; c < 16; ++c)
-            if (jb + c < nb) dst[c] = val[c];
+            if (jb + c < nk) dst[c] = val[c];
         }
       }
     }
@@ -280,8 +280,8 @@ enum Bar : int { FULL = 0, EMPTY = FULL + kStages, ACC_FULL = EMPTY + kStages, A
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     select_feat_kernel(const __grid_constant__ CUtensorMap tm_fq, const __grid_constant__ CUtensorMap tm_fk,
-                       float *__restrict__ block_scores, int Hq, int Hkv, int N, int block, int nb,
-                       long long n_tiles, int n_tq) {
+                       float *__restrict__ block_scores, int Hq, int Hkv, int N, int kblock, int nq, int nk,
+                       long long n_tiles, int n_tq, int n_tk) {
   constexpr int GROUPS = D / 64;
   extern __shared__ uint8_t dyn_smem[];
   __shared__ uint64_t bars[NUM_BARS];
@@ -293,8 +293,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int G = Hq / Hkv;
   // tile t -> (bh, query tile, key tile)
   auto decode = [&](long long t, long long &bh, int &tq, int &tk) {
-    tk = static_cast<int>(t % n_tq);
-    const long long r = t / n_tq;
+    tk = static_cast<int>(t % n_tk);
+    const long long r = t / n_tk;
     tq = static_cast<int>(r % n_tq);
     bh = r / n_tq;
   };
@@ -324,8 +324,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       int tq, tk;
       decode(t, bh, tq, tk);
       const int b = static_cast<int>(bh / Hq), h = static_cast<int>(bh % Hq);
-      const int qrow = static_cast<int>(bh * nb) + tq * kTile;
-      const int krow = (b * Hkv + h / G) * nb + tk * kTile;
+      const int qrow = static_cast<int>(bh * nq) + tq * kTile;
+      const int krow = (b * Hkv + h / G) * nk + tk * kTile;
       for (int g = 0; g < GROUPS && !stop; ++g) {
         for (int p = 0; p < 3; ++p, ++it) {
           const int st = static_cast<int>(it % kStages);
@@ -386,9 +386,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp < 4) {
     // ------------------------------------------------------------ epilogue
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    const float ln_full = logf(static_cast<float>(block));
-    const float ln_last = logf(static_cast<float>(N - (nb - 1) * block));
-    const bool vec = (nb & 3) == 0;
+    const float ln_full = logf(static_cast<float>(kblock));
+    const float ln_last = logf(static_cast<float>(N - (nk - 1) * kblock));
+    const bool vec = (nk & 3) == 0;
     int tl = 0;
     for (long long t = blockIdx.x; t < n_tiles; t += gridDim.x, ++tl) {
       const int acc = tl & 1, use = tl >> 1;
@@ -405,20 +405,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t r[32];
         tmem_ld32(tmem + lane_off + acc * kTile + c0, r);
         tmem_ld_wait();
-        if (i < nb) {
+        if (i < nq) {
           const int jb = j0 + c0;
-          float *dst = block_scores + (bh * nb + i) * nb + jb;
+          float *dst = block_scores + (bh * nq + i) * nk + jb;
           float val[32];
 #pragma unroll
-          for (int c = 0; c < 32; ++c) val[c] = __uint_as_float(r[c]) + (jb + c == nb - 1 ? ln_last : ln_full);
-          if (vec && jb + 32 <= nb) {
+          for (int c = 0; c < 32; ++c) val[c] = __uint_as_float(r[c]) + (jb + c == nk - 1 ? ln_last : ln_full);
+          if (vec && jb + 32 <= nk) {
 #pragma unroll
             for (int c = 0; c < 32; c += 4)
               *reinterpret_cast<float4 *>(dst + c) = make_float4(val[c], val[c + 1], val[c + 2], val[c + 3]);
           } else {
 #pragma unroll
             for (int c = 0; c < 32; ++c)
-              if (jb + c < nb) dst[c] = val[c];
+              if (jb + c < nk) dst[c] = val[c];
           }
         }
       }
@@ -440,40 +440,40 @@ __global__ void __launch_bounds__(kThreads, 1)
 // flags: the ba_att_select_ex bits (BA_SELECT_*).
 template <int D>
 cudaError_t launch_select_tc(const float *qm, const float *qv, const float *km, const float *kv, int32_t *idx,
-                             int32_t *cnt, float *scores, int B, int Hq, int Hkv, int N, int block, int k, int kmax,
-                             float sm_scale, uint32_t flags, float tau, int num_sms, cudaStream_t stream) {
+                             int32_t *cnt, float *scores, int B, int Hq, int Hkv, int N, int block, int kblock, int k,
+                             int kmax, float sm_scale, uint32_t flags, float tau, int num_sms, cudaStream_t stream) {
   const int var_product = (flags & BA_SELECT_NO_VAR_PRODUCT) ? 0 : 1;
-  const int nb = (N + block - 1) / block;
+  const int nq = (N + block - 1) / block, nk = (N + kblock - 1) / kblock;
   const long long bhs = static_cast<long long>(B) * Hq;
-  const int nq_tiles = (nb + seltc::kRows - 1) / seltc::kRows;
-  const bool wide = static_cast<long long>(nq_tiles) * ((nb + 127) / 128) * bhs >= num_sms / 2;
+  const int nq_tiles = (nq + seltc::kRows - 1) / seltc::kRows;
+  const bool wide = static_cast<long long>(nq_tiles) * ((nk + 127) / 128) * bhs >= num_sms / 2;
   cudaError_t e;
   if (wide) {
     using TL = seltc::Tile<128>;
     e = cudaFuncSetAttribute(seltc::select_tc_kernel<D, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(TL::kDynSmem));
     if (e != cudaSuccess) return e;
-    dim3 grid(((nb + 127) / 128) * nq_tiles, Hq, B);
+    dim3 grid(((nk + 127) / 128) * nq_tiles, Hq, B);
     seltc::select_tc_kernel<D, 128><<<grid, seltc::kThreads, TL::kDynSmem, stream>>>(qm, qv, km, kv, scores, Hq, Hkv,
-                                                                                      N, block, nb, sm_scale,
+                                                                                      N, kblock, nq, nk, sm_scale,
                                                                                       var_product);
   } else {
     using TL = seltc::Tile<64>;
     e = cudaFuncSetAttribute(seltc::select_tc_kernel<D, 64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(TL::kDynSmem));
     if (e != cudaSuccess) return e;
-    dim3 grid(((nb + 63) / 64) * nq_tiles, Hq, B);
+    dim3 grid(((nk + 63) / 64) * nq_tiles, Hq, B);
     seltc::select_tc_kernel<D, 64><<<grid, seltc::kThreads, TL::kDynSmem, stream>>>(qm, qv, km, kv, scores, Hq, Hkv,
-                                                                                     N, block, nb, sm_scale,
+                                                                                     N, kblock, nq, nk, sm_scale,
                                                                                      var_product);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const bool shared = (flags & BA_SELECT_SHARED_GQA) != 0, diag = (flags & BA_SELECT_FORCE_DIAGONAL) != 0;
   const bool mass = (flags & BA_SELECT_BY_MASS) != 0;
-  if (!shared && !diag && !mass) return launch_topk(scores, nb, k, idx, kmax, cnt, bhs * nb, num_sms, stream);
-  const TopkVariant var{shared ? Hq / Hkv : 1, Hq, nb, diag, mass, tau};
-  return launch_topk_variant(scores, nb, k, idx, kmax, cnt, static_cast<long long>(B) * (Hq / var.group) * nb, var,
+  if (!shared && !diag && !mass) return launch_topk(scores, nk, k, idx, kmax, cnt, bhs * nq, num_sms, stream);
+  const TopkVariant var{shared ? Hq / Hkv : 1, Hq, nq, diag, mass, tau};
+  return launch_topk_variant(scores, nk, k, idx, kmax, cnt, static_cast<long long>(B) * (Hq / var.group) * nq, var,
                              num_sms, stream);
 }
 

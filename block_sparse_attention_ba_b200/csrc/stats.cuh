@@ -27,7 +27,7 @@ __global__ void __launch_bounds__(kStatsThreads) stats_kernel(const T *__restric
                                                               float *__restrict__ q_mean, float *__restrict__ q_var,
                                                               float *__restrict__ k_mean, float *__restrict__ k_var,
                                                               int B, int Hq, int Hkv, int N, int N_alloc, int block,
-                                                              int nb) {
+                                                              int nb, int kblock, int nbk) {
   constexpr int VEC = Elem<T>::kVec;
   constexpr int COLS = D / VEC;                   // 16-byte vectors per row
   constexpr int RPP = kStatsThreads / COLS;       // rows covered per pass
@@ -38,14 +38,15 @@ __global__ void __launch_bounds__(kStatsThreads) stats_kernel(const T *__restric
   long long cta = blockIdx.x;
   const bool is_q = cta < n_q_ctas;
   if (!is_q) cta -= n_q_ctas;
-  const int blk = static_cast<int>(cta % nb);
-  const long long bh = cta / nb;                 // b*H + h
+  const int nbx = is_q ? nb : nbk, bsize = is_q ? block : kblock;    // query or key blocks
+  const int blk = static_cast<int>(cta % nbx);
+  const long long bh = cta / nbx;                // b*H + h
   const T *X = is_q ? Q : K;
   float *out_mean = is_q ? q_mean : k_mean;
   float *out_var = is_q ? q_var : k_var;
 
-  const int row0 = blk * block;
-  const int n_rows = min(block, N - row0);
+  const int row0 = blk * bsize;
+  const int n_rows = min(bsize, N - row0);
   const int tid = threadIdx.x;
   const int col = tid % COLS;
   const int rsub = tid / COLS;
@@ -112,7 +113,7 @@ __global__ void __launch_bounds__(kStatsThreads) stats_kernel(const T *__restric
     float s = 0.f;
 #pragma unroll 8
     for (int r = 0; r < RPP; ++r) s += red[r][tid];
-    const long long o = (bh * nb + blk) * static_cast<long long>(D) + tid;
+    const long long o = (bh * nbx + blk) * static_cast<long long>(D) + tid;
     out_mean[o] = mean_s[tid];
     out_var[o] = s * inv_n;
   }
@@ -273,7 +274,8 @@ template <typename T, int D>
 __global__ void __launch_bounds__(kStatsThreads, 2)
     stats_bulk_kernel(const T *__restrict__ Q, const T *__restrict__ K, float *__restrict__ q_mean,
                       float *__restrict__ q_var, float *__restrict__ k_mean, float *__restrict__ k_var, int B,
-                      int Hq, int Hkv, int N, int N_alloc, int block, int nb, FeatOut feat) {
+                      int Hq, int Hkv, int N, int N_alloc, int block, int nb, int kblock, int nbk,
+                      FeatOut feat) {
   constexpr int VEC = Elem<T>::kVec;
   constexpr int COLS = D / VEC;                     // threads per row (16-byte vectors)
   constexpr int RPP = kStatsThreads / COLS;         // rows per pass of the CTA
@@ -291,7 +293,7 @@ __global__ void __launch_bounds__(kStatsThreads, 2)
   __shared__ int meta_rows[kStatsStages];
 
   const long long n_q = static_cast<long long>(B) * Hq * nb;
-  const long long total = n_q + static_cast<long long>(B) * Hkv * nb;
+  const long long total = n_q + static_cast<long long>(B) * Hkv * nbk;
   const int tid = threadIdx.x, col = tid % COLS, rsub = tid / COLS, warp = tid >> 5;
   const uint32_t ring = smem_u32(stage_mem);
 
@@ -299,11 +301,12 @@ __global__ void __launch_bounds__(kStatsThreads, 2)
   auto locate = [&](long long w, const T *&src, int &n_rows, long long &orow, bool &is_q) {
     is_q = w < n_q;
     const long long c = is_q ? w : w - n_q;
-    const int blk = static_cast<int>(c % nb);
-    const long long bh = c / nb;
-    src = (is_q ? Q : K) + (bh * N_alloc + static_cast<long long>(blk) * block) * D;
-    n_rows = min(block, N - blk * block);
-    orow = (bh * nb + blk) * static_cast<long long>(D);
+    const int nbx = is_q ? nb : nbk, bsize = is_q ? block : kblock;   // query or key blocks
+    const int blk = static_cast<int>(c % nbx);
+    const long long bh = c / nbx;
+    src = (is_q ? Q : K) + (bh * N_alloc + static_cast<long long>(blk) * bsize) * D;
+    n_rows = min(bsize, N - blk * bsize);
+    orow = (bh * nbx + blk) * static_cast<long long>(D);
   };
   auto issue = [&](long long w, int s) {
     const T *src;
@@ -441,11 +444,12 @@ constexpr bool stats_bulk_fits(int block) {
 
 template <typename T, int D>
 cudaError_t launch_stats(const T *Q, const T *K, float *qm, float *qv, float *km, float *kv, int B, int Hq, int Hkv,
-                         int N, int N_alloc, int block, int num_sms, cudaStream_t stream,
+                         int N, int N_alloc, int block, int kblock, int num_sms, cudaStream_t stream,
                          FeatOut feat = FeatOut{nullptr, nullptr, 0.f, 0.f, 0, 0}) {
-  const int nb = (N + block - 1) / block;
-  const long long grid = static_cast<long long>(B) * (Hq + Hkv) * nb;
-  if (stats_bulk_fits<T, D>(block)) {
+  const int nb = (N + block - 1) / block, nbk = (N + kblock - 1) / kblock;
+  const long long grid = static_cast<long long>(B) * Hq * nb + static_cast<long long>(B) * Hkv * nbk;
+  const int bmax = block > kblock ? block : kblock;
+  if (stats_bulk_fits<T, D>(bmax)) {
     const size_t smem = static_cast<size_t>(kStatsStages) * kStatsStageBytes;
     cudaError_t e = cudaFuncSetAttribute(stats_bulk_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
@@ -456,22 +460,27 @@ cudaError_t launch_stats(const T *Q, const T *K, float *qm, float *qv, float *km
     const long long persistent = static_cast<long long>(num_sms) * (per_sm > 0 ? per_sm : 1);
     const unsigned g = static_cast<unsigned>(grid < persistent ? grid : persistent);
     stats_bulk_kernel<T, D><<<g, kStatsThreads, smem, stream>>>(Q, K, qm, qv, km, kv, B, Hq, Hkv, N, N_alloc, block,
-                                                                 nb, feat);
+                                                                 nb, kblock, nbk, feat);
     return cudaGetLastError();
   }
   if (feat.q != nullptr) return cudaErrorInvalidValue;    // features only from the one-copy kernel
-  const int need = stats_rpt_needed<T, D>(block);
+  const int need = stats_rpt_needed<T, D>(bmax);
   dim3 g(static_cast<unsigned>(grid));
   if (need <= 2) {
-    stats_kernel<T, D, 2><<<g, kStatsThreads, 0, stream>>>(Q, K, qm, qv, km, kv, B, Hq, Hkv, N, N_alloc, block, nb);
+    stats_kernel<T, D, 2><<<g, kStatsThreads, 0, stream>>>(Q, K, qm, qv, km, kv, B, Hq, Hkv, N, N_alloc, block, nb,
+                                                              kblock, nbk);
   } else if (need <= 4) {
-    stats_kernel<T, D, 4><<<g, kStatsThreads, 0, stream>>>(Q, K, qm, qv, km, kv, B, Hq, Hkv, N, N_alloc, block, nb);
+    stats_kernel<T, D, 4><<<g, kStatsThreads, 0, stream>>>(Q, K, qm, qv, km, kv, B, Hq, Hkv, N, N_alloc, block, nb,
+                                                              kblock, nbk);
   } else if (need <= 8) {
-    stats_kernel<T, D, 8><<<g, kStatsThreads, 0, stream>>>(Q, K, qm, qv, km, kv, B, Hq, Hkv, N, N_alloc, block, nb);
+    stats_kernel<T, D, 8><<<g, kStatsThreads, 0, stream>>>(Q, K, qm, qv, km, kv, B, Hq, Hkv, N, N_alloc, block, nb,
+                                                              kblock, nbk);
   } else if (need <= 16) {
-    stats_kernel<T, D, 16><<<g, kStatsThreads, 0, stream>>>(Q, K, qm, qv, km, kv, B, Hq, Hkv, N, N_alloc, block, nb);
+    stats_kernel<T, D, 16><<<g, kStatsThreads, 0, stream>>>(Q, K, qm, qv, km, kv, B, Hq, Hkv, N, N_alloc, block, nb,
+                                                              kblock, nbk);
   } else {
-    stats_kernel<T, D, 32><<<g, kStatsThreads, 0, stream>>>(Q, K, qm, qv, km, kv, B, Hq, Hkv, N, N_alloc, block, nb);
+    stats_kernel<T, D, 32><<<g, kStatsThreads, 0, stream>>>(Q, K, qm, qv, km, kv, B, Hq, Hkv, N, N_alloc, block, nb,
+                                                              kblock, nbk);
   }
   return cudaGetLastError();
 }

@@ -38,10 +38,21 @@ class Workload:
     needle: bool = False
     split: bool = False
     grid: tuple | None = None   # (t, h, w) for video_field
+    block_k: int = 0            # key block size when it differs from block (0: equal)
 
     @property
     def nb(self) -> int:
+        """Query blocks."""
         return -(-self.N // self.block)
+
+    @property
+    def kb(self) -> int:
+        return self.block_k if self.block_k > 0 else self.block
+
+    @property
+    def nk(self) -> int:
+        """Key blocks."""
+        return -(-self.N // self.kb)
 
     def with_(self, **kw) -> "Workload":
         return dataclasses.replace(self, **kw)
@@ -124,7 +135,7 @@ def _gen_shared_dir(w: Workload):
         Q[:, :, rows] += a * wv
         meta.update(needle_span=[start, start + span], needle_rows=rows.tolist())
     if w.split:
-        meta["split_block"] = int(meta_rng.integers(1, w.nb))
+        meta["split_block"] = int(meta_rng.integers(1, w.nk))
     if w.N_alloc > w.N:
         Q[:, :, w.N:] = 0
         K[:, :, w.N:] = 0
@@ -187,6 +198,6 @@ def make_inputs(w: Workload | str, **overrides):
            "video_field": _gen_video_field}[w.kind]
     Q, K, V, meta = gen(w)
     if w.split and "split_block" not in meta:      # generators without their own split point
-        meta["split_block"] = int(np.random.default_rng([w.seed, 2]).integers(1, w.nb))
+        meta["split_block"] = int(np.random.default_rng([w.seed, 2]).integers(1, w.nk))
     meta["workload"] = w
     return round_to(Q, w.dtype), round_to(K, w.dtype), round_to(V, w.dtype), meta

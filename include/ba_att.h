@@ -76,7 +76,16 @@ typedef struct {
   int32_t block;    /* block size b: a multiple of 16 in [16, 256]           */
   int32_t dtype;    /* ba_dtype of Q, K and V (and of O unless stated)      */
   float sm_scale;   /* softmax scale s; <= 0 selects d^-1/2                  */
+  int32_t block_k;  /* key block size b_k when it differs from b (asymmetric
+                       blocks): a multiple of 16 in [16, 256]; 0 = b          */
 } ba_att_shape;
+
+/* Block geometry: query blocks have b = block rows, key blocks b_k rows
+ * (b_k = block_k, or block when block_k is 0); nq = ceil(N / b) and
+ * nk = ceil(N / b_k). Query-side arrays (statistics of Q, lists, counts,
+ * score rows) have nq blocks, key-side ones (statistics of K, score
+ * columns, list entries) nk. The pages use one block size for both; unequal
+ * sizes are an extension. */
 
 /* Library version string, e.g. "0.1.0 sm_100a". Never NULL. */
 const char *ba_att_version(void);
@@ -84,8 +93,11 @@ const char *ba_att_version(void);
 /* Human-readable name of a status. Never NULL. */
 const char *ba_att_status_string(ba_status status);
 
-/* nq = nk = ceil(N / block); -1 if the shape is invalid. */
+/* nq = ceil(N / block), query blocks; -1 if the shape is invalid. */
 int32_t ba_att_num_blocks(const ba_att_shape *shape);
+
+/* nk = ceil(N / b_k), key blocks; -1 if the shape is invalid. */
+int32_t ba_att_num_key_blocks(const ba_att_shape *shape);
 
 /* Kept blocks per query block: max(1, ceil(keep * nk)) (the selector keeps
  * the top fraction of key blocks; "Core claim"). -1 if keep is outside (0,1]

@@ -71,7 +71,7 @@ MIS = ctypes.c_void_p(0x10008)
 
 
 @pytest.mark.parametrize("bad,status", [
-    (dict(d=96), 2), (dict(block=100), 2), (dict(block=512), 2), (dict(Hq=3, Hkv=2), 1), (dict(N=0), 1),
+    (dict(d=96), 2), (dict(block=100), 2), (dict(block=512), 2), (dict(block_k=100), 2), (dict(block_k=512), 2), (dict(Hq=3, Hkv=2), 1), (dict(N=0), 1),
     (dict(N_alloc=10), 1), (dict(dtype=7), 1), (dict(B=0), 1), (dict(sm_scale=float("nan")), 1),
 ])
 def test_bad_shapes_rejected(lib, bad, status):
@@ -205,3 +205,14 @@ def test_selector_workspace_and_arguments(lib):
     assert call(s, 0.5, *ptrs, kmax=3) == 1    # kmax below the keep count
     big = shape(N=4097 * 16, N_alloc=4097 * 16, block=16)
     assert call(big, 0.5, *ptrs, kmax=4097) == 2
+
+
+def test_key_block_geometry(lib):
+    s = shape(N=1000, block=128, block_k=64)
+    assert lib.ba_att_num_blocks(ctypes.byref(s)) == 8
+    assert lib.ba_att_num_key_blocks(ctypes.byref(s)) == 16
+    assert lib.ba_att_keep_count(ctypes.byref(s), ctypes.c_double(0.5)) == 8       # a fraction of the key blocks
+    assert lib.ba_att_num_key_blocks(ctypes.byref(shape())) == lib.ba_att_num_blocks(ctypes.byref(shape()))
+    # the forced diagonal pairs query block i with key block i: equal sizes only
+    assert lib.ba_att_select_ex(ctypes.byref(s), ctypes.c_double(0.5), ctypes.c_uint32(api.SELECT_FORCE_DIAGONAL),
+                                P, P, P, P, P, P, 8, P, None) == 2

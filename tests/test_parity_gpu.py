@@ -31,7 +31,7 @@ def _cuda():
 
 def run_gpu(Q, K, V, w, keep, kmax=None, with_scores=True):
     Qd, Kd, Vd = to_dev(Q, w.dtype), to_dev(K, w.dtype), to_dev(V, w.dtype)
-    shape = api.Shape.of(Qd, Kd, w.N, w.block)
+    shape = api.Shape.of(Qd, Kd, w.N, w.block, block_k=w.block_k)
     st = api.stats(Qd, Kd, shape)
     idx, cnt, sc = api.select(st, shape, keep, kmax=kmax, with_scores=True)
     Od, Ld = api.sparse_fwd(Qd, Kd, Vd, idx, cnt, shape)
@@ -43,7 +43,7 @@ def run_gpu(Q, K, V, w, keep, kmax=None, with_scores=True):
 
 def check_stats(r, Q, K, w):
     qm, qv, _ = O.block_stats(Q, w.N, w.block)
-    km, kv, kc = O.block_stats(K, w.N, w.block)
+    km, kv, kc = O.block_stats(K, w.N, w.kb)            # key blocks (asymmetric shapes: w.kb rows)
     for got, ref, name in zip(r["stats"], (qm, qv, km, kv), ("q_mean", "q_var", "k_mean", "k_var")):
         err = np.abs(got - ref)
         assert np.all(err <= 1e-5 * np.abs(ref) + 2e-6 * (1 + np.abs(ref).max())), (name, err.max())
@@ -54,13 +54,13 @@ def check_selection(r, stats_ref, w, keep):
     qm, qv, km, kv, kc = stats_ref
     s = w.d ** -0.5
     S = O.corrected_scores(qm, qv, km, kv, kc, s)
-    k = O.keep_count(keep, w.nb)
+    k = O.keep_count(keep, w.nk)
     err = np.abs(r["scores"] - S)
     assert np.all(err <= 1e-5 * np.abs(S) + 5e-5), err.max()
     idx_ref, cnt_ref = O.select_topk(S, k)
     assert (r["cnt"] == k).all()
-    got = mask_of(r["idx"], r["cnt"], w.nb)
-    ref = mask_of(idx_ref, cnt_ref, w.nb)
+    got = mask_of(r["idx"], r["cnt"], w.nk)
+    ref = mask_of(idx_ref, cnt_ref, w.nk)
     near = O.near_tie_mask(S, k, NEAR_TIE_REL)
     mism = (got != ref) & ~near
     assert not mism.any(), f"{int(mism.sum())} mask mismatches outside the near-tie band"
@@ -75,7 +75,8 @@ def check_selection(r, stats_ref, w, keep):
 
 def check_attention(r, Q, K, V, w, blocks):
     s = w.d ** -0.5
-    Oref, Lref = O.masked_attention(Q, K, V, r["idx"], r["cnt"], w.N, w.block, s, query_blocks=blocks)
+    Oref, Lref = O.masked_attention(Q, K, V, r["idx"], r["cnt"], w.N, w.block, s, query_blocks=blocks,
+                                    b_k=w.kb)
     tol = TOL[w.dtype]
     rows = []
     for (bb, h, i) in blocks:
@@ -124,6 +125,13 @@ SMALL = [
     ("dlm_16k", dict(N=4096, Hq=4, Hkv=2, block=256), 0.5),          # tcgen05 path, 256-row blocks
     ("dlm_16k", dict(N=3 * 256 + 200, N_alloc=1024, Hq=2, Hkv=1, block=256), 0.5),   # 256-row blocks, ragged
     ("dlm_16k", dict(N=2048 - 40, N_alloc=2048, Hq=4, Hkv=2, d=64, block=256), 0.5),  # 256-row blocks, d = 64
+    # asymmetric blocks: query blocks of `block` rows, key blocks of `block_k` rows
+    ("dlm_16k", dict(N=2048 - 30, N_alloc=2048, Hq=4, Hkv=2, block_k=64), 0.5),      # tcgen05, 128 x 64
+    ("dlm_16k", dict(N=2048, Hq=4, Hkv=2, block=256, block_k=128), 0.5),             # tcgen05, 256 x 128
+    ("dlm_16k", dict(N=3000, N_alloc=3072, Hq=2, Hkv=1, block=128, block_k=256), 0.3),  # tcgen05, 128 x 256
+    ("dlm_16k", dict(N=1500, N_alloc=1536, Hq=2, Hkv=1, d=64, block=128, block_k=64), 0.5),  # tcgen05, d 64
+    ("dlm_16k", dict(N=1024 - 9, N_alloc=1024, Hq=2, Hkv=1, block=64, block_k=128), 0.5),   # CUDA cores, 64 x 128
+    ("tiny_fp32", dict(block=32, block_k=64), 0.5),                                  # fp32, 32 x 64
 ]
 
 
@@ -146,13 +154,14 @@ def test_small_full_parity(name, over, keep):
 @pytest.mark.parametrize("name,over", [("tiny_fp32", {}), ("dlm_16k", dict(N=1536, Hq=4, Hkv=2)),
                                        ("dlm_16k", dict(N=1536 - 9, N_alloc=1536, Hq=4, Hkv=2, d=64)),
                                        ("dlm_16k", dict(N=1536, Hq=4, Hkv=2, block=256)),
+                                       ("dlm_16k", dict(N=1536, Hq=4, Hkv=2, block=256, block_k=64)),
                                        ("video_32k", dict(N=600, N_alloc=640, Hq=2, Hkv=2, grid=(3, 10, 20)))])
 def test_keep_all_equals_dense(name, over):
     # check (1): keep = 1.0 selects every block and equals dense attention
     Q, K, V, meta = make_inputs(name, **over)
     w = meta["workload"]
     r = run_gpu(Q, K, V, w, 1.0)
-    assert (r["cnt"] == w.nb).all()
+    assert (r["cnt"] == w.nk).all()
     Od, Ld = O.dense_attention(Q, K, V, w.N, w.d ** -0.5)
     tol = TOL[w.dtype]
     assert max_abs(r["O"][:, :, : w.N], Od) <= tol["max_abs"]

@@ -23,6 +23,8 @@ CASES = [
     ("dlm_16k", dict(N=1024, Hq=2, Hkv=1, d=64, block=64), 0.5),       # bf16 block 64
     ("dlm_16k", dict(N=1024, B=2, Hq=4, Hkv=2), 0.5),                  # two batches
     ("dlm_16k", dict(N=2048 - 40, N_alloc=2048, Hq=4, Hkv=2, d=64, block=256), 0.5),   # 256-row blocks, d 64
+    ("dlm_16k", dict(N=2048 - 30, N_alloc=2048, Hq=4, Hkv=2, block_k=64), 0.5),      # asymmetric: 16 x 32 blocks
+    ("dlm_16k", dict(N=3000, N_alloc=3072, Hq=2, Hkv=1, d=64, block_k=256), 0.3),    # asymmetric: 24 x 12 blocks
     ("tiny_fp32", dict(N=2048, d=128, block=128), 0.5),                # 64 KB blocks: plain stats + select
 ]
 
@@ -32,7 +34,7 @@ def _run_both(name, over, keep):
     w = meta["workload"]
     dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     Qd, Kd = (torch.from_numpy(np.ascontiguousarray(x)).to(dt).cuda() for x in (Q, K))
-    shape = api.Shape.of(Qd, Kd, w.N, w.block)
+    shape = api.Shape.of(Qd, Kd, w.N, w.block, block_k=w.block_k)
     st_ref = api.stats(Qd, Kd, shape)
     idx_ref, cnt_ref, sc_ref = api.select(st_ref, shape, keep, with_scores=True)
     # poison the outputs so that every written element is checked
