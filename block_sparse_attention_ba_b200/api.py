@@ -46,6 +46,7 @@ _SIGS = {
     "ba_att_select": (ctypes.c_int, [ctypes.POINTER(CShape), ctypes.c_double, _P, _P, _P, _P, _P, _P, _I32, _P, _P]),
     "ba_att_select_ex": (ctypes.c_int, [ctypes.POINTER(CShape), ctypes.c_double, ctypes.c_uint32, _P, _P, _P, _P, _P,
                                          _P, _I32, _P, _P]),
+    "ba_att_topk": (ctypes.c_int, [_P, ctypes.c_int64, _I32, _I32, _P, _P, _I32, _P]),
     "ba_att_selector_workspace": (ctypes.c_int64, [ctypes.POINTER(CShape)]),
     "ba_att_selector": (ctypes.c_int, [ctypes.POINTER(CShape), ctypes.c_double, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                         _P, _I32, _P]),
@@ -210,6 +211,24 @@ def select(stats_out, shape: Shape, keep: float, kmax: int | None = None, with_s
         _dev(qv, "q_var"), _dev(km, "k_mean"), _dev(kv, "k_var"), _dev(idx, "kv_idx"), _dev(cnt, "kv_cnt"),
         idx.shape[-1], _dev(sc, "block_scores"), _stream(qm)))
     return (idx, cnt, sc) if with_scores else (idx, cnt)
+
+
+def topk(scores: torch.Tensor, k: int, kmax: int | None = None, out=None):
+    """Norm sorting of a given fp32 score map [..., nk] (ba_att_topk) -> (idx [..., kmax], cnt [...])."""
+    lib = load_library()
+    if scores.dtype != torch.float32 or not scores.is_contiguous():
+        raise ValueError("scores must be a contiguous float32 tensor")
+    nk = scores.shape[-1]
+    rows = scores.numel() // nk
+    kmax = k if kmax is None else kmax
+    if out is None:
+        idx = torch.empty(scores.shape[:-1] + (kmax,), device=scores.device, dtype=torch.int32)
+        cnt = torch.empty(scores.shape[:-1], device=scores.device, dtype=torch.int32)
+    else:
+        idx, cnt = out
+    _check("ba_att_topk", lib.ba_att_topk(_dev(scores, "block_scores"), rows, nk, k, _dev(idx, "kv_idx"),
+                                          _dev(cnt, "kv_cnt"), idx.shape[-1], _stream(scores)))
+    return idx, cnt
 
 
 def selector_workspace_bytes(shape: Shape) -> int:

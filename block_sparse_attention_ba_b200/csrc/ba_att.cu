@@ -342,6 +342,16 @@ ba_status ba_att_selector(const ba_att_shape *s, double keep, const void *Q, con
                                sms, cs));
 }
 
+ba_status ba_att_topk(const float *block_scores, int64_t rows, int32_t nk, int32_t k, int32_t *kv_idx,
+                      int32_t *kv_cnt, int32_t kmax, ba_stream_t stream) {
+  if (!block_scores || !kv_idx || !kv_cnt) return BA_ERR_INVALID_ARG;
+  if (!aligned16(block_scores) || !aligned16(kv_idx) || !aligned16(kv_cnt)) return BA_ERR_MISALIGNED;
+  if (rows < 1 || nk < 1 || k < 1 || kmax < k) return BA_ERR_INVALID_ARG;
+  if (nk > 4096) return BA_ERR_UNSUPPORTED;
+  return from_cuda(launch_topk(block_scores, nk, k, kv_idx, kmax, kv_cnt, rows, num_sms_of_current_device(),
+                               reinterpret_cast<cudaStream_t>(stream)));
+}
+
 ba_status ba_att_complement_lists(const ba_att_shape *s, const int32_t *kv_idx, const int32_t *kv_cnt, int32_t kmax,
                                   int32_t *c_idx, int32_t *c_cnt, int32_t c_kmax, ba_stream_t stream) {
   ba_status st = check_shape(s);

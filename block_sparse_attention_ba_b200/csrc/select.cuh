@@ -11,9 +11,12 @@
 // of the fp32 scores (topk_row_keys: a sampled key window, 8-bit radix
 // passes, then direct ranking of at most 32 candidates); equal scores go to
 // the lower block index, and the kept indices are emitted ascending. Rows of
-// up to 256 keys are held in registers (topk_rows_kernel), up to 1024 in
-// shared memory (topk_rows_smem_kernel), longer ones are re-read from global
-// memory (topk_row_warp). topk_variant_kernel serves the selection variants
+// up to 1024 keys are held in registers lane-major (topk_rows_lm_kernel: each
+// lane a contiguous run of columns, 16-byte loads, kept columns emitted from
+// per-lane bit masks); the chunk-major register and shared-memory kernels
+// (topk_rows_kernel, topk_rows_smem_kernel) remain behind
+// BA_TOPK_LANE_MAJOR=0; longer rows are re-read from global memory
+// (topk_row_warp). topk_variant_kernel serves the selection variants
 // of ba_att_select_ex (shared per GQA group, forced diagonal, cumulative
 // softmax share: topk_row_mass).
 #pragma once
@@ -164,11 +167,32 @@ __device__ void topk_row_warp(const float *__restrict__ srow, int nk, int k, int
 // Scores of a row are concentrated in a narrow band with a long upper tail,
 // so a window placed by the sample spreads the band over many bins where the
 // row's full range would put most keys into one bin.
-template <int KPL, typename KeyAt>
+// Lane-major emission: lane l holds columns l*KPL .. l*KPL+KPL-1 and bit c of
+// `mask` marks column l*KPL + c as kept. Writes every kept column in
+// ascending order (lanes in order, each its set bits in order) and returns the
+// total, identical in every lane.
+template <int KPL>
+__device__ __forceinline__ int emit_lane_runs(uint32_t mask, int lane, int32_t *__restrict__ out_idx) {
+  const int n = __popc(mask);
+  int incl = n;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int y = __shfl_up_sync(0xFFFFFFFFu, incl, off);
+    if (lane >= off) incl += y;
+  }
+  int w = incl - n;
+  for (uint32_t m = mask; m != 0u; m &= m - 1u) out_idx[w++] = lane * KPL + (__ffs(m) - 1);
+  return __shfl_sync(0xFFFFFFFFu, incl, 31);
+}
+
+template <int KPL, bool LM = false, typename KeyAt>
 __device__ __forceinline__ void topk_row_keys(const KeyAt &key, int nk, int k, int32_t *__restrict__ out_idx,
                                               int kmax, int32_t *__restrict__ out_cnt, uint32_t hist_s, int lane) {
   const unsigned full = 0xFFFFFFFFu;
   const unsigned lt_mask = (1u << lane) - 1u;
+  // column of key c of this lane: chunk-major (c*32 + lane) or lane-major
+  // (lane*KPL + c, each lane a contiguous run of columns)
+  auto colof = [&](int c) { return LM ? lane * KPL + c : c * 32 + lane; };
   if (k >= nk) {
     for (int j = lane; j < kmax; j += 32) out_idx[j] = j < nk ? j : -1;
     if (lane == 0) *out_cnt = nk;
@@ -225,11 +249,18 @@ __device__ __forceinline__ void topk_row_keys(const KeyAt &key, int nk, int k, i
   int nbits = 32, need = k, in_bin = nk;
   bool bracketed = false;
   if (KPL >= 2 && nk >= 64) {
-    const int cs = lane % KPL;
     uint32_t smp = key(0);
+    if constexpr (LM) {
+      // the first key of every lane holding keys (evenly spaced columns);
+      // lanes past the row's end take a copy of one of them
+      const int nvl = (nk + KPL - 1) / KPL;
+      smp = __shfl_sync(full, smp, lane < nvl ? lane : lane % nvl);
+    } else {
+      const int cs = lane % KPL;
 #pragma unroll
-    for (int c = 1; c < KPL; ++c)
-      if (c == cs && c * 32 + lane < nk) smp = key(c);
+      for (int c = 1; c < KPL; ++c)
+        if (c == cs && c * 32 + lane < nk) smp = key(c);
+    }
 #pragma unroll
     for (int size = 2; size <= 32; size <<= 1) {       // bitonic sort, descending across lanes
 #pragma unroll
@@ -248,7 +279,7 @@ __device__ __forceinline__ void topk_row_keys(const KeyAt &key, int nk, int k, i
     int n_above = 0;
 #pragma unroll
     for (int c = 0; c < KPL; ++c) {
-      if (c * 32 + lane < nk && key(c) >= lo) {
+      if (colof(c) < nk && key(c) >= lo) {
         const uint32_t bin = (key(c) - lo) >> shift;
         if (bin > 255u)
           ++n_above;
@@ -275,7 +306,7 @@ __device__ __forceinline__ void topk_row_keys(const KeyAt &key, int nk, int k, i
     uint32_t umin = 0xFFFFFFFFu, umax = 0u;
 #pragma unroll
     for (int c = 0; c < KPL; ++c) {
-      if (c * 32 + lane < nk) {
+      if (colof(c) < nk) {
         umin = min(umin, key(c));
         umax = max(umax, key(c));
       }
@@ -299,7 +330,7 @@ __device__ __forceinline__ void topk_row_keys(const KeyAt &key, int nk, int k, i
 #pragma unroll
     for (int c = 0; c < KPL; ++c) {
       const uint32_t v = key(c) - base;
-      if (in_range(key(c), c * 32 + lane) && (v & mask) == prefix)
+      if (in_range(key(c), colof(c)) && (v & mask) == prefix)
         red_shared_add(hist_s + 4u * ((v >> shift) & 255u), 1u);
     }
     __syncwarp();
@@ -318,7 +349,7 @@ __device__ __forceinline__ void topk_row_keys(const KeyAt &key, int nk, int k, i
     int cnt = 0;
 #pragma unroll
     for (int c = 0; c < KPL; ++c) {
-      const int j = c * 32 + lane;
+      const int j = colof(c);
       const bool cand = in_range(key(c), j) && ((key(c) - base) & mask) == prefix;
       const unsigned cb = __ballot_sync(full, cand);
       if (cand) {
@@ -341,14 +372,47 @@ __device__ __forceinline__ void topk_row_keys(const KeyAt &key, int nk, int k, i
     const int cut = __ffs(__ballot_sync(full, lane < cnt && rank == need - 1)) - 1;
     const uint32_t thr_u = __shfl_sync(full, cv, cut);
     const int thr_j = __shfl_sync(full, cj, cut);
+    if constexpr (LM) {
+      uint32_t km = 0u;
+#pragma unroll
+      for (int c = 0; c < KPL; ++c) {
+        const int j = colof(c);
+        if (j < nk && (key(c) > thr_u || (key(c) == thr_u && j <= thr_j))) km |= 1u << c;
+      }
+      pos = emit_lane_runs<KPL>(km, lane, out_idx);
+    } else {
+#pragma unroll
+      for (int c = 0; c < KPL; ++c) {
+        const int j = c * 32 + lane;
+        const bool kept = j < nk && (key(c) > thr_u || (key(c) == thr_u && j <= thr_j));
+        const unsigned kb = __ballot_sync(full, kept);
+        if (kept) out_idx[pos + __popc(kb & lt_mask)] = j;
+        pos += __popc(kb);
+      }
+    }
+  } else if constexpr (LM) {
+    // the range is one key value (the k-th largest): every larger key and the
+    // first `need` equal keys in column order (lanes hold ascending runs)
+    const uint32_t thr = base + prefix;
+    uint32_t gm = 0u, em = 0u;
 #pragma unroll
     for (int c = 0; c < KPL; ++c) {
-      const int j = c * 32 + lane;
-      const bool kept = j < nk && (key(c) > thr_u || (key(c) == thr_u && j <= thr_j));
-      const unsigned kb = __ballot_sync(full, kept);
-      if (kept) out_idx[pos + __popc(kb & lt_mask)] = j;
-      pos += __popc(kb);
+      if (colof(c) < nk) {
+        if (key(c) > thr) gm |= 1u << c;
+        if (key(c) == thr) em |= 1u << c;
+      }
     }
+    const int ne = __popc(em);
+    int eincl = ne;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(full, eincl, off);
+      if (lane >= off) eincl += y;
+    }
+    int room = need - (eincl - ne);                    // equal keys this lane may still take
+    uint32_t take = 0u;
+    for (uint32_t m = em; m != 0u && room > 0; m &= m - 1u, --room) take |= m & (0u - m);
+    pos = emit_lane_runs<KPL>(gm | take, lane, out_idx);
   } else {
     const uint32_t thr = base + prefix;                 // the range is one key value: the k-th largest
     int eq_seen = 0;
@@ -414,6 +478,48 @@ __global__ void __launch_bounds__(kTopkWarps * 32) topk_rows_kernel(const float 
   } else {
     if (row >= rows) return;
     topk_row_warp(scores + row * nk, nk, k, kv_idx + row * kmax, kmax, kv_cnt + row, &hist[warp][0], lane);
+  }
+}
+
+// Lane-major rows of up to 32*KPL keys in registers: lane l holds the
+// contiguous columns l*KPL .. l*KPL+KPL-1, fetched with 16-byte loads when the
+// rows are 16-byte aligned; persistent warps prefetch the next row while the
+// current one is selected. The selection is topk_row_keys in lane-major mode
+// (same exact result as the chunk-major kernels).
+template <int KPL>
+__global__ void __launch_bounds__(kTopkWarps * 32) topk_rows_lm_kernel(const float *__restrict__ scores, int nk,
+                                                                       int k, int32_t *__restrict__ kv_idx, int kmax,
+                                                                       int32_t *__restrict__ kv_cnt, long long rows) {
+  __shared__ __align__(16) unsigned hist[kTopkWarps][256];   // also holds (key, column) pairs
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  long long row = blockIdx.x * static_cast<long long>(kTopkWarps) + warp;
+  const long long stride = static_cast<long long>(gridDim.x) * kTopkWarps;
+  const bool vec = (nk & 3) == 0 && (lane + 1) * KPL <= nk;
+  float nxt[KPL];
+  auto fetch = [&](long long r) {
+    const float *src = scores + r * nk + lane * KPL;
+    if (r < rows && vec) {
+#pragma unroll
+      for (int q = 0; q < KPL / 4; ++q) {
+        const float4 v = __ldg(reinterpret_cast<const float4 *>(src) + q);
+        nxt[4 * q] = v.x;
+        nxt[4 * q + 1] = v.y;
+        nxt[4 * q + 2] = v.z;
+        nxt[4 * q + 3] = v.w;
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < KPL; ++c) nxt[c] = (r < rows && lane * KPL + c < nk) ? __ldg(src + c) : 0.f;
+    }
+  };
+  fetch(row);
+  for (; row < rows; row += stride) {
+    uint32_t u[KPL];
+#pragma unroll
+    for (int c = 0; c < KPL; ++c) u[c] = order_key(nxt[c]);
+    fetch(row + stride);
+    topk_row_keys<KPL, true>([&](int c) { return u[c]; }, nk, k, kv_idx + row * kmax, kmax, kv_cnt + row,
+                             smem_u32(&hist[warp][0]), lane);
   }
 }
 
@@ -509,9 +615,28 @@ inline cudaError_t launch_topk_smem(const float *scores, int nk, int k, int32_t 
   return cudaGetLastError();
 }
 
+#ifndef BA_TOPK_LANE_MAJOR
+#define BA_TOPK_LANE_MAJOR 1
+#endif
+
+template <int KPL>
+inline cudaError_t launch_topk_lm(const float *scores, int nk, int k, int32_t *idx, int kmax, int32_t *cnt,
+                                  long long rows, int num_sms, cudaStream_t stream) {
+  const int threads = kTopkWarps * 32;
+  int per_sm = 0;
+  const cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, topk_rows_lm_kernel<KPL>, threads, 0);
+  if (e != cudaSuccess) return e;
+  long long grid = (rows + kTopkWarps - 1) / kTopkWarps;
+  const long long slots = static_cast<long long>(num_sms) * (per_sm > 0 ? per_sm : 1);
+  grid = grid < slots ? grid : slots;
+  topk_rows_lm_kernel<KPL><<<static_cast<unsigned>(grid), threads, 0, stream>>>(scores, nk, k, idx, kmax, cnt, rows);
+  return cudaGetLastError();
+}
+
 template <int KPL>
 inline cudaError_t launch_topk_kpl(const float *scores, int nk, int k, int32_t *idx, int kmax, int32_t *cnt,
                                    long long rows, int num_sms, cudaStream_t stream) {
+  if (BA_TOPK_LANE_MAJOR && KPL > 0) return launch_topk_lm<(KPL > 0 ? KPL : 8)>(scores, nk, k, idx, kmax, cnt, rows, num_sms, stream);
   if (KPL >= BA_TOPK_SMEM_MIN_KPL) return launch_topk_smem<(KPL > 0 ? KPL : 8)>(scores, nk, k, idx, kmax, cnt, rows, num_sms, stream);
   const int threads = kTopkWarps * 32;
   long long grid = (rows + kTopkWarps - 1) / kTopkWarps;

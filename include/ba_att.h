@@ -157,6 +157,24 @@ ba_status ba_att_select(const ba_att_shape *shape, double keep,
                         float *block_scores, ba_stream_t stream);
 
 /*
+ * ba_att_topk — the norm sorting step alone, on a score map the caller gives
+ * (BA-Att "The pith", abstract, Figure 2: the downsampled blocks are ranked
+ * and the top fraction is kept). Per row of `block_scores`, the k columns
+ * with the largest scores are kept (ranking by score descending, equal
+ * scores to the lower column, NaN last) and written ascending. This is the
+ * step ba_att_select runs after its score GEMM.
+ *
+ * block_scores  device fp32 [rows, nk], 16-byte aligned.
+ * kv_idx        device int32 [rows, kmax]: kept columns, ascending; entries
+ *               at positions >= k are -1.
+ * kv_cnt        device int32 [rows]: k (nk when k >= nk).
+ * 1 <= k, k <= kmax, 1 <= nk <= 4096, rows >= 1 (else BA_ERR_INVALID_ARG or,
+ * for nk, BA_ERR_UNSUPPORTED).
+ */
+ba_status ba_att_topk(const float *block_scores, int64_t rows, int32_t nk, int32_t k,
+                      int32_t *kv_idx, int32_t *kv_cnt, int32_t kmax, ba_stream_t stream);
+
+/*
  * ba_att_selector_workspace — device workspace bytes that ba_att_selector
  * needs for this shape: the augmented score features of every block,
  * 6 planes (3 parts x {hi, lo}) x (B*Hq*nq + B*Hkv*nk) rows x d bf16, rounded

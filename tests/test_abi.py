@@ -216,3 +216,12 @@ def test_key_block_geometry(lib):
     # the forced diagonal pairs query block i with key block i: equal sizes only
     assert lib.ba_att_select_ex(ctypes.byref(s), ctypes.c_double(0.5), ctypes.c_uint32(api.SELECT_FORCE_DIAGONAL),
                                 P, P, P, P, P, P, 8, P, None) == 2
+
+
+def test_topk_arguments(lib):
+    assert lib.ba_att_topk(None, 4, 16, 8, P, P, 8, None) == 1
+    assert lib.ba_att_topk(MIS, 4, 16, 8, P, P, 8, None) == 3
+    assert lib.ba_att_topk(P, 0, 16, 8, P, P, 8, None) == 1
+    assert lib.ba_att_topk(P, 4, 16, 0, P, P, 8, None) == 1
+    assert lib.ba_att_topk(P, 4, 16, 8, P, P, 7, None) == 1
+    assert lib.ba_att_topk(P, 4, 4097, 8, P, P, 8, None) == 2
