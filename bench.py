@@ -204,6 +204,17 @@ def cpu_cores():
 
 # --------------------------------------------------------------------------- our arm
 
+def step_config(w, keep: float, k: int, split_block: int, world: int) -> dict:
+    """The JSON `config` of a step on workload w; both arms report the same one."""
+    in_mib = (w.B * w.Hq + 2 * w.B * w.Hkv) * w.N_alloc * w.d * 2 / 2**20
+    return {"workload": f"{w.name}: B={w.B} Hq={w.Hq} Hkv={w.Hkv} N={w.N} d={w.d} block={w.block} "
+                        f"bf16 keep={keep}; step = selector(stats+scores+top-k)+split(block {split_block})"
+                        f"+sparse_fwd+sparse_fwd_merge",
+            "keep": keep, "kept_blocks_per_query_block": k, "split_block": split_block,
+            "parallelism": f"{world} independent replica(s)",
+            "l2": f"inputs {in_mib:.0f} MiB > L2 126 MiB; no flush"}
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -329,13 +340,7 @@ def run_ours(args):
             "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": f"{w.name}: B={w.B} Hq={w.Hq} Hkv={w.Hkv} N={w.N} d={w.d} block={w.block} "
-                                   f"bf16 keep={keep}; step = selector(stats+scores+top-k)+split(block {split_block})"
-                                   f"+sparse_fwd+sparse_fwd_merge",
-                       "keep": keep, "kept_blocks_per_query_block": k, "split_block": split_block,
-                       "parallelism": f"{world} independent replica(s)",
-                       "l2": f"inputs {(Qd.numel() + Kd.numel() + Vd.numel()) * 2 / 2**20:.0f} MiB > L2 "
-                             f"126 MiB; no flush"},
+            "config": step_config(w, keep, k, split_block, world),
             "roofline": roofline, "selector": selector,
             "stages_ms": {n: round(v, 4) for n, v in stage_ms.items()},
             "stages_ms_median": {n: round(v, 4) for n, v in stage_ms_median.items()},
@@ -557,8 +562,7 @@ def run_reference(args):
     out = {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": 1,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 1), "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-           "config": {"workload": f"{w.name}: B={w.B} Hq={w.Hq} Hkv={w.Hkv} N={w.N} d={w.d} block={w.block} "
-                                  f"keep={args.keep}", "keep": args.keep},
+           "config": step_config(w, args.keep, k, meta["split_block"], dist_env()[0]),
            "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
                             "sample": desc + "; one sample per step", "wall_seconds": round(wall, 1)},
            "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
