@@ -383,6 +383,8 @@ def test_fused_merge_equals_separate_merge(name, over):
     ("extreme_128k", dict(N=4096, Hq=8, Hkv=4), False, 3),                      # chunks of 3 + 1 KV heads
     ("dlm_16k", dict(N=2048, Hq=4, Hkv=2, B=2), True, 2),                       # one chunk per batch entry
     ("tiny_fp32", dict(N=1000, N_alloc=1024), False, 1),                        # fp32, CUDA-core attention
+    ("dlm_16k", dict(N=3000, N_alloc=3072, Hq=4, Hkv=2, block_k=64), True, 1),   # asymmetric 128 x 64, split
+    ("dlm_16k", dict(N=2048 - 20, N_alloc=2048, Hq=4, Hkv=2, block=256), False, 0),  # 256-row blocks
 ])
 def test_forward_host_pipeline(name, over, split, chunk):
     # host buffers in and out, chunked and pipelined: bit-identical to the
@@ -392,10 +394,11 @@ def test_forward_host_pipeline(name, over, split, chunk):
     keep = 0.5
     tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
     Qh, Kh, Vh = (torch.from_numpy(np.ascontiguousarray(x)).to(tdt).pin_memory() for x in (Q, K, V))
-    split_block = meta.get("split_block", w.nb // 2) if split else -1
+    split_block = meta.get("split_block", w.nk // 2) if split else -1
     Oh = torch.full(Qh.shape, 7.0, dtype=tdt).pin_memory()              # padding rows must stay untouched
     Lh = torch.full(Qh.shape[:3], 7.0, dtype=torch.float32).pin_memory()
-    api.forward_host(Qh, Kh, Vh, w.N, w.block, keep, split_block=split_block, kv_heads_per_chunk=chunk, out=(Oh, Lh))
+    api.forward_host(Qh, Kh, Vh, w.N, w.block, keep, split_block=split_block, kv_heads_per_chunk=chunk, out=(Oh, Lh),
+                     block_k=w.block_k)
     torch.cuda.synchronize()
     # the same steps on device-resident buffers
     r = run_gpu(Q, K, V, w, keep)
@@ -412,7 +415,7 @@ def test_forward_host_pipeline(name, over, split, chunk):
     assert torch.equal(Lh[:, :, :n], Ld[:, :, :n].cpu())
     assert (Oh[:, :, n:] == 7.0).all() and (Lh[:, :, n:] == 7.0).all()
     tol = TOL[w.dtype]
-    Oref, Lref = O.masked_attention(Q, K, V, r["idx"], r["cnt"], w.N, w.block, w.d ** -0.5)
+    Oref, Lref = O.masked_attention(Q, K, V, r["idx"], r["cnt"], w.N, w.block, w.d ** -0.5, b_k=w.kb)
     got = Oh[:, :, :n].float().numpy()
     assert max_abs(got, Oref[:, :, :n]) <= tol["max_abs"] and rel_l2(got, Oref[:, :, :n]) <= tol["rel_l2"]
     assert max_abs(Lh[:, :, :n].numpy(), Lref[:, :, :n]) <= tol["lse_abs"]
