@@ -428,6 +428,220 @@ __global__ void __launch_bounds__(kStatsThreads, 2)
   }
 }
 
+// One warp per block (the statistics pass of the one-copy path): the warp's
+// lanes own D/32 columns each across all rows of the block, so no value
+// crosses lanes and no barrier joins warps. Each lane accumulates, in fp32,
+// the deviations d = x - c from the block's first row c (exact in fp32 for
+// bf16 and small for fp32 inputs), S1 = sum d and S2 = sum d^2 over two
+// interleaved accumulator sets; then
+//   mean = c + S1/n,  var = (S2 - S1 * (S1/n)) / n   (clamped at 0).
+// A column that does not vary gives d = 0 and a variance of exactly 0.
+// Each warp double-buffers its own 32 KB bulk copies (two ring stages with
+// their own mbarriers); kStatsWarpsPerCta warps share a CTA and its shared
+// memory, one CTA per SM.
+constexpr int kStatsWarpsPerCta = 3;
+constexpr long long kStatsWarpMinBlocks = 16384;     // blocks of work from which the warp kernel is used
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kStatsWarpsPerCta * 32, 1)
+    stats_warp_kernel(const T *__restrict__ Q, const T *__restrict__ K, float *__restrict__ q_mean,
+                      float *__restrict__ q_var, float *__restrict__ k_mean, float *__restrict__ k_var, int B,
+                      int Hq, int Hkv, int N, int N_alloc, int block, int nb, int kblock, int nbk, FeatOut feat) {
+  constexpr int E = D / 32;                         // columns per lane
+  constexpr int P = E / 2;                          // packed fp32 pairs per lane
+  constexpr int RB = D * static_cast<int>(sizeof(T));   // bytes per row
+  static_assert(E == 2 || E == 4, "head dimension");
+  extern __shared__ __align__(128) uint8_t stage_mem[];
+  __shared__ uint64_t full[kStatsWarpsPerCta][2];
+  __shared__ long long meta_orow[kStatsWarpsPerCta][2];
+  __shared__ int meta_rows[kStatsWarpsPerCta][2];
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t ring = smem_u32(stage_mem) + static_cast<uint32_t>(warp) * 2u * kStatsStageBytes;
+  const long long n_q = static_cast<long long>(B) * Hq * nb;
+  const long long total = n_q + static_cast<long long>(B) * Hkv * nbk;
+  const long long tw = static_cast<long long>(gridDim.x) * kStatsWarpsPerCta;
+  const long long gw = static_cast<long long>(blockIdx.x) * kStatsWarpsPerCta + warp;
+  const uint64_t policy = l2_evict_first_policy();
+
+  // item w -> its slab (Q rows of a query block or K rows of a key block)
+  auto issue = [&](long long w, int st) {
+    const bool is_q = w < n_q;
+    const long long c = is_q ? w : w - n_q;
+    const int nbx = is_q ? nb : nbk, bsize = is_q ? block : kblock;
+    const int blk = static_cast<int>(c % nbx);
+    const long long bh = c / nbx;
+    const T *src = (is_q ? Q : K) + (bh * N_alloc + static_cast<long long>(blk) * bsize) * D;
+    const int n_rows = min(bsize, N - blk * bsize);
+    const long long orow = (bh * nbx + blk) * static_cast<long long>(D);
+    meta_orow[warp][st] = is_q ? orow : -1 - orow;   // sign carries Q-or-K
+    meta_rows[warp][st] = n_rows;
+    mbar_arrive_expect_tx(smem_u32(&full[warp][st]), static_cast<uint32_t>(n_rows) * RB);
+    bulk_load_hint(ring + st * kStatsStageBytes, src, static_cast<uint32_t>(n_rows) * RB, smem_u32(&full[warp][st]),
+                   policy);
+  };
+
+  long long issued = 0, consumed = 0;               // this warp's items handed to the copy engine / read
+  if (lane == 0) {
+    mbar_init(smem_u32(&full[warp][0]), 1);
+    mbar_init(smem_u32(&full[warp][1]), 1);
+    fence_mbar_init();
+    for (int st = 0; st < 2; ++st)
+      if (gw + st * tw < total) issue(gw + st * tw, st);
+  }
+  issued = (gw < total) + (gw + tw < total);
+  __syncwarp();
+
+  bool ok = true;
+  for (long long w = gw; w < total; w += tw) {
+    const int st = static_cast<int>(consumed & 1);
+    const bool got = mbar_wait_bounded(smem_u32(&full[warp][st]), static_cast<uint32_t>((consumed >> 1) & 1), nullptr);
+    if (!__all_sync(0xFFFFFFFFu, got)) {
+      ok = false;
+      break;
+    }
+    const long long mo = meta_orow[warp][st];
+    const int n = meta_rows[warp][st];
+    const bool is_q = mo >= 0;
+    const long long orow = is_q ? mo : -1 - mo;
+    const uint8_t *rows = stage_mem + (static_cast<size_t>(warp) * 2 + st) * kStatsStageBytes + lane * E * sizeof(T);
+
+    // this lane's E columns of row r as P packed fp32 pairs
+    auto row_pairs = [&](int r, uint64_t (&x)[P]) {
+      const uint8_t *a = rows + static_cast<size_t>(r) * RB;
+      if constexpr (sizeof(T) == 2) {
+        if constexpr (E == 4) {
+          const uint2 v = *reinterpret_cast<const uint2 *>(a);
+          x[0] = pack_u32x2(v.x << 16, v.x & 0xFFFF0000u);
+          x[1] = pack_u32x2(v.y << 16, v.y & 0xFFFF0000u);
+        } else {
+          const uint32_t v = *reinterpret_cast<const uint32_t *>(a);
+          x[0] = pack_u32x2(v << 16, v & 0xFFFF0000u);
+        }
+      } else {
+        if constexpr (E == 4) {
+          const uint4 v = *reinterpret_cast<const uint4 *>(a);
+          x[0] = pack_u32x2(v.x, v.y);
+          x[1] = pack_u32x2(v.z, v.w);
+        } else {
+          const uint2 v = *reinterpret_cast<const uint2 *>(a);
+          x[0] = pack_u32x2(v.x, v.y);
+        }
+      }
+    };
+    uint64_t c[P], nc[P], s1[2][P], s2[2][P];
+    row_pairs(0, c);
+#pragma unroll
+    for (int i = 0; i < P; ++i) {
+      nc[i] = pack_f32x2(-lo_f32(c[i]), -hi_f32(c[i]));
+      s1[0][i] = s1[1][i] = s2[0][i] = s2[1][i] = 0ull;       // +0.0f pairs
+    }
+    int r = 1;
+#pragma unroll 4
+    for (; r + 1 < n; r += 2) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint64_t x[P];
+        row_pairs(r + h, x);
+#pragma unroll
+        for (int i = 0; i < P; ++i) {
+          const uint64_t d = add_f32x2(x[i], nc[i]);
+          s1[h][i] = add_f32x2(s1[h][i], d);
+          s2[h][i] = fma_f32x2(d, d, s2[h][i]);
+        }
+      }
+    }
+    if (r < n) {
+      uint64_t x[P];
+      row_pairs(r, x);
+#pragma unroll
+      for (int i = 0; i < P; ++i) {
+        const uint64_t d = add_f32x2(x[i], nc[i]);
+        s1[0][i] = add_f32x2(s1[0][i], d);
+        s2[0][i] = fma_f32x2(d, d, s2[0][i]);
+      }
+    }
+    __syncwarp();                                   // every lane is done with this stage
+    ++consumed;
+    if (lane == 0 && w + 2 * tw < total) {
+      fence_proxy_async_smem();                     // the reads above before the bulk write
+      issue(w + 2 * tw, st);
+    }
+    if (w + 2 * tw < total) ++issued;
+
+    const float inv_n = 1.f / static_cast<float>(n);
+    float mean[E], var[E];
+#pragma unroll
+    for (int i = 0; i < P; ++i) {
+      const uint64_t S1 = add_f32x2(s1[0][i], s1[1][i]), S2 = add_f32x2(s2[0][i], s2[1][i]);
+      const float a1[2] = {lo_f32(S1), hi_f32(S1)}, a2[2] = {lo_f32(S2), hi_f32(S2)};
+      const float cc[2] = {lo_f32(c[i]), hi_f32(c[i])};
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float md = a1[e] * inv_n;
+        mean[2 * i + e] = cc[e] + md;
+        var[2 * i + e] = fmaxf(fmaf(-a1[e], md, a2[e]) * inv_n, 0.f);
+      }
+    }
+    float *om = (is_q ? q_mean : k_mean) + orow + lane * E;
+    float *ov = (is_q ? q_var : k_var) + orow + lane * E;
+    if constexpr (E == 4) {
+      *reinterpret_cast<float4 *>(om) = make_float4(mean[0], mean[1], mean[2], mean[3]);
+      *reinterpret_cast<float4 *>(ov) = make_float4(var[0], var[1], var[2], var[3]);
+    } else {
+      *reinterpret_cast<float2 *>(om) = make_float2(mean[0], mean[1]);
+      *reinterpret_cast<float2 *>(ov) = make_float2(var[0], var[1]);
+    }
+    if (feat.q != nullptr) {
+      // the lane's E columns of each plane packed into one store: a warp
+      // writes each plane's D contiguous values at once
+      float x[3][E];
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        if (is_q) {
+          x[0][e] = __fmul_rn(feat.s, mean[e]);
+          x[1][e] = __fmul_rn(feat.hs2, var[e]);
+          x[2][e] = __fmul_rn(__fmul_rn(feat.hs2, mean[e]), mean[e]);
+        } else {
+          x[0][e] = mean[e];
+          x[1][e] = __fmaf_rn(mean[e], mean[e], var[e]);
+          x[2][e] = var[e];
+        }
+      }
+      __nv_bfloat16 *base = is_q ? feat.q : feat.k;
+      const long long plane = (is_q ? feat.q_rows : feat.k_rows) * D;
+#pragma unroll
+      for (int pp = 0; pp < 3; ++pp) {
+        uint32_t hw[E / 2], lw[E / 2];
+#pragma unroll
+        for (int e = 0; e < E; e += 2) {
+          const __nv_bfloat16 h0 = __float2bfloat16_rn(x[pp][e]), h1 = __float2bfloat16_rn(x[pp][e + 1]);
+          const __nv_bfloat16 l0 = __float2bfloat16_rn(x[pp][e] - __bfloat162float(h0));
+          const __nv_bfloat16 l1 = __float2bfloat16_rn(x[pp][e + 1] - __bfloat162float(h1));
+          hw[e / 2] = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) |
+                      (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
+          lw[e / 2] = static_cast<uint32_t>(__bfloat16_as_ushort(l0)) |
+                      (static_cast<uint32_t>(__bfloat16_as_ushort(l1)) << 16);
+        }
+        __nv_bfloat16 *ph = base + (2 * pp) * plane + orow + lane * E;
+        __nv_bfloat16 *pl = base + (2 * pp + 1) * plane + orow + lane * E;
+        if constexpr (E == 4) {
+          *reinterpret_cast<uint2 *>(ph) = make_uint2(hw[0], hw[1]);
+          *reinterpret_cast<uint2 *>(pl) = make_uint2(lw[0], lw[1]);
+        } else {
+          *reinterpret_cast<uint32_t *>(ph) = hw[0];
+          *reinterpret_cast<uint32_t *>(pl) = lw[0];
+        }
+      }
+    }
+  }
+  // after an abandoned wait, let this warp's copies in flight land first
+  if (!ok && lane == 0) {
+    for (long long u = consumed; u < issued; ++u)
+      mbar_wait_bounded(smem_u32(&full[warp][u & 1]), static_cast<uint32_t>((u >> 1) & 1), nullptr);
+  }
+}
+
 // Rows each thread holds for a given block size (power-of-two bucket).
 template <typename T, int D>
 inline int stats_rpt_needed(int block) {
@@ -449,6 +663,21 @@ cudaError_t launch_stats(const T *Q, const T *K, float *qm, float *qv, float *km
   const int nb = (N + block - 1) / block, nbk = (N + kblock - 1) / kblock;
   const long long grid = static_cast<long long>(B) * Hq * nb + static_cast<long long>(B) * Hkv * nbk;
   const int bmax = block > kblock ? block : kblock;
+  // The warp-per-block kernel has no cross-warp merge and reaches ~0.97 of
+  // HBM on long runs (128K: 40960 blocks); below ~16K blocks its three warps
+  // per SM ramp up and drain more slowly than the CTA-per-block kernel.
+  if (stats_bulk_fits<T, D>(bmax) && grid >= kStatsWarpMinBlocks) {
+    const size_t smem = static_cast<size_t>(kStatsWarpsPerCta) * 2 * kStatsStageBytes;
+    cudaError_t e = cudaFuncSetAttribute(stats_warp_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    const long long warps = (grid + 0);                 // one warp per block
+    const long long ctas_needed = (warps + kStatsWarpsPerCta - 1) / kStatsWarpsPerCta;
+    const unsigned g = static_cast<unsigned>(ctas_needed < num_sms ? ctas_needed : num_sms);
+    stats_warp_kernel<T, D><<<g, kStatsWarpsPerCta * 32, smem, stream>>>(Q, K, qm, qv, km, kv, B, Hq, Hkv, N, N_alloc,
+                                                                       block, nb, kblock, nbk, feat);
+    return cudaGetLastError();
+  }
   if (stats_bulk_fits<T, D>(bmax)) {
     const size_t smem = static_cast<size_t>(kStatsStages) * kStatsStageBytes;
     cudaError_t e = cudaFuncSetAttribute(stats_bulk_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -596,3 +596,23 @@ def test_full_size_workloads(name):
             check_attention(r2, Q, K, V, w, sample_blocks(w, per_head=1, seed=1))
         del r
         torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("name,over", [
+    ("tiny_fp32", dict(N=16384 - 5, N_alloc=16384, Hq=8, Hkv=8, block=16)),       # fp32, d 64: 16384 blocks
+    ("dlm_16k", dict(N=16384, Hq=16, Hkv=4, d=64, block=16, block_k=32)),        # bf16, asymmetric: 18432 blocks
+])
+def test_stats_many_blocks(name, over):
+    # enough blocks for the warp-per-block statistics kernel: statistics and
+    # selection against the oracle
+    Q, K, V, meta = make_inputs(name, **over)
+    w = meta["workload"]
+    Qd, Kd = to_dev(Q, w.dtype), to_dev(K, w.dtype)
+    shape = api.Shape.of(Qd, Kd, w.N, w.block, block_k=w.block_k)
+    assert w.B * (w.Hq * w.nb + w.Hkv * w.nk) >= 16384
+    st = api.stats(Qd, Kd, shape)
+    idx, cnt, sc = api.select(st, shape, 0.5, with_scores=True)
+    torch.cuda.synchronize()
+    r = dict(stats=[t.cpu().numpy() for t in st], scores=sc.cpu().numpy(), idx=idx.cpu().numpy(), cnt=cnt.cpu().numpy())
+    stats_ref = check_stats(r, Q, K, w)
+    check_selection(r, stats_ref, w, 0.5)
