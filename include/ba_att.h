@@ -113,7 +113,10 @@ int32_t ba_att_keep_count(const ba_att_shape *shape, double keep);
  *   mean[i, m] = (1/n_i) sum_r x[r, m]
  *   var [i, m] = (1/n_i) sum_r (x[r, m] - mean[i, m])^2     (population)
  * computed in fp32: exact two-pass moments of each thread's register-resident
- * rows, merged with the pairwise update for centred moments.
+ * rows, merged with the pairwise update for centred moments; or, for runs of
+ * 16384 blocks or more, per column the sums of the deviations from the
+ * block's first row (mean = c + S1/n, var = (S2 - S1^2/n)/n, at least 0).
+ * Either way a column that does not vary within a block has variance 0.
  *
  * Q, K      device, [B,Hq|Hkv,N_alloc,d] of shape->dtype; read once.
  * q_mean, q_var   device fp32 [B, Hq,  nq, d]  (written)
