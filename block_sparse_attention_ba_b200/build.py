@@ -54,6 +54,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
         "-lineinfo", "-O3", "-std=c++17",
         "-Xcompiler", "-fPIC,-O3",
         "-shared", "-cudart", "static",
+        "-Xfatbin=-compress-all",
         "-I", INCLUDE,
         "-o", LIB + ".tmp",
     ] + SOURCES

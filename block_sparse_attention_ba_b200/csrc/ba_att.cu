@@ -256,12 +256,7 @@ long long feat_rows_k(const ba_att_shape *s) { return static_cast<long long>(s->
 // Whether the shape takes the feature path (else the selector is the plain
 // ba_att_stats + ba_att_select sequence).
 bool selector_feature_path(const ba_att_shape *s) {
-  const int bmax = s->block > kblock(s) ? s->block : kblock(s);
-  const bool bulk = s->dtype == BA_DTYPE_BF16
-                        ? (s->d == 128 ? stats_bulk_fits<__nv_bfloat16, 128>(bmax)
-                                       : stats_bulk_fits<__nv_bfloat16, 64>(bmax))
-                        : (s->d == 128 ? stats_bulk_fits<float, 128>(bmax) : stats_bulk_fits<float, 64>(bmax));
-  return bulk && feat_rows_q(s) + selft::kTile < 0x7FFFFFFFLL;
+  return feat_rows_q(s) + selft::kTile < 0x7FFFFFFFLL;
 }
 
 template <int D>

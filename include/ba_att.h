@@ -112,11 +112,10 @@ int32_t ba_att_keep_count(const ba_att_shape *shape, double keep);
  * For every block i and head h, over the valid rows r of the block:
  *   mean[i, m] = (1/n_i) sum_r x[r, m]
  *   var [i, m] = (1/n_i) sum_r (x[r, m] - mean[i, m])^2     (population)
- * computed in fp32: exact two-pass moments of each thread's register-resident
- * rows, merged with the pairwise update for centred moments; or, for runs of
- * 16384 blocks or more, per column the sums of the deviations from the
- * block's first row (mean = c + S1/n, var = (S2 - S1^2/n)/n, at least 0).
- * Either way a column that does not vary within a block has variance 0.
+ * computed in fp32 from the per-column sums of the deviations from the
+ * block's first row c: mean = c + S1/n, var = (S2 - S1^2/n)/n, at least 0
+ * (S1 = sum (x - c), S2 = sum (x - c)^2, rows summed in order). A column
+ * that does not vary within a block has variance exactly 0.
  *
  * Q, K      device, [B,Hq|Hkv,N_alloc,d] of shape->dtype; read once.
  * q_mean, q_var   device fp32 [B, Hq,  nq, d]  (written)
@@ -204,9 +203,8 @@ int64_t ba_att_selector_workspace(const ba_att_shape *shape);
  * ba_att_stats and ba_att_select (block_scores holds the score map on return).
  * workspace   device, caller-owned, >= ba_att_selector_workspace(shape)
  *             bytes, 16-byte aligned; its contents on return are unspecified.
- * Shapes whose block of d values does not fit one 32 KB copy (bf16 with
- * block * d > 16384, fp32 with block * d > 8192) run ba_att_stats and
- * ba_att_select instead, leaving the workspace unused. NULL pointers ->
+ * Shapes with more than 2^31 - 129 feature rows (B*Hq*nq) run ba_att_stats
+ * and ba_att_select instead, leaving the workspace unused. NULL pointers ->
  * BA_ERR_INVALID_ARG; misaligned -> BA_ERR_MISALIGNED; nk > 4096 ->
  * BA_ERR_UNSUPPORTED.
  */
