@@ -25,7 +25,8 @@ CASES = [
     ("dlm_16k", dict(N=2048 - 40, N_alloc=2048, Hq=4, Hkv=2, d=64, block=256), 0.5),   # 256-row blocks, d 64
     ("dlm_16k", dict(N=2048 - 30, N_alloc=2048, Hq=4, Hkv=2, block_k=64), 0.5),      # asymmetric: 16 x 32 blocks
     ("dlm_16k", dict(N=3000, N_alloc=3072, Hq=2, Hkv=1, d=64, block_k=256), 0.3),    # asymmetric: 24 x 12 blocks
-    ("tiny_fp32", dict(N=2048, d=128, block=128), 0.5),                # 64 KB blocks: plain stats + select
+    ("tiny_fp32", dict(N=2048, d=128, block=128), 0.5),                # fp32 64 KB blocks, streamed in chunks
+    ("dlm_16k", dict(N=4096 - 100, N_alloc=4096, Hq=4, Hkv=2, block=256), 0.5),   # bf16 d 128, 64 KB blocks
 ]
 
 
