@@ -268,10 +268,9 @@ cudaError_t launch_select_feat(const CUtensorMap &mq, const CUtensorMap &mk, flo
                                        static_cast<int>(selft::kDynSmem));
   if (e != cudaSuccess) return e;
   const unsigned grid = static_cast<unsigned>(n_tiles < sms ? n_tiles : sms);
-  selft::select_feat_kernel<D><<<grid, selft::kThreads, selft::kDynSmem, cs>>>(mq, mk, scores, s->Hq, s->Hkv, s->N,
-                                                                              kblock(s), nq, nk, n_tiles, n_tq,
-                                                                              n_tk);
-  return cudaGetLastError();
+  // a programmatic dependent of the statistics pass that writes its features
+  return launch_dependent(selft::select_feat_kernel<D>, dim3(grid), dim3(selft::kThreads), selft::kDynSmem, cs, mq, mk,
+                          scores, s->Hq, s->Hkv, s->N, kblock(s), nq, nk, n_tiles, n_tq, n_tk);
 }
 }  // namespace
 
@@ -334,7 +333,7 @@ ba_status ba_att_selector(const ba_att_shape *s, double keep, const void *Q, con
                   : launch_select_feat<64>(mq, mk, block_scores, s, nq, nk, sms, cs);
   if (e != cudaSuccess) return from_cuda(e);
   return from_cuda(launch_topk(block_scores, nk, k, kv_idx, kmax, kv_cnt, static_cast<long long>(s->B) * s->Hq * nq,
-                               sms, cs));
+                               sms, cs, /*dependent=*/true));
 }
 
 ba_status ba_att_topk(const float *block_scores, int64_t rows, int32_t nk, int32_t k, int32_t *kv_idx,

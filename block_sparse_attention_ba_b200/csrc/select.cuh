@@ -22,6 +22,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "pdl.cuh"
 
 namespace baatt {
 
@@ -512,6 +513,7 @@ __global__ void __launch_bounds__(kTopkWarps * 32) topk_rows_lm_kernel(const flo
       for (int c = 0; c < KPL; ++c) nxt[c] = (r < rows && lane * KPL + c < nk) ? __ldg(src + c) : 0.f;
     }
   };
+  pdl_wait();                                       // the score map is complete from here on
   fetch(row);
   for (; row < rows; row += stride) {
     uint32_t u[KPL];
@@ -621,7 +623,7 @@ inline cudaError_t launch_topk_smem(const float *scores, int nk, int k, int32_t 
 
 template <int KPL>
 inline cudaError_t launch_topk_lm(const float *scores, int nk, int k, int32_t *idx, int kmax, int32_t *cnt,
-                                  long long rows, int num_sms, cudaStream_t stream) {
+                                  long long rows, int num_sms, cudaStream_t stream, bool dependent) {
   const int threads = kTopkWarps * 32;
   int per_sm = 0;
   const cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, topk_rows_lm_kernel<KPL>, threads, 0);
@@ -629,14 +631,18 @@ inline cudaError_t launch_topk_lm(const float *scores, int nk, int k, int32_t *i
   long long grid = (rows + kTopkWarps - 1) / kTopkWarps;
   const long long slots = static_cast<long long>(num_sms) * (per_sm > 0 ? per_sm : 1);
   grid = grid < slots ? grid : slots;
+  if (dependent)
+    return launch_dependent(topk_rows_lm_kernel<KPL>, dim3(static_cast<unsigned>(grid)), dim3(threads), 0, stream,
+                            scores, nk, k, idx, kmax, cnt, rows);
   topk_rows_lm_kernel<KPL><<<static_cast<unsigned>(grid), threads, 0, stream>>>(scores, nk, k, idx, kmax, cnt, rows);
   return cudaGetLastError();
 }
 
 template <int KPL>
 inline cudaError_t launch_topk_kpl(const float *scores, int nk, int k, int32_t *idx, int kmax, int32_t *cnt,
-                                   long long rows, int num_sms, cudaStream_t stream) {
-  if (BA_TOPK_LANE_MAJOR && KPL > 0) return launch_topk_lm<(KPL > 0 ? KPL : 8)>(scores, nk, k, idx, kmax, cnt, rows, num_sms, stream);
+                                   long long rows, int num_sms, cudaStream_t stream, bool dependent = false) {
+  if (BA_TOPK_LANE_MAJOR && KPL > 0)
+    return launch_topk_lm<(KPL > 0 ? KPL : 8)>(scores, nk, k, idx, kmax, cnt, rows, num_sms, stream, dependent);
   if (KPL >= BA_TOPK_SMEM_MIN_KPL) return launch_topk_smem<(KPL > 0 ? KPL : 8)>(scores, nk, k, idx, kmax, cnt, rows, num_sms, stream);
   const int threads = kTopkWarps * 32;
   long long grid = (rows + kTopkWarps - 1) / kTopkWarps;
@@ -833,11 +839,13 @@ inline cudaError_t launch_topk_variant(const float *scores, int nk, int k, int32
   return launch_topk_variant_kpl<32>(scores, nk, k, idx, kmax, cnt, sel_rows, var, num_sms, stream);
 }
 
+// dependent: launch the lane-major kernel as a programmatic dependent of the
+// kernel before it on the stream (which must be the one writing `scores`).
 inline cudaError_t launch_topk(const float *scores, int nk, int k, int32_t *idx, int kmax, int32_t *cnt,
-                               long long rows, int num_sms, cudaStream_t stream) {
-  if (nk <= 256) return launch_topk_kpl<8>(scores, nk, k, idx, kmax, cnt, rows, num_sms, stream);
-  if (nk <= 512) return launch_topk_kpl<16>(scores, nk, k, idx, kmax, cnt, rows, num_sms, stream);
-  if (nk <= 1024) return launch_topk_kpl<32>(scores, nk, k, idx, kmax, cnt, rows, num_sms, stream);
+                               long long rows, int num_sms, cudaStream_t stream, bool dependent = false) {
+  if (nk <= 256) return launch_topk_kpl<8>(scores, nk, k, idx, kmax, cnt, rows, num_sms, stream, dependent);
+  if (nk <= 512) return launch_topk_kpl<16>(scores, nk, k, idx, kmax, cnt, rows, num_sms, stream, dependent);
+  if (nk <= 1024) return launch_topk_kpl<32>(scores, nk, k, idx, kmax, cnt, rows, num_sms, stream, dependent);
   return launch_topk_kpl<0>(scores, nk, k, idx, kmax, cnt, rows, num_sms, stream);
 }
 

@@ -28,6 +28,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "pdl.cuh"
 #include "select.cuh"
 
 namespace baatt {
@@ -312,6 +313,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = tmem_base_s;
   volatile int *abort = &abort_flag;
+  // launched as a dependent of the statistics pass: its features (and the
+  // score map's earlier readers) are settled only from here on
+  pdl_wait();
+  pdl_allow_dependents();
 
   if (warp == 4 && lane == 0) {
     // ------------------------------------------------------------ producer

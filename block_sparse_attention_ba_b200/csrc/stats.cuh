@@ -27,6 +27,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "pdl.cuh"
 
 #ifndef BA_STATS_LONG_RUN_ITEMS
 #define BA_STATS_LONG_RUN_ITEMS 16384
@@ -129,6 +130,7 @@ __global__ void __launch_bounds__(3 * SPLIT * 32, 1)
   load_item();
   issued += issue_next(0);
   issued += issue_next(1);
+  pdl_allow_dependents();                           // the score GEMM may launch as SMs free up
 
   uint64_t c[P], nc[P], s1[2][P], s2[2][P];
 #pragma unroll
