@@ -86,7 +86,7 @@ def selector_bytes(w, k: int) -> int:
     return qk + lists
 
 
-LAUNCHES_PER_STEP = 6   # stats_bulk, select_tc + topk_rows, split_lists, attn_tc x2
+LAUNCHES_PER_STEP = 6   # stats_warp, select_feat, topk_rows_lm, split_lists, attn_tc x2
 
 
 def kernel_sources_sha(files):
