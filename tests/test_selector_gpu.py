@@ -27,6 +27,10 @@ CASES = [
     ("dlm_16k", dict(N=3000, N_alloc=3072, Hq=2, Hkv=1, d=64, block_k=256), 0.3),    # asymmetric: 24 x 12 blocks
     ("tiny_fp32", dict(N=2048, d=128, block=128), 0.5),                # fp32 64 KB blocks, streamed in chunks
     ("dlm_16k", dict(N=4096 - 100, N_alloc=4096, Hq=4, Hkv=2, block=256), 0.5),   # bf16 d 128, 64 KB blocks
+    # long key ranges: 4 to 6 key tiles per query tile, ragged last tile
+    ("dlm_16k", dict(N=32768 - 100, N_alloc=32768, Hq=2, Hkv=1, block_k=64), 0.5),   # 256 x 511 blocks
+    ("dlm_16k", dict(N=32768, B=2, Hq=4, Hkv=2, d=64, block_k=64), 0.3),            # d 64, two batches
+    ("dlm_16k", dict(N=16384 * 3 - 7, N_alloc=16384 * 3, Hq=3, Hkv=1, block=64), 0.5),   # 768 x 768 blocks
 ]
 
 
