@@ -24,9 +24,9 @@ plain reading of that prose, stated in the docstring of the function that
 implements it.
 
 Parity status: every public function is pinned by tests in
-``tests/test_oracle.py`` except the two diagnostics marked "parity unpinned"
-(``spearman_vs_post`` and ``topk_recall_vs_post``): the pages print no value to
-pin them to.
+``tests/test_oracle.py``. The two diagnostics (``spearman_vs_post`` and
+``topk_recall_vs_post``) have no value on the pages; they are pinned to a
+library routine, closed forms and brute force instead.
 """
 
 from .ba_att_oracle import (  # noqa: F401

@@ -516,8 +516,9 @@ def _rank(x):
 def spearman_vs_post(S, A):
     """Mean per-row Spearman rank correlation between a block score and A.
 
-    Diagnostic for the correlation the Figure 2 caption of [BA-Att] refers to.
-    Parity unpinned: the pages print no value for it.
+    Diagnostic for the correlation the Figure 2 caption of [BA-Att] refers to;
+    the pages print no value for it. Pinned to scipy's Spearman rho and the
+    closed form on tie-free rows, and to +1 / -1 for equal / reversed order.
     """
     S = np.asarray(S).reshape(-1, S.shape[-1])
     A = np.asarray(A).reshape(-1, A.shape[-1])
@@ -534,7 +535,8 @@ def spearman_vs_post(S, A):
 def topk_recall_vs_post(S, A, k: int):
     """Fraction of the exact-A top-k blocks that the S~ top-k also keeps.
 
-    Diagnostic of selection quality. Parity unpinned: no value on the pages.
+    Diagnostic of selection quality; no value on the pages. Pinned by a
+    hand-worked row, brute-force set intersection, and the 1 / 0 limits.
     """
     idx_s, _ = select_topk(S, k)
     idx_a, _ = select_topk(A, k)

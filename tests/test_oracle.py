@@ -513,3 +513,53 @@ def test_asymmetric_post_downsample_map():
     assert A16.shape == (1, 2, 3, 6) and A32.shape == (1, 2, 3, 3)
     np.testing.assert_allclose(A16.sum(-1), 1.0, rtol=1e-13)
     np.testing.assert_allclose(A16[..., 0::2] + A16[..., 1::2], A32, rtol=1e-12, atol=1e-15)
+
+
+# ------------------------------------------------- diagnostics: rank agreement and top-k recall
+
+def test_spearman_vs_post_matches_library_and_closed_form():
+    # tie-free rows: the mean of scipy's per-row Spearman rho, and the closed
+    # form rho = 1 - 6 sum d^2 / (n (n^2 - 1)) on the ranks
+    import scipy.stats
+    rng = np.random.default_rng(11)
+    S = rng.standard_normal((3, 4, 37))
+    A = S + 0.7 * rng.standard_normal(S.shape)
+    got = O.spearman_vs_post(S, A)
+    rows_s, rows_a = S.reshape(-1, 37), A.reshape(-1, 37)
+    lib = np.mean([scipy.stats.spearmanr(a, b).statistic for a, b in zip(rows_s, rows_a)])
+    np.testing.assert_allclose(got, lib, rtol=0, atol=1e-12)
+    n = 37
+    closed = []
+    for a, b in zip(rows_s, rows_a):
+        ra = np.argsort(np.argsort(a))
+        rb = np.argsort(np.argsort(b))
+        closed.append(1.0 - 6.0 * float(((ra - rb) ** 2).sum()) / (n * (n * n - 1)))
+    np.testing.assert_allclose(got, np.mean(closed), rtol=0, atol=1e-12)
+
+
+def test_spearman_vs_post_special_cases():
+    rng = np.random.default_rng(12)
+    A = rng.random((2, 5, 16))
+    assert O.spearman_vs_post(A, A) == pytest.approx(1.0, abs=1e-12)
+    assert O.spearman_vs_post(-A, A) == pytest.approx(-1.0, abs=1e-12)
+    # any strictly increasing transform of the score leaves the ranks alone
+    assert O.spearman_vs_post(np.exp(3.0 * A) - 2.0, A) == pytest.approx(1.0, abs=1e-12)
+
+
+def test_topk_recall_vs_post_hand_worked_and_limits():
+    # top-2 of A is {0, 1}; top-2 of S is {0, 2}: one of two kept -> 0.5
+    A = np.array([[[5.0, 4.0, 3.0, 2.0, 1.0]]])
+    S = np.array([[[5.0, 1.0, 4.0, 2.0, 3.0]]])
+    assert O.topk_recall_vs_post(S, A, 2) == pytest.approx(0.5)
+    rng = np.random.default_rng(13)
+    A = rng.random((2, 3, 20))
+    assert O.topk_recall_vs_post(A, A, 7) == pytest.approx(1.0)
+    # the top 7 of -A are the bottom 7 of A: disjoint from its top 7 (no ties)
+    assert O.topk_recall_vs_post(-A, A, 7) == pytest.approx(0.0)
+    # brute force over rows: |top_k(S) & top_k(A)| / k by full sorts
+    S = A + 0.3 * rng.standard_normal(A.shape)
+    k = 5
+    hits = 0
+    for a, s in zip(A.reshape(-1, 20), S.reshape(-1, 20)):
+        hits += len(set(np.argsort(-a, kind="stable")[:k]) & set(np.argsort(-s, kind="stable")[:k]))
+    assert O.topk_recall_vs_post(S, A, k) == pytest.approx(hits / (k * 6))
