@@ -5,7 +5,7 @@
 // the downsampled block space, the pooled score is corrected with diagonal
 // Q/K variances, blocks are sorted and the top fraction is kept.
 //
-// The scores S~[i,j] are written by select_tc_kernel (select_tc.cuh, tensor
+// The scores S~[i,j] are written by the score kernels (select_tc.cuh, tensor
 // cores); this file ranks each (batch, head, query block) row of that map.
 // One warp per row selects the top k exactly on order-preserving 32-bit keys
 // of the fp32 scores (topk_row_keys: a sampled key window, 8-bit radix
@@ -13,12 +13,11 @@
 // the lower block index, and the kept indices are emitted ascending. Rows of
 // up to 1024 keys are held in registers lane-major (topk_rows_lm_kernel: each
 // lane a contiguous run of columns, 16-byte loads, kept columns emitted from
-// per-lane bit masks); the chunk-major register and shared-memory kernels
-// (topk_rows_kernel, topk_rows_smem_kernel) remain behind
-// BA_TOPK_LANE_MAJOR=0; longer rows are re-read from global memory
-// (topk_row_warp). topk_variant_kernel serves the selection variants
-// of ba_att_select_ex (shared per GQA group, forced diagonal, cumulative
-// softmax share: topk_row_mass).
+// per-lane bit masks); longer rows are re-read from global memory
+// (topk_rows_long_kernel, topk_row_warp). topk_variant_kernel serves the
+// selection variants of ba_att_select_ex (shared per GQA group, forced
+// diagonal, cumulative softmax share: topk_row_mass); it holds its rows
+// chunk-major (lane l has columns c*32 + l).
 #pragma once
 
 #include "common.cuh"
@@ -446,40 +445,16 @@ __device__ __forceinline__ void topk_row_regs(const uint32_t (&u)[KPL], int nk, 
 // 32*KPL keys are held in registers, longer rows are re-read per pass.
 constexpr int kTopkWarps = 8;
 
-// Rows up to 32*KPL keys: persistent warps walk the rows with a stride of all
-// warps of the grid, and the next row's scores are loaded into registers
-// before the current row is selected, so the load latency overlaps the
-// selection. Longer rows: one warp per row, re-read from global memory.
-template <int KPL>
-__global__ void __launch_bounds__(kTopkWarps * 32) topk_rows_kernel(const float *__restrict__ scores, int nk, int k,
-                                                                    int32_t *__restrict__ kv_idx, int kmax,
-                                                                    int32_t *__restrict__ kv_cnt, long long rows) {
-  __shared__ __align__(16) unsigned hist[kTopkWarps][256];   // also holds (key, column) pairs
+// Rows longer than 1024 keys: one warp per row, re-read from global memory
+// on every pass (topk_row_warp).
+__global__ void __launch_bounds__(kTopkWarps * 32) topk_rows_long_kernel(const float *__restrict__ scores, int nk,
+                                                                         int k, int32_t *__restrict__ kv_idx, int kmax,
+                                                                         int32_t *__restrict__ kv_cnt, long long rows) {
+  __shared__ __align__(16) unsigned hist[kTopkWarps][256];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  long long row = blockIdx.x * static_cast<long long>(kTopkWarps) + warp;
-  if constexpr (KPL > 0) {
-    const long long stride = static_cast<long long>(gridDim.x) * kTopkWarps;
-    float nxt[KPL];
-    auto fetch = [&](long long r) {
-      const float *srow = scores + r * nk;
-#pragma unroll
-      for (int c = 0; c < KPL; ++c) {
-        const int j = c * 32 + lane;
-        nxt[c] = (r < rows && j < nk) ? __ldg(srow + j) : 0.f;
-      }
-    };
-    fetch(row);
-    for (; row < rows; row += stride) {
-      uint32_t u[KPL];
-#pragma unroll
-      for (int c = 0; c < KPL; ++c) u[c] = order_key(nxt[c]);
-      fetch(row + stride);
-      topk_row_regs<KPL>(u, nk, k, kv_idx + row * kmax, kmax, kv_cnt + row, smem_u32(&hist[warp][0]), lane);
-    }
-  } else {
-    if (row >= rows) return;
-    topk_row_warp(scores + row * nk, nk, k, kv_idx + row * kmax, kmax, kv_cnt + row, &hist[warp][0], lane);
-  }
+  const long long row = blockIdx.x * static_cast<long long>(kTopkWarps) + warp;
+  if (row >= rows) return;
+  topk_row_warp(scores + row * nk, nk, k, kv_idx + row * kmax, kmax, kv_cnt + row, &hist[warp][0], lane);
 }
 
 // Lane-major rows of up to 32*KPL keys in registers: lane l holds the
@@ -525,102 +500,6 @@ __global__ void __launch_bounds__(kTopkWarps * 32) topk_rows_lm_kernel(const flo
   }
 }
 
-// Rows staged in shared memory instead of registers (fewer registers, more
-// resident warps): each warp double-buffers its rows with cp.async (16-byte
-// copies when rows are 16-byte aligned, else 4-byte ones), converts its own
-// columns to order keys in place, and selects from there.
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src) {
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-
-template <int KPL>
-constexpr size_t topk_smem_bytes() {
-  return static_cast<size_t>(kTopkWarps) * (2 * KPL * 32 + 256) * sizeof(uint32_t);
-}
-
-template <int KPL>
-__global__ void __launch_bounds__(kTopkWarps * 32, KPL >= 32 ? 3 : 4) topk_rows_smem_kernel(const float *__restrict__ scores, int nk,
-                                                                         int k, int32_t *__restrict__ kv_idx,
-                                                                         int kmax, int32_t *__restrict__ kv_cnt,
-                                                                         long long rows) {
-  constexpr int ROW = KPL * 32;
-  extern __shared__ __align__(16) uint32_t tk_smem[];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  uint32_t *buf = tk_smem + warp * (2 * ROW + 256);
-  const uint32_t hist_s = smem_u32(buf + 2 * ROW);
-  const long long stride = static_cast<long long>(gridDim.x) * kTopkWarps;
-  long long row = blockIdx.x * static_cast<long long>(kTopkWarps) + warp;
-  const bool vec = (nk & 3) == 0;
-  auto fetch = [&](long long r, int slot) {
-    if (r < rows) {
-      const float *src = scores + r * nk;
-      const uint32_t dst = smem_u32(buf + slot * ROW);
-      if (vec) {
-        for (int ch = lane; ch < (nk >> 2); ch += 32) cp_async16(dst + 16u * ch, src + 4 * ch);
-      } else {
-        for (int j = lane; j < nk; j += 32) cp_async4(dst + 4u * j, src + j);
-      }
-    }
-    cp_async_commit();                         // one group per row, empty past the end
-  };
-  fetch(row, 0);
-  for (int it = 0; row < rows; row += stride, ++it) {
-    const int slot = it & 1;
-    fetch(row + stride, slot ^ 1);
-    cp_async_wait<1>();                        // this row's group has landed (the newest may not)
-    __syncwarp();
-    uint32_t *keys = buf + slot * ROW;
-#pragma unroll
-    for (int c = 0; c < KPL; ++c) {
-      const int j = c * 32 + lane;
-      if (j < nk) keys[j] = order_key(__uint_as_float(keys[j]));
-    }
-    // volatile loads: re-read per use rather than held in registers
-    const uint32_t keys_s = smem_u32(keys) + 4u * lane;
-    auto key_at = [&](int c) {
-      uint32_t x;
-      asm volatile("ld.shared.u32 %0, [%1];" : "=r"(x) : "r"(keys_s + 128u * c));
-      return x;
-    };
-    topk_row_keys<KPL>(key_at, nk, k, kv_idx + row * kmax, kmax, kv_cnt + row, hist_s, lane);
-    __syncwarp();                              // the slot is refilled two rows later
-  }
-  cp_async_wait<0>();
-}
-
-#ifndef BA_TOPK_SMEM_MIN_KPL
-#define BA_TOPK_SMEM_MIN_KPL 16
-#endif
-
-template <int KPL>
-inline cudaError_t launch_topk_smem(const float *scores, int nk, int k, int32_t *idx, int kmax, int32_t *cnt,
-                                    long long rows, int num_sms, cudaStream_t stream) {
-  const int threads = kTopkWarps * 32;
-  constexpr size_t smem = topk_smem_bytes<KPL>();
-  cudaError_t e = cudaFuncSetAttribute(topk_rows_smem_kernel<KPL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, topk_rows_smem_kernel<KPL>, threads, smem);
-  if (e != cudaSuccess) return e;
-  long long grid = (rows + kTopkWarps - 1) / kTopkWarps;
-  const long long slots = static_cast<long long>(num_sms) * (per_sm > 0 ? per_sm : 1);
-  grid = grid < slots ? grid : slots;
-  topk_rows_smem_kernel<KPL><<<static_cast<unsigned>(grid), threads, smem, stream>>>(scores, nk, k, idx, kmax, cnt,
-                                                                                     rows);
-  return cudaGetLastError();
-}
-
-#ifndef BA_TOPK_LANE_MAJOR
-#define BA_TOPK_LANE_MAJOR 1
-#endif
-
 template <int KPL>
 inline cudaError_t launch_topk_lm(const float *scores, int nk, int k, int32_t *idx, int kmax, int32_t *cnt,
                                   long long rows, int num_sms, cudaStream_t stream, bool dependent) {
@@ -641,20 +520,14 @@ inline cudaError_t launch_topk_lm(const float *scores, int nk, int k, int32_t *i
 template <int KPL>
 inline cudaError_t launch_topk_kpl(const float *scores, int nk, int k, int32_t *idx, int kmax, int32_t *cnt,
                                    long long rows, int num_sms, cudaStream_t stream, bool dependent = false) {
-  if (BA_TOPK_LANE_MAJOR && KPL > 0)
-    return launch_topk_lm<(KPL > 0 ? KPL : 8)>(scores, nk, k, idx, kmax, cnt, rows, num_sms, stream, dependent);
-  if (KPL >= BA_TOPK_SMEM_MIN_KPL) return launch_topk_smem<(KPL > 0 ? KPL : 8)>(scores, nk, k, idx, kmax, cnt, rows, num_sms, stream);
-  const int threads = kTopkWarps * 32;
-  long long grid = (rows + kTopkWarps - 1) / kTopkWarps;
-  if (KPL > 0) {                                    // persistent: every resident CTA slot once
-    int per_sm = 0;
-    const cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, topk_rows_kernel<KPL>, threads, 0);
-    if (e != cudaSuccess) return e;
-    const long long slots = static_cast<long long>(num_sms) * (per_sm > 0 ? per_sm : 1);
-    grid = grid < slots ? grid : slots;
+  if constexpr (KPL > 0) {
+    return launch_topk_lm<KPL>(scores, nk, k, idx, kmax, cnt, rows, num_sms, stream, dependent);
+  } else {
+    const long long grid = (rows + kTopkWarps - 1) / kTopkWarps;
+    topk_rows_long_kernel<<<static_cast<unsigned>(grid), kTopkWarps * 32, 0, stream>>>(scores, nk, k, idx, kmax, cnt,
+                                                                                      rows);
+    return cudaGetLastError();
   }
-  topk_rows_kernel<KPL><<<static_cast<unsigned>(grid), threads, 0, stream>>>(scores, nk, k, idx, kmax, cnt, rows);
-  return cudaGetLastError();
 }
 
 // Selection by cumulative share: keep the shortest prefix of the ranking
