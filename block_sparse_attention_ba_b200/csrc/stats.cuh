@@ -23,7 +23,8 @@
 // SPLIT or on the block size. Smaller chunks (SPLIT 4) give twelve warps per
 // SM, which ramp up and drain faster on short runs; on long runs 32 KB
 // chunks (SPLIT 1) keep fewer, longer streams in flight and reach ~0.97 of
-// HBM.
+// HBM. Once its first copies are issued, each CTA lets a programmatic
+// dependent (the score GEMM of ba_att_selector) launch as SMs free up.
 #pragma once
 
 #include "common.cuh"
