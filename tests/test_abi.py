@@ -225,3 +225,42 @@ def test_topk_arguments(lib):
     assert lib.ba_att_topk(P, 4, 16, 0, P, P, 8, None) == 1
     assert lib.ba_att_topk(P, 4, 16, 8, P, P, 7, None) == 1
     assert lib.ba_att_topk(P, 4, 4097, 8, P, P, 8, None) == 2
+
+
+C_CALLER = r"""
+#include <stdio.h>
+#include "ba_att.h"
+/* a plain C caller of the boundary: shape geometry and host-side checks only */
+int main(void) {
+  ba_att_shape s = {0};
+  s.B = 1; s.Hq = 4; s.Hkv = 2; s.N = 1000; s.N_alloc = 1024; s.d = 128; s.block = 128;
+  s.dtype = BA_DTYPE_BF16; s.sm_scale = 0.f; s.block_k = 0;
+  if (ba_att_num_blocks(&s) != 8 || ba_att_keep_count(&s, 0.5) != 4) return 1;
+  s.block_k = 64;
+  if (ba_att_num_key_blocks(&s) != 16) return 2;
+  if (ba_att_stats(&s, NULL, NULL, NULL, NULL, NULL, NULL, NULL) != BA_ERR_INVALID_ARG) return 3;
+  printf("%s\n", ba_att_status_string(BA_OK));
+  return 0;
+}
+"""
+
+
+def test_header_is_plain_c_and_links(lib):
+    # the boundary compiles as strict C99 (no C++ in the header) and a C
+    # program links against the library and calls it
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not found")
+    out = os.path.join(ROOT, "tests", "_build")
+    os.makedirs(out, exist_ok=True)
+    src, exe = os.path.join(out, "c_caller.c"), os.path.join(out, "c_caller")
+    with open(src, "w") as f:
+        f.write(C_CALLER)
+    so = os.path.abspath(api.library_path())
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    "-o", exe, src, so, "-Wl,-rpath," + os.path.dirname(so)], check=True)
+    res = subprocess.run([exe], capture_output=True, text=True)
+    assert res.returncode == 0, res.returncode
+    assert res.stdout.strip() == "BA_OK"
