@@ -24,6 +24,7 @@ import hashlib
 import json
 import os
 import statistics
+import shutil
 import subprocess
 import sys
 import time
@@ -112,11 +113,14 @@ def traffic_from_profile(sha: str):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons, sampled every 200 ms."""
+    """nvidia-smi clocks and throttle reasons, sampled every 50 ms with their
+    timestamps; summarise() keeps the samples taken inside a wall-clock window
+    (the timed region)."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
@@ -124,15 +128,22 @@ class ClockSampler:
         self.path = os.path.join("/tmp", f"ba_att_clocks_{os.getpid()}.csv")
 
     def start(self):
+        self.proc = None
+        if shutil.which("nvidia-smi") is None:
+            return
         try:
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=self.fh, stderr=subprocess.DEVNULL)
+                 "-lms", "50"], stdout=self.fh, stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
+            self.fh.close()
+            os.unlink(self.path)
 
-    def stop(self):
+    def stop(self, window=None):
+        """Stop sampling; summarise the samples inside window = (t0, t1) in
+        seconds since the epoch (all samples when none fall inside)."""
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -141,21 +152,39 @@ class ClockSampler:
         except subprocess.TimeoutExpired:
             self.proc.kill()
         self.fh.close()
-        rows = []
         with open(self.path) as f:
-            for line in f:
-                parts = [x.strip() for x in line.split(",")]
-                if len(parts) >= 9:
-                    rows.append(parts)
+            lines = f.readlines()
         os.unlink(self.path)
+        return self.summarise(lines, window)
+
+    @classmethod
+    def summarise(cls, lines, window=None):
+        import datetime
+        rows = []
+        for line in lines:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            except ValueError:
+                ts = None
+            rows.append((ts, parts[1:]))
         if not rows:
             return None
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[k] for r in rows for k in range(4) if r[5 + k].lower() == "active"})
+        inside = [r for ts, r in rows if window is not None and ts is not None and window[0] <= ts <= window[1]]
+        use = inside if inside else [r for _, r in rows]
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [v for v in (num(r[1]) for r in use) if v is not None]
+        smax = [v for v in (num(r[2]) for r in use) if v is not None]
+        reasons = sorted({cls.REASONS[k] for r in use for k in range(4) if r[5 + k].lower() == "active"})
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
-                "reasons": reasons, "samples": len(rows)}
+                "reasons": reasons, "samples": len(use), "in_timed_region": bool(inside)}
 
 
 # --------------------------------------------------------------------------- CPU oracle arms
@@ -285,19 +314,21 @@ def run_ours(args):
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)] for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)                                 # nvidia-smi is up and sampling before the timed region
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    clocks.start()
-    time.sleep(0.3)
+    wall0 = time.time()
     t_start.record(stream)
     for s_i in range(args.steps):
         step(ev[s_i])
     t_end.record(stream)
     torch.cuda.synchronize()
+    wall1 = time.time()
     if world > 1:
         dist.barrier()
-    clk = clocks.stop()
+    clk = clocks.stop(window=(wall0, wall1))
     elapsed_ms = t_start.elapsed_time(t_end)
     stage_ms = {n: float(np.mean([ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(args.steps)]))
                 for i, n in enumerate(names)}

@@ -75,3 +75,27 @@ def test_algorithmic_work_formulas():
         B, Hq, Hkv, N, d, nb, dtype = 1, 4, 2, 1024, 128, 8, "bf16"
     # Q and K read once (bf16), index lists (k + count) written once
     assert bench.selector_bytes(W, 4) == (4 + 2) * 1024 * 128 * 2 + 4 * 8 * 5 * 4
+
+
+def test_clock_summary_keeps_the_timed_window():
+    import datetime
+    base = datetime.datetime(2026, 1, 2, 3, 4, 5)
+
+    def line(dt_ms, mhz, cap="Not Active", thermal="Not Active"):
+        ts = (base + datetime.timedelta(milliseconds=dt_ms)).strftime("%Y/%m/%d %H:%M:%S.%f")[:-3]
+        return f"{ts}, 0, {mhz}, 1965, 700.5, 0x0, Not Active, {thermal}, Not Active, {cap}\n"
+
+    lines = [line(0, 1200), line(50, 1965), line(100, 1950, cap="Active"), line(150, 1965), line(400, 900,
+             thermal="Active")]
+    t0 = (base + datetime.timedelta(milliseconds=40)).timestamp()
+    t1 = (base + datetime.timedelta(milliseconds=160)).timestamp()
+    s = bench.ClockSampler.summarise(lines, (t0, t1))
+    assert s["samples"] == 3 and s["in_timed_region"] is True
+    assert s["sm_mhz"] == 1965 and s["sm_max_mhz"] == 1965
+    assert s["reasons"] == ["sw_power_cap"]
+    # no sample inside the window: every sample is summarised, and it says so
+    s = bench.ClockSampler.summarise(lines, (t1 + 10, t1 + 11))
+    assert s["samples"] == 5 and s["in_timed_region"] is False
+    assert s["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]
+    assert bench.ClockSampler.summarise([], (t0, t1)) is None
+    assert bench.ClockSampler.summarise(["garbage\n"], None) is None
