@@ -2,10 +2,12 @@
 //
 // Every entry point validates its arguments on the host first and launches
 // nothing on a bad argument. Launches are asynchronous on the caller's
-// stream; no call synchronises except ba_att_get_device_error. The library
-// allocates no device memory: its global state is the device error word (a
-// __device__ variable), a cache of per-device SM counts, and per device the
-// two copy streams and events of the host-buffer pipeline.
+// stream; no call synchronises except ba_att_get_device_error. No call
+// allocates device memory: the global state is the device error word (a
+// __device__ variable), a cache of per-device SM counts, per device the two
+// copy streams and events of the host-buffer pipeline, and the static
+// scratch of ba_att_forward_host_noalloc, a __device__ array that the module
+// reserves on every device where it loads, whichever entry points are used.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -786,8 +788,9 @@ ba_status ba_att_forward_host_noalloc(const ba_att_shape *s, double keep, int32_
   PipeLayout L;
   ba_status st = validate_host_call(s, keep, split_block, 0, Q, K, V, O, LSE, &L);
   if (st != BA_OK) return st;
-  // the widest chunk whose workspace fits the static scratch
-  int chunk = s->Hkv;
+  // the chunk ba_att_forward_host would pick (about 1024 query tiles, so that
+  // copies and compute overlap), narrowed until its workspace fits the scratch
+  int chunk = auto_chunk(s);
   for (; chunk >= 1; --chunk) {
     if (!pipe_layout(s, keep, split_block, chunk, &L)) return BA_ERR_INVALID_ARG;
     if (L.total <= static_cast<size_t>(BA_ATT_STATIC_SCRATCH_BYTES)) break;

@@ -182,6 +182,96 @@ def _gen_video_field(w: Workload):
     return out[0], out[1], out[2], {"grid": list(w.grid)}
 
 
+def make_inputs_device(w: Workload | str, device, **overrides):
+    """The same recipe drawn on a CUDA device with torch's generator, for
+    timing runs at full size: (Q, K, V, meta) as bf16 (or fp32) device
+    tensors. The structure (shared direction per KV head, planted x3 key
+    blocks, needle, smoothed video field, zero padding rows, split point)
+    matches make_inputs; the values differ, since the generator does. Parity
+    tests use make_inputs, whose arrays the oracle also reads."""
+    import torch
+    import torch.nn.functional as F
+
+    if isinstance(w, str):
+        w = WORKLOADS[w]
+    if overrides:
+        if "N" in overrides and "N_alloc" not in overrides:
+            overrides["N_alloc"] = overrides["N"]
+        w = w.with_(**overrides)
+    dev = torch.device(device)
+    g = torch.Generator(device=dev)
+    g.manual_seed(1_000_003 * w.seed + 17)
+    meta_rng = np.random.default_rng([w.seed, 1])
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+
+    def randn(*shape):
+        return torch.randn(*shape, generator=g, device=dev, dtype=torch.float32)
+
+    meta = {}
+    if w.kind == "video_field":
+        T, Hh, Ww = w.grid
+        sigma = 3.0
+        radius = int(math.ceil(4 * sigma))
+        t = torch.arange(-radius, radius + 1, device=dev, dtype=torch.float32)
+        kern = torch.exp(-0.5 * (t / sigma) ** 2)
+        kern = (kern / kern.sum()).view(1, 1, -1)
+        out = []
+        for H in (w.Hq, w.Hkv, w.Hkv):
+            f = randn(H * w.d, T, Hh, Ww)
+            for ax in (1, 2, 3):                   # separable smoothing along t, h, w
+                x = f.movedim(ax, -1)
+                shp = x.shape
+                x = F.conv1d(x.reshape(-1, 1, shp[-1]), kern, padding=radius).reshape(shp)
+                f = x.movedim(-1, ax)
+            f = f / (f.reshape(H * w.d, -1).std(dim=-1).view(-1, 1, 1, 1) + 1e-12)
+            f = f + randn(*f.shape)
+            X = torch.zeros((1, H, w.N_alloc, w.d), device=dev, dtype=tdt)
+            X[0, :, :T * Hh * Ww] = f.reshape(H, w.d, -1).transpose(1, 2).to(tdt)
+            out.append(X)
+        Q, K, V = out
+        meta["grid"] = list(w.grid)
+    else:
+        Q = randn(w.B, w.Hq, w.N_alloc, w.d)
+        K = randn(w.B, w.Hkv, w.N_alloc, w.d)
+        V = randn(w.B, w.Hkv, w.N_alloc, w.d)
+        if w.kind == "shared_dir":
+            group = w.Hq // w.Hkv
+            u = randn(w.B, w.Hkv, w.d)
+            u = u / u.norm(dim=-1, keepdim=True)
+            Q += 0.5 * u.repeat_interleave(group, dim=1)[:, :, None, :]
+            K += 0.5 * u[:, :, None, :]
+            n_planted = max(1, int(round(0.05 * w.nb)))
+        else:
+            n_planted = 2
+        for bb in range(w.B):
+            for gg in range(w.Hkv if w.kind == "shared_dir" else 1):
+                for j in np.sort(meta_rng.choice(w.nb, size=n_planted, replace=False)):
+                    rows = slice(j * w.block, min(w.N, (j + 1) * w.block))
+                    if w.kind == "shared_dir":
+                        K[bb, gg, rows] *= 3.0
+                    else:
+                        K[:, :, rows] *= 3.0
+        if w.needle:
+            span = min(512, w.N)
+            start = int(meta_rng.integers(0, w.N - span + 1))
+            rows = np.sort(meta_rng.choice(w.N, size=min(8, w.N), replace=False))
+            wv = randn(w.d)
+            wv = wv / wv.norm()
+            a = 2.0 * w.d ** 0.25
+            K[:, :, start:start + span] += a * wv
+            Q[:, :, torch.as_tensor(rows, device=dev)] += a * wv
+            meta.update(needle_span=[start, start + span], needle_rows=rows.tolist())
+        if w.N_alloc > w.N:
+            Q[:, :, w.N:] = 0
+            K[:, :, w.N:] = 0
+            V[:, :, w.N:] = 0
+        Q, K, V = Q.to(tdt), K.to(tdt), V.to(tdt)
+    if w.split:
+        meta["split_block"] = int(meta_rng.integers(1, w.nk))
+    meta["workload"] = w
+    return Q, K, V, meta
+
+
 def make_inputs(w: Workload | str, **overrides):
     """Draw (Q, K, V, meta) for a workload; float32 arrays rounded to w.dtype.
 

@@ -24,9 +24,12 @@
  *    block i covers rows [i*b, min(N, (i+1)*b)) (the last may be ragged).
  *  - Grouped-query attention: query head h uses KV head h / (Hq / Hkv).
  *  - Memory: the caller allocates and owns every buffer. Device pointers are
- *    CUDA device (or managed) memory, 16-byte aligned. The library allocates
- *    no device memory; its global state is one device-side error word and,
- *    per device, the two copy streams and events of ba_att_forward_host.
+ *    CUDA device (or managed) memory, 16-byte aligned. No call allocates
+ *    device memory; the global state is one device-side error word, per
+ *    device the two copy streams and events of ba_att_forward_host, and the
+ *    static scratch of ba_att_forward_host_noalloc: a __device__ array of
+ *    BA_ATT_STATIC_SCRATCH_BYTES (512 MiB) that the library's device code
+ *    reserves on every device where it is loaded, whichever calls are made.
  *  - Streams: every call is asynchronous on `stream` (NULL = legacy default
  *    stream) and never synchronises, except ba_att_get_device_error.
  *  - Errors: arguments are checked on the host before anything is launched;
@@ -407,11 +410,14 @@ ba_status ba_att_forward_host(const ba_att_shape *shape, double keep, int32_t sp
  * the same computation.
  *
  * The workspace is a static __device__ array of BA_ATT_STATIC_SCRATCH_BYTES
- * inside the library (reserved once, when the library's device code is
- * loaded; nothing is allocated at call time). The chunk is the largest number
- * of KV heads whose workspace (ba_att_forward_host_workspace) fits it;
- * BA_ERR_UNSUPPORTED when one KV head per chunk does not fit (e.g. 32 query
- * heads per KV head at N = 128K with a split). Results are bit-identical to
+ * inside the library (reserved on every device where the library's device
+ * code is loaded, at load time, whether or not this call is ever made;
+ * nothing is allocated at call time). The chunk is the one
+ * ba_att_forward_host picks for kv_heads_per_chunk <= 0 (about 1024 query
+ * tiles, so that copies overlap compute), narrowed until its workspace
+ * (ba_att_forward_host_workspace) fits the scratch; BA_ERR_UNSUPPORTED when
+ * one KV head per chunk does not fit (e.g. 32 query heads per KV head at
+ * N = 128K with a split). Results are bit-identical to
  * ba_att_forward_host. The scratch is shared by all calls on a device: each
  * call starts on `stream` only after the previous call on the scratch has
  * ended, whatever stream that call used.

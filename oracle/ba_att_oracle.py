@@ -261,16 +261,22 @@ def mass_share_before(R, idx, cnt):
 def near_tie_mask(S, k: int, rel: float = 1e-3):
     """Blocks whose score lies within ``rel`` of the selection threshold.
 
-    The threshold is the k-th ranked block of the row. Closeness is measured
-    on the normalised map A^ (a relative band on probabilities):
-    |A^_ij - A^_thr| <= rel * A^_thr, which is |exp(S~_ij - S~_thr) - 1| <= rel
-    because A^ is proportional to exp(S~) within a row. Blocks in this band
-    may legitimately fall either side of the cut under different rounding.
+    The threshold is the k-th ranked block of the row. "Within rel of the
+    threshold" is read two ways, and a block counts as a near-tie only when
+    it is close in both (the narrower band):
+      - on the corrected score itself: |S~_ij - S~_thr| <= rel * |S~_thr|;
+      - on the normalised map A^ (a relative band on probabilities):
+        |A^_ij - A^_thr| <= rel * A^_thr, i.e. |exp(S~_ij - S~_thr) - 1| <= rel,
+        because A^ is proportional to exp(S~) within a row.
+    Blocks in this band may legitimately fall either side of the cut under
+    different rounding; outside it the kept set is fixed.
     """
     S = np.asarray(S, dtype=np.float64)
     srt = -np.sort(-S, axis=-1)
     thr = srt[..., min(k, S.shape[-1]) - 1][..., None]
-    return np.abs(np.expm1(S - thr)) <= rel
+    in_map_band = np.abs(np.expm1(S - thr)) <= rel
+    in_score_band = np.abs(S - thr) <= rel * np.abs(thr)
+    return in_map_band & in_score_band
 
 
 # ---------------------------------------------------------------------------

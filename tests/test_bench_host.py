@@ -99,3 +99,27 @@ def test_clock_summary_keeps_the_timed_window():
     assert s["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]
     assert bench.ClockSampler.summarise([], (t0, t1)) is None
     assert bench.ClockSampler.summarise(["garbage\n"], None) is None
+
+
+def test_clock_sampler_names_the_gpu_by_pci_bus_id(monkeypatch):
+    # With CUDA_VISIBLE_DEVICES=3 the process sees that GPU as CUDA device 0,
+    # while nvidia-smi's index 0 is another GPU; the bus id names the right one.
+    monkeypatch.setenv("CUDA_VISIBLE_DEVICES", "3")
+
+    class Props:
+        pci_domain_id, pci_bus_id, pci_device_id = 0, 0x9B, 0
+    gid = bench.smi_gpu_id(Props)
+    assert gid == "00000000:9B:00.0"
+    cmd = bench.ClockSampler(gid).command()
+    assert f"--id={gid}" in cmd and "--id=0" not in cmd and "--id=3" not in cmd
+    assert any(a.startswith("--query-gpu=") and "pci.bus_id" in a for a in cmd)
+
+
+def test_step_config_names_the_step_form():
+    from block_sparse_attention_ba_b200.workloads import WORKLOADS
+    single = bench.step_config(WORKLOADS["sweep_32k"], 0.5, 128, None, 1)
+    assert "split" not in single["workload"] and "split_block" not in single
+    assert single["workload"].endswith("selector(stats+scores+top-k)+sparse_fwd")
+    split = bench.step_config(WORKLOADS["extreme_128k"], 0.5, 512, 77, 1)
+    assert split["split_block"] == 77 and "sparse_fwd_merge" in split["workload"]
+    assert bench.LAUNCHES_PER_STEP[False] == 4 and bench.LAUNCHES_PER_STEP[True] == 6

@@ -241,6 +241,15 @@ def test_near_tie_band():
     # k=3: ranking 3 (2.0), 4 (1.002), 2 (1.0005) -> threshold 1.0005
     nt = O.near_tie_mask(row, 3)
     assert nt[0].tolist() == [False, True, True, False, False]
+    # the band is the narrower of the score-relative and the map-relative one:
+    # near a small threshold the score band decides (0.1005 is 5e-4 above 0.1,
+    # inside the map band but outside 1e-3 * 0.1) ...
+    row = np.array([[3.0, 0.1, 0.1005, 0.10005, -1.0]])      # k = 4: threshold 0.1
+    assert O.near_tie_mask(row, 4)[0].tolist() == [False, True, False, True, False]
+    # ... and near a large one the map band does (100.05 is within 1e-3 * 100
+    # of 100 but exp(0.05) - 1 = 0.051 on the map)
+    row = np.array([[200.0, 100.0, 100.05, 100.0004, 0.0]])   # k = 4: threshold 100
+    assert O.near_tie_mask(row, 4)[0].tolist() == [False, True, False, True, False]
 
 
 # ------------------------------------------------------------------ attention
@@ -398,6 +407,19 @@ def test_select_by_mass():
     idx, cnt = O.select_by_mass(R, 1e-12)
     assert (cnt == 1).all() and (idx[..., 0] == R.argmax(-1)).all()
     assert (O.select_by_mass(R, 1.0)[1] == R.shape[-1]).all()
+
+
+def test_select_by_mass_hand_worked_row():
+    # scores ln 1, ln 4, ln 1, ln 2 (+ any constant): the normalised map is
+    # exp(S) / sum = 1/8, 1/2, 1/8, 1/4, so the ranking is 1, 3, 0, 2 (the
+    # two 1/8 shares tie and go to the lower index) with running shares
+    # 1/2, 3/4, 7/8, 1
+    for shift in (0.0, 7.3, -40.0):
+        R = np.log(np.array([[[1.0, 4.0, 1.0, 2.0]]])) + shift
+        for tau, want in ((0.4, [1]), (0.6, [1, 3]), (0.8, [0, 1, 3]), (0.95, [0, 1, 2, 3])):
+            idx, cnt = O.select_by_mass(R, tau)
+            assert int(cnt[0, 0]) == len(want), (shift, tau)
+            assert idx[0, 0, : len(want)].tolist() == want and (idx[0, 0, len(want):] == -1).all()
 
 
 def test_merge_edge_cases():
