@@ -54,6 +54,8 @@ _SIGS = {
     "ba_att_complement_lists": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _I32, _P, _P, _I32, _P]),
     "ba_att_sparse_fwd": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _P, _P, _P, _I32, _P, _I32, _P, _P]),
     "ba_att_merge_lse": (ctypes.c_int, [ctypes.c_int64, _I32, _I32, _I32, _P, _P, _P, _P, _P, _P, _P]),
+    "ba_att_sparse_fwd_rows": (ctypes.c_int, [ctypes.POINTER(CShape), _I32, _I32, _P, _P, _P, _P, _P, _I32, _P, _P,
+                                               _P, _I32, _P, _P]),
     "ba_att_sparse_fwd_merge": (ctypes.c_int, [ctypes.POINTER(CShape), _P, _P, _P, _P, _P, _I32, _P, _P, _P, _I32, _P,
                                                 _P]),
     "ba_att_get_device_error": (ctypes.c_int, [_P, ctypes.POINTER(ctypes.c_uint32)]),
@@ -331,6 +333,63 @@ def sparse_fwd_merge(Q, K, V, idx, cnt, shape: Shape, O_prev, L_prev, out=None, 
         ctypes.byref(shape.c()), _dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), _dev(idx, "kv_idx"), _dev(cnt, "kv_cnt"),
         idx.shape[-1], _dev(O_prev, "O_prev"), _dev(L_prev, "L_prev"), _dev(O, "O"), _TORCH_DT[O.dtype],
         _dev(LSE, "LSE"), _stream(Q)))
+    return out
+
+
+def _rows_view(t: torch.Tensor, name: str, q_rows: int, d: int | None) -> int:
+    """Row stride of a [B, H, rows, d] (or [B, H, rows]) CUDA tensor that is
+    either contiguous or a slice of rows of a contiguous one (heads at a fixed
+    stride of whole rows); the call reads and writes through its data pointer."""
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    inner = 1 if d is None else d
+    st = t.stride()
+    if (d is not None and st[3] != 1) or st[2] != inner or st[1] % inner != 0:
+        raise ValueError(f"{name} must be contiguous or a slice of rows of a contiguous tensor")
+    stride = st[1] // inner
+    if stride < q_rows or st[0] != t.shape[1] * st[1]:
+        raise ValueError(f"{name} must be contiguous or a slice of rows of a contiguous tensor")
+    return stride
+
+
+def sparse_fwd_rows(Qr, K, V, idx, cnt, shape: Shape, q_rows: int | None = None, O_prev=None, L_prev=None,
+                    out=None, out_dtype=None):
+    """Attention for one range of query rows only (ba_att_sparse_fwd_rows) -> (O, LSE).
+
+    Qr [B, Hq, R, d] holds the range's rows: a contiguous tensor, or a slice of
+    rows of a full one (e.g. Q[:, :, r0:r0 + R], r0 a multiple of 8), whose head
+    stride becomes the call's row stride; q_rows defaults to R. K, V and `shape`
+    describe the keys. idx/cnt list key blocks per query block of the range
+    ([B, Hq, ceil(q_rows / block), kmax]). With (O_prev, L_prev), fp32, laid out
+    like Qr, the result is merged with that cached partial in the epilogue; out
+    (laid out like Qr, e.g. slices of full O/LSE tensors) may be (O_prev, L_prev)
+    for an in-place fp32 merge."""
+    lib = load_library()
+    B, Hq, R, d = Qr.shape
+    q_rows = R if q_rows is None else q_rows
+    q_stride = _rows_view(Qr, "Q", q_rows, d)
+    if (O_prev is None) != (L_prev is None):
+        raise ValueError("pass both O_prev and L_prev, or neither")
+    if O_prev is not None:
+        if O_prev.dtype != torch.float32 or L_prev.dtype != torch.float32:
+            raise TypeError("O_prev and L_prev must be float32")
+        if _rows_view(O_prev, "O_prev", q_rows, d) != q_stride or _rows_view(L_prev, "L_prev", q_rows, None) != q_stride:
+            raise ValueError("O_prev and L_prev must have Q's row stride")
+    if out is None:
+        odt = Qr.dtype if out_dtype is None else out_dtype
+        full = (torch.empty((B, Hq, q_stride, d), device=Qr.device, dtype=odt),
+                torch.empty((B, Hq, q_stride), device=Qr.device, dtype=torch.float32))
+        out = (full[0][:, :, :R], full[1][:, :, :R])
+    O, LSE = out
+    if _rows_view(O, "O", q_rows, d) != q_stride or _rows_view(LSE, "LSE", q_rows, None) != q_stride:
+        raise ValueError("O and LSE must have Q's row stride")
+    null = ctypes.c_void_p(0)
+    ptr = lambda t: ctypes.c_void_p(t.data_ptr())
+    _check("ba_att_sparse_fwd_rows", lib.ba_att_sparse_fwd_rows(
+        ctypes.byref(shape.c()), int(q_rows), int(q_stride), ptr(Qr), _dev(K, "K"), _dev(V, "V"),
+        _dev(idx, "kv_idx"), _dev(cnt, "kv_cnt"), idx.shape[-1],
+        null if O_prev is None else ptr(O_prev), null if L_prev is None else ptr(L_prev),
+        ptr(O), _TORCH_DT[O.dtype], ptr(LSE), _stream(Qr)))
     return out
 
 

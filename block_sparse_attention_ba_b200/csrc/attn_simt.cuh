@@ -36,7 +36,8 @@ template <typename T, typename TO, int D, bool MERGE>
 __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(
     const T *__restrict__ Q, const T *__restrict__ K, const T *__restrict__ V, const int32_t *__restrict__ kv_idx,
     const int32_t *__restrict__ kv_cnt, int kmax, TO *O, float *LSE, const float *O_prev, const float *L_prev, int Hq,
-    int Hkv, int N, int N_alloc, int block, int nb, int kblock, int nk, int subs, float scale_log2) {
+    int Hkv, int N, int N_alloc, int Nq, int q_stride, int block, int nb, int kblock, int nk, int subs,
+    float scale_log2) {
   constexpr int DPL = D / 32;
   constexpr int RPW = kSimtRows / (kSimtThreads / 32);      // rows per warp
   __shared__ float q_s[kSimtRows][D];
@@ -47,12 +48,12 @@ __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(
   const int i = blockIdx.x / subs, sub = blockIdx.x % subs;
   const int g = h / (Hq / Hkv);
   const int row0 = i * block + sub * kSimtRows;
-  const int row_end = min(min(i * block + block, N), row0 + kSimtRows);
+  const int row_end = min(min(i * block + block, Nq), row0 + kSimtRows);
   if (row0 >= row_end) return;
   const int nrows = row_end - row0;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-  const long long qhead = (static_cast<long long>(b) * Hq + h) * N_alloc;
+  const long long qhead = (static_cast<long long>(b) * Hq + h) * q_stride;
   const long long khead = (static_cast<long long>(b) * Hkv + g) * N_alloc;
   for (int e = tid; e < kSimtRows * D; e += kSimtThreads) {
     const int r = e / D, m = e % D;
@@ -147,18 +148,20 @@ __global__ void __launch_bounds__(kSimtThreads) attn_simt_kernel(
   }
 }
 
+// Nq query rows per head at a stride of q_stride rows (Nq = N, q_stride =
+// N_alloc for a full call); keys: N valid rows at a stride of N_alloc.
 template <typename T, typename TO, int D, bool MERGE = false>
 cudaError_t launch_attn_simt(const T *Q, const T *K, const T *V, const int32_t *idx, const int32_t *cnt, int kmax, TO *O,
-                             float *LSE, int B, int Hq, int Hkv, int N, int N_alloc, int block, int kblock,
-                             float sm_scale, cudaStream_t stream, const float *O_prev = nullptr,
+                             float *LSE, int B, int Hq, int Hkv, int N, int N_alloc, int Nq, int q_stride, int block,
+                             int kblock, float sm_scale, cudaStream_t stream, const float *O_prev = nullptr,
                              const float *L_prev = nullptr) {
-  const int nb = (N + block - 1) / block, nk = (N + kblock - 1) / kblock;
+  const int nb = (Nq + block - 1) / block, nk = (N + kblock - 1) / kblock;
   const int subs = (block + kSimtRows - 1) / kSimtRows;
   dim3 grid(static_cast<unsigned>(nb * subs), Hq, B);
   const float scale_log2 = sm_scale * 1.4426950408889634f;
   attn_simt_kernel<T, TO, D, MERGE><<<grid, kSimtThreads, 0, stream>>>(Q, K, V, idx, cnt, kmax, O, LSE, O_prev, L_prev,
-                                                                    Hq, Hkv, N, N_alloc, block, nb, kblock, nk, subs,
-                                                                    scale_log2);
+                                                                    Hq, Hkv, N, N_alloc, Nq, q_stride, block, nb,
+                                                                    kblock, nk, subs, scale_log2);
   return cudaGetLastError();
 }
 

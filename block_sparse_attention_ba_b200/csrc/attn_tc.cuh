@@ -1,5 +1,6 @@
 // attn_tc.cuh — K8: block-sparse attention forward on the 5th-generation
-// tensor cores (tcgen05 + TMEM), bf16 inputs, d = 64 or 128, block = 128.
+// tensor cores (tcgen05 + TMEM), bf16 inputs, d = 64 or 128, query blocks of
+// 64, 128 or 256 rows, key blocks of 64, 128 or 256 rows.
 //
 // Operator: "Efficient Long-Context Modeling in DLMs via Block Approximate
 // Sparse Attention" (abstract; Figure 4) — bidirectional attention over the
@@ -136,6 +137,10 @@ __device__ __forceinline__ void exp_pack_store(const uint32_t (&sr)[2][32], floa
   }
 }
 
+// Query rows: Nq valid rows per head at a stride of q_stride rows (Q, O, LSE,
+// O_prev, L_prev), in nq blocks of `block`; keys: N valid rows per KV head
+// (the K/V tensor maps). A full call has Nq = N; a call for one range of
+// query rows (ba_att_sparse_fwd_rows) has its own Nq and stride.
 // TO: output element type, bf16 (final output) or float (a partial that is
 // merged later, so the merged result is rounded only once).
 // MERGE: the epilogue merges this span's result with an earlier fp32 partial
@@ -147,8 +152,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const int32_t *__restrict__ kv_idx,
                    const int32_t *__restrict__ kv_cnt, int kmax, TO *O, float *LSE, const float *O_prev,
-                   const float *L_prev, int Hq, int Hkv, int N, int N_alloc, int nq, int block, int nk,
-                   int kblock, float scale_log2) {
+                   const float *L_prev, int Hq, int Hkv, int N, int Nq, int q_stride, int nq, int block,
+                   int nk, int kblock, float scale_log2) {
   extern __shared__ uint8_t dyn_smem[];
   __shared__ Ctl ctl;
   const uint32_t smem_base = (smem_u32(dyn_smem) + 1023u) & ~1023u;
@@ -162,12 +167,18 @@ __global__ void __launch_bounds__(kThreads, 2)
   // rows (128 or 256) is block/128 query tiles, which share its list; a key
   // block of `kblock` rows (64, 128 or 256) is kblock/64 key halves.
   const int G = Hq / Hkv;
-  const int qpb = block >> 7, hpe_log2 = kblock == 256 ? 2 : (kblock == 128 ? 1 : 0), hpe = 1 << hpe_log2;
+  const int qpb = block >= kTileRows ? block >> 7 : 1;
+  const int hpe_log2 = kblock == 256 ? 2 : (kblock == 128 ? 1 : 0), hpe = 1 << hpe_log2;
   long long tile = blockIdx.x;
   const int hg = static_cast<int>(tile % G);
   tile /= G;
   const int it = static_cast<int>(tile % (static_cast<long long>(nq) * qpb));   // query tile within the head
   const int i = it / qpb;                                                        // its query block
+  // the tile's first query row and its rows of this block: 128, or 64 for a
+  // 64-row block, whose tile also loads (and computes, but never stores) the
+  // next block's 64 rows
+  const int tile_row0 = i * block + (it % qpb) * kTileRows;
+  const int tile_rows = block < kTileRows ? block : kTileRows;
   tile /= static_cast<long long>(nq) * qpb;
   const int g = static_cast<int>(tile % Hkv);
   const int b = static_cast<int>(tile / Hkv);
@@ -212,7 +223,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       tma_prefetch_desc(&tm_q);
       mbar_arrive_expect_tx(bar(Q_FULL), DM::kTileBytes);
 #pragma unroll
-      for (int sp = 0; sp < DM::kSpans; ++sp) tma_load_3d(&tm_q, sQ + sp * kHalfBytes, bar(Q_FULL), 64 * sp, it * kTileRows, qz);
+      for (int sp = 0; sp < DM::kSpans; ++sp) tma_load_3d(&tm_q, sQ + sp * kHalfBytes, bar(Q_FULL), 64 * sp, tile_row0, qz);
     }
     int issued = -1;                    // last half-block index u loaded
     bool bad_index = false, bad_order = false;
@@ -292,8 +303,9 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int row = threadIdx.x;                       // TMEM lane = query row in tile
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
     const uint32_t tS = tmem + lane_off + kColS, tO = tmem + lane_off + kColO;
-    const int qrow = it * kTileRows + row;
-    const long long orow = static_cast<long long>(qz) * N_alloc + qrow;
+    const int qrow = tile_row0 + row;
+    const bool owned = row < tile_rows && qrow < Nq;   // a row of this tile's block, and a token
+    const long long orow = static_cast<long long>(qz) * q_stride + qrow;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     int n_keys = 0;
@@ -370,7 +382,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       const float inv = has ? 1.f / l : 0.f;
       const float lse_new = has ? (m_used + __log2f(l)) * 0.6931471805599453f : -INFINITY;
       MergeWeights mw{0.f, 0.f, 0.f, lse_new};
-      if constexpr (MERGE) mw = merge_weights(qrow < N ? L_prev[orow] : -INFINITY, lse_new);
+      if constexpr (MERGE) mw = merge_weights(owned ? L_prev[orow] : -INFINITY, lse_new);
       const float *prev = MERGE ? O_prev + orow * D : nullptr;
       uint4 *dst = reinterpret_cast<uint4 *>(O + orow * D);
 #pragma unroll
@@ -383,7 +395,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
           for (int c = 0; c < 32; ++c) orr[c] = 0u;
         }
-        if (qrow < N) {
+        if (owned) {
           float o[32];
 #pragma unroll
           for (int c = 0; c < 32; ++c) o[c] = __uint_as_float(orr[c]) * inv;
@@ -410,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           }
         }
       }
-      if (qrow < N) LSE[orow] = mw.lse;
+      if (owned) LSE[orow] = mw.lse;
     }
     tc_fence_before();
   }

@@ -106,8 +106,8 @@ bool make_head_map(CUtensorMap *map, const void *ptr, int d, int N_valid, int N_
 
 bool use_tensor_core_path(const ba_att_shape *s) {
   const int kb = s->block_k > 0 ? s->block_k : s->block;
-  return s->dtype == BA_DTYPE_BF16 && (s->d == 128 || s->d == 64) && (s->block == 128 || s->block == 256) &&
-         (kb == 64 || kb == 128 || kb == 256);
+  return s->dtype == BA_DTYPE_BF16 && (s->d == 128 || s->d == 64) &&
+         (s->block == 64 || s->block == 128 || s->block == 256) && (kb == 64 || kb == 128 || kb == 256);
 }
 
 __global__ void bounded_wait_selftest_kernel(unsigned long long limit_ns) {
@@ -383,12 +383,16 @@ ba_status ba_att_split_lists(const ba_att_shape *s, int32_t split_block, const i
 namespace {
 
 // Attention over the listed blocks; with O_prev/L_prev (both non-null) the
-// epilogue merges the result with that earlier fp32 partial.
+// epilogue merges the result with that earlier fp32 partial. Query side: Nq
+// rows per head at a stride of q_stride rows (Nq = N, q_stride = N_alloc for
+// the whole sequence).
 ba_status sparse_fwd_impl(const ba_att_shape *s, const void *Q, const void *K, const void *V, const int32_t *kv_idx,
                           const int32_t *kv_cnt, int32_t kmax, void *O, int32_t o_dtype, float *LSE,
-                          const float *O_prev, const float *L_prev, ba_stream_t stream) {
+                          const float *O_prev, const float *L_prev, int Nq, int q_stride, ba_stream_t stream) {
   ba_status st = check_shape(s);
   if (st != BA_OK) return st;
+  if (Nq < 1 || q_stride < Nq) return BA_ERR_INVALID_ARG;
+  if (static_cast<long long>(s->B) * s->Hq * q_stride > (1LL << 36)) return BA_ERR_UNSUPPORTED;
   if (!Q || !K || !V || !kv_idx || !kv_cnt || !O || !LSE) return BA_ERR_INVALID_ARG;
   if (o_dtype != s->dtype && o_dtype != BA_DTYPE_F32) return BA_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(kv_idx) || !aligned16(kv_cnt) || !aligned16(O) ||
@@ -397,18 +401,20 @@ ba_status sparse_fwd_impl(const ba_att_shape *s, const void *Q, const void *K, c
   const bool merge = O_prev != nullptr;
   if (merge && (!aligned16(O_prev) || (reinterpret_cast<uintptr_t>(L_prev) & 3u))) return BA_ERR_MISALIGNED;
   if (kmax < 1) return BA_ERR_INVALID_ARG;
-  const int nb = nblocks(s);
+  const int nb = (Nq + s->block - 1) / s->block;        // query blocks of this call
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   const float scale = effective_scale(s);
   const bool out_f32 = (o_dtype == BA_DTYPE_F32);
   if (use_tensor_core_path(s)) {
     CUtensorMap mq, mk, mv;
-    if (!make_head_map(&mq, Q, s->d, s->N, s->N_alloc, static_cast<long long>(s->B) * s->Hq, tc::kTileRows) ||
+    if (!make_head_map(&mq, Q, s->d, Nq, q_stride, static_cast<long long>(s->B) * s->Hq, tc::kTileRows) ||
         !make_head_map(&mk, K, s->d, s->N, s->N_alloc, static_cast<long long>(s->B) * s->Hkv, tc::kKvBoxRows) ||
         !make_head_map(&mv, V, s->d, s->N, s->N_alloc, static_cast<long long>(s->B) * s->Hkv, tc::kKvBoxRows))
       return BA_ERR_CUDA;
-    // one CTA per 128-row query tile (a 256-row block is two tiles sharing its list)
-    const long long tiles = static_cast<long long>(s->B) * s->Hq * nb * (s->block / tc::kTileRows);
+    // one CTA per 128-row query tile (a 256-row block is two tiles sharing its
+    // list; a 64-row block is one tile whose second half is not stored)
+    const long long tiles =
+        static_cast<long long>(s->B) * s->Hq * nb * (s->block >= tc::kTileRows ? s->block / tc::kTileRows : 1);
     if (tiles > 0x7FFFFFFFLL) return BA_ERR_UNSUPPORTED;
     const float sl2 = scale * 1.4426950408889634f;
     const uint32_t smem = tc::dyn_smem_bytes(s->d);
@@ -416,8 +422,8 @@ ba_status sparse_fwd_impl(const ba_att_shape *s, const void *Q, const void *K, c
       cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
       if (e != cudaSuccess) return BA_ERR_CUDA;
       kernel<<<static_cast<unsigned>(tiles), tc::kThreads, smem, cs>>>(
-          mq, mk, mv, kv_idx, kv_cnt, kmax, out, LSE, O_prev, L_prev, s->Hq, s->Hkv, s->N, s->N_alloc, nb, s->block,
-          nkblocks(s), kblock(s), sl2);
+          mq, mk, mv, kv_idx, kv_cnt, kmax, out, LSE, O_prev, L_prev, s->Hq, s->Hkv, s->N, Nq, q_stride, nb,
+          s->block, nkblocks(s), kblock(s), sl2);
       return from_cuda(cudaGetLastError());
     };
     float *of = static_cast<float *>(O);
@@ -437,12 +443,12 @@ ba_status sparse_fwd_impl(const ba_att_shape *s, const void *Q, const void *K, c
 #define BA_SIMT(T, TO, DD)                                                                                           \
   (merge ? launch_attn_simt<T, TO, DD, true>(static_cast<const T *>(Q), static_cast<const T *>(K),                   \
                                              static_cast<const T *>(V), kv_idx, kv_cnt, kmax, static_cast<TO *>(O), \
-                                             LSE, s->B, s->Hq, s->Hkv, s->N, s->N_alloc, s->block, kblock(s), scale, \
-                                             cs, O_prev, L_prev)                                                      \
+                                             LSE, s->B, s->Hq, s->Hkv, s->N, s->N_alloc, Nq, q_stride, s->block,   \
+                                             kblock(s), scale, cs, O_prev, L_prev)                                   \
          : launch_attn_simt<T, TO, DD, false>(static_cast<const T *>(Q), static_cast<const T *>(K),                  \
                                               static_cast<const T *>(V), kv_idx, kv_cnt, kmax, static_cast<TO *>(O), \
-                                              LSE, s->B, s->Hq, s->Hkv, s->N, s->N_alloc, s->block, kblock(s), scale, \
-                                              cs))
+                                              LSE, s->B, s->Hq, s->Hkv, s->N, s->N_alloc, Nq, q_stride, s->block,  \
+                                              kblock(s), scale, cs))
   if (s->dtype == BA_DTYPE_BF16) {
     if (out_f32)
       e = s->d == 128 ? BA_SIMT(__nv_bfloat16, float, 128) : BA_SIMT(__nv_bfloat16, float, 64);
@@ -462,14 +468,26 @@ extern "C" {
 ba_status ba_att_sparse_fwd(const ba_att_shape *s, const void *Q, const void *K, const void *V, const int32_t *kv_idx,
                             const int32_t *kv_cnt, int32_t kmax, void *O, int32_t o_dtype, float *LSE,
                             ba_stream_t stream) {
-  return sparse_fwd_impl(s, Q, K, V, kv_idx, kv_cnt, kmax, O, o_dtype, LSE, nullptr, nullptr, stream);
+  if (s == nullptr) return BA_ERR_INVALID_ARG;
+  return sparse_fwd_impl(s, Q, K, V, kv_idx, kv_cnt, kmax, O, o_dtype, LSE, nullptr, nullptr, s->N, s->N_alloc,
+                         stream);
 }
 
 ba_status ba_att_sparse_fwd_merge(const ba_att_shape *s, const void *Q, const void *K, const void *V,
                                   const int32_t *kv_idx, const int32_t *kv_cnt, int32_t kmax, const float *O_prev,
                                   const float *LSE_prev, void *O, int32_t o_dtype, float *LSE, ba_stream_t stream) {
-  if (!O_prev || !LSE_prev) return BA_ERR_INVALID_ARG;
-  return sparse_fwd_impl(s, Q, K, V, kv_idx, kv_cnt, kmax, O, o_dtype, LSE, O_prev, LSE_prev, stream);
+  if (s == nullptr || !O_prev || !LSE_prev) return BA_ERR_INVALID_ARG;
+  return sparse_fwd_impl(s, Q, K, V, kv_idx, kv_cnt, kmax, O, o_dtype, LSE, O_prev, LSE_prev, s->N, s->N_alloc,
+                         stream);
+}
+
+ba_status ba_att_sparse_fwd_rows(const ba_att_shape *s, int32_t q_rows, int32_t q_stride, const void *Q,
+                                 const void *K, const void *V, const int32_t *kv_idx, const int32_t *kv_cnt,
+                                 int32_t kmax, const float *O_prev, const float *LSE_prev, void *O, int32_t o_dtype,
+                                 float *LSE, ba_stream_t stream) {
+  if (s == nullptr || (O_prev == nullptr) != (LSE_prev == nullptr)) return BA_ERR_INVALID_ARG;
+  return sparse_fwd_impl(s, Q, K, V, kv_idx, kv_cnt, kmax, O, o_dtype, LSE, O_prev, LSE_prev, q_rows, q_stride,
+                         stream);
 }
 
 ba_status ba_att_merge_lse(int64_t rows, int32_t d, int32_t in_dtype, int32_t out_dtype, const void *O1,

@@ -305,10 +305,12 @@ ba_status ba_att_complement_lists(const ba_att_shape *shape, const int32_t *kv_i
  * o_dtype   shape->dtype, or BA_DTYPE_F32 to keep a partial output in fp32
  *           (one rounding in total when partials are merged later).
  * LSE       device fp32 [B, Hq, N_alloc], natural log (written).
- * Paths: bf16 with d = 64 or 128 and block = 128 or 256 runs the tcgen05/TMEM
- * tensor-core kernel (a 256-row block is two 128-row query tiles sharing its
- * list, its key blocks four 64-key halves); every other supported shape runs
- * an fp32 CUDA-core kernel.
+ * Paths: bf16 with d = 64 or 128, block = 64, 128 or 256 and key blocks of
+ * 64, 128 or 256 rows runs the tcgen05/TMEM tensor-core kernel (a 256-row
+ * block is two 128-row query tiles sharing its list; a 64-row block is one
+ * 128-row tile of which only the block's 64 rows are stored; key blocks are
+ * taken as 64-key halves); every other supported shape runs an fp32
+ * CUDA-core kernel.
  */
 ba_status ba_att_sparse_fwd(const ba_att_shape *shape,
                             const void *Q, const void *K, const void *V,
@@ -336,6 +338,45 @@ ba_status ba_att_sparse_fwd_merge(const ba_att_shape *shape,
                                   const int32_t *kv_idx, const int32_t *kv_cnt, int32_t kmax,
                                   const float *O_prev, const float *LSE_prev,
                                   void *O, int32_t o_dtype, float *LSE, ba_stream_t stream);
+
+/*
+ * ba_att_sparse_fwd_rows — block-sparse attention for one range of query
+ * rows only, optionally merged with a cached partial of those rows
+ * (FlashBlock "Core claim" and "What carries the argument": during block
+ * diffusion the attention of the current block's queries to the tokens
+ * outside the block changes little between steps, so its (O, LSE) is cached
+ * and only the attention inside the current block is recomputed, then merged
+ * in log space by Eq. 9; the key access per step then scales with the block,
+ * not with the sequence).
+ *
+ * Query side: q_rows valid rows per (batch, query head), at a stride of
+ * q_stride rows (q_stride >= q_rows), cut into nqr = ceil(q_rows / block)
+ * query blocks of shape->block rows (the last may be ragged). Q is
+ * [B, Hq, q_stride, d] of shape->dtype; O, LSE, O_prev and LSE_prev use the
+ * same row stride. Q may be a compact buffer of the range (q_stride = q_rows)
+ * or point at row r0 of a full [B, Hq, N_alloc, d] tensor (Q + r0*d, with
+ * q_stride = N_alloc; r0 a multiple of 8 keeps the 16-byte alignment).
+ * Key side: K, V, N, N_alloc, Hkv, block_k and sm_scale as in shape.
+ * kv_idx  device int32 [B, Hq, nqr, kmax], kv_cnt [B, Hq, nqr]: per query
+ *         block of the range, its key blocks in [0, nk), strictly ascending.
+ * O_prev, LSE_prev   nullable (both or neither): fp32 [B, Hq, q_stride, d]
+ *         and [B, Hq, q_stride], the cached partial of these rows over a key
+ *         set disjoint from the listed blocks; the epilogue merges it exactly
+ *         as ba_att_sparse_fwd_merge does. With o_dtype = BA_DTYPE_F32, O may
+ *         be O_prev and LSE may be LSE_prev (in place).
+ * O       device [B, Hq, q_stride, d] of o_dtype (shape->dtype or fp32);
+ *         LSE device fp32 [B, Hq, q_stride]. Rows >= q_rows are not written.
+ * One CTA (or CUDA-core block) is launched per query tile of the range only,
+ * B * Hq * nqr tiles in all. Results equal ba_att_sparse_fwd (or _merge) on
+ * the same rows bit for bit. Paths as for ba_att_sparse_fwd. q_rows < 1 or
+ * q_stride < q_rows -> BA_ERR_INVALID_ARG; one of O_prev, LSE_prev NULL ->
+ * BA_ERR_INVALID_ARG.
+ */
+ba_status ba_att_sparse_fwd_rows(const ba_att_shape *shape, int32_t q_rows, int32_t q_stride,
+                                 const void *Q, const void *K, const void *V,
+                                 const int32_t *kv_idx, const int32_t *kv_cnt, int32_t kmax,
+                                 const float *O_prev, const float *LSE_prev,
+                                 void *O, int32_t o_dtype, float *LSE, ba_stream_t stream);
 
 /*
  * ba_att_merge_lse — log-space merge of two partial attentions over disjoint

@@ -43,6 +43,7 @@ from .ba_att_oracle import (  # noqa: F401
     mass_share_before,
     near_tie_mask,
     masked_attention,
+    block_rows_attention,
     dense_attention,
     merge_lse,
     split_lists,

@@ -340,6 +340,50 @@ def masked_attention(Q, K, V, idx, cnt, N: int, b: int, sm_scale: float,
     return O, LSE
 
 
+def block_rows_attention(Qr, K, V, idx, cnt, q_rows: int, N: int, b: int, sm_scale: float,
+                         O_prev=None, L_prev=None, dtype=np.float64, b_k: int | None = None):
+    """Attention of one range of query rows over listed key blocks, merged
+    with a cached partial of those rows when one is given.
+
+    [FlashBlock, "Core claim" and "What carries the argument"]: in block
+    diffusion the current block's attention to the tokens outside it is
+    cached as (A_out, L_out); each step recomputes only the attention inside
+    the current block and combines the two in log space (Eq. 9, with the
+    split of Eq. 5). Here: Qr [B, Hq, q_stride, d] holds the range's q_rows
+    query rows, cut into query blocks of b rows (the last may be ragged);
+    idx [B, Hq, nqr, kmax] / cnt [B, Hq, nqr] list, per query block of the
+    range, the key blocks (of b_k keys, default b) it attends; keys >= N are
+    not tokens. For every row r < q_rows of block i:
+        L_r = ln sum_{c in C_i} exp(s q_r . k_c),
+        O_r = sum_{c in C_i} exp(s q_r . k_c - L_r) v_c,
+    then, with (O_prev, L_prev) [B, Hq, q_stride, d] / [B, Hq, q_stride],
+    (O_r, L_r) = merge_lse(O_prev_r, L_prev_r, O_r, L_r).
+    Rows >= q_rows are NaN. Returns O [B, Hq, q_stride, d], LSE [B, Hq, q_stride].
+    """
+    Qr = np.asarray(Qr)
+    K = np.asarray(K)
+    V = np.asarray(V)
+    B, Hq, q_stride, d = Qr.shape
+    Hkv = K.shape[1]
+    bk = b if b_k is None else b_k
+    O = np.full((B, Hq, q_stride, d), np.nan, dtype=dtype)
+    LSE = np.full((B, Hq, q_stride), np.nan, dtype=dtype)
+    for bb in range(B):
+        for h in range(Hq):
+            g = _kv_head(h, Hq, Hkv)
+            for i in range(num_blocks(q_rows, b)):
+                rows = _block_rows(q_rows, b, i)
+                blocks = [int(j) for j in idx[bb, h, i, : int(cnt[bb, h, i])]]
+                keys = (np.concatenate([_block_rows(N, bk, j) for j in blocks]) if blocks
+                        else np.zeros(0, dtype=np.int64))
+                o, l = _attend(Qr[bb, h, rows].astype(dtype), K[bb, g, keys].astype(dtype),
+                               V[bb, g, keys].astype(dtype), sm_scale, dtype)
+                if O_prev is not None:
+                    o, l = merge_lse(np.asarray(O_prev)[bb, h, rows], np.asarray(L_prev)[bb, h, rows], o, l, dtype)
+                O[bb, h, rows], LSE[bb, h, rows] = o, l
+    return O, LSE
+
+
 def dense_attention(Q, K, V, N: int, sm_scale: float, rows=None, dtype=np.float64):
     """Textbook dense softmax attention over all N valid keys (no mask).
 

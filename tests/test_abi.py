@@ -158,6 +158,21 @@ def test_sparse_fwd_merge_arguments(lib):
     assert lib.ba_att_sparse_fwd_merge(ctypes.byref(shape(d=96)), P, P, P, P, P, 4, P, P, P, 1, P, None) == 2
 
 
+def test_sparse_fwd_rows_arguments(lib):
+    s = shape()
+    call = lambda sh, rows, stride, op, lp, *rest: lib.ba_att_sparse_fwd_rows(
+        ctypes.byref(sh), rows, stride, P, P, P, P, P, 4, op, lp, *rest)
+    assert call(s, 0, 64, None, None, P, 1, P, None) == 1             # no query rows
+    assert call(s, 65, 64, None, None, P, 1, P, None) == 1            # stride below the row count
+    assert call(s, 64, 64, P, None, P, 1, P, None) == 1               # the cached partial comes in pairs
+    assert call(s, 64, 64, None, P, P, 1, P, None) == 1
+    assert call(s, 64, 64, None, None, None, 1, P, None) == 1         # no output
+    assert call(s, 64, 64, None, None, MIS, 1, P, None) == 3
+    assert call(s, 64, 64, MIS, P, P, 1, P, None) == 3
+    assert call(shape(d=96), 64, 64, None, None, P, 1, P, None) == 2
+    assert lib.ba_att_sparse_fwd_rows(None, 64, 64, P, P, P, P, P, 4, None, None, P, 1, P, None) == 1
+
+
 def test_complement_lists_arguments(lib):
     s = shape()                                          # nb = 8
     assert lib.ba_att_complement_lists(ctypes.byref(s), P, P, 4, P, P, 7, None) == 1       # stride below nb

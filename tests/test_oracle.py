@@ -320,6 +320,61 @@ def test_merge_of_disjoint_spans_equals_union():
         np.testing.assert_allclose(Lm, Lu[:, :, :N], rtol=1e-12, atol=1e-12)
 
 
+def test_block_rows_attention_cached_external_plus_internal_is_dense():
+    # FlashBlock's block-external caching: the current block's rows attend the
+    # prefix (cached as one partial) and the block itself (recomputed); the
+    # merge equals textbook dense attention of those rows over every key
+    rng = np.random.default_rng(21)
+    B, Hq, Hkv, d, b, s = 1, 4, 2, 16, 16, 16 ** -0.5
+    for r0, R, bk in ((64, 37, 16), (32, 48, 32), (0, 20, 16), (96, 16, 16)):
+        N = r0 + R                                      # tokens so far: prefix + current block
+        Q = rng.standard_normal((B, Hq, N + 5, d))
+        K = rng.standard_normal((B, Hkv, N + 5, d))
+        V = rng.standard_normal((B, Hkv, N + 5, d))
+        rows = np.arange(r0, N)
+        Qr = np.zeros((B, Hq, R + 3, d))                # compact range buffer with a few spare rows
+        Qr[:, :, :R] = Q[:, :, rows]
+        if r0 > 0:
+            Oe, Le = O.dense_attention(Q, K, V, r0, s, rows=rows)          # external: keys [0, r0)
+        else:
+            Oe, Le = np.zeros((B, Hq, R, d)), np.full((B, Hq, R), -np.inf)
+        Oc = np.zeros((B, Hq, R + 3, d))
+        Lc = np.zeros((B, Hq, R + 3))
+        Oc[:, :, :R], Lc[:, :, :R] = Oe, Le
+        # internal: the key blocks of [r0, N) (r0 is a multiple of the key block size)
+        internal = np.arange(r0 // bk, -(-N // bk), dtype=np.int32)
+        nqr = O.num_blocks(R, b)
+        idx = np.tile(internal, (B, Hq, nqr, 1))
+        cnt = np.full((B, Hq, nqr), internal.size, dtype=np.int32)
+        Og, Lg = O.block_rows_attention(Qr, K, V, idx, cnt, R, N, b, s, O_prev=Oc, L_prev=Lc, b_k=bk)
+        Od, Ld = O.dense_attention(Q, K, V, N, s, rows=rows)
+        np.testing.assert_allclose(Og[:, :, :R], Od, rtol=1e-11, atol=1e-12)
+        np.testing.assert_allclose(Lg[:, :, :R], Ld, rtol=1e-12, atol=1e-12)
+        assert np.isnan(Og[:, :, R:]).all() and np.isnan(Lg[:, :, R:]).all()
+
+
+def test_block_rows_attention_without_cache_is_masked_attention_on_those_rows():
+    Q, K, V = _qkv()
+    N, b, s = 200, 32, 16 ** -0.5
+    nb = O.num_blocks(N, b)
+    S = np.random.default_rng(8).standard_normal((1, 4, nb, nb))
+    idx, cnt = O.select_topk(S, 3, kmax=5)
+    cnt[0, 1, 2] = 0                                    # an empty list: O = 0, LSE = -inf
+    Om, Lm = O.masked_attention(Q, K, V, idx, cnt, N, b, s)
+    i0, R = 2, 200 - 64                                 # query blocks 2.. of the sequence, ragged at N
+    rows = slice(i0 * b, i0 * b + R)
+    Og, Lg = O.block_rows_attention(Q[:, :, rows], K, V, idx[:, :, i0:], cnt[:, :, i0:], R, N, b, s)
+    np.testing.assert_array_equal(Og, Om[:, :, rows])
+    np.testing.assert_array_equal(Lg, Lm[:, :, rows])
+    assert (Og[0, 1, 0:32] == 0).all() and np.isneginf(Lg[0, 1, 0:32]).all()
+    # an empty list with a cached partial passes the partial through
+    Oc = np.random.default_rng(9).standard_normal(Og.shape)
+    Lc = np.random.default_rng(10).standard_normal(Lg.shape)
+    Ox, Lx = O.block_rows_attention(Q[:, :, rows], K, V, idx[:, :, i0:], cnt[:, :, i0:], R, N, b, s, Oc, Lc)
+    np.testing.assert_allclose(Ox[0, 1, 0:32], Oc[0, 1, 0:32], rtol=1e-15)
+    np.testing.assert_array_equal(Lx[0, 1, 0:32], Lc[0, 1, 0:32])
+
+
 def test_complement_lists_partition_and_kept_plus_rest_is_dense():
     # the complement is the exact set difference (ascending, -1 padded), and
     # merging attention over the kept blocks with attention over the rest
