@@ -115,7 +115,8 @@ SMALL = [
     ("dlm_16k", dict(N=1920 + 77, N_alloc=2048, Hq=4, Hkv=2), 0.5),   # tcgen05 path, ragged last block
     ("sweep_32k", dict(N=4096, Hq=4, Hkv=1), 0.25),                   # needle generator, 32 blocks
     ("video_32k", dict(N=600, N_alloc=640, Hq=2, Hkv=2, grid=(3, 10, 20)), 0.5),
-    ("dlm_16k", dict(N=1024, Hq=2, Hkv=1, d=64, block=64), 0.5),      # bf16 on the CUDA-core path
+    ("dlm_16k", dict(N=1024, Hq=2, Hkv=1, d=64, block=64), 0.5),      # tcgen05, 64-row query blocks, d = 64
+    ("dlm_16k", dict(N=1600 - 23, N_alloc=1600, Hq=4, Hkv=2, block=64), 0.5),   # tcgen05, 64-row blocks, ragged
     ("tiny_fp32", dict(N=768, d=128, block=32), 0.3),                 # fp32 d=128, block 32
     ("tiny_fp32", dict(N=9600 - 7, N_alloc=9600, block=16, Hq=2, Hkv=1), 0.5),   # 600 blocks: 5x5 score tiles
     ("dlm_16k", dict(N=64 * 128, Hq=2, Hkv=1), 0.5),                 # 512 blocks: 16 keys per lane in the top-k
@@ -130,7 +131,8 @@ SMALL = [
     ("dlm_16k", dict(N=2048, Hq=4, Hkv=2, block=256, block_k=128), 0.5),             # tcgen05, 256 x 128
     ("dlm_16k", dict(N=3000, N_alloc=3072, Hq=2, Hkv=1, block=128, block_k=256), 0.3),  # tcgen05, 128 x 256
     ("dlm_16k", dict(N=1500, N_alloc=1536, Hq=2, Hkv=1, d=64, block=128, block_k=64), 0.5),  # tcgen05, d 64
-    ("dlm_16k", dict(N=1024 - 9, N_alloc=1024, Hq=2, Hkv=1, block=64, block_k=128), 0.5),   # CUDA cores, 64 x 128
+    ("dlm_16k", dict(N=1024 - 9, N_alloc=1024, Hq=2, Hkv=1, block=64, block_k=128), 0.5),   # tcgen05, 64 x 128
+    ("dlm_16k", dict(N=1024, Hq=2, Hkv=1, block=32), 0.5),                         # CUDA cores, bf16 block 32
     ("tiny_fp32", dict(block=32, block_k=64), 0.5),                                  # fp32, 32 x 64
 ]
 
@@ -155,6 +157,7 @@ def test_small_full_parity(name, over, keep):
                                        ("dlm_16k", dict(N=1536 - 9, N_alloc=1536, Hq=4, Hkv=2, d=64)),
                                        ("dlm_16k", dict(N=1536, Hq=4, Hkv=2, block=256)),
                                        ("dlm_16k", dict(N=1536, Hq=4, Hkv=2, block=256, block_k=64)),
+                                       ("dlm_16k", dict(N=1536 - 5, N_alloc=1536, Hq=4, Hkv=2, block=64)),
                                        ("video_32k", dict(N=600, N_alloc=640, Hq=2, Hkv=2, grid=(3, 10, 20)))])
 def test_keep_all_equals_dense(name, over):
     # check (1): keep = 1.0 selects every block and equals dense attention
@@ -344,7 +347,8 @@ def test_complement_lists_and_cached_residual_is_dense(name, over, keep):
 @pytest.mark.parametrize("name,over", [
     ("extreme_128k", dict(N=4096 - 50, N_alloc=4096, Hq=4, Hkv=2)),      # tensor-core path, ragged tail
     ("tiny_fp32", dict(N=1000, N_alloc=1024)),                             # CUDA-core path, fp32
-    ("dlm_16k", dict(N=1024, Hq=2, Hkv=1, d=64, block=64)),                # CUDA-core path, bf16 inputs
+    ("dlm_16k", dict(N=1024, Hq=2, Hkv=1, d=64, block=64)),                # tensor-core path, 64-row blocks
+    ("dlm_16k", dict(N=1024 - 3, N_alloc=1024, Hq=2, Hkv=1, block=32)),    # CUDA-core path, bf16 inputs
     ("dlm_16k", dict(N=2048 - 40, N_alloc=2048, Hq=4, Hkv=2, d=64)),       # tensor-core path, d = 64
 ])
 def test_fused_merge_equals_separate_merge(name, over):

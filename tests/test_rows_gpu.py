@@ -37,7 +37,8 @@ CASES = [
     ("dlm_16k", dict(Hq=2, Hkv=1, block=256), 1024, 256 + 100),       # 256-row query blocks (two tiles each)
     ("dlm_16k", dict(Hq=2, Hkv=1), 0, 300),                           # no prefix: the cache is empty
     ("tiny_fp32", dict(Hq=2, Hkv=2), 256, 100),                       # fp32 on the CUDA cores, block 64
-    ("dlm_16k", dict(Hq=2, Hkv=1, d=64, block=64), 320, 64 + 30),     # bf16 block 64 (CUDA cores)
+    ("dlm_16k", dict(Hq=2, Hkv=1, d=64, block=64), 320, 64 + 30),     # tcgen05, 64-row query blocks
+    ("dlm_16k", dict(Hq=2, Hkv=1, block=32), 320, 64 + 30),           # bf16 block 32 (CUDA cores)
 ]
 
 
