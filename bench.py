@@ -298,7 +298,7 @@ class Step:
                           torch.empty((w.B, w.Hkv, nb, w.d), device=dev))
         self.idx = torch.empty((w.B, w.Hq, nb, k), device=dev, dtype=torch.int32)
         self.cnt = torch.empty((w.B, w.Hq, nb), device=dev, dtype=torch.int32)
-        self.scores = torch.empty((w.B, w.Hq, nb, nb), device=dev, dtype=torch.float32)
+        # the score map is not asked for: ba_att_selector keeps it in its workspace
         self.sel_ws = torch.empty(api.selector_workspace_bytes(shape), device=dev, dtype=torch.uint8)
         self.O = torch.empty_like(Qd)
         self.L = torch.empty((w.B, w.Hq, w.N_alloc), device=dev)
@@ -323,7 +323,7 @@ class Step:
                 events[i].record(self.stream)
         mark(0)
         api.selector(self.Qd, self.Kd, self.shape, self.keep, kmax=self.k,
-                     out=(self.stats_buf, self.idx, self.cnt, self.scores), workspace=self.sel_ws)
+                     out=(self.stats_buf, self.idx, self.cnt, None), workspace=self.sel_ws)
         mark(1)
         if self.split_block is None:
             api.sparse_fwd(self.Qd, self.Kd, self.Vd, self.idx, self.cnt, self.shape, out=(self.O, self.L))
@@ -543,8 +543,9 @@ def run_selector_isolated(step, reps=20):
     intervals. Q and K exceed L2, so each pass streams them from HBM."""
     import torch
     api, shape, keep, w = step.api, step.shape, step.keep, step.w
-    stats_buf, idx, cnt, scores = step.stats_buf, step.idx, step.cnt, step.scores
-    one_call = lambda: api.selector(step.Qd, step.Kd, shape, keep, kmax=step.k, out=(stats_buf, idx, cnt, scores),
+    stats_buf, idx, cnt = step.stats_buf, step.idx, step.cnt
+    scores = torch.empty((w.B, w.Hq, w.nb, w.nb), device=step.dev, dtype=torch.float32)   # the two-call form's map
+    one_call = lambda: api.selector(step.Qd, step.Kd, shape, keep, kmax=step.k, out=(stats_buf, idx, cnt, None),
                                     workspace=step.sel_ws)
     one_call()
     api.stats(step.Qd, step.Kd, shape, out=stats_buf)

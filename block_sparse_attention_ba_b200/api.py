@@ -242,12 +242,14 @@ def selector_workspace_bytes(shape: Shape) -> int:
 
 
 def selector(Q: torch.Tensor, K: torch.Tensor, shape: Shape, keep: float, kmax: int | None = None, out=None,
-             workspace: torch.Tensor | None = None):
+             workspace: torch.Tensor | None = None, with_scores: bool = True):
     """The whole selector in one call (ba_att_selector): stats, scores and top-k.
 
     Returns (stats, idx, cnt, scores) with stats = (q_mean, q_var, k_mean, k_var); out may
-    pass the same tuple preallocated, workspace a uint8 device tensor of at least
-    selector_workspace_bytes(shape)."""
+    pass the same tuple preallocated (its scores may be None), workspace a uint8 device
+    tensor of at least selector_workspace_bytes(shape). With with_scores=False (or a None
+    scores entry in out) no score map is returned (scores is None): the map stays in the
+    workspace."""
     lib = load_library()
     k = keep_count(shape, keep)
     if k < 1:
@@ -261,7 +263,8 @@ def selector(Q: torch.Tensor, K: torch.Tensor, shape: Shape, keep: float, kmax: 
               torch.empty((shape.B, shape.Hkv, shape.nk, shape.d), device=dev, dtype=torch.float32))
         idx = torch.empty((shape.B, shape.Hq, shape.nb, kmax), device=dev, dtype=torch.int32)
         cnt = torch.empty((shape.B, shape.Hq, shape.nb), device=dev, dtype=torch.int32)
-        sc = torch.empty((shape.B, shape.Hq, shape.nb, shape.nk), device=dev, dtype=torch.float32)
+        sc = (torch.empty((shape.B, shape.Hq, shape.nb, shape.nk), device=dev, dtype=torch.float32)
+              if with_scores else None)
     else:
         st, idx, cnt, sc = out
     if workspace is None:
@@ -270,7 +273,8 @@ def selector(Q: torch.Tensor, K: torch.Tensor, shape: Shape, keep: float, kmax: 
     _check("ba_att_selector", lib.ba_att_selector(
         ctypes.byref(shape.c()), ctypes.c_double(keep), _dev(Q, "Q"), _dev(K, "K"), _dev(qm, "q_mean"),
         _dev(qv, "q_var"), _dev(km, "k_mean"), _dev(kv, "k_var"), _dev(workspace, "workspace"),
-        _dev(sc, "block_scores"), _dev(idx, "kv_idx"), _dev(cnt, "kv_cnt"), idx.shape[-1], _stream(Q)))
+        ctypes.c_void_p(0) if sc is None else _dev(sc, "block_scores"), _dev(idx, "kv_idx"), _dev(cnt, "kv_cnt"),
+        idx.shape[-1], _stream(Q)))
     return st, idx, cnt, sc
 
 

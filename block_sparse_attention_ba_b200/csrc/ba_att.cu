@@ -238,13 +238,13 @@ ba_status ba_att_select(const ba_att_shape *s, double keep, const float *q_mean,
 // ---------------------------------------------------------------- one-call selector
 
 namespace {
-// [6 planes][rows][d] bf16 feature array read in boxes of 64 dims x 128 rows.
-bool make_feat_map(CUtensorMap *map, const void *ptr, int d, long long rows) {
+// [6 planes][rows][d] bf16 feature array read in boxes of 64 dims x box_rows rows.
+bool make_feat_map(CUtensorMap *map, const void *ptr, int d, long long rows, int box_rows = selft::kTile) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows), 6u};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2u, static_cast<cuuint64_t>(rows) * d * 2u};
-  cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(selft::kTile), 1u};
+  cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(box_rows), 1u};
   cuuint32_t estr[3] = {1u, 1u, 1u};
   CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), dims, strides, box, estr,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -260,6 +260,15 @@ long long feat_rows_k(const ba_att_shape *s) { return static_cast<long long>(s->
 bool selector_feature_path(const ba_att_shape *s) {
   return feat_rows_q(s) + selft::kTile < 0x7FFFFFFFLL;
 }
+
+// Workspace of ba_att_selector: the score features, then room for the score
+// map when the caller passes none; each part 256-byte aligned.
+size_t ws_align(long long x) { return static_cast<size_t>((x + 255) & ~255LL); }
+long long feat_bytes(const ba_att_shape *s) { return 6LL * (feat_rows_q(s) + feat_rows_k(s)) * s->d * 2; }
+long long score_map_bytes(const ba_att_shape *s) {
+  return static_cast<long long>(s->B) * s->Hq * nblocks(s) * nkblocks(s) * 4;
+}
+size_t ws_scores_offset(const ba_att_shape *s) { return ws_align(feat_bytes(s)); }
 
 template <int D>
 cudaError_t launch_select_feat(const CUtensorMap &mq, const CUtensorMap &mk, float *scores, const ba_att_shape *s,
@@ -280,8 +289,7 @@ extern "C" {
 
 int64_t ba_att_selector_workspace(const ba_att_shape *s) {
   if (check_shape(s) != BA_OK) return -1;
-  const long long bytes = 6LL * (feat_rows_q(s) + feat_rows_k(s)) * s->d * 2;
-  return (bytes + 255) & ~255LL;
+  return static_cast<int64_t>(ws_scores_offset(s) + ws_align(score_map_bytes(s)));
 }
 
 ba_status ba_att_selector(const ba_att_shape *s, double keep, const void *Q, const void *K, float *q_mean,
@@ -289,7 +297,7 @@ ba_status ba_att_selector(const ba_att_shape *s, double keep, const void *Q, con
                           int32_t *kv_idx, int32_t *kv_cnt, int32_t kmax, ba_stream_t stream) {
   ba_status st = check_shape(s);
   if (st != BA_OK) return st;
-  if (!Q || !K || !q_mean || !q_var || !k_mean || !k_var || !workspace || !block_scores || !kv_idx || !kv_cnt)
+  if (!Q || !K || !q_mean || !q_var || !k_mean || !k_var || !workspace || !kv_idx || !kv_cnt)
     return BA_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(q_mean) || !aligned16(q_var) || !aligned16(k_mean) ||
       !aligned16(k_var) || !aligned16(workspace) || !aligned16(block_scores) || !aligned16(kv_idx) ||
@@ -299,16 +307,18 @@ ba_status ba_att_selector(const ba_att_shape *s, double keep, const void *Q, con
   if (k < 1 || kmax < k) return BA_ERR_INVALID_ARG;
   const int nq = nblocks(s), nk = nkblocks(s);
   if (nk > 4096 || nq > 1048576) return BA_ERR_UNSUPPORTED;
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  // without a caller map the scores live in the workspace (read back by the top-k, never returned)
+  float *scores = block_scores != nullptr ? block_scores : reinterpret_cast<float *>(ws + ws_scores_offset(s));
   if (!selector_feature_path(s)) {
     st = ba_att_stats(s, Q, K, q_mean, q_var, k_mean, k_var, stream);
-    return st == BA_OK ? ba_att_select(s, keep, q_mean, q_var, k_mean, k_var, kv_idx, kv_cnt, kmax, block_scores,
-                                       stream)
+    return st == BA_OK ? ba_att_select(s, keep, q_mean, q_var, k_mean, k_var, kv_idx, kv_cnt, kmax, scores, stream)
                        : st;
   }
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   const int sms = num_sms_of_current_device();
   const float scale = effective_scale(s);
-  auto *fq = static_cast<__nv_bfloat16 *>(workspace);
+  auto *fq = reinterpret_cast<__nv_bfloat16 *>(ws);
   auto *fk = fq + 6 * feat_rows_q(s) * s->d;
   const FeatOut feat{fq, fk, scale, 0.5f * scale * scale, feat_rows_q(s), feat_rows_k(s)};
   cudaError_t e;
@@ -331,10 +341,10 @@ ba_status ba_att_selector(const ba_att_shape *s, double keep, const void *Q, con
   CUtensorMap mq, mk;
   if (!make_feat_map(&mq, fq, s->d, feat_rows_q(s)) || !make_feat_map(&mk, fk, s->d, feat_rows_k(s)))
     return BA_ERR_CUDA;
-  e = s->d == 128 ? launch_select_feat<128>(mq, mk, block_scores, s, nq, nk, sms, cs)
-                  : launch_select_feat<64>(mq, mk, block_scores, s, nq, nk, sms, cs);
+  e = s->d == 128 ? launch_select_feat<128>(mq, mk, scores, s, nq, nk, sms, cs)
+                  : launch_select_feat<64>(mq, mk, scores, s, nq, nk, sms, cs);
   if (e != cudaSuccess) return from_cuda(e);
-  return from_cuda(launch_topk(block_scores, nk, k, kv_idx, kmax, kv_cnt, static_cast<long long>(s->B) * s->Hq * nq,
+  return from_cuda(launch_topk(scores, nk, k, kv_idx, kmax, kv_cnt, static_cast<long long>(s->B) * s->Hq * nq,
                                sms, cs, /*dependent=*/true));
 }
 
@@ -551,7 +561,7 @@ size_t round_up(size_t x) { return (x + kWsAlign - 1) / kWsAlign * kWsAlign; }
 struct PipeLayout {
   int C = 0, G = 0, nb = 0, k = 0;
   size_t q[2], kk[2], v[2], o[2], l[2];                 // double-buffered chunk inputs and outputs
-  size_t qm, qv, km, kv, idx, cnt, sc, feat;            // selector buffers of one chunk
+  size_t qm, qv, km, kv, idx, cnt, feat;                // selector buffers of one chunk
   size_t lo_idx, lo_cnt, hi_idx, hi_cnt, o1, l1;         // split buffers and the first span's fp32 partial
   size_t total = 0;
 };
@@ -596,8 +606,11 @@ bool pipe_layout(const ba_att_shape *s, double keep, int32_t split_block, int32_
   L->kv = take(hk * nk * s->d * 4);
   L->idx = take(hq * nb * k * 4);
   L->cnt = take(hq * nb * 4);
-  L->sc = take(hq * nb * static_cast<size_t>(nk) * 4);
-  L->feat = take(6 * (hq * nb + hk * nk) * s->d * 2);     // ba_att_selector's feature workspace
+  ba_att_shape cs = *s;                                     // one chunk of C KV heads of one batch entry
+  cs.B = 1;
+  cs.Hq = static_cast<int32_t>(hq);
+  cs.Hkv = static_cast<int32_t>(hk);
+  L->feat = take(static_cast<size_t>(ba_att_selector_workspace(&cs)));   // features, counters, score map
   if (split_block >= 0) {
     L->lo_idx = take(hq * nb * k * 4);
     L->lo_cnt = take(hq * nb * 4);
@@ -710,8 +723,7 @@ ba_status forward_host_impl(PipeResources *r, const ba_att_shape *s, double keep
     float *qm = reinterpret_cast<float *>(ws + L.qm), *qv = reinterpret_cast<float *>(ws + L.qv);
     float *km = reinterpret_cast<float *>(ws + L.km), *kv = reinterpret_cast<float *>(ws + L.kv);
     int32_t *idx = reinterpret_cast<int32_t *>(ws + L.idx), *cnt = reinterpret_cast<int32_t *>(ws + L.cnt);
-    st = ba_att_selector(&sc, keep, Qc, Kc, qm, qv, km, kv, ws + L.feat, reinterpret_cast<float *>(ws + L.sc), idx,
-                         cnt, L.k, stream);
+    st = ba_att_selector(&sc, keep, Qc, Kc, qm, qv, km, kv, ws + L.feat, nullptr, idx, cnt, L.k, stream);
     if (st == BA_OK && split_block >= 0) {
       int32_t *lo_idx = reinterpret_cast<int32_t *>(ws + L.lo_idx), *lo_cnt = reinterpret_cast<int32_t *>(ws + L.lo_cnt);
       int32_t *hi_idx = reinterpret_cast<int32_t *>(ws + L.hi_idx), *hi_cnt = reinterpret_cast<int32_t *>(ws + L.hi_cnt);

@@ -53,6 +53,161 @@ struct FeatOut {
   long long q_rows, k_rows;    // rows per plane
 };
 
+// Per-lane pieces of the statistics pass (stats_warp_kernel). A lane owns
+// E = D/32 columns of a block, as P = E/2 packed fp32 pairs.
+template <typename T, int D>
+struct LaneStats {
+  static constexpr int E = D / 32;
+  static constexpr int P = E / 2;
+  static constexpr int RB = D * static_cast<int>(sizeof(T));   // bytes per row
+  uint64_t c[P], nc[P], s1[2][P], s2[2][P];
+
+  // this lane's E columns of row r of a staged chunk as P packed fp32 pairs
+  __device__ __forceinline__ static void row_pairs(const uint8_t *rows, int r, uint64_t (&x)[P]) {
+    const uint8_t *a = rows + static_cast<size_t>(r) * RB;
+    if constexpr (sizeof(T) == 2) {
+      if constexpr (E == 4) {
+        const uint2 v = *reinterpret_cast<const uint2 *>(a);
+        x[0] = pack_u32x2(v.x << 16, v.x & 0xFFFF0000u);
+        x[1] = pack_u32x2(v.y << 16, v.y & 0xFFFF0000u);
+      } else {
+        const uint32_t v = *reinterpret_cast<const uint32_t *>(a);
+        x[0] = pack_u32x2(v << 16, v & 0xFFFF0000u);
+      }
+    } else {
+      if constexpr (E == 4) {
+        const uint4 v = *reinterpret_cast<const uint4 *>(a);
+        x[0] = pack_u32x2(v.x, v.y);
+        x[1] = pack_u32x2(v.z, v.w);
+      } else {
+        const uint2 v = *reinterpret_cast<const uint2 *>(a);
+        x[0] = pack_u32x2(v.x, v.y);
+      }
+    }
+  }
+
+  __device__ __forceinline__ void clear() {
+#pragma unroll
+    for (int i = 0; i < P; ++i) c[i] = nc[i] = s1[0][i] = s1[1][i] = s2[0][i] = s2[1][i] = 0ull;
+  }
+
+  // Adds the nr rows of one staged chunk (rows: this lane's first column of
+  // the chunk's row 0); the first chunk of a block also takes its first row
+  // as the shift c. Rows go in pairs (even row -> set 0, odd row -> set 1;
+  // the first row contributes exactly +0).
+  __device__ __forceinline__ void add_chunk(const uint8_t *rows, int nr, bool first_chunk) {
+    if (first_chunk) {
+      row_pairs(rows, 0, c);
+#pragma unroll
+      for (int i = 0; i < P; ++i) {
+        nc[i] = pack_f32x2(-lo_f32(c[i]), -hi_f32(c[i]));
+        s1[0][i] = s1[1][i] = s2[0][i] = s2[1][i] = 0ull;     // +0.0f pairs
+      }
+    }
+    int r = 0;
+#pragma unroll 4
+    for (; r + 1 < nr; r += 2) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint64_t x[P];
+        row_pairs(rows, r + h, x);
+#pragma unroll
+        for (int i = 0; i < P; ++i) {
+          const uint64_t d = add_f32x2(x[i], nc[i]);
+          s1[h][i] = add_f32x2(s1[h][i], d);
+          s2[h][i] = fma_f32x2(d, d, s2[h][i]);
+        }
+      }
+    }
+    if (r < nr) {
+      uint64_t x[P];
+      row_pairs(rows, r, x);
+#pragma unroll
+      for (int i = 0; i < P; ++i) {
+        const uint64_t d = add_f32x2(x[i], nc[i]);
+        s1[0][i] = add_f32x2(s1[0][i], d);
+        s2[0][i] = fma_f32x2(d, d, s2[0][i]);
+      }
+    }
+  }
+
+  // mean = c + S1/n, var = (S2 - S1*(S1/n))/n clamped at 0, for a block of n rows
+  __device__ __forceinline__ void finish(int n, float (&mean)[E], float (&var)[E]) const {
+    const float inv_n = 1.f / static_cast<float>(n);
+#pragma unroll
+    for (int i = 0; i < P; ++i) {
+      const uint64_t S1 = add_f32x2(s1[0][i], s1[1][i]), S2 = add_f32x2(s2[0][i], s2[1][i]);
+      const float a1[2] = {lo_f32(S1), hi_f32(S1)}, a2[2] = {lo_f32(S2), hi_f32(S2)};
+      const float cc[2] = {lo_f32(c[i]), hi_f32(c[i])};
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float md = a1[e] * inv_n;
+        mean[2 * i + e] = cc[e] + md;
+        var[2 * i + e] = fmaxf(fmaf(-a1[e], md, a2[e]) * inv_n, 0.f);
+      }
+    }
+  }
+};
+
+// Writes one lane's E columns of a block's mean and variance (at element
+// offset orow + lane*E of the mean/var arrays) and, with feat.q set, the
+// block's augmented score features (the lane's columns of each plane packed
+// into one store, so a warp writes each plane's D contiguous values at once).
+template <int D>
+__device__ __forceinline__ void write_block_stats(bool is_q, long long orow, int lane, const float (&mean)[D / 32],
+                                                  const float (&var)[D / 32], float *q_mean, float *q_var,
+                                                  float *k_mean, float *k_var, const FeatOut &feat) {
+  constexpr int E = D / 32;
+  float *om = (is_q ? q_mean : k_mean) + orow + lane * E;
+  float *ov = (is_q ? q_var : k_var) + orow + lane * E;
+  if constexpr (E == 4) {
+    *reinterpret_cast<float4 *>(om) = make_float4(mean[0], mean[1], mean[2], mean[3]);
+    *reinterpret_cast<float4 *>(ov) = make_float4(var[0], var[1], var[2], var[3]);
+  } else {
+    *reinterpret_cast<float2 *>(om) = make_float2(mean[0], mean[1]);
+    *reinterpret_cast<float2 *>(ov) = make_float2(var[0], var[1]);
+  }
+  if (feat.q == nullptr) return;
+  float x[3][E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    if (is_q) {
+      x[0][e] = __fmul_rn(feat.s, mean[e]);
+      x[1][e] = __fmul_rn(feat.hs2, var[e]);
+      x[2][e] = __fmul_rn(__fmul_rn(feat.hs2, mean[e]), mean[e]);
+    } else {
+      x[0][e] = mean[e];
+      x[1][e] = __fmaf_rn(mean[e], mean[e], var[e]);
+      x[2][e] = var[e];
+    }
+  }
+  __nv_bfloat16 *base = is_q ? feat.q : feat.k;
+  const long long plane = (is_q ? feat.q_rows : feat.k_rows) * D;
+#pragma unroll
+  for (int pp = 0; pp < 3; ++pp) {
+    uint32_t hw[E / 2], lw[E / 2];
+#pragma unroll
+    for (int e = 0; e < E; e += 2) {
+      const __nv_bfloat16 h0 = __float2bfloat16_rn(x[pp][e]), h1 = __float2bfloat16_rn(x[pp][e + 1]);
+      const __nv_bfloat16 l0 = __float2bfloat16_rn(x[pp][e] - __bfloat162float(h0));
+      const __nv_bfloat16 l1 = __float2bfloat16_rn(x[pp][e + 1] - __bfloat162float(h1));
+      hw[e / 2] = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) |
+                  (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
+      lw[e / 2] = static_cast<uint32_t>(__bfloat16_as_ushort(l0)) |
+                  (static_cast<uint32_t>(__bfloat16_as_ushort(l1)) << 16);
+    }
+    __nv_bfloat16 *ph = base + (2 * pp) * plane + orow + lane * E;
+    __nv_bfloat16 *pl = base + (2 * pp + 1) * plane + orow + lane * E;
+    if constexpr (E == 4) {
+      *reinterpret_cast<uint2 *>(ph) = make_uint2(hw[0], hw[1]);
+      *reinterpret_cast<uint2 *>(pl) = make_uint2(lw[0], lw[1]);
+    } else {
+      *reinterpret_cast<uint32_t *>(ph) = hw[0];
+      *reinterpret_cast<uint32_t *>(pl) = lw[0];
+    }
+  }
+}
+
 template <typename T, int D, int SPLIT>
 __global__ void __launch_bounds__(3 * SPLIT * 32, 1)
     stats_warp_kernel(const T *__restrict__ Q, const T *__restrict__ K, float *__restrict__ q_mean,
@@ -133,9 +288,8 @@ __global__ void __launch_bounds__(3 * SPLIT * 32, 1)
   issued += issue_next(1);
   pdl_allow_dependents();                           // the score GEMM may launch as SMs free up
 
-  uint64_t c[P], nc[P], s1[2][P], s2[2][P];
-#pragma unroll
-  for (int i = 0; i < P; ++i) c[i] = nc[i] = s1[0][i] = s1[1][i] = s2[0][i] = s2[1][i] = 0ull;
+  LaneStats<T, D> acc;
+  acc.clear();
   bool ok = true;
   while (consumed < issued) {
     const int st = static_cast<int>(consumed & 1);
@@ -151,136 +305,16 @@ __global__ void __launch_bounds__(3 * SPLIT * 32, 1)
     const bool is_q = mo >= 0;
     const long long orow = is_q ? mo : -1 - mo;
     const uint8_t *rows = stage_mem + (static_cast<size_t>(warp) * 2 + st) * CB + lane * E * sizeof(T);
-
-    // this lane's E columns of row r of the chunk as P packed fp32 pairs
-    auto row_pairs = [&](int r, uint64_t (&x)[P]) {
-      const uint8_t *a = rows + static_cast<size_t>(r) * RB;
-      if constexpr (sizeof(T) == 2) {
-        if constexpr (E == 4) {
-          const uint2 v = *reinterpret_cast<const uint2 *>(a);
-          x[0] = pack_u32x2(v.x << 16, v.x & 0xFFFF0000u);
-          x[1] = pack_u32x2(v.y << 16, v.y & 0xFFFF0000u);
-        } else {
-          const uint32_t v = *reinterpret_cast<const uint32_t *>(a);
-          x[0] = pack_u32x2(v << 16, v & 0xFFFF0000u);
-        }
-      } else {
-        if constexpr (E == 4) {
-          const uint4 v = *reinterpret_cast<const uint4 *>(a);
-          x[0] = pack_u32x2(v.x, v.y);
-          x[1] = pack_u32x2(v.z, v.w);
-        } else {
-          const uint2 v = *reinterpret_cast<const uint2 *>(a);
-          x[0] = pack_u32x2(v.x, v.y);
-        }
-      }
-    };
-    if (r0 == 0) {                                  // a new block: its first row is the shift
-      row_pairs(0, c);
-#pragma unroll
-      for (int i = 0; i < P; ++i) {
-        nc[i] = pack_f32x2(-lo_f32(c[i]), -hi_f32(c[i]));
-        s1[0][i] = s1[1][i] = s2[0][i] = s2[1][i] = 0ull;     // +0.0f pairs
-      }
-    }
-    // rows in pairs (even row -> set 0, odd row -> set 1; the first row
-    // contributes exactly +0)
-    int r = 0;
-#pragma unroll 4
-    for (; r + 1 < nr; r += 2) {
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint64_t x[P];
-        row_pairs(r + h, x);
-#pragma unroll
-        for (int i = 0; i < P; ++i) {
-          const uint64_t d = add_f32x2(x[i], nc[i]);
-          s1[h][i] = add_f32x2(s1[h][i], d);
-          s2[h][i] = fma_f32x2(d, d, s2[h][i]);
-        }
-      }
-    }
-    if (r < nr) {
-      uint64_t x[P];
-      row_pairs(r, x);
-#pragma unroll
-      for (int i = 0; i < P; ++i) {
-        const uint64_t d = add_f32x2(x[i], nc[i]);
-        s1[0][i] = add_f32x2(s1[0][i], d);
-        s2[0][i] = fma_f32x2(d, d, s2[0][i]);
-      }
-    }
+    acc.add_chunk(rows, nr, r0 == 0);              // a new block: its first row is the shift
     __syncwarp();                                   // every lane is done with this stage
     ++consumed;
     if (lane == 0 && iw < total) fence_proxy_async_smem();   // the reads above before the bulk write
     issued += issue_next(st);
     if (r0 + nr < n) continue;                      // the block goes on in the next chunk
 
-    const float inv_n = 1.f / static_cast<float>(n);
     float mean[E], var[E];
-#pragma unroll
-    for (int i = 0; i < P; ++i) {
-      const uint64_t S1 = add_f32x2(s1[0][i], s1[1][i]), S2 = add_f32x2(s2[0][i], s2[1][i]);
-      const float a1[2] = {lo_f32(S1), hi_f32(S1)}, a2[2] = {lo_f32(S2), hi_f32(S2)};
-      const float cc[2] = {lo_f32(c[i]), hi_f32(c[i])};
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const float md = a1[e] * inv_n;
-        mean[2 * i + e] = cc[e] + md;
-        var[2 * i + e] = fmaxf(fmaf(-a1[e], md, a2[e]) * inv_n, 0.f);
-      }
-    }
-    float *om = (is_q ? q_mean : k_mean) + orow + lane * E;
-    float *ov = (is_q ? q_var : k_var) + orow + lane * E;
-    if constexpr (E == 4) {
-      *reinterpret_cast<float4 *>(om) = make_float4(mean[0], mean[1], mean[2], mean[3]);
-      *reinterpret_cast<float4 *>(ov) = make_float4(var[0], var[1], var[2], var[3]);
-    } else {
-      *reinterpret_cast<float2 *>(om) = make_float2(mean[0], mean[1]);
-      *reinterpret_cast<float2 *>(ov) = make_float2(var[0], var[1]);
-    }
-    if (feat.q != nullptr) {
-      // the lane's E columns of each plane packed into one store: a warp
-      // writes each plane's D contiguous values at once
-      float x[3][E];
-#pragma unroll
-      for (int e = 0; e < E; ++e) {
-        if (is_q) {
-          x[0][e] = __fmul_rn(feat.s, mean[e]);
-          x[1][e] = __fmul_rn(feat.hs2, var[e]);
-          x[2][e] = __fmul_rn(__fmul_rn(feat.hs2, mean[e]), mean[e]);
-        } else {
-          x[0][e] = mean[e];
-          x[1][e] = __fmaf_rn(mean[e], mean[e], var[e]);
-          x[2][e] = var[e];
-        }
-      }
-      __nv_bfloat16 *base = is_q ? feat.q : feat.k;
-      const long long plane = (is_q ? feat.q_rows : feat.k_rows) * D;
-#pragma unroll
-      for (int pp = 0; pp < 3; ++pp) {
-        uint32_t hw[E / 2], lw[E / 2];
-#pragma unroll
-        for (int e = 0; e < E; e += 2) {
-          const __nv_bfloat16 h0 = __float2bfloat16_rn(x[pp][e]), h1 = __float2bfloat16_rn(x[pp][e + 1]);
-          const __nv_bfloat16 l0 = __float2bfloat16_rn(x[pp][e] - __bfloat162float(h0));
-          const __nv_bfloat16 l1 = __float2bfloat16_rn(x[pp][e + 1] - __bfloat162float(h1));
-          hw[e / 2] = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) |
-                      (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
-          lw[e / 2] = static_cast<uint32_t>(__bfloat16_as_ushort(l0)) |
-                      (static_cast<uint32_t>(__bfloat16_as_ushort(l1)) << 16);
-        }
-        __nv_bfloat16 *ph = base + (2 * pp) * plane + orow + lane * E;
-        __nv_bfloat16 *pl = base + (2 * pp + 1) * plane + orow + lane * E;
-        if constexpr (E == 4) {
-          *reinterpret_cast<uint2 *>(ph) = make_uint2(hw[0], hw[1]);
-          *reinterpret_cast<uint2 *>(pl) = make_uint2(lw[0], lw[1]);
-        } else {
-          *reinterpret_cast<uint32_t *>(ph) = hw[0];
-          *reinterpret_cast<uint32_t *>(pl) = lw[0];
-        }
-      }
-    }
+    acc.finish(n, mean, var);
+    write_block_stats<D>(is_q, orow, lane, mean, var, q_mean, q_var, k_mean, k_var, feat);
   }
   // after an abandoned wait, let this warp's copies in flight land first
   if (!ok && lane == 0) {

@@ -181,9 +181,10 @@ ba_status ba_att_topk(const float *block_scores, int64_t rows, int32_t nk, int32
 
 /*
  * ba_att_selector_workspace — device workspace bytes that ba_att_selector
- * needs for this shape: the augmented score features of every block,
- * 6 planes (3 parts x {hi, lo}) x (B*Hq*nq + B*Hkv*nk) rows x d bf16, rounded
- * up to 256. -1 for an invalid shape.
+ * needs for this shape: the augmented score features of every block
+ * (6 planes (3 parts x {hi, lo}) x (B*Hq*nq + B*Hkv*nk) rows x d bf16), then
+ * room for the score map [B, Hq, nq, nk] fp32 for callers that pass no
+ * block_scores; each part rounded up to 256 bytes. -1 for an invalid shape.
  */
 int64_t ba_att_selector_workspace(const ba_att_shape *shape);
 
@@ -202,12 +203,16 @@ int64_t ba_att_selector_workspace(const ba_att_shape *shape);
  * `workspace`; the score GEMM reads them instead of deriving them per tile.
  * Outputs are bit-identical to ba_att_stats followed by ba_att_select.
  *
- * Q, K, q_mean..k_var, kv_idx, kv_cnt, kmax, block_scores: as for
- * ba_att_stats and ba_att_select (block_scores holds the score map on return).
+ * Q, K, q_mean..k_var, kv_idx, kv_cnt, kmax: as for ba_att_stats and
+ * ba_att_select.
+ * block_scores  nullable: device fp32 [B, Hq, nq, nk], 16-byte aligned,
+ *             which then holds the score map on return; NULL keeps the map
+ *             inside the workspace (it is not returned).
  * workspace   device, caller-owned, >= ba_att_selector_workspace(shape)
  *             bytes, 16-byte aligned; its contents on return are unspecified.
  * Shapes with more than 2^31 - 129 feature rows (B*Hq*nq) run ba_att_stats
- * and ba_att_select instead, leaving the workspace unused. NULL pointers ->
+ * and ba_att_select instead (the score map then still goes to block_scores or
+ * the workspace). NULL pointers other than block_scores ->
  * BA_ERR_INVALID_ARG; misaligned -> BA_ERR_MISALIGNED; nk > 4096 ->
  * BA_ERR_UNSUPPORTED.
  */

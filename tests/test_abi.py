@@ -204,16 +204,19 @@ def test_select_variant_arguments(lib):
 def test_selector_workspace_and_arguments(lib):
     s = shape()
     nb = lib.ba_att_num_blocks(ctypes.byref(s))
-    want = 6 * s.B * (s.Hq + s.Hkv) * nb * s.d * 2
-    assert lib.ba_att_selector_workspace(ctypes.byref(s)) == (want + 255) // 256 * 256
+    up = lambda x: (x + 255) // 256 * 256
+    feats = 6 * s.B * (s.Hq + s.Hkv) * nb * s.d * 2          # score features, hi and lo
+    scores = 4 * s.B * s.Hq * nb * nb                          # room for the map when none is passed
+    assert lib.ba_att_selector_workspace(ctypes.byref(s)) == up(feats) + up(scores)
     assert lib.ba_att_selector_workspace(ctypes.byref(shape(d=96))) == -1
     call = lambda sh, keep, *ptrs, kmax=8: lib.ba_att_selector(ctypes.byref(sh), ctypes.c_double(keep), *ptrs[:9],
                                                                ptrs[9], kmax, None)
     ptrs = [P] * 10
-    for i in range(10):                        # every pointer is required
+    for i in range(10):                        # every pointer but block_scores (index 7) is required
         bad = list(ptrs)
-        bad[i] = None
-        assert call(s, 0.5, *bad) == 1
+        if i != 7:
+            bad[i] = None
+            assert call(s, 0.5, *bad) == 1
         bad[i] = MIS
         assert call(s, 0.5, *bad) == 3
     assert call(s, 0.0, *ptrs) == 1            # keep outside (0, 1]

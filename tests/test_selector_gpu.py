@@ -85,3 +85,28 @@ def test_selector_against_oracle():
          "cnt": cnt.cpu().numpy()}
     stats_ref = check_stats(r, Q, K, w)
     check_selection(r, stats_ref, w, keep)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("name,over", [("dlm_16k", dict(N=2048 - 40, N_alloc=2048, Hq=8, Hkv=2)),
+                                       ("dlm_16k", dict(N=300 * 128 - 5, Hq=2, Hkv=2)),
+                                       ("dlm_16k", dict(N=1024, B=2, Hq=4, Hkv=2, d=64))])
+def test_selector_without_score_map_and_reused_workspace(name, over):
+    # block_scores NULL: the map stays in the workspace and the lists are the
+    # same; a second call on the same (now used) workspace gives them again
+    keep = 0.5
+    (st_ref, idx_ref, cnt_ref, _), _, _ = _run_both(name, over, keep)
+    Q, K, V, meta = make_inputs(name, **over)
+    w = meta["workload"]
+    Qd, Kd = (torch.from_numpy(np.ascontiguousarray(x)).to(torch.bfloat16).cuda() for x in (Q, K))
+    shape = api.Shape.of(Qd, Kd, w.N, w.block)
+    ws = torch.full((api.selector_workspace_bytes(shape),), 0x5A, device="cuda", dtype=torch.uint8)
+    for _ in range(2):
+        st, idx, cnt, sc = api.selector(Qd, Kd, shape, keep, workspace=ws, with_scores=False)
+        torch.cuda.synchronize()
+        assert sc is None
+        assert torch.equal(idx, idx_ref) and torch.equal(cnt, cnt_ref)
+        for a, b in zip(st, st_ref):
+            assert torch.equal(a, b)
+    status, word = api.get_device_error()
+    assert status == 0, f"device error word {word:#x}"
