@@ -166,6 +166,13 @@ class ClockSampler:
             self.proc = None
             self.fh.close()
             os.unlink(self.path)
+            return
+        # nvidia-smi is sampling once its first line is out (bounded wait)
+        t0 = time.time()
+        while time.time() - t0 < 3.0 and self.proc.poll() is None:
+            if os.path.getsize(self.path) > 0:
+                break
+            time.sleep(0.05)
 
     def stop(self, window=None):
         """Stop sampling; summarise the samples inside window = (t0, t1) in
@@ -347,8 +354,7 @@ def timed_steps(step, steps, clock_id, barrier=None):
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(step.names) + 1)] for _ in range(steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(clock_id)
-    clocks.start()
-    time.sleep(0.3)                                 # nvidia-smi is up and sampling before the timed region
+    clocks.start()                                  # returns once nvidia-smi is sampling
     if barrier:
         barrier()
     torch.cuda.synchronize()
@@ -361,6 +367,7 @@ def timed_steps(step, steps, clock_id, barrier=None):
     wall1 = time.time()
     if barrier:
         barrier()
+    time.sleep(0.06)                                # the sample that covers the region's end
     clk = clocks.stop(window=(wall0, wall1))
     per = {n: [ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(steps)] for i, n in enumerate(step.names)}
     return {"elapsed_ms": t_start.elapsed_time(t_end), "clocks": clk,
@@ -475,7 +482,6 @@ def run_sustained(ctx, seconds=SUSTAINED_SECONDS):
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(n + 1)]
     clocks = ClockSampler(ctx["clock_id"])
     clocks.start()
-    time.sleep(0.3)
     torch.cuda.synchronize()
     wall0 = time.time()
     ev[0].record(step.stream)
