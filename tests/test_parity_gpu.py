@@ -389,6 +389,8 @@ def test_fused_merge_equals_separate_merge(name, over):
     ("tiny_fp32", dict(N=1000, N_alloc=1024), False, 1),                        # fp32, CUDA-core attention
     ("dlm_16k", dict(N=3000, N_alloc=3072, Hq=4, Hkv=2, block_k=64), True, 1),   # asymmetric 128 x 64, split
     ("dlm_16k", dict(N=2048 - 20, N_alloc=2048, Hq=4, Hkv=2, block=256), False, 0),  # 256-row blocks
+    ("dlm_16k", dict(N=2048, Hq=12, Hkv=4), False, 1),        # 3 query heads per KV head, 4 chunks
+    ("dlm_16k", dict(N=1024, B=2, Hq=4, Hkv=2), True, 1),     # chunks across batch entries, split
 ])
 def test_forward_host_pipeline(name, over, split, chunk):
     # host buffers in and out, chunked and pipelined: bit-identical to the
