@@ -430,6 +430,8 @@ def run_ours(args):
     barrier = dist.barrier if world > 1 else None
 
     w = WORKLOADS[args.workload]
+    if args.block:
+        w = w.with_(block=args.block)
     keep = args.keep
     Q, K, V, meta = make_inputs(w)
     split_block = meta.get("split_block") if w.split else None
@@ -454,7 +456,7 @@ def run_ours(args):
     result = None
     if rank == 0:
         peaks, peak_src = load_peaks()
-        step_key = f"{w.name}/{'split' if split_block is not None else 'single'}/keep{keep}"
+        step_key = f"{w.name}/b{w.block}/{'split' if split_block is not None else 'single'}/keep{keep}"
         traffic = traffic_from_profile(kernel_sources_sha(["attn_tc.cuh", "common.cuh"]), step_key)
         result = {
             "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -679,6 +681,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="sweep_32k")
     ap.add_argument("--keep", type=float, default=0.5)
+    ap.add_argument("--block", type=int, default=0,
+                    help="query and key block size in place of the workload's (0: the workload's own)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true",
                     help="only the timed K steps (no sustained loop, other workloads, e2e, dense, merge)")
@@ -705,7 +709,7 @@ def main(argv=None):
         result["dense_keep1"] = run_dense(ctx["step"])
         result["merge_lse_standalone"] = run_merge_standalone(ctx)
         by = {}
-        for name in EXTRA_WORKLOADS:
+        for name in EXTRA_WORKLOADS if not args.block else ():
             if name != args.workload:
                 by[name] = run_workload_entry(name, args.keep, ctx["dev"], ctx["clock_id"])
         result["by_workload"] = by
@@ -730,6 +734,8 @@ def run_reference(args):
     import oracle as O
 
     w = WORKLOADS[args.workload]
+    if args.block:
+        w = w.with_(block=args.block)
     Q, K, V, meta = make_inputs(w)
     split_block = meta.get("split_block") if w.split else None
     k = O.keep_count(args.keep, w.nb)
