@@ -7,7 +7,10 @@
 // kept key blocks only, emitting O and the per-row log-sum-exp; the online
 // softmax over blocks is the FlashAttention recurrence the pages compare to.
 //
-// One CTA = one 128-row query block of one (batch, head) = one tile. Two CTAs
+// One CTA = one 128-row query tile of one (batch, head): a 128-row query
+// block, half of a 256-row one, or two 64-row ones whose tile attends the
+// union of their two lists, each row masking the key blocks its own list
+// leaves out (UnionCursor). Two CTAs
 // share an SM (up to 96 KB shared memory and 256 TMEM columns each), so one CTA's
 // softmax overlaps the other CTA's MMAs. Roles (192 threads):
 //   warps 0-3  softmax + correction + epilogue; thread t owns query row t,
@@ -72,23 +75,48 @@ struct Ctl {
   int abort;
 };
 
-// Validity of list entries, computed identically by every role from the raw
-// list: entry t is valid when it lies in [0, nb) and strictly above the
-// previous raw entry. Walks the list in order, with the next entry's load
-// issued one step ahead so that its latency hides behind the current block.
-struct ListCursor {
-  const int32_t *list;
-  int cnt, nb, prev, next;
-  __device__ __forceinline__ ListCursor(const int32_t *l, int c, int n) : list(l), cnt(c), nb(n), prev(-1), next(0) {
-    if (cnt > 0) next = __ldg(list);
+// The key blocks a tile attends, walked in ascending order by every role
+// alike: the kept list of its query block, or, for a 128-row tile that holds
+// two 64-row query blocks, the union of their two lists. An entry of a list
+// is valid when it lies in [0, nb) and above the previous raw entry of that
+// list. Each step is one key block: raw entries of equal value in both lists
+// make one step; a step valid in neither list is block 0, which the softmax
+// masks for every row. Next entries are loaded one step ahead.
+struct UnionCursor {
+  const int32_t *la, *lb;
+  int ca, cb, nb, ta, tb, pa, pb, va, vb;
+  __device__ __forceinline__ UnionCursor(const int32_t *a, int na, const int32_t *b, int nbl, int n)
+      : la(a), lb(b), ca(na), cb(nbl), nb(n), ta(0), tb(0), pa(-1), pb(-1) {
+    va = ca > 0 ? __ldg(la) : 0;
+    vb = cb > 0 ? __ldg(lb) : 0;
   }
-  // entry t (called for t = 0, 1, 2, ... in order); returns its validity
-  __device__ __forceinline__ bool step(int t, int &j) {
-    j = next;
-    if (t + 1 < cnt) next = __ldg(list + t + 1);
-    const bool ok = j >= 0 && j < nb && (t == 0 || j > prev);
-    prev = j;
-    return ok;
+  __device__ __forceinline__ bool done() const { return ta >= ca && tb >= cb; }
+  // the next step's block j and whether it is a valid entry of list A / B;
+  // a taken entry out of range or out of order sets bad_index / bad_order
+  __device__ __forceinline__ void step(int &j, bool &in_a, bool &in_b, bool &bad_index, bool &bad_order) {
+    const bool take_a = ta < ca && (tb >= cb || va <= vb);
+    const bool take_b = tb < cb && (ta >= ca || vb <= va);
+    int v = 0;
+    in_a = in_b = false;
+    if (take_a) {
+      v = va;
+      const bool range = va >= 0 && va < nb, order = ta == 0 || va > pa;
+      in_a = range && order;
+      bad_index |= !range;
+      bad_order |= range && !order;
+      pa = va;
+      if (++ta < ca) va = __ldg(la + ta);
+    }
+    if (take_b) {
+      v = vb;                                        // equal to A's entry when both are taken
+      const bool range = vb >= 0 && vb < nb, order = tb == 0 || vb > pb;
+      in_b = range && order;
+      bad_index |= !range;
+      bad_order |= range && !order;
+      pb = vb;
+      if (++tb < cb) vb = __ldg(lb + tb);
+    }
+    j = (in_a || in_b) ? v : 0;
   }
 };
 
@@ -164,32 +192,39 @@ __global__ void __launch_bounds__(kThreads, 2)
 
   // tile -> (b, kv head, 128-row query tile, head within group): consecutive
   // CTAs share a KV head, so its K/V stay hot in L2. A query block of `block`
-  // rows (128 or 256) is block/128 query tiles, which share its list; a key
+  // rows (128 or 256) is block/128 query tiles, which share its list; two
+  // 64-row query blocks 2t and 2t+1 share one tile, which attends the union
+  // of their lists (each row masks the blocks its own list leaves out). A key
   // block of `kblock` rows (64, 128 or 256) is kblock/64 key halves.
   const int G = Hq / Hkv;
-  const int qpb = block >= kTileRows ? block >> 7 : 1;
+  const bool pair = block < kTileRows;               // 64-row blocks, two per tile
+  const int qpb = pair ? 1 : block >> 7;
+  const long long tiles_per_head = pair ? (nq + 1) / 2 : static_cast<long long>(nq) * qpb;
   const int hpe_log2 = kblock == 256 ? 2 : (kblock == 128 ? 1 : 0), hpe = 1 << hpe_log2;
   long long tile = blockIdx.x;
   const int hg = static_cast<int>(tile % G);
   tile /= G;
-  const int it = static_cast<int>(tile % (static_cast<long long>(nq) * qpb));   // query tile within the head
-  const int i = it / qpb;                                                        // its query block
-  // the tile's first query row and its rows of this block: 128, or 64 for a
-  // 64-row block, whose tile also loads (and computes, but never stores) the
-  // next block's 64 rows
-  const int tile_row0 = i * block + (it % qpb) * kTileRows;
-  const int tile_rows = block < kTileRows ? block : kTileRows;
-  tile /= static_cast<long long>(nq) * qpb;
+  const int it = static_cast<int>(tile % tiles_per_head);                        // query tile within the head
+  const int ia = pair ? 2 * it : it / qpb;                                       // its (first) query block
+  const int tile_row0 = pair ? it * kTileRows : ia * block + (it % qpb) * kTileRows;
+  tile /= tiles_per_head;
   const int g = static_cast<int>(tile % Hkv);
   const int b = static_cast<int>(tile / Hkv);
   const int h = g * G + hg;
-  const long long list_row = (static_cast<long long>(b) * Hq + h) * nq + i;
-  const int32_t *list = kv_idx + list_row * kmax;
-  int cnt = __ldg(kv_cnt + list_row);
-  if (cnt < 0 || cnt > kmax) {
-    if (threadIdx.x == 0) raise_error(BA_DEVERR_BAD_COUNT);
-    cnt = cnt < 0 ? 0 : kmax;
-  }
+  auto list_of = [&](int i, const int32_t *&list) -> int {
+    const long long list_row = (static_cast<long long>(b) * Hq + h) * nq + i;
+    list = kv_idx + list_row * kmax;
+    int c = __ldg(kv_cnt + list_row);
+    if (c < 0 || c > kmax) {
+      if (threadIdx.x == 0) raise_error(BA_DEVERR_BAD_COUNT);
+      c = c < 0 ? 0 : kmax;
+    }
+    return c;
+  };
+  const int32_t *list_a = nullptr, *list_b = nullptr;
+  const int cnt_a = list_of(ia, list_a);
+  const int cnt_b = (pair && ia + 1 < nq) ? list_of(ia + 1, list_b) : 0;
+  const bool has_work = cnt_a + cnt_b > 0;
 
   if (threadIdx.x == 0) {
     for (int k = 0; k < NUM_BARS; ++k) mbar_init(smem_u32(&ctl.bar[k]), (k == P_FULL0 || k == P_FULL1) ? 128u : 1u);
@@ -210,7 +245,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int qz = b * Hq + h;          // row of the [B*H] head axis in the tensor maps
   const int kz = b * Hkv + g;
 
-  if (cnt > 0 && warp == 4 && lane < 2) {
+  if (has_work && warp == 4 && lane < 2) {
     // ------------------------------------------------------------ producers
     // lane 0: Q, then the K halves; lane 1: the V halves. Half h of block t
     // reuses the slot rows of half h of block t-1 once its MMAs are done.
@@ -227,13 +262,11 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     int issued = -1;                    // last half-block index u loaded
     bool bad_index = false, bad_order = false;
-    ListCursor cur(list, cnt, nk);
-    for (int t = 0; t < cnt; ++t) {
+    UnionCursor cur(list_a, cnt_a, list_b, cnt_b, nk);
+    for (int t = 0; !cur.done(); ++t) {
       int j;
-      if (!cur.step(t, j)) {
-        if (j < 0 || j >= nk) bad_index = true; else bad_order = true;
-        j = 0;                            // load a valid block; softmax masks it out
-      }
+      bool in_a, in_b;
+      cur.step(j, in_a, in_b, bad_index, bad_order);   // j = 0 when invalid: loaded, then masked
       bool stop = false;
       for (int hh = 0; hh < hpe; ++hh) {
         const int u = t * hpe + hh, h = u & 1;          // half index; halves alternate the two slots
@@ -258,11 +291,23 @@ __global__ void __launch_bounds__(kThreads, 2)
       for (int u = issued; u >= 0 && u > issued - 2; --u) mbar_wait_bounded(bar(full0 + (u & 1)), (u >> 1) & 1, nullptr);
       if (is_k) mbar_wait_bounded(bar(Q_FULL), 0, nullptr);
     }
-  } else if (cnt > 0 && warp == 5 && lane == 0) {
+  } else if (has_work && warp == 5 && lane == 0) {
     // ------------------------------------------------------------ MMA issuer
     constexpr uint32_t idesc_qk = idesc_bf16_f32(128, kHalfKeys, 0, 0);
     constexpr uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
-    const int n_half = hpe * cnt;
+    // whether half u exists: the steps are counted from the same walk
+    UnionCursor mc(list_a, cnt_a, list_b, cnt_b, nk);
+    int steps_seen = 0;
+    auto half_exists = [&](int u) -> bool {
+      const int st = u >> hpe_log2;
+      while (steps_seen <= st && !mc.done()) {
+        int j;
+        bool in_a, in_b, bi = false, bo = false;
+        mc.step(j, in_a, in_b, bi, bo);
+        ++steps_seen;
+      }
+      return st < steps_seen;
+    };
     // S_u = Q K_u^T into S columns h*64..h*64+63
     auto issue_s = [&](int u) -> bool {
       const int h = u & 1;
@@ -279,9 +324,9 @@ __global__ void __launch_bounds__(kThreads, 2)
       return true;
     };
     bool ok = mbar_wait_bounded(bar(Q_FULL), 0, abort);
-    if (ok) ok = issue_s(0);
-    if (ok && n_half > 1) ok = issue_s(1);
-    for (int u = 0; ok && u < n_half; ++u) {
+    if (ok) ok = issue_s(0);                           // a tile with work has at least one step
+    if (ok && half_exists(1)) ok = issue_s(1);
+    for (int u = 0; ok && half_exists(u); ++u) {
       const int h = u & 1;
       if (!mbar_wait_bounded(bar(V_FULL0 + h), (u >> 1) & 1, abort)) break;
       if (!mbar_wait_bounded(bar(P_FULL0 + h), (u >> 1) & 1, abort)) break;
@@ -293,7 +338,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       mma_commit(bar(V_EMPTY0 + h));
       mma_commit(bar(PV_DONE0 + h));
-      if (u + 2 < n_half && !issue_s(u + 2)) break;   // after PV_u: S_{u+2} overwrites P_u
+      if (half_exists(u + 2) && !issue_s(u + 2)) break;   // after PV_u: S_{u+2} overwrites P_u
     }
     mma_commit(bar(O_FINAL));
     mma_commit(bar(DRAIN));
@@ -304,18 +349,21 @@ __global__ void __launch_bounds__(kThreads, 2)
     const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
     const uint32_t tS = tmem + lane_off + kColS, tO = tmem + lane_off + kColO;
     const int qrow = tile_row0 + row;
-    const bool owned = row < tile_rows && qrow < Nq;   // a row of this tile's block, and a token
+    const bool owned = qrow < Nq;                      // a token (rows past the range are not written)
+    const bool row_in_b = pair && row >= 64;           // this row's block is the tile's second one
     const long long orow = static_cast<long long>(qz) * q_stride + qrow;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
     int n_keys = 0;
-    ListCursor cur(list, cnt, nk);
-    for (int u = 0; u < hpe * cnt; ++u) {
+    UnionCursor cur(list_a, cnt_a, list_b, cnt_b, nk);
+    for (int u = 0;; ++u) {
       const int h = u & 1, hh = u & (hpe - 1);          // S slot; half within the key block
       if (hh == 0) {
+        if (cur.done()) break;
         int j;
-        const bool valid = cur.step(u >> hpe_log2, j);
-        n_keys = valid ? min(kblock, N - j * kblock) : 0;
+        bool in_a, in_b, bi = false, bo = false;
+        cur.step(j, in_a, in_b, bi, bo);
+        n_keys = (row_in_b ? in_b : in_a) ? min(kblock, N - j * kblock) : 0;
       }
       const int n_half = min(max(n_keys - hh * kHalfKeys, 0), kHalfKeys);
       bool w = mbar_wait_bounded(bar(S_FULL0 + h), (u >> 1) & 1, abort);
@@ -326,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       tmem_ld32(tSu, sr[0]);
       tmem_ld32(tSu + 32, sr[1]);
       tmem_ld_wait();
-      if (n_half < kHalfKeys) {                        // ragged last block or a skipped entry (rare)
+      if (n_half < kHalfKeys) {                        // ragged last block, a block of the other list, a skipped entry
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
 #pragma unroll
@@ -369,10 +417,10 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_arrive(bar(P_FULL0 + h));
     }
     // ------------------------------------------------------------ epilogue
-    // (cnt == 0: nothing was accumulated; this span contributes O = 0,
+    // (no listed block: nothing was accumulated; this span contributes O = 0,
     // LSE = -inf, and a merge passes the earlier partial through)
-    bool go = (cnt == 0);
-    if (cnt > 0 && ok) {
+    bool go = !has_work;
+    if (has_work && ok) {
       const bool w = mbar_wait_bounded(bar(O_FINAL), 0, abort);
       go = __all_sync(0xFFFFFFFFu, w);
       if (go) tc_fence_after();
@@ -388,7 +436,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
       for (int q = 0; q < D / 32; ++q) {
         uint32_t orr[32];
-        if (cnt > 0) {
+        if (has_work) {
           tmem_ld32(tO + q * 32, orr);
           tmem_ld_wait();
         } else {

@@ -422,9 +422,10 @@ ba_status sparse_fwd_impl(const ba_att_shape *s, const void *Q, const void *K, c
         !make_head_map(&mv, V, s->d, s->N, s->N_alloc, static_cast<long long>(s->B) * s->Hkv, tc::kKvBoxRows))
       return BA_ERR_CUDA;
     // one CTA per 128-row query tile (a 256-row block is two tiles sharing its
-    // list; a 64-row block is one tile whose second half is not stored)
-    const long long tiles =
-        static_cast<long long>(s->B) * s->Hq * nb * (s->block >= tc::kTileRows ? s->block / tc::kTileRows : 1);
+    // list; two 64-row blocks share one tile, which attends both lists)
+    const long long tiles = static_cast<long long>(s->B) * s->Hq *
+                            (s->block >= tc::kTileRows ? static_cast<long long>(nb) * (s->block / tc::kTileRows)
+                                                       : (nb + 1) / 2);
     if (tiles > 0x7FFFFFFFLL) return BA_ERR_UNSUPPORTED;
     const float sl2 = scale * 1.4426950408889634f;
     const uint32_t smem = tc::dyn_smem_bytes(s->d);
