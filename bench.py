@@ -640,7 +640,7 @@ def run_dense(step, steps=3):
             "sparse_fwd_tflops": round(fl / (att_ms * 1e-3) / 1e12, 1)}
 
 
-def run_workload_entry(name, keep, dev, clock_id, steps=5, warmup=3):
+def run_workload_entry(name, keep, dev, clock_id, steps=5, warmup=3, block=0):
     """A full-size workload timed like the headline (its own recipe's step
     form: single pass, or split + fused merge for the 128K case), with inputs
     drawn on the device (timing only; parity at full size is in the tests)."""
@@ -649,6 +649,8 @@ def run_workload_entry(name, keep, dev, clock_id, steps=5, warmup=3):
     from block_sparse_attention_ba_b200.workloads import WORKLOADS, make_inputs_device
 
     w = WORKLOADS[name]
+    if block:
+        w = w.with_(block=block)
     Qd, Kd, Vd, meta = make_inputs_device(w, dev)
     split_block = meta.get("split_block") if w.split else None
     step = Step(w, keep, Qd, Kd, Vd, split_block, dev)
@@ -712,6 +714,11 @@ def main(argv=None):
         for name in EXTRA_WORKLOADS if not args.block else ():
             if name != args.workload:
                 by[name] = run_workload_entry(name, args.keep, ctx["dev"], ctx["clock_id"])
+        if not args.block and args.workload == "sweep_32k":
+            # the rest of the 32K keep sweep, and the 64-row query blocks at keep 0.5
+            by["sweep_32k@keep0.25"] = run_workload_entry("sweep_32k", 0.25, ctx["dev"], ctx["clock_id"])
+            by["sweep_32k@block64"] = run_workload_entry("sweep_32k", args.keep, ctx["dev"], ctx["clock_id"],
+                                                         block=64)
         result["by_workload"] = by
     if rank == 0:
         if not args.no_cpu_baseline:

@@ -215,7 +215,6 @@ __global__ void __launch_bounds__(3 * SPLIT * 32, 1)
                       int Hq, int Hkv, int N, int N_alloc, int block, int nb, int kblock, int nbk, FeatOut feat) {
   static_assert(SPLIT == 1 || SPLIT == 2 || SPLIT == 4, "chunks per 32 KB");
   constexpr int E = D / 32;                         // columns per lane
-  constexpr int P = E / 2;                          // packed fp32 pairs per lane
   constexpr int RB = D * static_cast<int>(sizeof(T));   // bytes per row
   constexpr int W = 3 * SPLIT;                      // warps per CTA
   constexpr uint32_t CB = kStatsStageBytes / SPLIT; // bytes per chunk
