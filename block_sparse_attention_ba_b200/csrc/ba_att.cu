@@ -23,6 +23,7 @@
 #include "merge.cuh"
 #include "attn_simt.cuh"
 #include "attn_tc.cuh"
+#include "attn_tc2.cuh"
 
 using namespace baatt;
 
@@ -415,6 +416,34 @@ ba_status sparse_fwd_impl(const ba_att_shape *s, const void *Q, const void *K, c
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
   const float scale = effective_scale(s);
   const bool out_f32 = (o_dtype == BA_DTYPE_F32);
+  if (use_tensor_core_path(s) && s->block == 256 && s->d == 128) {
+    // a 256-row query block on a CTA pair (cta_group::2): each CTA holds 32
+    // keys of every K half, so the K map has 32-row boxes
+    CUtensorMap mq, mk, mv;
+    if (!make_head_map(&mq, Q, s->d, Nq, q_stride, static_cast<long long>(s->B) * s->Hq, tc::kTileRows) ||
+        !make_head_map(&mk, K, s->d, s->N, s->N_alloc, static_cast<long long>(s->B) * s->Hkv, tc2::kKRows) ||
+        !make_head_map(&mv, V, s->d, s->N, s->N_alloc, static_cast<long long>(s->B) * s->Hkv, tc::kKvBoxRows))
+      return BA_ERR_CUDA;
+    const long long ctas = 2LL * s->B * s->Hq * nb;
+    if (ctas > 0x7FFFFFFFLL) return BA_ERR_UNSUPPORTED;
+    const float sl2 = scale * 1.4426950408889634f;
+    const uint32_t smem = tc2::kDynSmem;
+    auto run = [&](auto kernel, auto *out) -> ba_status {
+      cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+      if (e != cudaSuccess) return BA_ERR_CUDA;
+      kernel<<<static_cast<unsigned>(ctas), tc::kThreads, smem, cs>>>(mq, mk, mv, kv_idx, kv_cnt, kmax, out, LSE, O_prev,
+                                                                   L_prev, s->Hq, s->Hkv, s->N, Nq, q_stride, nb,
+                                                                   nkblocks(s), kblock(s), sl2);
+      return from_cuda(cudaGetLastError());
+    };
+    if (out_f32) {
+      float *of = static_cast<float *>(O);
+      return merge ? run(tc2::attn_tc2_kernel<float, true>, of) : run(tc2::attn_tc2_kernel<float, false>, of);
+    }
+    __nv_bfloat16 *ob = static_cast<__nv_bfloat16 *>(O);
+    return merge ? run(tc2::attn_tc2_kernel<__nv_bfloat16, true>, ob)
+                 : run(tc2::attn_tc2_kernel<__nv_bfloat16, false>, ob);
+  }
   if (use_tensor_core_path(s)) {
     CUtensorMap mq, mk, mv;
     if (!make_head_map(&mq, Q, s->d, Nq, q_stride, static_cast<long long>(s->B) * s->Hq, tc::kTileRows) ||

@@ -126,6 +126,9 @@ SMALL = [
     ("dlm_16k", dict(N=4096, Hq=4, Hkv=2, block=256), 0.5),          # tcgen05 path, 256-row blocks
     ("dlm_16k", dict(N=3 * 256 + 200, N_alloc=1024, Hq=2, Hkv=1, block=256), 0.5),   # 256-row blocks, ragged
     ("dlm_16k", dict(N=2048 - 40, N_alloc=2048, Hq=4, Hkv=2, d=64, block=256), 0.5),  # 256-row blocks, d = 64
+    ("dlm_16k", dict(N=2 * 256 + 60, N_alloc=640, Hq=2, Hkv=1, block=256), 0.5),   # CTA pair: rank 1 of the last block holds no row
+    ("dlm_16k", dict(N=3072 - 50, N_alloc=3072, B=2, Hq=8, Hkv=2, block=256), 0.3),   # CTA pair: B = 2, 4 heads per KV head
+    ("dlm_16k", dict(N=4096 - 70, N_alloc=4096, Hq=2, Hkv=1, block=256, block_k=256), 0.5),   # CTA pair, 256 x 256
     # asymmetric blocks: query blocks of `block` rows, key blocks of `block_k` rows
     ("dlm_16k", dict(N=2048 - 30, N_alloc=2048, Hq=4, Hkv=2, block_k=64), 0.5),      # tcgen05, 128 x 64
     ("dlm_16k", dict(N=2048, Hq=4, Hkv=2, block=256, block_k=128), 0.5),             # tcgen05, 256 x 128
@@ -461,8 +464,9 @@ def test_merge_parity_and_edges(dtype, out, d):
         assert torch.equal(O1d, Om) and torch.equal(L1d, Lm)
 
 
-def test_empty_lists_and_single_block_lists():
-    Q, K, V, meta = make_inputs("dlm_16k", N=1024, Hq=2, Hkv=1)
+@pytest.mark.parametrize("block", [128, 256])
+def test_empty_lists_and_single_block_lists(block):
+    Q, K, V, meta = make_inputs("dlm_16k", N=1024, Hq=2, Hkv=1, block=block)
     w = meta["workload"]
     Qd, Kd, Vd = to_dev(Q, "bf16"), to_dev(K, "bf16"), to_dev(V, "bf16")
     shape = api.Shape.of(Qd, Kd, w.N, w.block)
@@ -506,7 +510,7 @@ def test_post_downsample_mass_via_single_block_lists():
 def test_device_checks_flag_bad_lists_without_trapping():
     Q, K, V, meta = make_inputs("dlm_16k", N=1024, Hq=2, Hkv=1)
     w = meta["workload"]
-    for dtype, d, block in (("bf16", 128, 128), ("f32", 128, 64)):
+    for dtype, d, block in (("bf16", 128, 128), ("bf16", 128, 256), ("f32", 128, 64)):
         Qd, Kd, Vd = to_dev(Q, dtype), to_dev(K, dtype), to_dev(V, dtype)
         shape = api.Shape.of(Qd, Kd, w.N, block)
         nb = shape.nb
