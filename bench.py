@@ -384,11 +384,18 @@ def check_device(api, when):
         raise RuntimeError(f"device error word {word:#x} {when}")
 
 
+def attention_kernel_name(w):
+    """The attention kernel the library runs for this workload's shape."""
+    if w.dtype != "bf16" or w.block not in (64, 128, 256) or w.d not in (64, 128):
+        return "attn_simt_kernel"
+    return "attn_tc2_kernel (256-row blocks on a CTA pair)" if (w.block == 256 and w.d == 128) else "attn_tc_kernel"
+
+
 def attention_roofline(step, t, flops, peaks, peak_src, traffic=None):
     att_ms = sum(t["stage_ms"][n] for n in step.attention)
     achieved = flops / (att_ms * 1e-3) / 1e12
     return {"bound": "tensor",
-            "kernel": "attn_tc_kernel" + (" (both span launches of a step; the second also merges the first "
+            "kernel": attention_kernel_name(step.w) + (" (both span launches of a step; the second also merges the first "
                                           "span's fp32 partial in its epilogue)" if step.split_block is not None
                                           else " (one launch per step)"),
             "achieved": round(achieved, 1), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
@@ -715,10 +722,12 @@ def main(argv=None):
             if name != args.workload:
                 by[name] = run_workload_entry(name, args.keep, ctx["dev"], ctx["clock_id"])
         if not args.block and args.workload == "sweep_32k":
-            # the rest of the 32K keep sweep, and the 64-row query blocks at keep 0.5
+            # the rest of the 32K keep sweep, and 64- and 256-row query blocks at keep 0.5
             by["sweep_32k@keep0.25"] = run_workload_entry("sweep_32k", 0.25, ctx["dev"], ctx["clock_id"])
             by["sweep_32k@block64"] = run_workload_entry("sweep_32k", args.keep, ctx["dev"], ctx["clock_id"],
                                                          block=64)
+            by["sweep_32k@block256"] = run_workload_entry("sweep_32k", args.keep, ctx["dev"], ctx["clock_id"],
+                                                          block=256)
         result["by_workload"] = by
     if rank == 0:
         if not args.no_cpu_baseline:

@@ -311,11 +311,13 @@ ba_status ba_att_complement_lists(const ba_att_shape *shape, const int32_t *kv_i
  *           (one rounding in total when partials are merged later).
  * LSE       device fp32 [B, Hq, N_alloc], natural log (written).
  * Paths: bf16 with d = 64 or 128, block = 64, 128 or 256 and key blocks of
- * 64, 128 or 256 rows runs the tcgen05/TMEM tensor-core kernel (a 256-row
- * block is two 128-row query tiles sharing its list; two 64-row blocks
- * share one 128-row tile, which attends the union of their lists, each row
- * masking the key blocks its own list leaves out; key blocks are taken as
- * 64-key halves); every other supported shape runs an fp32 CUDA-core kernel.
+ * 64, 128 or 256 rows runs the tcgen05/TMEM tensor-core kernel (key blocks
+ * are taken as 64-key halves). A 256-row block with d = 128 runs on a pair
+ * of CTAs (a 2-CTA cluster, cta_group::2 MMAs of 256 rows) that share each
+ * K/V half; with d = 64 it is two 128-row tiles sharing its list. Two
+ * 64-row blocks share one 128-row tile, which attends the union of their
+ * lists, each row masking the key blocks its own list leaves out. Every
+ * other supported shape runs an fp32 CUDA-core kernel.
  */
 ba_status ba_att_sparse_fwd(const ba_att_shape *shape,
                             const void *Q, const void *K, const void *V,

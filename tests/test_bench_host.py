@@ -123,3 +123,14 @@ def test_step_config_names_the_step_form():
     split = bench.step_config(WORKLOADS["extreme_128k"], 0.5, 512, 77, 1)
     assert split["split_block"] == 77 and "sparse_fwd_merge" in split["workload"]
     assert bench.LAUNCHES_PER_STEP[False] == 4 and bench.LAUNCHES_PER_STEP[True] == 6
+
+
+def test_attention_kernel_name_follows_the_library_dispatch():
+    from block_sparse_attention_ba_b200.workloads import WORKLOADS
+    w = WORKLOADS["sweep_32k"]
+    assert bench.attention_kernel_name(w) == "attn_tc_kernel"
+    assert bench.attention_kernel_name(w.with_(block=64)) == "attn_tc_kernel"
+    assert bench.attention_kernel_name(w.with_(block=256)).startswith("attn_tc2_kernel")
+    assert bench.attention_kernel_name(w.with_(block=256, d=64)) == "attn_tc_kernel"
+    assert bench.attention_kernel_name(w.with_(block=32)) == "attn_simt_kernel"
+    assert bench.attention_kernel_name(WORKLOADS["tiny_fp32"]) == "attn_simt_kernel"
