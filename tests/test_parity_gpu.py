@@ -156,6 +156,44 @@ def test_small_full_parity(name, over, keep):
         assert (Od[:, :, w.N:] == 7.0).all() and (Ld[:, :, w.N:] == 7.0).all()
 
 
+@pytest.mark.parametrize("block_k", [128, 256])
+@pytest.mark.parametrize("merge", [False, True])
+def test_cta_pair_equals_two_single_tiles(block_k, merge):
+    # A 256-row query block on the CTA pair computes, per 128-row half, what
+    # the one-CTA kernel computes for a 128-row block holding the same list:
+    # the same key halves in the same order, the same MMA k-steps. The two
+    # are compared bit for bit (the pair against the kernel the oracle pins).
+    Q, K, V, meta = make_inputs("dlm_16k", N=1536 - 70, N_alloc=1536, Hq=4, Hkv=2)
+    w = meta["workload"]
+    Qd, Kd, Vd = to_dev(Q, "bf16"), to_dev(K, "bf16"), to_dev(V, "bf16")
+    s256 = api.Shape.of(Qd, Kd, w.N, 256, block_k=block_k)
+    s128 = api.Shape.of(Qd, Kd, w.N, 128, block_k=block_k)
+    idx, cnt = api.select(api.stats(Qd, Kd, s256), s256, 0.5)
+    idx[0, 1, 2] = torch.arange(idx.shape[-1], device="cuda", dtype=torch.int32)    # consecutive blocks
+    cnt[0, 2, 1] = 0                                                   # one empty list
+    idx128 = idx.repeat_interleave(2, dim=2)[:, :, : s128.nb].contiguous()
+    cnt128 = cnt.repeat_interleave(2, dim=2)[:, :, : s128.nb].contiguous()
+    if merge:
+        g = torch.Generator(device="cuda").manual_seed(5)
+        Op = torch.randn(Qd.shape, device="cuda", generator=g)
+        Lp = torch.randn((w.B, w.Hq, w.N_alloc), device="cuda", generator=g)
+        O2, L2 = api.sparse_fwd_merge(Qd, Kd, Vd, idx, cnt, s256, Op, Lp)
+        O1, L1 = api.sparse_fwd_merge(Qd, Kd, Vd, idx128, cnt128, s128, Op, Lp)
+    else:
+        O2, L2 = api.sparse_fwd(Qd, Kd, Vd, idx, cnt, s256)
+        O1, L1 = api.sparse_fwd(Qd, Kd, Vd, idx128, cnt128, s128)
+    torch.cuda.synchronize()
+    n = w.N
+    assert torch.equal(O2[:, :, :n], O1[:, :, :n]) and torch.equal(L2[:, :, :n], L1[:, :, :n])
+    Oref, Lref = O.masked_attention(Q, K, V, idx.cpu().numpy(), cnt.cpu().numpy(), n, 256, w.d ** -0.5, b_k=block_k)
+    if not merge:
+        assert max_abs(O2[:, :, :n].float().cpu().numpy(), Oref[:, :, :n]) <= TOL["bf16"]["max_abs"]
+        got_l = L2[:, :, :n].cpu().numpy()
+        fin = np.isfinite(Lref[:, :, :n])
+        assert (np.isneginf(got_l) == ~fin).all()
+        assert np.abs(got_l[fin] - Lref[:, :, :n][fin]).max() <= TOL["bf16"]["lse_abs"]
+
+
 @pytest.mark.parametrize("name,over", [("tiny_fp32", {}), ("dlm_16k", dict(N=1536, Hq=4, Hkv=2)),
                                        ("dlm_16k", dict(N=1536 - 9, N_alloc=1536, Hq=4, Hkv=2, d=64)),
                                        ("dlm_16k", dict(N=1536, Hq=4, Hkv=2, block=256)),
