@@ -19,7 +19,8 @@
 //     multicast to the same barrier in both CTAs (S ready, K/V slot free,
 //     PV done, O final).
 //   - Each CTA's softmax warps work on its own 128 rows in its own TMEM, as
-//     in attn_tc.cuh, and arrive on the leader's P barrier (256 arrivals).
+//     in attn_tc.cuh, and arrive on the leader's P barrier (one arrival per
+//     warp, eight in all).
 //   - A cluster barrier after the barrier set-up and before teardown keeps
 //     either CTA from signalling, or writing into, a CTA that is not there.
 // TMEM: S (128 columns) and O (128 columns) in each CTA, allocated for the
