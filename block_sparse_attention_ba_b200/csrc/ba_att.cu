@@ -450,8 +450,9 @@ ba_status sparse_fwd_impl(const ba_att_shape *s, const void *Q, const void *K, c
         !make_head_map(&mk, K, s->d, s->N, s->N_alloc, static_cast<long long>(s->B) * s->Hkv, tc::kKvBoxRows) ||
         !make_head_map(&mv, V, s->d, s->N, s->N_alloc, static_cast<long long>(s->B) * s->Hkv, tc::kKvBoxRows))
       return BA_ERR_CUDA;
-    // one CTA per 128-row query tile (a 256-row block is two tiles sharing its
-    // list; two 64-row blocks share one tile, which attends both lists)
+    // one CTA per 128-row query tile (a 256-row block at d = 64 is two tiles
+    // sharing its list; two 64-row blocks share one tile, which attends both
+    // lists)
     const long long tiles = static_cast<long long>(s->B) * s->Hq *
                             (s->block >= tc::kTileRows ? static_cast<long long>(nb) * (s->block / tc::kTileRows)
                                                        : (nb + 1) / 2);
