@@ -617,6 +617,33 @@ def test_fuzz_small_shapes(seed):
     check_attention(r, Q, K, V, w, all_blocks(w))
 
 
+@pytest.mark.parametrize("seed", range(5))
+def test_fuzz_cta_pair(seed):
+    # 256-row query blocks at d = 128 (the CTA pair) on random shapes: ragged
+    # tails (a pair whose second CTA holds no row included), GQA ratios, key
+    # blocks of 64, 128 or 256 rows, keep ratios from sparse to dense
+    rng = np.random.default_rng(500 + seed)
+    block_k = int(rng.choice([64, 128, 256]))
+    Hkv = int(rng.integers(1, 3))
+    Hq = Hkv * int(rng.integers(1, 4))
+    N = int(rng.integers(257, 9 * 256))
+    if seed == 0:
+        N = 2 * 256 + 40                          # the last pair's second CTA is past the end
+    N_alloc = N + int(rng.integers(0, 40))
+    B = int(rng.integers(1, 3))
+    keep = float(rng.uniform(0.05, 1.0))
+    Q = rng.standard_normal((B, Hq, N_alloc, 128)).astype(np.float32)
+    K = rng.standard_normal((B, Hkv, N_alloc, 128)).astype(np.float32)
+    V = rng.standard_normal((B, Hkv, N_alloc, 128)).astype(np.float32)
+    from block_sparse_attention_ba_b200.workloads import Workload, round_to
+    Q, K, V = (round_to(x, "bf16") for x in (Q, K, V))
+    w = Workload("fuzz", B, Hq, Hkv, N, N_alloc, 128, 256, "bf16", (keep,), seed, "iid_planted", block_k=block_k)
+    r = run_gpu(Q, K, V, w, keep, kmax=O.keep_count(keep, w.nk) + 2)
+    st = check_stats(r, Q, K, w)
+    check_selection(r, st, w, keep)
+    check_attention(r, Q, K, V, w, all_blocks(w))
+
+
 # ------------------------------------------------------------- full-size cases
 
 @pytest.mark.parametrize("name", ["dlm_16k", "sweep_32k", "video_32k", "extreme_128k"])
